@@ -1,0 +1,214 @@
+/*
+ * mx.h -- C ABI of libmx: the MX (microscaling) cast and the block-scaled
+ * GEMM on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the pages:
+ *  - "Microscaling Data Formats for Deep Learning" (summary page), section 2
+ *    "Microscaling": an MX block holds k = 32 values as one shared E8M0 scale X
+ *    and 32 narrow elements P_i, v_i = X * P_i; a NaN scale (code 0xFF) makes
+ *    the whole block NaN; the storage layout is left to the implementation.
+ *  - same page, section 3 "Scalar Float to MX Format Conversion" (Algorithm 1):
+ *    X = 2^(floor(log2 amax) - emax_elem), P_i = quantize(V_i / X) with
+ *    overflow clamped to the element format's largest normal, and FP32
+ *    subnormal inputs set to zero; the block axis is a parameter because the
+ *    cast does not commute with a transpose.
+ *  - same page, section 4, compute flow: dot products consume MX operands and
+ *    return scalar floats (here fp32 accumulation, fp32 or bf16 output).
+ *  - "Format-Aware Fusion for Fast FP4 Pretraining" (abstract): stochastic
+ *    rounding and a fixed-sign 32-point Hadamard before the FP4 cast of the
+ *    weight-gradient operands.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers named x, codes, scales, y, c, a_*, b_* are DEVICE pointers
+ *    (cudaMalloc'd or torch-allocated on the current device) unless the name
+ *    says otherwise.  The caller owns all of them; the library never frees,
+ *    retains or allocates device buffers (it keeps one status word per device
+ *    in a static __device__ variable).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Every call only enqueues work on it and returns; nothing
+ *    synchronises unless stated.
+ *  - Return value: MX_OK (0) or a negative mx_status.  Argument errors are
+ *    detected on the host before anything is launched; the output buffers are
+ *    then untouched.  An empty tensor (a zero size) is a no-op returning MX_OK,
+ *    and its pointers may then be NULL.
+ *  - All 2-D tensors are row-major with an explicit leading dimension
+ *    (elements between consecutive rows).
+ *
+ * Storage layout (section 2 leaves it to the implementation)
+ *  - Element codes are stored "block-axis-major": one row per line along the
+ *    block axis ("outer" rows of "inner" elements, inner % 32 == 0).  Quantizing
+ *    an R x C tensor along C gives R rows of C codes; along R it gives C rows of
+ *    R codes (transposed on the way out).  Rows are packed with no padding:
+ *    8-bit formats one code per byte; FP6 four codes per 3 bytes (code j of a
+ *    group in bits 6j..6j+5 of a little-endian 24-bit word); FP4 two codes per
+ *    byte, the even element in the low nibble.
+ *  - Element encodings: E4M3 (bias 7, NaN S.1111.111, no Inf), E5M2 (bias 15,
+ *    IEEE Inf/NaN), E2M3 (bias 1), E3M2 (bias 3), E2M1 (bias 1), INT8 (two's
+ *    complement, value = code * 2^-6).  Scale codes are E8M0: 2^(s-127), 0xFF
+ *    is NaN.
+ *  - Scales, MX_SCALES_PLAIN: outer x (inner/32) bytes, row-major.
+ *    MX_SCALES_MMA: the layout the tensor cores read.  Rows are padded to a
+ *    multiple of 128 and k-blocks to a multiple of 4; the buffer is a sequence
+ *    of 512-byte atoms, one per (128-row block, 4-k-block group), k-groups
+ *    fastest; inside an atom the byte for row r, k-block kb is at
+ *    (r % 32) * 16 + ((r / 32) % 4) * 4 + (kb % 4).  Padding bytes are never
+ *    written by mx_quantize.
+ */
+#ifndef MX_H
+#define MX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__) || defined(__clang__)
+#define MX_API __attribute__((visibility("default")))
+#else
+#define MX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MX_E4M3 = 0,  /* MXFP8, 4-bit exponent, 3-bit mantissa, emax 8,  max 448   */
+    MX_E5M2 = 1,  /* MXFP8, 5-bit exponent, 2-bit mantissa, emax 15, max 57344 */
+    MX_E2M3 = 2,  /* MXFP6, emax 2, max 7.5 */
+    MX_E3M2 = 3,  /* MXFP6, emax 4, max 28  */
+    MX_E2M1 = 4,  /* MXFP4, emax 2, max 6   */
+    MX_INT8 = 5   /* MXINT8, emax 0, max 127/64 (symmetric; -128 is never produced) */
+} mx_fmt;
+
+typedef enum { MX_F32 = 0, MX_BF16 = 1 } mx_dtype;
+
+typedef enum {
+    MX_RNE = 0,   /* round to nearest, ties to even mantissa (even integer for INT8) */
+    MX_SR = 1     /* stochastic rounding, see mx_quantize */
+} mx_round;
+
+typedef enum { MX_SCALES_PLAIN = 0, MX_SCALES_MMA = 1 } mx_scale_layout;
+
+/* Optional preconditioning of each 32-block before the cast.
+ * hadamard != 0: x_j <- s_j * x_j with s_j = +1 where bit j of sign_mask is
+ * set and -1 elsewhere (j = position inside the block along the block axis),
+ * then the unnormalised 32-point Sylvester Hadamard transform as five fp32
+ * butterfly stages (h = 1, 2, 4, 8, 16; (a, b) -> (a + b, a - b)).  The
+ * transform is orthogonal up to a factor 32, so a GEMM of two operands
+ * preconditioned with the same mask along the reduction axis recovers the
+ * plain product with alpha = 1/32. */
+typedef struct {
+    int32_t hadamard;
+    uint32_t sign_mask;
+} mx_precond;
+
+#define MX_DEFAULT_SIGN_MASK 0x6A09E667u
+
+typedef enum {
+    MX_OK = 0,
+    MX_ERR_ARG = -1,          /* null pointer, bad enum, negative size, ld too small   */
+    MX_ERR_ALIGN = -2,        /* pointer or leading dimension breaks the 16-byte rules  */
+    MX_ERR_SHAPE = -3,        /* block-axis length not a multiple of 32                 */
+    MX_ERR_UNSUPPORTED = -4,  /* valid request that this build does not implement       */
+    MX_ERR_SR_RANGE = -5,     /* stochastic rounding index space exceeds 2^34 elements  */
+    MX_ERR_CUDA = -6,         /* a CUDA runtime/driver call or launch failed            */
+    MX_ERR_TIMEOUT = -7       /* a bounded device-side wait expired (see below)         */
+} mx_status;
+
+/*
+ * mx_quantize -- Algorithm 1 of section 3 on every 32-block along block_axis.
+ *
+ *  x          device, rows x cols, leading dimension ldx (elements), dtype xdt.
+ *             16-byte aligned; ldx * sizeof(elem) must be a multiple of 16.
+ *  block_axis 1: blocks run along a row (contiguous).  codes: rows x cols.
+ *             0: blocks run down a column (strided).   codes: cols x rows.
+ *  fmt        element format.
+ *  rnd        MX_RNE, or MX_SR: with lo <= |u| < hi the neighbouring grid
+ *             points of u = V/X, F = floor(256 (|u| - lo) / (hi - lo)), and the
+ *             magnitude rounds up iff F + r >= 256, where r is byte (i mod 4)
+ *             of fmix32(floor(i / 4) xor (fmix32(seed_lo32) xor seed_hi32)),
+ *             i the element's linear index in the output (outer * inner +
+ *             position along the block axis) and fmix32 the MurmurHash3
+ *             32-bit finaliser.  Results therefore do not depend on tiling.
+ *  seed       only read for MX_SR.
+ *  pre        NULL, or preconditioning (see mx_precond).  Non-NULL with
+ *             hadamard != 0 is supported for block_axis 0 only.
+ *  codes      device, mx_codes_bytes(fmt, outer, inner) bytes, 16-byte aligned.
+ *  scales     device, mx_scales_bytes(sl, outer, inner) bytes.
+ *  sl         scale layout to write.
+ *
+ * Per block: FP32 subnormals (after preconditioning, and bf16 subnormals,
+ * which widen to FP32 subnormals) become signed zeros; a NaN or Inf anywhere
+ * gives scale 0xFF and all-zero codes; amax == 0 gives scale code 0; else
+ * e = clamp(floor(log2 amax) - emax, -127, 127) and the scale code is e + 127.
+ * Elements are rounded to the grid with overflow clamped to +-max; FP formats
+ * keep the sign of zero.
+ * Errors: MX_ERR_ARG, MX_ERR_ALIGN, MX_ERR_SHAPE (inner % 32 != 0),
+ * MX_ERR_UNSUPPORTED, MX_ERR_SR_RANGE, MX_ERR_CUDA.
+ */
+MX_API int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
+                const mx_precond *pre, void *codes, void *scales, mx_scale_layout sl,
+                void *stream);
+
+/*
+ * mx_dequantize -- v = X * P (section 2), exact, rounded once to ydt.
+ *
+ *  codes, scales  device, as written by mx_quantize for (outer, inner).
+ *  y              device, outer x inner, leading dimension ldy (elements),
+ *                 16-byte aligned, ldy * sizeof(ydt) a multiple of 16.
+ * A 0xFF scale gives NaN for its whole block; values beyond the output
+ * type's range become +-Inf.
+ * Errors: MX_ERR_ARG, MX_ERR_ALIGN, MX_ERR_SHAPE, MX_ERR_CUDA.
+ */
+MX_API int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_scale_layout sl,
+                  int64_t outer, int64_t inner, void *y, mx_dtype ydt, int64_t ldy,
+                  void *stream);
+
+/*
+ * mx_gemm -- C = alpha * A * B^T, the block-scaled matmul of section 4's
+ * compute flow on the fifth-generation tensor cores.
+ *
+ *  a_codes  device, M x K codes of format fa, quantized along K
+ *           (block_axis 1 of an M x K tensor), 16-byte aligned.
+ *  a_scales device, MX_SCALES_MMA layout for (M, K).
+ *  b_codes  device, N x K codes of format fb, quantized along K.
+ *  b_scales device, MX_SCALES_MMA layout for (N, K).
+ *  c        device, M x N, leading dimension ldc, type cdt (fp32 or bf16,
+ *           rounded to nearest even from the fp32 accumulator).
+ *  workspace / ws_bytes  reserved; pass NULL / 0 (mx_gemm_workspace_bytes
+ *           returns 0 in this build).
+ * Supported: fa == fb in {MX_E4M3, MX_E5M2} (kind::mxf8f6f4, K % 128 == 0)
+ * and fa == fb == MX_E2M1 (kind::mxf4, K % 256 == 0); any M, N >= 1.
+ * Accumulation is fp32 on the tensor cores; |C - C_exact| stays within
+ * 1e-5 * |alpha| * sum_k |a_mk b_nk| in the tested configurations.
+ * Errors: MX_ERR_ARG, MX_ERR_ALIGN, MX_ERR_SHAPE, MX_ERR_UNSUPPORTED,
+ * MX_ERR_CUDA.  A pipeline wait that exceeds its bound ends the kernel early
+ * and records MX_ERR_TIMEOUT, read with mx_last_device_status.
+ */
+MX_API int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
+            const void *b_codes, const void *b_scales, mx_fmt fb,
+            int64_t M, int64_t N, int64_t K, float alpha,
+            void *c, mx_dtype cdt, int64_t ldc, void *workspace, size_t ws_bytes,
+            void *stream);
+
+/* Byte sizes of the buffers above (0 for invalid arguments). */
+MX_API size_t mx_codes_bytes(mx_fmt fmt, int64_t outer, int64_t inner);
+MX_API size_t mx_scales_bytes(mx_scale_layout sl, int64_t outer, int64_t inner);
+MX_API size_t mx_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Synchronises `stream`, then returns and clears the current device's status
+ * word: MX_OK, or MX_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * last call.  MX_ERR_CUDA if the synchronisation itself failed. */
+MX_API int mx_last_device_status(void *stream);
+
+/* Static description of a status code. */
+MX_API const char *mx_status_str(int status);
+
+/* ABI version of this header: 1. */
+MX_API int mx_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MX_H */

@@ -1,0 +1,163 @@
+// mx_api.cu -- the C ABI of libmx (declared in include/mx.h): argument
+// validation, status codes and launches on the caller's stream.  No entry
+// point allocates device memory or synchronises, except
+// mx_last_device_status, which synchronises the given stream by contract.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "mx.h"
+#include "mx_internal.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];   // 0 = not queried yet
+
+int sm_count(int *device_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (device_out) *device_out = dev;
+    if (dev < 0 || dev >= kMaxDevices) return -1;
+    if (g_sm_count[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        g_sm_count[dev] = n;
+    }
+    return g_sm_count[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bits(int fmt) {
+    switch (fmt) {
+        case MX_E4M3: case MX_E5M2: case MX_INT8: return 8;
+        case MX_E2M3: case MX_E3M2: return 6;
+        case MX_E2M1: return 4;
+        default: return 0;
+    }
+}
+
+int dtype_bytes(int dt) { return dt == MX_F32 ? 4 : (dt == MX_BF16 ? 2 : 0); }
+
+}  // namespace
+
+extern "C" {
+
+int mx_abi_version(void) { return 1; }
+
+const char *mx_status_str(int status) {
+    switch (status) {
+        case MX_OK: return "MX_OK";
+        case MX_ERR_ARG: return "MX_ERR_ARG: invalid argument (null pointer, bad enum or size)";
+        case MX_ERR_ALIGN: return "MX_ERR_ALIGN: pointer or leading dimension not 16-byte aligned";
+        case MX_ERR_SHAPE: return "MX_ERR_SHAPE: block-axis length is not a multiple of 32";
+        case MX_ERR_UNSUPPORTED: return "MX_ERR_UNSUPPORTED: combination not implemented";
+        case MX_ERR_SR_RANGE: return "MX_ERR_SR_RANGE: stochastic-rounding index space exceeds 2^34";
+        case MX_ERR_CUDA: return "MX_ERR_CUDA: CUDA call or kernel launch failed";
+        case MX_ERR_TIMEOUT: return "MX_ERR_TIMEOUT: a bounded device wait expired";
+        default: return "unknown mx status";
+    }
+}
+
+size_t mx_codes_bytes(mx_fmt fmt, int64_t outer, int64_t inner) {
+    const int b = elem_bits(fmt);
+    if (b == 0 || outer < 0 || inner < 0 || inner % 32 != 0) return 0;
+    return static_cast<size_t>(outer) * static_cast<size_t>(inner / 32 * 4 * b);
+}
+
+size_t mx_scales_bytes(mx_scale_layout sl, int64_t outer, int64_t inner) {
+    if (outer < 0 || inner < 0 || inner % 32 != 0) return 0;
+    const int64_t kb = inner / 32;
+    if (sl == MX_SCALES_PLAIN) return static_cast<size_t>(outer * kb);
+    if (sl != MX_SCALES_MMA) return 0;
+    return static_cast<size_t>((outer + 127) / 128 * 128) * static_cast<size_t>((kb + 3) / 4 * 4);
+}
+
+size_t mx_gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+
+int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
+                const mx_precond *pre, void *codes, void *scales, mx_scale_layout sl,
+                void *stream) {
+    if ((xdt != MX_F32 && xdt != MX_BF16) || elem_bits(fmt) == 0) return MX_ERR_ARG;
+    if ((rnd != MX_RNE && rnd != MX_SR) || (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA)) return MX_ERR_ARG;
+    if (block_axis != 0 && block_axis != 1) return MX_ERR_ARG;
+    if (rows < 0 || cols < 0) return MX_ERR_ARG;
+    const int64_t outer = block_axis == 1 ? rows : cols;
+    const int64_t inner = block_axis == 1 ? cols : rows;
+    if (inner % 32 != 0) return MX_ERR_SHAPE;
+    if (outer == 0 || inner == 0) return MX_OK;          // empty: pointers may be NULL
+    if (!x || !codes || !scales) return MX_ERR_ARG;
+    if (ldx < cols) return MX_ERR_ARG;
+    if (!aligned16(x) || (ldx * dtype_bytes(xdt)) % 16 != 0 || !aligned16(codes)) return MX_ERR_ALIGN;
+    const bool had = pre && pre->hadamard;
+    if (had && block_axis != 0) return MX_ERR_UNSUPPORTED;
+    if (rnd == MX_SR && static_cast<uint64_t>(outer) * static_cast<uint64_t>(inner) > (1ull << 34))
+        return MX_ERR_SR_RANGE;
+
+    MxQuantizeArgs a;
+    a.x = x; a.xdt = xdt; a.rows = rows; a.cols = cols; a.ldx = ldx;
+    a.block_axis = block_axis; a.fmt = fmt; a.rnd = rnd; a.seed = seed;
+    a.hadamard = had; a.sign_mask = had ? pre->sign_mask : 0u;
+    a.codes = codes; a.scales = scales; a.sl = sl;
+    a.num_sms = sm_count(nullptr);
+    if (a.num_sms <= 0) return MX_ERR_CUDA;
+    return mx_launch_quantize(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_scale_layout sl,
+                  int64_t outer, int64_t inner, void *y, mx_dtype ydt, int64_t ldy, void *stream) {
+    if (elem_bits(fmt) == 0 || (ydt != MX_F32 && ydt != MX_BF16)) return MX_ERR_ARG;
+    if (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA) return MX_ERR_ARG;
+    if (outer < 0 || inner < 0) return MX_ERR_ARG;
+    if (inner % 32 != 0) return MX_ERR_SHAPE;
+    if (outer == 0 || inner == 0) return MX_OK;          // empty: pointers may be NULL
+    if (!codes || !scales || !y || ldy < inner) return MX_ERR_ARG;
+    if (!aligned16(codes) || !aligned16(y) || (ldy * dtype_bytes(ydt)) % 16 != 0) return MX_ERR_ALIGN;
+    MxDequantArgs a;
+    a.codes = codes; a.scales = scales; a.fmt = fmt; a.sl = sl;
+    a.outer = outer; a.inner = inner; a.y = y; a.ydt = ydt; a.ldy = ldy;
+    a.num_sms = sm_count(nullptr);
+    if (a.num_sms <= 0) return MX_ERR_CUDA;
+    return mx_launch_dequantize(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
+            const void *b_codes, const void *b_scales, mx_fmt fb,
+            int64_t M, int64_t N, int64_t K, float alpha,
+            void *c, mx_dtype cdt, int64_t ldc, void *workspace, size_t ws_bytes, void *stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    if (elem_bits(fa) == 0 || elem_bits(fb) == 0 || (cdt != MX_F32 && cdt != MX_BF16)) return MX_ERR_ARG;
+    if (M < 0 || N < 0 || K < 0) return MX_ERR_ARG;
+    if (K % 32 != 0) return MX_ERR_SHAPE;
+    if (M == 0 || N == 0) return MX_OK;                  // empty: pointers may be NULL
+    if (!c || ldc < N) return MX_ERR_ARG;
+    if (K > 0 && (!a_codes || !a_scales || !b_codes || !b_scales)) return MX_ERR_ARG;
+    const bool fp8 = (fa == MX_E4M3 || fa == MX_E5M2) && (fb == MX_E4M3 || fb == MX_E5M2);
+    const bool fp4 = fa == MX_E2M1 && fb == MX_E2M1;
+    if (!fp8 && !fp4) return MX_ERR_UNSUPPORTED;
+    if ((fp8 && K % 128 != 0) || (fp4 && K % 256 != 0)) return MX_ERR_UNSUPPORTED;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
+        !aligned16(c) || (ldc * dtype_bytes(cdt)) % 16 != 0)
+        return MX_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) {
+        const size_t esz = static_cast<size_t>(dtype_bytes(cdt));
+        return cudaMemset2DAsync(c, ldc * esz, 0, N * esz, M, st) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+    }
+    MxGemmArgs a;
+    a.a_codes = a_codes; a.a_scales = a_scales; a.b_codes = b_codes; a.b_scales = b_scales;
+    a.fa = fa; a.fb = fb; a.M = M; a.N = N; a.K = K; a.alpha = alpha;
+    a.c = c; a.cdt = cdt; a.ldc = ldc;
+    a.num_sms = sm_count(&a.device);
+    if (a.num_sms <= 0) return MX_ERR_CUDA;
+    return mx_launch_gemm(a, st);
+}
+
+int mx_last_device_status(void *stream) {
+    return mx_read_device_status(static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+// mx_device.cuh -- device-side MX element formats for sm_100a.
+//
+// The cast of "Microscaling Data Formats for Deep Learning" (summary page,
+// section 3, Algorithm 1): per 32-block, X = 2^(floor(log2 amax) - emax),
+// P_i = round(V_i / X) with overflow clamped to the largest normal and FP32
+// subnormal inputs set to zero.  Rounding to the element grid uses the
+// hardware conversions (cvt.rn.satfinite.{e4m3,e5m2,e2m3,e3m2,e2m1}x2.f32),
+// whose round-to-nearest-even with saturation to the largest finite value is
+// exactly the clamp that section asks for.  Stochastic rounding (the
+// row-gradient rounding of "Format-Aware Fusion for Fast FP4 Pretraining")
+// truncates onto the grid and adds one grid step when the 8 bits below it plus
+// a random byte carry out.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "mx.h"
+
+namespace mxk {
+
+// Per-format constants: code width, emax (exponent of the largest binade),
+// mantissa bits, smallest normal exponent, largest finite value.
+template <int FMT> struct Fmt;
+template <> struct Fmt<MX_E4M3> { static constexpr int bits = 8, emax = 8,  mbits = 3, emin = -6;  static constexpr float maxv = 448.0f; };
+template <> struct Fmt<MX_E5M2> { static constexpr int bits = 8, emax = 15, mbits = 2, emin = -14; static constexpr float maxv = 57344.0f; };
+template <> struct Fmt<MX_E2M3> { static constexpr int bits = 6, emax = 2,  mbits = 3, emin = 0;   static constexpr float maxv = 7.5f; };
+template <> struct Fmt<MX_E3M2> { static constexpr int bits = 6, emax = 4,  mbits = 2, emin = -2;  static constexpr float maxv = 28.0f; };
+template <> struct Fmt<MX_E2M1> { static constexpr int bits = 4, emax = 2,  mbits = 1, emin = 0;   static constexpr float maxv = 6.0f; };
+// INT8: fixed point with 6 fraction bits; treated as one binade with spacing 2^-6.
+template <> struct Fmt<MX_INT8> { static constexpr int bits = 8, emax = 0,  mbits = 6, emin = 0;   static constexpr float maxv = 127.0f / 64.0f; };
+
+__device__ __forceinline__ float pow2f(int k) {  // 2^k for k in [-126, 127]
+    return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+}
+
+// E8M0 scale exponent of a block from the largest |bits| (sign cleared) of
+// its FP32 values.  Returns e with X = 2^e; 0x7f800000 or above means the
+// block held an Inf or NaN (handled by the caller).  Subnormal magnitudes
+// count as zero: they are flushed before the cast.
+template <int FMT>
+__device__ __forceinline__ int block_exponent(uint32_t amax_bits) {
+    if (amax_bits < 0x00800000u) return -127;               // all zero after the flush
+    int e = static_cast<int>(amax_bits >> 23) - 127 - Fmt<FMT>::emax;
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// V * 2^-e with the FP32-subnormal flush folded in: mul.ftz treats subnormal
+// inputs as signed zeros (the section-3 flush); a subnormal product is also
+// flushed, which is harmless because every element format rounds anything
+// below 2^-126 to zero.  e = 127 (only reachable for INT8) takes two steps so
+// that no factor is itself subnormal.
+template <int FMT>
+__device__ __forceinline__ float scale_down(float v, int e) {
+    float r;
+    if (Fmt<FMT>::emax == 0 && e > 126) {
+        asm("mul.rn.ftz.f32 %0, %1, %2;" : "=f"(r) : "f"(v), "f"(pow2f(-64)));
+        asm("mul.rn.ftz.f32 %0, %1, %2;" : "=f"(r) : "f"(r), "f"(pow2f(64 - e)));
+    } else {
+        asm("mul.rn.ftz.f32 %0, %1, %2;" : "=f"(r) : "f"(v), "f"(pow2f(-e)));
+    }
+    return r;
+}
+
+// Round-to-nearest-even with saturation of two FP32 values; returns the codes
+// of a (bits 0..7) and b (bits 8..15), sign bits included.  For FP6 each code
+// sits in the low 6 bits of its byte, for FP4 in the low nibble of bits 0..7
+// (a) and the high nibble (b).
+template <int FMT> __device__ __forceinline__ uint32_t cvt_pair(float a, float b);
+
+template <> __device__ __forceinline__ uint32_t cvt_pair<MX_E4M3>(float a, float b) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(b), "f"(a));
+    return d;
+}
+template <> __device__ __forceinline__ uint32_t cvt_pair<MX_E5M2>(float a, float b) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(d) : "f"(b), "f"(a));
+    return d;
+}
+template <> __device__ __forceinline__ uint32_t cvt_pair<MX_E2M3>(float a, float b) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(b), "f"(a));
+    return d;
+}
+template <> __device__ __forceinline__ uint32_t cvt_pair<MX_E3M2>(float a, float b) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e3m2x2.f32 %0, %1, %2;" : "=h"(d) : "f"(b), "f"(a));
+    return d;
+}
+template <> __device__ __forceinline__ uint32_t cvt_pair<MX_E2M1>(float a, float b) {
+    uint32_t d;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}" : "=r"(d) : "f"(b), "f"(a));
+    return d;
+}
+// INT8: round |v| * 64 to the nearest even integer, clamp to 127, two's complement.
+template <> __device__ __forceinline__ uint32_t cvt_pair<MX_INT8>(float a, float b) {
+    auto one = [](float v) -> uint32_t {
+        float m = rintf(fabsf(v) * 64.0f);
+        int q = static_cast<int>(fminf(m, 127.0f));
+        if (__float_as_uint(v) >> 31) q = -q;
+        return static_cast<uint32_t>(q) & 0xffu;
+    };
+    return one(a) | (one(b) << 8);
+}
+
+// Stochastic rounding of a non-negative FP32 value onto the element grid: with
+// lo the grid point at or below a and s the grid step there, take the 8 bits
+// of (a - lo) / s just below the step, F; the result is lo + s when
+// F + r >= 256, else lo; a >= max gives max.  Every step is exact in FP32.
+template <int FMT>
+__device__ __forceinline__ float sr_magnitude(float a, uint32_t r) {
+    using F = Fmt<FMT>;
+    if (a >= F::maxv) return F::maxv;
+    int ea = static_cast<int>(__float_as_uint(a) >> 23) - 127;   // -127 for 0 / subnormal
+    int E = ea < F::emin ? F::emin : ea;
+    if (FMT == MX_INT8) E = 0;
+    float inv_step = pow2f(F::mbits - E);
+    float step = pow2f(E - F::mbits);
+    float q = a * inv_step;
+    float lo = floorf(q);
+    uint32_t frac8 = static_cast<uint32_t>((q - lo) * 256.0f);
+    float t = (frac8 + r >= 256u) ? lo + 1.0f : lo;
+    return t * step;
+}
+
+// MurmurHash3 32-bit finaliser (public domain, A. Appleby).
+__device__ __forceinline__ uint32_t fmix32(uint32_t h) {
+    h ^= h >> 16;
+    h *= 0x85ebca6bu;
+    h ^= h >> 13;
+    h *= 0xc2b2ae35u;
+    h ^= h >> 16;
+    return h;
+}
+
+// Byte offset of the scale of (outer row o, k-block kb) in the MMA layout:
+// 512-byte atoms of 128 rows x 4 k-blocks, k-groups fastest; inside an atom
+// (o % 32) * 16 + ((o / 32) % 4) * 4 + kb % 4.
+__device__ __forceinline__ int64_t mma_scale_offset(int64_t o, int64_t kb, int64_t k_groups) {
+    int64_t atom = (o >> 7) * k_groups + (kb >> 2);
+    return (atom << 9) + ((o & 31) << 4) + (((o >> 5) & 3) << 2) + (kb & 3);
+}
+
+}  // namespace mxk

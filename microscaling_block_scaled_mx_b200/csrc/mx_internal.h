@@ -1,0 +1,66 @@
+// mx_internal.h -- host-side glue between the C ABI (mx_api.cu) and the
+// kernel launchers.  Arguments reaching these functions are already
+// validated.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "mx.h"
+
+struct MxQuantizeArgs {
+    const void *x;
+    int xdt;
+    int64_t rows, cols, ldx;
+    int block_axis;
+    int fmt;
+    int rnd;
+    uint64_t seed;
+    bool hadamard;
+    uint32_t sign_mask;
+    void *codes;
+    void *scales;
+    int sl;
+    int num_sms;
+};
+
+struct MxDequantArgs {
+    const void *codes;
+    const void *scales;
+    int fmt;
+    int sl;
+    int64_t outer, inner;
+    void *y;
+    int ydt;
+    int64_t ldy;
+    int num_sms;
+};
+
+struct MxGemmArgs {
+    const void *a_codes, *a_scales, *b_codes, *b_scales;
+    int fa, fb;
+    int64_t M, N, K;
+    float alpha;
+    void *c;
+    int cdt;
+    int64_t ldc;
+    int num_sms;
+    int device;
+};
+
+// MurmurHash3 32-bit finaliser on the host (seed key of stochastic rounding).
+inline uint32_t fmix32_host(uint32_t h) {
+    h ^= h >> 16;
+    h *= 0x85ebca6bu;
+    h ^= h >> 13;
+    h *= 0xc2b2ae35u;
+    h ^= h >> 16;
+    return h;
+}
+
+cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st);
+cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st);
+// returns an mx_status (MX_OK, MX_ERR_CUDA, MX_ERR_UNSUPPORTED)
+int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st);
+// reads and clears the device status word of the current device (after a sync)
+int mx_read_device_status(cudaStream_t st);

@@ -408,7 +408,8 @@ int mxref_quantize(const void *x, int xdt, int64_t rows, int64_t cols, int64_t l
     int64_t outer = block_axis == 1 ? rows : cols;
     int64_t inner = block_axis == 1 ? cols : rows;
     if (inner % BLOCK != 0) return MXO_ERR_SHAPE;
-    if (rnd == RND_SR && (uint64_t)(outer * inner) / 4u > 0xffffffffull) return MXO_ERR_SR_RANGE;
+    /* the random-word counter floor(i / 4) must fit 32 bits: at most 2^34 elements */
+    if (rnd == RND_SR && (uint64_t)(outer * inner) > (1ull << 34)) return MXO_ERR_SR_RANGE;
     int64_t kb_total = inner / BLOCK;
     int64_t row_bytes = mxref_codes_bytes(fmt, 1, inner);
 

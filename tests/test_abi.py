@@ -1,0 +1,118 @@
+"""The C ABI (include/mx.h) without a GPU: the library loads, exports every
+declared entry point, sizes agree with the oracle, and host-side argument
+validation returns the documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from microscaling_block_scaled_mx_b200 import build, mx as m
+    build.build()
+    return m
+
+
+def declared_functions():
+    txt = open(os.path.join(ROOT, "include", "mx.h")).read()
+    return sorted(set(re.findall(r"MX_API\s+[\w\s\*]+?\b(mx_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["mx_quantize", "mx_dequantize", "mx_gemm", "mx_codes_bytes", "mx_scales_bytes",
+              "mx_gemm_workspace_bytes", "mx_last_device_status", "mx_status_str", "mx_abi_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(mx):
+    L = mx.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert L.mx_abi_version() == 1
+
+
+def test_status_strings(mx):
+    for code, name in mx.STATUS_NAMES.items():
+        assert mx.status_str(code).startswith(name)
+
+
+@pytest.mark.parametrize("fmt", list(range(6)))
+@pytest.mark.parametrize("outer,inner", [(0, 32), (7, 64), (128, 4096), (300, 96)])
+def test_sizes_agree_with_oracle(mx, oracle, fmt, outer, inner):
+    assert mx.codes_bytes(fmt, outer, inner) == oracle.codes_bytes(fmt, outer, inner)
+    for sl in (0, 1):
+        assert mx.scales_bytes(sl, outer, inner) == oracle.scales_bytes(sl, outer, inner)
+
+
+def test_sizes_reject_bad_shapes(mx):
+    assert mx.codes_bytes(0, 4, 33) == 0
+    assert mx.codes_bytes(9, 4, 32) == 0
+    assert mx.scales_bytes(2, 4, 32) == 0
+
+
+def _q(mx, x=16, dt=1, rows=64, cols=64, ldx=64, axis=1, fmt=0, rnd=0, codes=16, scales=16,
+       sl=1, pre=None):
+    L = mx.lib()
+    return L.mx_quantize(x, dt, rows, cols, ldx, axis, fmt, rnd, 0, pre, codes, scales, sl, None)
+
+
+def test_quantize_validation(mx):
+    assert _q(mx, x=None) == -1
+    assert _q(mx, codes=None) == -1
+    assert _q(mx, dt=7) == -1
+    assert _q(mx, fmt=6) == -1
+    assert _q(mx, rnd=2) == -1
+    assert _q(mx, axis=2) == -1
+    assert _q(mx, sl=3) == -1
+    assert _q(mx, ldx=32) == -1                   # ldx < cols
+    assert _q(mx, rows=-1) == -1
+    assert _q(mx, cols=48, ldx=48) == -3          # along cols, 48 % 32
+    assert _q(mx, rows=48, axis=0) == -3          # along rows, 48 % 32
+    assert _q(mx, x=8) == -2                      # misaligned input
+    assert _q(mx, ldx=68) == -2                   # 68 * 2 bytes is not a multiple of 16
+    assert _q(mx, codes=24) == -2
+    pre = mx._Precond(1, 0xFFFFFFFF)
+    assert _q(mx, pre=ctypes.byref(pre), axis=1) == -4   # Hadamard only on the strided axis
+    assert _q(mx, rnd=1, rows=(1 << 20) + 1, cols=1 << 14, ldx=1 << 14) == -5
+
+
+def test_dequantize_validation(mx):
+    L = mx.lib()
+    assert L.mx_dequantize(None, 16, 0, 1, 4, 64, 16, 0, 64, None) == -1
+    assert L.mx_dequantize(16, 16, 0, 1, 4, 48, 16, 0, 48, None) == -3
+    assert L.mx_dequantize(16, 16, 0, 1, 4, 64, 8, 0, 64, None) == -2
+    assert L.mx_dequantize(16, 16, 0, 1, 4, 32, 16, 1, 36, None) == -2
+
+
+def _g(mx, fa=0, fb=0, M=128, N=128, K=256, c=16, cdt=1, ldc=128, a=16):
+    L = mx.lib()
+    return L.mx_gemm(a, 16, fa, 16, 16, fb, M, N, K, 1.0, c, cdt, ldc, None, 0, None)
+
+
+def test_gemm_validation(mx):
+    assert _g(mx, a=None) == -1
+    assert _g(mx, fa=8) == -1
+    assert _g(mx, M=-1) == -1
+    assert _g(mx, ldc=64) == -1
+    assert _g(mx, K=48) == -3
+    assert _g(mx, fa=5, fb=5) == -4               # no block-scaled INT8 MMA
+    assert _g(mx, fa=0, fb=4) == -4               # mixed FP8 x FP4 not built
+    assert _g(mx, fa=2, fb=2) == -4               # FP6 not built
+    assert _g(mx, K=160) == -4                    # FP8 needs K % 128
+    assert _g(mx, fa=4, fb=4, K=384) == -4        # FP4 needs K % 256
+    assert _g(mx, c=8) == -2
+    assert _g(mx, ldc=129, cdt=1) == -2
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from microscaling_block_scaled_mx_b200 import mx as m
+    monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(m, "_lib", None)
+    with pytest.raises(RuntimeError, match="libmx.so not found"):
+        m.lib()
