@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the MX hot path on B200: the cast (GB/s against HBM) and the
+block-scaled GEMM (TFLOP/s against the tensor cores).
+
+Default workload (one "step"): the cast bandwidth sweep -- one bf16
+8192 x 8192 tensor (N(0,1), 0.01% outliers x 1e3) cast along rows to all six
+element formats (E4M3, E5M2, E2M3, E3M2, E2M1, INT8), RNE, MMA scale layout.
+Inputs rotate over three device copies (3 x 128 MiB > the 126 MB L2) so no cast
+reads its input from L2.  `value` = algorithmic bytes of all casts / device
+time (GB/s).  The same line carries a "gemm" object: the Llama-3-8B-shaped
+MXFP4 GEMMs (M=8192: 4096->6144, 4096->14336, 14336->4096, bf16 out) timed the
+same way on operands cast in advance.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mx|reference]
+
+Multi-GPU: one process per GPU (torchrun); each rank runs the same per-GPU
+workload on its own data (weak scaling, no data-path collective); the time is
+the max over ranks.  `--impl reference` times the CPU oracle on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MX cast GB/s vs HBM peak; MX GEMM TFLOP/s vs block-scaled tensor peak"
+FMTS = ["e4m3", "e5m2", "e2m3", "e3m2", "e2m1", "int8"]
+BITS = {"e4m3": 8, "e5m2": 8, "e2m3": 6, "e3m2": 6, "e2m1": 4, "int8": 8}
+ROWS = COLS = 8192
+N_ROTATE = 3
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def cast_alg_bytes(fmt: str, rows: int = ROWS, cols: int = COLS, in_bytes: int = 2) -> int:
+    """Bytes a cast must move: read the input once, write codes and E8M0 scales once."""
+    n = rows * cols
+    return n * in_bytes + n * BITS[fmt] // 8 + n // 32
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.samples = []
+        if self.proc is None:
+            return False
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                self.samples.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                                     "hw_slowdown": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7],
+                                     "sw_power_cap": parts[8]})
+            except ValueError:
+                continue
+        return False
+
+    def summary(self):
+        s = getattr(self, "samples", [])
+        if not s:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        busy = [x for x in s if x["power"] > 200] or s
+        reasons = set()
+        for x in busy:
+            for k in ("hw_slowdown", "hw_thermal", "sw_thermal", "sw_power_cap"):
+                if x[k].lower() == "active":
+                    reasons.add({"hw_thermal": "hw_thermal_slowdown", "sw_thermal": "sw_thermal_slowdown"}.get(k, k))
+        return {"sm_mhz": statistics.median(x["sm"] for x in busy), "sm_max_mhz": max(x["max"] for x in s),
+                "samples": len(busy), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_cast_sample(rows: int):
+    """Time the oracle casting `rows` rows of the sweep input to all six formats."""
+    import oracle
+    from microscaling_block_scaled_mx_b200 import inputs as I
+    x = I.cast_sweep_input(rows, COLS)
+    oracle.build()
+    t0 = time.perf_counter()
+    for f in FMTS:
+        oracle.quantize(x, 1, oracle.FORMATS[f], scale_layout=oracle.MMA)
+    dt = time.perf_counter() - t0
+    nbytes = sum(cast_alg_bytes(f, rows, COLS) for f in FMTS)
+    return nbytes / dt / 1e9, dt, nbytes
+
+
+def cpu_threads() -> int:
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = 512
+    oracle_cast_sample(64)                     # warm the library
+    vals = []
+    for _ in range(args.warmup):
+        oracle_cast_sample(rows)
+    t_total = 0.0
+    nbytes = 0
+    for _ in range(args.steps):
+        v, dt, nb = oracle_cast_sample(rows)
+        vals.append(v)
+        t_total += dt
+        nbytes += nb
+    value = nbytes / t_total / 1e9
+    sample = f"{rows} x {COLS} rows of the sweep input, six formats per step"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * t_total / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "cast_sweep_bf16_8192x8192_6fmt", "global_batch": args.gpus,
+                       "parallelism": f"replicas{args.gpus}", "sampled_rows": rows},
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": cpu_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# product arm
+# ---------------------------------------------------------------------------
+
+def run_mx(args):
+    import torch
+    import torch.distributed as dist
+    from microscaling_block_scaled_mx_b200 import inputs as I
+    from microscaling_block_scaled_mx_b200 import mx
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream()
+    if args.no_cast:
+        gemm = run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world)
+        if rank == 0:
+            print(json.dumps({"gemm_only": True, "gemm": gemm}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # ---- inputs (host generation, then resident in HBM) ----
+    bits = I.cast_sweep_input(ROWS, COLS, seed_stream=rank)
+    host = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    xs = [host.to(dev) for _ in range(N_ROTATE)]
+    outs = {}
+    for f in FMTS:
+        outs[f] = [(torch.empty((ROWS, mx.codes_row_bytes(f, COLS)), dtype=torch.uint8, device=dev),
+                    torch.empty(mx.scales_bytes("mma", ROWS, COLS), dtype=torch.uint8, device=dev))
+                   for _ in range(N_ROTATE)]
+    stream = torch.cuda.current_stream()
+
+    launches = 0
+    events = []
+
+    def step(i, record=False):
+        nonlocal launches
+        for j, f in enumerate(FMTS):
+            r = (i * len(FMTS) + j) % N_ROTATE
+            c, s = outs[f][r]
+            if record:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            mx.quantize(xs[r], 1, f, codes=c, scales=s, scale_layout="mma")
+            if record:
+                e1.record(stream)
+                events.append((f, e0, e1))
+            launches += 1
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # timed region: K steps, barrier + synchronize on both sides
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        launches = 0
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i, record=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_total = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(ms_total)
+    alg_bytes_step = sum(cast_alg_bytes(f) for f in FMTS)
+    value = world * alg_bytes_step * args.steps / (ms_total * 1e-3) / 1e9
+
+    per_fmt = {}
+    for f in FMTS:
+        durs = [a.elapsed_time(b) for (g, a, b) in events if g == f]
+        per_fmt[f] = {"us": round(1e3 * statistics.mean(durs), 2),
+                      "gbs": round(cast_alg_bytes(f) / (statistics.mean(durs) * 1e-3) / 1e9, 1)}
+    all_durs_ms = sum(a.elapsed_time(b) for (_, a, b) in events)
+    achieved = alg_bytes_step * args.steps / (all_durs_ms * 1e-3) / 1e9
+    hbm_peak = float(peaks["hbm_gbs"])
+    roofline = {"bound": "hbm", "kernel": "cast_rows_kernel (six format instantiations)",
+                "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "peak_kind": f"{peak_kind} copy bandwidth (burst)",
+                "traffic": None, "per_format": per_fmt}
+
+    # ---- end to end through the C ABI with host buffers ----
+    pinned = host.pin_memory()
+    host_out = {f: (torch.empty(outs[f][0][0].shape, dtype=torch.uint8).pin_memory(),
+                    torch.empty(outs[f][0][1].shape, dtype=torch.uint8).pin_memory()) for f in FMTS}
+    d2h = sum(host_out[f][0].numel() + host_out[f][1].numel() for f in FMTS)
+    h2d = pinned.numel() * 2
+
+    def e2e_step():
+        xs[0].copy_(pinned, non_blocking=True)
+        for f in FMTS:
+            c, s = outs[f][0]
+            mx.quantize(xs[0], 1, f, codes=c, scales=s, scale_layout="mma")
+            host_out[f][0].copy_(c, non_blocking=True)
+            host_out[f][1].copy_(s, non_blocking=True)
+
+    e2e_steps = min(args.steps, 50)
+    e2e_val = None
+    if not args.no_e2e:
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e2e_val = world * alg_bytes_step * e2e_steps / (e2e_ms * 1e-3) / 1e9
+
+    gemm = run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world)
+    if gemm is not None:
+        launches_gemm = gemm.pop("_launches")
+    else:
+        launches_gemm = 0
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, nb = oracle_cast_sample(2048)
+        cpu = {"value": round(v, 3), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"2048 x {COLS} rows of the sweep input cast to all six formats ({dt:.1f} s wall)"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_total / args.steps, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": "cast_sweep_bf16_8192x8192_6fmt", "global_batch": world,
+                           "seq_len": None, "parallelism": f"replicas{world}",
+                           "formats": FMTS, "block_axis": "rows", "rounding": "rne",
+                           "l2": f"inputs rotate over {N_ROTATE} device buffers of 128 MiB (> L2)"},
+                "roofline": roofline,
+                "cpu_baseline": cpu,
+                "e2e": None if e2e_val is None else
+                       {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                        "path": "pinned host bf16 -> H2D -> mx_quantize (6 formats) -> D2H codes+scales"},
+                "gpu_launches": launches + launches_gemm,
+                "clocks": clocks.summary()}
+        if gemm is not None:
+            line["gemm"] = gemm
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world):
+    """Llama-3-8B-shaped MXFP4 GEMMs on operands cast in advance; None if the
+    GEMM is not available in this build."""
+    import torch
+    from microscaling_block_scaled_mx_b200 import inputs as I
+    from microscaling_block_scaled_mx_b200 import mx
+    if args.no_gemm:
+        return None
+    ops = []
+    for idx, (M, N, K) in enumerate(I.LLAMA3_GEMMS):
+        if str(idx) not in args.gemm_shapes.split(","):
+            continue
+        xb, wb = I.linear_operands(M, K, N, 3, stream=idx)
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
+        ac, as_ = mx.quantize(x, 1, "e2m1")
+        bc, bs = mx.quantize(w, 1, "e2m1")
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ops.append((M, N, K, ac, as_, bc, bs, c))
+        del x, w
+    try:
+        M, N, K, ac, as_, bc, bs, c = ops[0]
+        mx.gemm(ac, as_, bc, bs, M, N, K, fa="e2m1", out=c)
+    except mx.MxError as e:
+        if e.status == -4:
+            return None
+        raise
+    flops_step = sum(2.0 * M * N * K for (M, N, K, *_r) in ops)
+    for _ in range(args.warmup):
+        for (M, N, K, ac, as_, bc, bs, c) in ops:
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa="e2m1", out=c)
+    torch.cuda.synchronize()
+    barrier()
+    evs = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    t0.record(stream)
+    for _ in range(args.steps):
+        for (M, N, K, ac, as_, bc, bs, c) in ops:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa="e2m1", out=c)
+            e1.record(stream)
+            evs.append(((M, N, K), e0, e1))
+            launches += 1
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1))
+    value = world * flops_step * args.steps / (ms * 1e-3) / 1e12
+    per_shape = {}
+    for (M, N, K, *_r) in ops:
+        d = [a.elapsed_time(b) for (s, a, b) in evs if s == (M, N, K)]
+        per_shape[f"{M}x{N}x{K}"] = {"us": round(1e3 * statistics.mean(d), 1),
+                                     "tflops": round(2.0 * M * N * K / (statistics.mean(d) * 1e-3) / 1e12, 1)}
+    kern_ms = sum(a.elapsed_time(b) for (_, a, b) in evs)
+    achieved = flops_step * args.steps / (kern_ms * 1e-3) / 1e12
+    fp4_peak = 4.0 * float(peaks["bf16_tflops"])      # nominal fp4 : bf16 = 9 : 2.25
+    return {"metric": "MX GEMM TFLOP/s", "value": round(value, 1), "unit": "TFLOP/s",
+            "workload": "llama3_8b_mxfp4_gemms_m8192 (4096->6144, 4096->14336, 14336->4096), bf16 out",
+            "ms_per_step": round(ms / args.steps, 4),
+            "roofline": {"bound": "tensor", "kernel": "mx_gemm_kernel (kind::mxf4)",
+                         "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(achieved / fp4_peak, 4),
+                         "peak_kind": f"{peak_kind} bf16 burst x 4 (nominal MXFP4:bf16 ratio)",
+                         "traffic": None, "per_shape": per_shape},
+            "_launches": launches}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mx", "reference"], default="mx")
+    ap.add_argument("--no-gemm", action="store_true", help="skip the GEMM phase")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phase")
+    ap.add_argument("--no-cast", action="store_true", help="GEMM phase only (profiling)")
+    ap.add_argument("--fmts", default=",".join(FMTS), help="comma-separated cast formats (profiling)")
+    ap.add_argument("--gemm-shapes", default="0,1,2", help="indices of the Llama-3 GEMM shapes to time")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)      # at least three untimed warm-up steps
+    FMTS[:] = [f for f in args.fmts.split(",") if f]
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mx(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -131,7 +131,8 @@ typedef enum {
  *             32-bit finaliser.  Results therefore do not depend on tiling.
  *  seed       only read for MX_SR.
  *  pre        NULL, or preconditioning (see mx_precond).  Non-NULL with
- *             hadamard != 0 is supported for block_axis 0 only.
+ *             hadamard != 0 is supported for block_axis 0 only.  Scale
+ *             buffers of 4 GiB or more are not supported (MX_ERR_UNSUPPORTED).
  *  codes      device, mx_codes_bytes(fmt, outer, inner) bytes, 16-byte aligned.
  *  scales     device, mx_scales_bytes(sl, outer, inner) bytes.
  *  sl         scale layout to write.

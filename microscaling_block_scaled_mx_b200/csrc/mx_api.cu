@@ -95,6 +95,7 @@ int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t
     if (had && block_axis != 0) return MX_ERR_UNSUPPORTED;
     if (rnd == MX_SR && static_cast<uint64_t>(outer) * static_cast<uint64_t>(inner) > (1ull << 34))
         return MX_ERR_SR_RANGE;
+    if (mx_scales_bytes(sl, outer, inner) >= (1ull << 32)) return MX_ERR_UNSUPPORTED;  // 32-bit scale offsets
 
     MxQuantizeArgs a;
     a.x = x; a.xdt = xdt; a.rows = rows; a.cols = cols; a.ldx = ldx;

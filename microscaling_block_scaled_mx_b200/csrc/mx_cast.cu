@@ -35,7 +35,10 @@ struct CastParams {
 };
 
 __device__ __forceinline__ void store_scale(const CastParams &p, int64_t o, int64_t kb, uint32_t s) {
-    int64_t off = p.mma_scales ? mma_scale_offset(o, kb, p.k_groups) : o * p.k_blocks + kb;
+    // scale buffers are far below 4 GiB: offsets in 32-bit arithmetic
+    const uint32_t oo = static_cast<uint32_t>(o), k = static_cast<uint32_t>(kb);
+    const uint32_t off = p.mma_scales ? mma_scale_offset32(oo, k, static_cast<uint32_t>(p.k_groups))
+                                      : oo * static_cast<uint32_t>(p.k_blocks) + k;
     p.scales[off] = static_cast<uint8_t>(s);
 }
 
@@ -58,93 +61,134 @@ __device__ __forceinline__ void encode_values(float *u, int n, const uint32_t *r
 // ---------------------------------------------------------------------------
 // Row cast: block axis contiguous.
 // ---------------------------------------------------------------------------
+// One oct = 8 consecutive values of a row, owned by one lane; the four lanes
+// 4b..4b+3 of a warp hold one 32-block.  A warp walks 32-oct segments of one
+// row; U segments are loaded before any of them is processed so that every
+// thread keeps U 16-byte loads (bf16; 2U for fp32) in flight.
+template <bool BF16_IN>
+struct OctLoad {
+    uint4 w[BF16_IN ? 1 : 2];
+};
+
+template <bool BF16_IN>
+__device__ __forceinline__ void load_oct(const CastParams &p, int64_t row, int64_t col8, bool valid,
+                                         OctLoad<BF16_IN> &o) {
+    if (BF16_IN) {
+        o.w[0] = make_uint4(0, 0, 0, 0);
+        if (valid)
+            o.w[0] = __ldcs(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.x) + row * p.ldx + col8 * 8));
+    } else {
+        o.w[0] = o.w[BF16_IN ? 0 : 1] = make_uint4(0, 0, 0, 0);
+        if (valid) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const float *>(p.x) + row * p.ldx + col8 * 8);
+            o.w[0] = __ldcs(src);
+            o.w[BF16_IN ? 0 : 1] = __ldcs(src + 1);
+        }
+    }
+}
+
+template <int FMT, bool SR, bool BF16_IN>
+__device__ __forceinline__ void cast_oct(const CastParams &p, int64_t row, int64_t col8, bool valid,
+                                         const OctLoad<BF16_IN> &o, int lane) {
+    constexpr int BITS = Fmt<FMT>::bits;
+    float v[8];
+    uint32_t amax_bits;
+    if (BF16_IN) {
+        const uint4 w = o.w[0];
+        const uint32_t m = __vmaxu2(__vmaxu2(w.x & 0x7fff7fffu, w.y & 0x7fff7fffu),
+                                    __vmaxu2(w.z & 0x7fff7fffu, w.w & 0x7fff7fffu));
+        amax_bits = max(m & 0xffffu, m >> 16) << 16;
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(ws[i] << 16);
+            v[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+        }
+    } else {
+        const uint4 a = o.w[0], b = o.w[BF16_IN ? 0 : 1];
+        const uint32_t ws[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        amax_bits = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v[i] = __uint_as_float(ws[i]);
+            amax_bits = max(amax_bits, ws[i] & 0x7fffffffu);
+        }
+    }
+    amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 1));
+    amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 2));
+    if (!valid) return;
+
+    const bool nan_block = amax_bits >= 0x7f800000u;
+    const int e = block_exponent<FMT>(amax_bits);
+    float u[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = scale_down<FMT>(v[i], e);
+
+    uint32_t rw[2] = {0u, 0u};
+    if (SR) {
+        const uint64_t idx0 = static_cast<uint64_t>(row * p.cols + col8 * 8);
+        const uint32_t g = static_cast<uint32_t>(idx0 >> 2);
+        rw[0] = fmix32(g ^ p.key);
+        rw[1] = fmix32((g + 1u) ^ p.key);
+    }
+    uint32_t c[4];
+    encode_values<FMT, SR>(u, 8, rw, c);
+    if (nan_block) c[0] = c[1] = c[2] = c[3] = 0u;
+
+    if (BITS == 8) {
+        uint2 out = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+        *reinterpret_cast<uint2 *>(p.codes + row * p.cols + col8 * 8) = out;
+    } else if (BITS == 4) {
+        uint32_t out = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+        *reinterpret_cast<uint32_t *>(p.codes + row * (p.cols >> 1) + col8 * 4) = out;
+    } else {
+        uint64_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            w |= static_cast<uint64_t>(c[i] & 0x3fu) << (12 * i);
+            w |= static_cast<uint64_t>((c[i] >> 8) & 0x3fu) << (12 * i + 6);
+        }
+        uint8_t *dst = p.codes + row * (p.cols / 4 * 3) + col8 * 6;
+        if ((col8 & 1) == 0) {
+            *reinterpret_cast<uint32_t *>(dst) = static_cast<uint32_t>(w);
+            *reinterpret_cast<uint16_t *>(dst + 4) = static_cast<uint16_t>(w >> 32);
+        } else {
+            *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(w);
+            *reinterpret_cast<uint32_t *>(dst + 2) = static_cast<uint32_t>(w >> 16);
+        }
+    }
+    if ((lane & 3) == 0) store_scale(p, row, col8 >> 2, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+}
+
 template <int FMT, bool SR, bool BF16_IN>
 __global__ void __launch_bounds__(256) cast_rows_kernel(CastParams p) {
+    constexpr int U = BF16_IN ? 4 : 2;                  // segments in flight per warp
     const int lane = threadIdx.x & 31;
     const int64_t octs_per_row = p.cols >> 3;
-    const int64_t segs_per_row = (octs_per_row + 31) >> 5;
-    const int64_t n_segs = p.rows * segs_per_row;
+    const int64_t spr = (octs_per_row + 31) >> 5;       // 32-oct segments per row
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    constexpr int BITS = Fmt<FMT>::bits;
+    // segment s = row * spr + seg; consecutive visits of a warp are n_warps
+    // apart, stepped without a division inside the loop
+    int64_t row = warp0 / spr, seg = warp0 - row * spr;
+    const int64_t step_rows = n_warps / spr, step_seg = n_warps - step_rows * spr;
 
-    for (int64_t s = warp0; s < n_segs; s += n_warps) {
-        const int64_t row = s / segs_per_row;
-        const int64_t col8 = (s - row * segs_per_row) * 32 + lane;
-        const bool valid = col8 < octs_per_row;
-
-        float v[8];
-        uint32_t amax_bits;
-        if (BF16_IN) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            const uint16_t *src = static_cast<const uint16_t *>(p.x) + row * p.ldx + col8 * 8;
-            if (valid) w = __ldcs(reinterpret_cast<const uint4 *>(src));
-            uint32_t m = __vmaxu2(__vmaxu2(w.x & 0x7fff7fffu, w.y & 0x7fff7fffu),
-                                  __vmaxu2(w.z & 0x7fff7fffu, w.w & 0x7fff7fffu));
-            amax_bits = max(m & 0xffffu, m >> 16) << 16;
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    while (row < p.rows) {
+        int64_t r[U], c8[U];
+        bool ok[U];
+        OctLoad<BF16_IN> ld[U];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                v[2 * i] = __uint_as_float(ws[i] << 16);
-                v[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
-            }
-        } else {
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-            const float *src = static_cast<const float *>(p.x) + row * p.ldx + col8 * 8;
-            if (valid) {
-                a = __ldcs(reinterpret_cast<const float4 *>(src));
-                b = __ldcs(reinterpret_cast<const float4 *>(src) + 1);
-            }
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-            amax_bits = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) amax_bits = max(amax_bits, __float_as_uint(v[i]) & 0x7fffffffu);
+        for (int u = 0; u < U; ++u) {
+            r[u] = row;
+            c8[u] = seg * 32 + lane;
+            ok[u] = row < p.rows && c8[u] < octs_per_row;
+            load_oct<BF16_IN>(p, row, c8[u], ok[u], ld[u]);
+            seg += step_seg;
+            row += step_rows;
+            if (seg >= spr) { seg -= spr; ++row; }
         }
-        amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 1));
-        amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 2));
-        if (!valid) continue;
-
-        const bool nan_block = amax_bits >= 0x7f800000u;
-        const int e = block_exponent<FMT>(amax_bits);
-        float u[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) u[i] = scale_down<FMT>(v[i], e);
-
-        uint32_t rw[2] = {0u, 0u};
-        if (SR) {
-            const uint64_t idx0 = static_cast<uint64_t>(row * p.cols + col8 * 8);
-            const uint32_t g = static_cast<uint32_t>(idx0 >> 2);
-            rw[0] = fmix32(g ^ p.key);
-            rw[1] = fmix32((g + 1u) ^ p.key);
-        }
-        uint32_t c[4];
-        encode_values<FMT, SR>(u, 8, rw, c);
-        if (nan_block) c[0] = c[1] = c[2] = c[3] = 0u;
-
-        if (BITS == 8) {
-            uint2 out = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-            *reinterpret_cast<uint2 *>(p.codes + row * p.cols + col8 * 8) = out;
-        } else if (BITS == 4) {
-            uint32_t out = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-            *reinterpret_cast<uint32_t *>(p.codes + row * (p.cols >> 1) + col8 * 4) = out;
-        } else {
-            uint64_t w = 0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                w |= static_cast<uint64_t>(c[i] & 0x3fu) << (12 * i);
-                w |= static_cast<uint64_t>((c[i] >> 8) & 0x3fu) << (12 * i + 6);
-            }
-            uint8_t *dst = p.codes + row * (p.cols / 4 * 3) + col8 * 6;
-            if ((col8 & 1) == 0) {
-                *reinterpret_cast<uint32_t *>(dst) = static_cast<uint32_t>(w);
-                *reinterpret_cast<uint16_t *>(dst + 4) = static_cast<uint16_t>(w >> 32);
-            } else {
-                *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(w);
-                *reinterpret_cast<uint32_t *>(dst + 2) = static_cast<uint32_t>(w >> 16);
-            }
-        }
-        if ((lane & 3) == 0) store_scale(p, row, col8 >> 2, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+        for (int u = 0; u < U; ++u) cast_oct<FMT, SR, BF16_IN>(p, r[u], c8[u], ok[u], ld[u], lane);
     }
 }
 

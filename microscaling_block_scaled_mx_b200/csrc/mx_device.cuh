@@ -144,4 +144,9 @@ __device__ __forceinline__ int64_t mma_scale_offset(int64_t o, int64_t kb, int64
     return (atom << 9) + ((o & 31) << 4) + (((o >> 5) & 3) << 2) + (kb & 3);
 }
 
+__device__ __forceinline__ uint32_t mma_scale_offset32(uint32_t o, uint32_t kb, uint32_t k_groups) {
+    const uint32_t atom = (o >> 7) * k_groups + (kb >> 2);
+    return (atom << 9) + ((o & 31u) << 4) + (((o >> 5) & 3u) << 2) + (kb & 3u);
+}
+
 }  // namespace mxk

@@ -1,13 +1,538 @@
-// mx_gemm.cu -- block-scaled GEMM (placeholder until the tcgen05 kernel lands).
+// mx_gemm.cu -- block-scaled GEMM C = alpha * A * B^T on the sm_100a tensor
+// cores: the quantized dot products of the compute flow in "Microscaling Data
+// Formats for Deep Learning" (summary page, section 4), which take MX inputs
+// and return scalar floats.
+//
+// Design (one persistent CTA per SM, 192 threads, warp-specialized):
+//   warp 0      TMA producer: 128 x 128-byte A tile and 256 x 128-byte B tile
+//               per stage (128-byte swizzle), plus the 512-byte E8M0 scale
+//               atoms of both operands (bulk copies; the MMA layout written by
+//               mx_quantize is already the tensor-core layout).
+//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.cp moves each
+//               scale atom smem -> TMEM (32x128b, replicated to the four lane
+//               quarters), then four tcgen05.mma.block_scale per stage
+//               (kind::mxf8f6f4 K=32 for MXFP8, kind::mxf4 K=64 for MXFP4)
+//               accumulate into a 128 x 256 fp32 TMEM accumulator.
+//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, times alpha,
+//               rounded to fp32 / bf16, stored to C with bounds checks.
+// Every mbarrier wait is bounded; on expiry the kernel records MX_ERR_TIMEOUT
+// in the device status word, drains what it issued (bounded again), frees
+// its TMEM and returns.
+#include <cstdint>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "mx.h"
+#include "mx_debug.h"
 #include "mx_internal.h"
 
 // Device status word: kernels that give up a bounded wait record MX_ERR_TIMEOUT here.
 __device__ int g_mx_status;
 
-int mx_launch_gemm(const MxGemmArgs &, cudaStream_t) { return MX_ERR_UNSUPPORTED; }
+namespace mxg {
+
+constexpr int BM = 128;            // tile rows (A rows, TMEM lanes)
+constexpr int BN = 256;            // tile columns (B rows, accumulator columns)
+constexpr int BK_BYTES = 128;      // K bytes per stage: 128 fp8 or 256 fp4 elements
+constexpr int STAGES = 4;
+constexpr int NUM_THREADS = 192;
+constexpr int A_STAGE_BYTES = BM * BK_BYTES;   // 16 KiB
+constexpr int B_STAGE_BYTES = BN * BK_BYTES;   // 32 KiB
+constexpr int ATOM = 512;                      // scale atom: 128 rows x 4 k-blocks
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;                // accumulator columns [0, 256)
+constexpr uint32_t SF_COL = 256;               // scale-factor columns from 256
+constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
+constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;   // 0.2 s when draining
+
+template <bool FP4> struct Cfg {
+    static constexpr int G = FP4 ? 2 : 1;             // scale atoms along K per stage
+    static constexpr int SFA_BYTES = ATOM * G;        // per stage
+    static constexpr int SFB_BYTES = 2 * ATOM * G;    // two 128-row halves of B
+    static constexpr int SFA_COLS = 4 * G;            // TMEM columns per stage
+    static constexpr int SFB_COLS = 8 * G;
+    static constexpr int SF_STAGE_COLS = SFA_COLS + SFB_COLS;
+};
+
+struct Smem {
+    // offsets inside the 1024-aligned dynamic shared buffer
+    static constexpr int A = 0;
+    static constexpr int B = A + STAGES * A_STAGE_BYTES;
+    static constexpr int SFA = B + STAGES * B_STAGE_BYTES;
+    static constexpr int SFB = SFA + STAGES * 2 * ATOM;       // sized for the FP4 case
+    static constexpr int BAR = SFB + STAGES * 4 * ATOM;
+    // full[STAGES], empty[STAGES], acc_full, acc_empty, drain
+    static constexpr int NUM_BARS = 2 * STAGES + 3;
+    static constexpr int TMEM_SLOT = BAR + NUM_BARS * 8;
+    static constexpr int ABORT = TMEM_SLOT + 4;
+    static constexpr int TOTAL = ABORT + 4;
+};
+constexpr int SMEM_BYTES = Smem::TOTAL + 1024;   // slack for 1024-byte alignment
+
+struct Params {
+    const uint8_t *a_scales;
+    const uint8_t *b_scales;
+    void *c;
+    int64_t ldc;
+    int M, N, K;
+    int k_tiles;     // K bytes / BK_BYTES
+    int k_groups;    // scale atoms along K per 128-row block (K / 128 elements)
+    int tiles_m, tiles_n;
+    float alpha;
+    uint32_t idesc;  // instruction descriptor without the scale-factor ids
+    int skip_k_tile; // testing hook: CTA 0 withholds this k-tile of its first tile (-1: off)
+};
+
+// ------------------------------------------------------------------------
+// PTX wrappers
+// ------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait.  Returns false (and flags the CTA and the device) when the
+// phase does not complete within `limit` ns or another role already aborted.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                             unsigned long long limit = WAIT_LIMIT_NS) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 63u) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > limit) {
+                *abort_flag = 1;
+                atomicExch(&g_mx_status, MX_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 format): start address, leading
+// and stride byte offsets in 16-byte units, version 1, layout type.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;                                   // descriptor version for sm_100
+    d |= static_cast<uint64_t>(layout & 7u) << 61;
+    return d;
+}
+constexpr uint32_t LAYOUT_SW128 = 2;
+constexpr uint32_t LAYOUT_NONE = 0;
+
+// K-major operand tile with 128-byte rows and 128-byte swizzle: 8-row groups
+// 1024 bytes apart.  k_off moves along K inside the swizzled row.
+__device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, uint32_t k_off_bytes) {
+    return smem_desc(tile_addr + k_off_bytes, 16, 1024, LAYOUT_SW128);
+}
+// One 512-byte scale atom: 32 rows of 16 bytes, no swizzle, 8-row core
+// matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t scale_atom_desc(uint32_t addr) {
+    return smem_desc(addr, 16, 128, LAYOUT_NONE);
+}
+
+__device__ __forceinline__ void tc_cp_scale_atom(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+template <bool FP4>
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    if (FP4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+            : "memory");
+    }
+}
+
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------
+// The kernel
+// ------------------------------------------------------------------------
+template <bool FP4, bool BF16_OUT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, Params p) {
+    using C = Cfg<FP4>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Smem::ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Smem::TMEM_SLOT);
+
+    auto full_bar = [&](int s) { return sbase + Smem::BAR + 8u * s; };
+    auto empty_bar = [&](int s) { return sbase + Smem::BAR + 8u * (STAGES + s); };
+    const uint32_t acc_full = sbase + Smem::BAR + 8u * (2 * STAGES);
+    const uint32_t acc_empty = acc_full + 8u;
+    const uint32_t drain_bar = acc_full + 16u;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 4);
+        mbar_init(drain_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t outstanding = 0;   // bit s: stage s has loads in flight not yet observed
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+                const int m0 = tm * BM, n0 = tn * BN;
+                const int rb_a = m0 / 128, rb_b = n0 / 128;
+                const bool b_hi = (n0 + 128) < p.N;   // second 128-row half of B exists
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
+                    if (kt == p.skip_k_tile && tile == static_cast<int>(blockIdx.x) && blockIdx.x == 0) {
+                        ok = false;          // injected stall: this stage is never filled
+                        break;
+                    }
+                    const uint32_t bytes = A_STAGE_BYTES + B_STAGE_BYTES + C::SFA_BYTES +
+                                           (b_hi ? 2 : 1) * (C::SFB_BYTES / 2);
+                    const uint32_t fb = full_bar(s);
+                    mbar_expect_tx(fb, bytes);
+                    tma_load_2d(sbase + Smem::A + s * A_STAGE_BYTES, &tma_a, kt * BK_BYTES, m0, fb);
+                    tma_load_2d(sbase + Smem::B + s * B_STAGE_BYTES, &tma_b, kt * BK_BYTES, n0, fb);
+                    const int kg = kt * C::G;
+                    bulk_load(sbase + Smem::SFA + s * 2 * ATOM,
+                              p.a_scales + (static_cast<int64_t>(rb_a) * p.k_groups + kg) * ATOM, C::SFA_BYTES, fb);
+                    bulk_load(sbase + Smem::SFB + s * 4 * ATOM,
+                              p.b_scales + (static_cast<int64_t>(rb_b) * p.k_groups + kg) * ATOM, C::SFB_BYTES / 2, fb);
+                    if (b_hi)
+                        bulk_load(sbase + Smem::SFB + s * 4 * ATOM + C::SFB_BYTES / 2,
+                                  p.b_scales + (static_cast<int64_t>(rb_b + 1) * p.k_groups + kg) * ATOM,
+                                  C::SFB_BYTES / 2, fb);
+                    outstanding |= 1u << s;
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                    outstanding &= ~(1u << s);   // its previous use was released by the MMA
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for every stage whose loads may still land
+                int ds = s;
+                uint32_t dph = ph;
+                for (int i = 0; i < STAGES; ++i) {
+                    ds = ds == 0 ? STAGES - 1 : ds - 1;
+                    if (ds == STAGES - 1) dph ^= 1u;
+                    if (outstanding & (1u << ds)) {
+                        volatile int no_abort = 0;
+                        (void)wait_bounded(full_bar(ds), dph, &no_abort, DRAIN_LIMIT_NS);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ----------------------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0, acc_ph = 0;
+            bool ok = true;
+            bool issued = false;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!wait_bounded(acc_empty, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!wait_bounded(full_bar(s), ph, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sfa_t = tmem + SF_COL + s * C::SF_STAGE_COLS;
+                    const uint32_t sfb_t = sfa_t + C::SFA_COLS;
+                    const uint32_t sfa_s = sbase + Smem::SFA + s * 2 * ATOM;
+                    const uint32_t sfb_s = sbase + Smem::SFB + s * 4 * ATOM;
+#pragma unroll
+                    for (int g = 0; g < C::G; ++g) {
+                        tc_cp_scale_atom(sfa_t + 4 * g, scale_atom_desc(sfa_s + g * ATOM));
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tc_cp_scale_atom(sfb_t + 8 * g + 4 * h,
+                                             scale_atom_desc(sfb_s + h * (C::SFB_BYTES / 2) + g * ATOM));
+                    }
+                    const uint32_t a_s = sbase + Smem::A + s * A_STAGE_BYTES;
+                    const uint32_t b_s = sbase + Smem::B + s * B_STAGE_BYTES;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        // FP8: k-block k of the atom; FP4: k-blocks 2k, 2k+1 (atom k/2, bytes 2k%4..)
+                        const uint32_t g = FP4 ? (k >> 1) : 0u;
+                        const uint32_t sf_id = FP4 ? ((2u * k) & 3u) : static_cast<uint32_t>(k);
+                        const uint32_t idesc = p.idesc | (sf_id << 4) | (sf_id << 29);
+                        tc_mma<FP4>(tmem + ACC_COL, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k), idesc,
+                                    sfa_t + 4 * g, sfb_t + 8 * g, (kt > 0 || k > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit(empty_bar(s));
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(acc_full);
+                acc_ph ^= 1u;
+            }
+            if (issued) {
+                // all issued MMAs must finish before TMEM is released
+                tc_commit(drain_bar);
+                volatile int no_abort = 0;
+                (void)wait_bounded(drain_bar, 0, &no_abort, ok ? WAIT_LIMIT_NS : DRAIN_LIMIT_NS);
+            }
+        }
+    } else {
+        // ------------------------------ epilogue ------------------------------
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        uint32_t acc_ph = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            // one lane waits, the warp follows its verdict: tcgen05.ld below
+            // must be executed by all 32 lanes together
+            int ok = 1;
+            if (lane == 0) ok = wait_bounded(acc_full, acc_ph, abort_flag) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+            const int m = tm * BM + q * 32 + lane;
+            const int n_base = tn * BN;
+#pragma unroll 1
+            for (int j = 0; j < BN / 32; ++j) {
+                uint32_t r[32];
+                tmem_ld_32cols(tmem + ACC_COL + (static_cast<uint32_t>(q * 32) << 16) + j * 32, r);
+                const int n0 = n_base + j * 32;
+                if (m < p.M && n0 < p.N) {
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), p.alpha);
+                    if (BF16_OUT) {
+                        __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
+                        if (n0 + 32 <= p.N) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 8) {
+                                uint32_t w[4];
+#pragma unroll
+                                for (int t = 0; t < 4; ++t) {
+                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * t], v[i + 2 * t + 1]);
+                                    w[t] = *reinterpret_cast<uint32_t *>(&b2);
+                                }
+                                *reinterpret_cast<uint4 *>(row + i) = make_uint4(w[0], w[1], w[2], w[3]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (n0 + i < p.N) row[i] = __float2bfloat16_rn(v[i]);
+                        }
+                    } else {
+                        float *row = static_cast<float *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
+                        if (n0 + 32 <= p.N) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (n0 + i < p.N) row[i] = v[i];
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            acc_ph ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D uint8 tensor map over a rows x row_bytes matrix, box of box_rows x 128
+// bytes, 128-byte swizzle; out-of-range rows read as zero.
+bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t row_bytes, int box_rows) {
+    auto encode = get_encode();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+uint32_t make_idesc(int fa, int fb, bool fp4) {
+    auto code = [&](int f) -> uint32_t {
+        if (fp4) return 1u;               // kind::mxf4: E2M1
+        return f == MX_E5M2 ? 1u : 0u;    // kind::mxf8f6f4: E4M3 = 0, E5M2 = 1
+    };
+    uint32_t d = 0;
+    d |= code(fa) << 7;
+    d |= code(fb) << 10;
+    d |= static_cast<uint32_t>(BN >> 3) << 17;
+    d |= 1u << 23;                         // scale factors are UE8M0
+    d |= static_cast<uint32_t>(BM >> 4) << 24;
+    return d;
+}
+
+template <bool FP4, bool BF16_OUT>
+cudaError_t launch(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int grid, cudaStream_t st) {
+    auto kern = mx_gemm_kernel<FP4, BF16_OUT>;
+    static bool configured = false;   // per instantiation; attribute setting is idempotent
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    kern<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+}  // namespace mxg
+
+namespace {
+std::atomic<int> g_skip_k_tile{-1};
+}
+
+extern "C" int mx_debug_gemm_skip_stage(int k_tile) {
+    g_skip_k_tile.store(k_tile < 0 ? -1 : k_tile);
+    return MX_OK;
+}
+
+int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
+    using namespace mxg;
+    const bool fp4 = a.fa == MX_E2M1;
+    const int64_t k_bytes = fp4 ? a.K / 2 : a.K;
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, a.a_codes, a.M, k_bytes, BM)) return MX_ERR_CUDA;
+    if (!make_operand_map(&tb, a.b_codes, a.N, k_bytes, BN)) return MX_ERR_CUDA;
+    Params p;
+    p.a_scales = static_cast<const uint8_t *>(a.a_scales);
+    p.b_scales = static_cast<const uint8_t *>(a.b_scales);
+    p.c = a.c;
+    p.ldc = a.ldc;
+    p.M = static_cast<int>(a.M);
+    p.N = static_cast<int>(a.N);
+    p.K = static_cast<int>(a.K);
+    p.k_tiles = static_cast<int>(k_bytes / BK_BYTES);
+    p.k_groups = static_cast<int>(a.K / 128);
+    p.tiles_m = static_cast<int>((a.M + BM - 1) / BM);
+    p.tiles_n = static_cast<int>((a.N + BN - 1) / BN);
+    p.alpha = a.alpha;
+    p.idesc = make_idesc(a.fa, a.fb, fp4);
+    p.skip_k_tile = g_skip_k_tile.exchange(-1);
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int grid = tiles < a.num_sms ? tiles : a.num_sms;
+    cudaError_t e;
+    const bool bf = a.cdt == MX_BF16;
+    if (fp4) e = bf ? launch<true, true>(ta, tb, p, grid, st) : launch<true, false>(ta, tb, p, grid, st);
+    else e = bf ? launch<false, true>(ta, tb, p, grid, st) : launch<false, false>(ta, tb, p, grid, st);
+    return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
 
 int mx_read_device_status(cudaStream_t st) {
     if (cudaStreamSynchronize(st) != cudaSuccess) return MX_ERR_CUDA;

@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             L.mx_status_str.argtypes = [i32]
             L.mx_abi_version.restype = i32
             L.mx_abi_version.argtypes = []
+            L.mx_debug_gemm_skip_stage.restype = i32
+            L.mx_debug_gemm_skip_stage.argtypes = [i32]
             _lib = L
     return _lib
 

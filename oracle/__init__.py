@@ -259,3 +259,21 @@ def gemm_entries(a_codes, a_scales, fa, b_codes, b_scales, fb, K, ms, ns, alpha=
                                   ms.size, _ptr(c), _ptr(bound))
     _check(rc, "mxref_gemm_entries")
     return c, bound
+
+
+def gemm_decoded(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha=1.0,
+                 rows=None, scale_layout: int = MMA):
+    """The same C = alpha * A * B^T with numpy's fp64 matmul as the summation step.
+
+    Both operands are decoded exactly by the oracle (mxref_dequantize); the
+    dot products are then an fp64 matrix product, whose rounding error
+    (about K * 2^-53 relative to sum |a b|) is far below any tolerance used.
+    `rows` restricts the result to those rows of A.  Returns (C, bound).
+    """
+    A = dequantize(a_codes, a_scales, fa, M, K, scale_layout)
+    B = dequantize(b_codes, b_scales, fb, N, K, scale_layout)
+    if rows is not None:
+        A = A[np.asarray(rows)]
+    c = alpha * (A @ B.T)
+    bound = abs(alpha) * (np.abs(A) @ np.abs(B).T)
+    return c, bound

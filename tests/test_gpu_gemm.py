@@ -1,0 +1,218 @@
+"""GPU parity of the block-scaled GEMM (compute flow of "Microscaling Data
+Formats for Deep Learning", summary page, section 4: dot products on MX inputs
+return scalar floats) against the oracle.
+
+Tolerance (stated for the GEMM): |C - C_ref| <= 1e-5 * |alpha| * sum_k |a_mk b_nk|
+for fp32 output, plus one bf16 ulp of C_ref for bf16 output.  Where every
+partial sum is exact in fp32 the result must be bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import dev, host, to_device
+from microscaling_block_scaled_mx_b200 import inputs as I
+from microscaling_block_scaled_mx_b200 import mx
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-5
+
+
+def bf16_ulp(x):
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    _, ex = np.frexp(a)
+    e = np.maximum(ex - 1, -126)
+    return np.exp2(e - 7.0)
+
+
+def check(got, ref, bound, out_dtype, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    tol = REL_TOL * bound
+    if out_dtype == torch.bfloat16:
+        tol = tol + bf16_ulp(ref)
+    err = np.abs(got - ref)
+    bad = err > tol
+    assert not np.any(np.isnan(got)), (what, "NaN in output")
+    if np.any(bad):
+        i = np.argwhere(bad)[:5]
+        raise AssertionError((what, int(bad.sum()), [(tuple(j), got[tuple(j)], ref[tuple(j)], tol[tuple(j)])
+                                                     for j in i]))
+
+
+def to_f64(t):
+    return host(t.float()).astype(np.float64) if t.dtype == torch.bfloat16 else host(t).astype(np.float64)
+
+
+def run_gemm(oracle, a, b, fmt, M, N, K, alpha=1.0, out_dtype=torch.float32, ldc=None, rows=None):
+    """a: M x K, b: N x K host arrays (float32 or bf16 bits); both cast along K
+    by the GPU (verified bit-exact elsewhere) and by the oracle."""
+    ac, as_ = mx.quantize(to_device(a), 1, fmt)
+    bc, bs = mx.quantize(to_device(b), 1, fmt)
+    if ldc is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev())
+    else:
+        out = torch.empty((M, ldc), dtype=out_dtype, device=dev())[:, :N]
+    out.fill_(float("nan"))
+    mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, alpha=alpha, out=out)
+    torch.cuda.synchronize()
+    f = oracle.FORMATS[fmt]
+    oac, oas = oracle.quantize(a, 1, f, scale_layout=oracle.MMA)
+    obc, obs = oracle.quantize(b, 1, f, scale_layout=oracle.MMA)
+    ref, bound = oracle.gemm_decoded(oac, oas, f, obc, obs, f, M, N, K, alpha=alpha, rows=rows)
+    got = to_f64(out)
+    if rows is not None:
+        got = got[np.asarray(rows)]
+    return got, ref, bound
+
+
+def small_int_operand(rng, rows, K):
+    """Small integers times a power of two per 32-block: every product and
+    partial sum is exact in fp32, and the block scales vary."""
+    v = rng.integers(-3, 4, (rows, K)).astype(np.float64)
+    v *= np.exp2(np.repeat(rng.integers(-2, 3, (rows, K // 32)), 32, axis=1))
+    return v.astype(np.float32)
+
+
+@pytest.mark.parametrize("fmt,K", [("e4m3", 128), ("e4m3", 512), ("e2m1", 256), ("e2m1", 1024),
+                                   ("e5m2", 256)])
+def test_gemm_single_tile_bit_exact(oracle, fmt, K):
+    rng = np.random.default_rng(K)
+    M, N = 128, 256
+    a = small_int_operand(rng, M, K)
+    b = small_int_operand(rng, N, K)
+    if fmt == "e2m1":   # keep the values on the E2M1 grid: {0, .5, 1, 1.5, 2, 3} x 2^k
+        a = np.clip(a, -3, 3)
+        b = np.clip(b, -3, 3)
+    got, ref, bound = run_gemm(oracle, a, b, fmt, M, N, K)
+    exact = oracle.round_f32(ref).astype(np.float64)
+    assert np.array_equal(got, exact), np.argwhere(got != exact)[:5]
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2", "e2m1"])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_multi_tile_tolerance(oracle, fmt, out_dtype):
+    rng = np.random.default_rng(7)
+    M, N, K = 384, 768, 2048
+    a = (rng.standard_normal((M, K)) * np.exp2(rng.uniform(-4, 4, (M, 1)))).astype(np.float32)
+    b = rng.standard_t(3, size=(N, K)).astype(np.float32)
+    got, ref, bound = run_gemm(oracle, a, b, fmt, M, N, K, alpha=0.75, out_dtype=out_dtype)
+    check(got, ref, bound, out_dtype, fmt)
+
+
+@pytest.mark.parametrize("fmt,K", [("e4m3", 384), ("e2m1", 512)])
+def test_gemm_ragged_m_n_and_pitched_c(oracle, fmt, K):
+    rng = np.random.default_rng(11)
+    for (M, N) in [(200, 300), (1, 1), (129, 257), (130, 100)]:
+        a = rng.standard_normal((M, K)).astype(np.float32)
+        b = rng.standard_normal((N, K)).astype(np.float32)
+        for out_dtype in (torch.float32, torch.bfloat16):
+            ldc = (N + 7) // 8 * 8 + 8        # padded pitch, a multiple of 16 bytes
+            got, ref, bound = run_gemm(oracle, a, b, fmt, M, N, K, out_dtype=out_dtype, ldc=ldc)
+            check(got, ref, bound, out_dtype, (fmt, M, N))
+
+
+def test_gemm_k_zero_and_empty():
+    c = torch.full((4, 8), 7.0, device=dev())
+    z = torch.empty(0, dtype=torch.uint8, device=dev())
+    mx.gemm(z, z, z, z, 4, 8, 0, fa="e4m3", out=c)
+    torch.cuda.synchronize()
+    assert torch.all(c == 0)
+    mx.gemm(z, z, z, z, 0, 8, 128, fa="e4m3", out=torch.empty((0, 8), device=dev()))
+
+
+def test_gemm_roundtrip_config(oracle):
+    """fp32 A 256x512 (blocks along K = rows of A) times B 512x256 (K x N,
+    blocks along K = down its columns), E4M3, fp32 out, every entry."""
+    d = I.config_roundtrip()
+    A, B = d["A"], d["B"]
+    M, K = A.shape
+    N = B.shape[1]
+    ac, as_ = mx.quantize(to_device(A), 1, "e4m3")
+    bc, bs = mx.quantize(to_device(B), 0, "e4m3")        # N x K codes
+    c = mx.gemm(ac, as_, bc, bs, M, N, K, fa="e4m3", out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    oac, oas = oracle.quantize(A, 1, 0, scale_layout=1)
+    obc, obs = oracle.quantize(B, 0, 0, scale_layout=1)
+    ref, bound = oracle.gemm(oac, oas, 0, obc, obs, 0, M, N, K)
+    check(to_f64(c), ref, bound, torch.float32)
+
+
+@pytest.mark.parametrize("idx", [0, 1])
+def test_gemm_gpt2_config(oracle, idx):
+    """GPT-2-small-shaped MXFP8 GEMMs (M=8192, 768->3072 and 3072->768), bf16
+    activations N(0,1) and weights N(0,0.02^2) cast along K, bf16 out: all of C."""
+    M, N, K = I.GPT2_GEMMS[idx]
+    x, w = I.linear_operands(M, K, N, 2, stream=idx)
+    got, ref, bound = run_gemm(oracle, x, w, "e4m3", M, N, K, out_dtype=torch.bfloat16)
+    check(got, ref, bound, torch.bfloat16, (M, N, K))
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2])
+def test_gemm_llama3_config(oracle, idx):
+    """Llama-3-8B-shaped MXFP4 GEMMs along K, bf16 out: 384 sampled rows of C
+    (every column)."""
+    M, N, K = I.LLAMA3_GEMMS[idx]
+    x, w = I.linear_operands(M, K, N, 3, stream=idx)
+    rows = np.sort(np.random.default_rng(idx).choice(M, 384, replace=False))
+    got, ref, bound = run_gemm(oracle, x, w, "e2m1", M, N, K, out_dtype=torch.bfloat16, rows=rows)
+    check(got, ref, bound, torch.bfloat16, (M, N, K))
+
+
+def test_gemm_llama3_along_m(oracle):
+    """The same activations cast along M (transposed blocks): the weight-gradient
+    shaped product C^T X contracts over the 8192 tokens.  C is the forward
+    output of the 4096->6144 GEMM (bf16), cast along M as well."""
+    M, N, K = I.LLAMA3_GEMMS[0]
+    x, w = I.linear_operands(M, K, N, 3, stream=0)
+    xd = to_device(x)
+    ac, as_ = mx.quantize(xd, 1, "e2m1")
+    bc, bs = mx.quantize(to_device(w), 1, "e2m1")
+    c = mx.gemm(ac, as_, bc, bs, M, N, K, fa="e2m1", out_dtype=torch.bfloat16)      # 8192 x 6144
+    gc, gs = mx.quantize(c, 0, "e2m1")            # 6144 x 8192 codes (blocks along tokens)
+    xc, xs = mx.quantize(xd, 0, "e2m1")           # 4096 x 8192 codes
+    dw = mx.gemm(gc, gs, xc, xs, N, K, M, fa="e2m1", out_dtype=torch.float32)       # 6144 x 4096
+    torch.cuda.synchronize()
+    c_bits = host(c)
+    ogc, ogs = oracle.quantize(c_bits, 0, oracle.E2M1, scale_layout=oracle.MMA)
+    oxc, oxs = oracle.quantize(x, 0, oracle.E2M1, scale_layout=oracle.MMA)
+    assert np.array_equal(host(gc), ogc) and np.array_equal(host(xc), oxc)
+    rows = np.sort(np.random.default_rng(5).choice(N, 256, replace=False))
+    ref, bound = oracle.gemm_decoded(ogc, ogs, oracle.E2M1, oxc, oxs, oracle.E2M1, N, K, M, rows=rows)
+    check(to_f64(dw)[rows], ref, bound, torch.float32, "along M")
+
+
+def test_gemm_wgrad_config(oracle):
+    """dW = alpha * dY^T X with tokens K=16384: dY 16384x4096 and X 16384x14336
+    (Student-t), both cast along tokens with the fixed-sign Hadamard and
+    stochastic rounding to E2M1, alpha = 1/32, fp32 out; 256 sampled rows."""
+    dy, xx = I.wgrad_operands()
+    T, Do = dy.shape
+    Di = xx.shape[1]
+    ac, as_ = mx.quantize(to_device(dy), 0, "e2m1", rnd="sr", seed=42, hadamard=True)
+    bc, bs = mx.quantize(to_device(xx), 0, "e2m1", rnd="sr", seed=43, hadamard=True)
+    dw = mx.gemm(ac, as_, bc, bs, Do, Di, T, fa="e2m1", alpha=1.0 / 32, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(9).choice(Do, 256, replace=False))
+    # the operands are bit-identical to the oracle's (checked by the cast tests)
+    ref, bound = oracle.gemm_decoded(host(ac), host(as_), oracle.E2M1, host(bc), host(bs), oracle.E2M1,
+                                     Do, Di, T, alpha=1.0 / 32, rows=rows)
+    check(to_f64(dw)[rows], ref, bound, torch.float32, "wgrad")
+
+
+def test_gemm_bounded_wait_reports_timeout():
+    """A stage that is never filled: the MMA issuer's bounded wait runs out, the
+    kernel records MX_ERR_TIMEOUT and returns; the context stays usable."""
+    rng = np.random.default_rng(1)
+    M, N, K = 256, 256, 1024
+    a = to_device(rng.standard_normal((M, K)).astype(np.float32))
+    ac, as_ = mx.quantize(a, 1, "e4m3")
+    assert mx.last_device_status() == 0
+    mx.lib().mx_debug_gemm_skip_stage(3)
+    mx.gemm(ac, as_, ac, as_, M, N, K, fa="e4m3", out_dtype=torch.float32)
+    assert mx.last_device_status() == -7
+    assert mx.last_device_status() == 0          # read-and-clear
+    c = mx.gemm(ac, as_, ac, as_, M, N, K, fa="e4m3", out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert mx.last_device_status() == 0
+    assert torch.isfinite(c).all()

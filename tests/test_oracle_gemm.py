@@ -87,3 +87,21 @@ def test_gemm_random_close_to_fp64_of_inputs(oracle):
     exact = a.astype(np.float64) @ b.astype(np.float64).T
     # E4M3 relative element error <= 2^-4, so |C - exact| <= ~2^-3 * sum|ab|
     assert np.all(np.abs(c - exact) <= 0.13 * bound)
+
+
+def test_gemm_decoded_matches_scalar_loop(oracle):
+    """The matmul route used for large shapes agrees with the scalar oracle."""
+    rng = np.random.default_rng(9)
+    M, N, K = 96, 80, 512
+    a = (rng.standard_normal((M, K)) * np.exp2(rng.integers(-20, 20, (M, 1)))).astype(np.float32)
+    b = rng.standard_t(3, size=(N, K)).astype(np.float32)
+    for f in (0, 1, 4):
+        ac, as_ = oracle.quantize(a, 1, f, scale_layout=1)
+        bc, bs = oracle.quantize(b, 1, f, scale_layout=1)
+        c1, b1 = oracle.gemm(ac, as_, f, bc, bs, f, M, N, K, alpha=0.03125)
+        c2, b2 = oracle.gemm_decoded(ac, as_, f, bc, bs, f, M, N, K, alpha=0.03125)
+        np.testing.assert_allclose(c2, c1, rtol=0, atol=1e-12 * b1.max())
+        np.testing.assert_allclose(b2, b1, rtol=1e-12)
+        rows = [3, 50, 95]
+        c3, _ = oracle.gemm_decoded(ac, as_, f, bc, bs, f, M, N, K, alpha=0.03125, rows=rows)
+        np.testing.assert_array_equal(c3, c2[rows])
