@@ -187,16 +187,11 @@ def run_mx(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    from microscaling_block_scaled_mx_b200 import dist as mxdist
+    barrier = mxdist.barrier
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return mxdist.max_over_ranks(x, dev)
 
     peaks, peak_kind = load_peaks()
     stream = torch.cuda.current_stream()
