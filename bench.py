@@ -303,6 +303,8 @@ def run_mx(args):
         launches_gemm = gemm.pop("_launches")
     else:
         launches_gemm = 0
+    wgrad = None if args.no_wgrad else run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier,
+                                                        max_over_ranks, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -329,6 +331,8 @@ def run_mx(args):
                 "clocks": clocks.summary()}
         if gemm is not None:
             line["gemm"] = gemm
+        if wgrad is not None:
+            line["wgrad"] = wgrad
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -404,6 +408,71 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
             "_launches": launches}
 
 
+def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world):
+    """Weight-gradient step: dY 16384x4096 and X 16384x14336 (bf16, Student-t)
+    cast along tokens with the fixed-sign Hadamard and stochastic rounding to
+    E2M1, then dW = dY^T X / 32 in fp32.  Times the two casts and the GEMM."""
+    import torch
+    from microscaling_block_scaled_mx_b200 import inputs as I
+    from microscaling_block_scaled_mx_b200 import mx
+    dyb, xb = I.wgrad_operands()
+    T, Do = dyb.shape
+    Di = xb.shape[1]
+    dy = torch.from_numpy(dyb.view(np.int16)).view(torch.bfloat16).to(dev)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+    del dyb, xb
+    ac = torch.empty((Do, T // 2), dtype=torch.uint8, device=dev)
+    as_ = torch.empty(mx.scales_bytes("mma", Do, T), dtype=torch.uint8, device=dev)
+    bc = torch.empty((Di, T // 2), dtype=torch.uint8, device=dev)
+    bs = torch.empty(mx.scales_bytes("mma", Di, T), dtype=torch.uint8, device=dev)
+    dw = torch.empty((Do, Di), dtype=torch.float32, device=dev)
+    evs = {"cast_dY": [], "cast_X": [], "gemm_dW": []}
+
+    def step(record):
+        for name, fn in (("cast_dY", lambda: mx.quantize(dy, 0, "e2m1", rnd="sr", seed=42, hadamard=True,
+                                                         codes=ac, scales=as_)),
+                         ("cast_X", lambda: mx.quantize(x, 0, "e2m1", rnd="sr", seed=43, hadamard=True,
+                                                        codes=bc, scales=bs)),
+                         ("gemm_dW", lambda: mx.gemm(ac, as_, bc, bs, Do, Di, T, fa="e2m1", alpha=1.0 / 32,
+                                                     out=dw))):
+            if record:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            fn()
+            if record:
+                e1.record(stream)
+                evs[name].append((e0, e1))
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1))
+    us = {k: 1e3 * statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in evs.items()}
+    cast_bytes = {"cast_dY": T * Do * 2 + T * Do // 2 + T * Do // 32,
+                  "cast_X": T * Di * 2 + T * Di // 2 + T * Di // 32}
+    flops = 2.0 * Do * Di * T
+    fp4_peak = 4.0 * float(peaks["bf16_tflops"])
+    hbm = float(peaks["hbm_gbs"])
+    out = {"workload": "wgrad_mxfp4 dY 16384x4096, X 16384x14336 (Student-t), Hadamard+SR along tokens, "
+                       "dW fp32", "steps": steps, "ms_per_step": round(ms / steps, 4)}
+    for k in ("cast_dY", "cast_X"):
+        gbs = cast_bytes[k] / (us[k] * 1e-6) / 1e9
+        out[k] = {"us": round(us[k], 1), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+    tf = flops / (us["gemm_dW"] * 1e-6) / 1e12
+    out["gemm_dW"] = {"us": round(us["gemm_dW"], 1), "tflops": round(tf, 1), "frac": round(tf / fp4_peak, 4),
+                      "peak": round(fp4_peak, 1)}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -414,6 +483,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phase")
     ap.add_argument("--no-cast", action="store_true", help="GEMM phase only (profiling)")
+    ap.add_argument("--no-wgrad", action="store_true", help="skip the weight-gradient phase")
     ap.add_argument("--fmts", default=",".join(FMTS), help="comma-separated cast formats (profiling)")
     ap.add_argument("--gemm-shapes", default="0,1,2", help="indices of the Llama-3 GEMM shapes to time")
     args = ap.parse_args()

@@ -61,258 +61,350 @@ __device__ __forceinline__ void encode_values(float *u, int n, const uint32_t *r
 // ---------------------------------------------------------------------------
 // Row cast: block axis contiguous.
 // ---------------------------------------------------------------------------
-// One oct = 8 consecutive values of a row, owned by one lane; the four lanes
-// 4b..4b+3 of a warp hold one 32-block.  A warp walks 32-oct segments of one
-// row; U segments are loaded before any of them is processed so that every
-// thread keeps U 16-byte loads (bf16; 2U for fp32) in flight.
+// One lane owns one 32-block (64 bytes of bf16, four 16-byte loads), so the
+// block's amax, exponent, scale byte and addresses are computed once per 32
+// values; a warp covers 32 consecutive blocks (1024 values) of one row.  The
+// next chunk's loads are issued before the current chunk is converted, so each
+// thread keeps up to eight 16-byte loads in flight.
 template <bool BF16_IN>
-struct OctLoad {
-    uint4 w[BF16_IN ? 1 : 2];
+struct BlockLoad {
+    uint4 w[BF16_IN ? 4 : 8];
+};
+
+struct ChunkPos {
+    int64_t row, chunk;   // chunk = 32 consecutive blocks of one row
 };
 
 template <bool BF16_IN>
-__device__ __forceinline__ void load_oct(const CastParams &p, int64_t row, int64_t col8, bool valid,
-                                         OctLoad<BF16_IN> &o) {
-    if (BF16_IN) {
-        o.w[0] = make_uint4(0, 0, 0, 0);
-        if (valid)
-            o.w[0] = __ldcs(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.x) + row * p.ldx + col8 * 8));
+__device__ __forceinline__ void load_block(const CastParams &p, const ChunkPos &cp, int64_t blocks_per_row, int lane,
+                                           BlockLoad<BF16_IN> &o) {
+    constexpr int NW = BF16_IN ? 4 : 8;
+    const int64_t kb = cp.chunk * 32 + lane;
+    if (cp.row < p.rows && kb < blocks_per_row) {
+        constexpr int EB = BF16_IN ? 2 : 4;
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.x) +
+                                                           (cp.row * p.ldx + kb * 32) * EB);
+#pragma unroll
+        for (int i = 0; i < NW; ++i) o.w[i] = __ldcs(src + i);
     } else {
-        o.w[0] = o.w[BF16_IN ? 0 : 1] = make_uint4(0, 0, 0, 0);
-        if (valid) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const float *>(p.x) + row * p.ldx + col8 * 8);
-            o.w[0] = __ldcs(src);
-            o.w[BF16_IN ? 0 : 1] = __ldcs(src + 1);
-        }
+#pragma unroll
+        for (int i = 0; i < NW; ++i) o.w[i] = make_uint4(0, 0, 0, 0);
     }
 }
 
+__device__ __forceinline__ uint64_t f2_mul_ftz(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 template <int FMT, bool SR, bool BF16_IN>
-__device__ __forceinline__ void cast_oct(const CastParams &p, int64_t row, int64_t col8, bool valid,
-                                         const OctLoad<BF16_IN> &o, int lane) {
+__device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &cp, int64_t blocks_per_row,
+                                           const BlockLoad<BF16_IN> &o, int lane) {
     constexpr int BITS = Fmt<FMT>::bits;
-    float v[8];
-    uint32_t amax_bits;
+    const int64_t kb = cp.chunk * 32 + lane;
+    if (cp.row >= p.rows || kb >= blocks_per_row) return;
+    // the 32 values as fp32 bit patterns
+    uint32_t b[32];
     if (BF16_IN) {
-        const uint4 w = o.w[0];
-        const uint32_t m = __vmaxu2(__vmaxu2(w.x & 0x7fff7fffu, w.y & 0x7fff7fffu),
-                                    __vmaxu2(w.z & 0x7fff7fffu, w.w & 0x7fff7fffu));
-        amax_bits = max(m & 0xffffu, m >> 16) << 16;
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            v[2 * i] = __uint_as_float(ws[i] << 16);
-            v[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+            const uint32_t ws[4] = {o.w[i].x, o.w[i].y, o.w[i].z, o.w[i].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                b[8 * i + 2 * k] = ws[k] << 16;
+                b[8 * i + 2 * k + 1] = ws[k] & 0xffff0000u;
+            }
         }
     } else {
-        const uint4 a = o.w[0], b = o.w[BF16_IN ? 0 : 1];
-        const uint32_t ws[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        amax_bits = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            v[i] = __uint_as_float(ws[i]);
-            amax_bits = max(amax_bits, ws[i] & 0x7fffffffu);
+            b[4 * i] = o.w[i].x; b[4 * i + 1] = o.w[i].y; b[4 * i + 2] = o.w[i].z; b[4 * i + 3] = o.w[i].w;
         }
     }
-    amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 1));
-    amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 2));
-    if (!valid) return;
-
+    uint32_t amax_bits = 0;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2)
+        amax_bits = __vimax3_u32(amax_bits, b[i] & 0x7fffffffu, b[i + 1] & 0x7fffffffu);
     const bool nan_block = amax_bits >= 0x7f800000u;
     const int e = block_exponent<FMT>(amax_bits);
-    float u[8];
+
+    // V * 2^-e with the subnormal flush (mul.ftz), two values per instruction
+    float u[32];
+    if (Fmt<FMT>::emax == 0) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) u[i] = scale_down<FMT>(v[i], e);
-
-    uint32_t rw[2] = {0u, 0u};
-    if (SR) {
-        const uint64_t idx0 = static_cast<uint64_t>(row * p.cols + col8 * 8);
-        const uint32_t g = static_cast<uint32_t>(idx0 >> 2);
-        rw[0] = fmix32(g ^ p.key);
-        rw[1] = fmix32((g + 1u) ^ p.key);
-    }
-    uint32_t c[4];
-    encode_values<FMT, SR>(u, 8, rw, c);
-    if (nan_block) c[0] = c[1] = c[2] = c[3] = 0u;
-
-    if (BITS == 8) {
-        uint2 out = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-        *reinterpret_cast<uint2 *>(p.codes + row * p.cols + col8 * 8) = out;
-    } else if (BITS == 4) {
-        uint32_t out = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-        *reinterpret_cast<uint32_t *>(p.codes + row * (p.cols >> 1) + col8 * 4) = out;
+        for (int i = 0; i < 32; ++i) u[i] = scale_down<FMT>(__uint_as_float(b[i]), e);
     } else {
-        uint64_t w = 0;
+        const uint32_t f = __float_as_uint(pow2f(-e));
+        const uint64_t ff = static_cast<uint64_t>(f) | (static_cast<uint64_t>(f) << 32);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            w |= static_cast<uint64_t>(c[i] & 0x3fu) << (12 * i);
-            w |= static_cast<uint64_t>((c[i] >> 8) & 0x3fu) << (12 * i + 6);
-        }
-        uint8_t *dst = p.codes + row * (p.cols / 4 * 3) + col8 * 6;
-        if ((col8 & 1) == 0) {
-            *reinterpret_cast<uint32_t *>(dst) = static_cast<uint32_t>(w);
-            *reinterpret_cast<uint16_t *>(dst + 4) = static_cast<uint16_t>(w >> 32);
-        } else {
-            *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(w);
-            *reinterpret_cast<uint32_t *>(dst + 2) = static_cast<uint32_t>(w >> 16);
+        for (int i = 0; i < 32; i += 2) {
+            const uint64_t r = f2_mul_ftz(static_cast<uint64_t>(b[i]) | (static_cast<uint64_t>(b[i + 1]) << 32), ff);
+            u[i] = __uint_as_float(static_cast<uint32_t>(r));
+            u[i + 1] = __uint_as_float(static_cast<uint32_t>(r >> 32));
         }
     }
-    if ((lane & 3) == 0) store_scale(p, row, col8 >> 2, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+    if (SR) {
+        const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(cp.row * p.cols + kb * 32) >> 2);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const uint32_t rw = fmix32((g + w) ^ p.key);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = 4 * w + k;
+                u[j] = copysignf(sr_magnitude_int<FMT>(fabsf(u[j]), (rw >> (8 * k)) & 255u), u[j]);
+            }
+        }
+    }
+    uint32_t c[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(u[j], u[j + 1]);
+    if (nan_block) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) c[i] = 0u;
+    }
+    uint8_t *dst = p.codes + cp.row * (p.cols * BITS / 8) + kb * (32 * BITS / 8);
+    if (BITS == 8) {
+        uint4 *d = reinterpret_cast<uint4 *>(dst);
+        d[0] = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+        d[1] = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16), c[14] | (c[15] << 16));
+    } else if (BITS == 4) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = c[4 * i] | (c[4 * i + 1] << 8) | (c[4 * i + 2] << 16) | (c[4 * i + 3] << 24);
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+        uint64_t *d = reinterpret_cast<uint64_t *>(dst);     // 24 bytes, 8-byte aligned
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+            uint64_t w = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int bit = 6 * j - 64 * q;
+                const uint64_t code = (c[j >> 1] >> (8 * (j & 1))) & 0x3fu;
+                if (bit >= 0 && bit < 64) w |= code << bit;
+                else if (bit < 0 && bit > -6) w |= code >> (-bit);
+            }
+            d[q] = w;
+        }
+    }
+    store_scale(p, cp.row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
 }
 
 template <int FMT, bool SR, bool BF16_IN>
-__global__ void __launch_bounds__(256) cast_rows_kernel(CastParams p) {
-    constexpr int U = BF16_IN ? 4 : 2;                  // segments in flight per warp
+__global__ void __launch_bounds__(256, 2) cast_rows_kernel(CastParams p) {
     const int lane = threadIdx.x & 31;
-    const int64_t octs_per_row = p.cols >> 3;
-    const int64_t spr = (octs_per_row + 31) >> 5;       // 32-oct segments per row
+    const int64_t blocks_per_row = p.cols >> 5;
+    const int64_t cpr = (blocks_per_row + 31) >> 5;      // chunks per row
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    // segment s = row * spr + seg; consecutive visits of a warp are n_warps
-    // apart, stepped without a division inside the loop
-    int64_t row = warp0 / spr, seg = warp0 - row * spr;
-    const int64_t step_rows = n_warps / spr, step_seg = n_warps - step_rows * spr;
-
-    while (row < p.rows) {
-        int64_t r[U], c8[U];
-        bool ok[U];
-        OctLoad<BF16_IN> ld[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            r[u] = row;
-            c8[u] = seg * 32 + lane;
-            ok[u] = row < p.rows && c8[u] < octs_per_row;
-            load_oct<BF16_IN>(p, row, c8[u], ok[u], ld[u]);
-            seg += step_seg;
-            row += step_rows;
-            if (seg >= spr) { seg -= spr; ++row; }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) cast_oct<FMT, SR, BF16_IN>(p, r[u], c8[u], ok[u], ld[u], lane);
+    const int64_t step_rows = n_warps / cpr, step_chunk = n_warps - step_rows * cpr;
+    auto advance = [&](ChunkPos &q) {
+        q.chunk += step_chunk;
+        q.row += step_rows;
+        if (q.chunk >= cpr) { q.chunk -= cpr; ++q.row; }
+    };
+    ChunkPos cur;
+    cur.row = warp0 / cpr;
+    cur.chunk = warp0 - cur.row * cpr;
+    BlockLoad<BF16_IN> cur_ld;
+    load_block<BF16_IN>(p, cur, blocks_per_row, lane, cur_ld);
+    while (cur.row < p.rows) {
+        ChunkPos nxt = cur;
+        advance(nxt);
+        BlockLoad<BF16_IN> nxt_ld;
+        load_block<BF16_IN>(p, nxt, blocks_per_row, lane, nxt_ld);
+        cast_block<FMT, SR, BF16_IN>(p, cur, blocks_per_row, cur_ld, lane);
+        cur = nxt;
+        cur_ld = nxt_ld;
     }
 }
 
 // ---------------------------------------------------------------------------
 // Column cast: block axis strided, output transposed.
 // ---------------------------------------------------------------------------
+// A CTA owns a 128-row x 128-column input tile at a time, staged in shared
+// memory by 16-byte cp.async copies (zero-filled outside the tensor) into one
+// of two buffers, so the next tile streams in while the current one is
+// converted.  Each thread owns two adjacent columns of one 32-row block: one
+// 4- or 8-byte shared load feeds both, and the Hadamard butterflies run as
+// packed f32x2 adds on the pair.
 constexpr int COL_TILE_R = 128;   // 4 blocks down
-constexpr int COL_TILE_C = 64;    // columns per tile
+constexpr int COL_TILE_C = 128;   // 64 column pairs
+constexpr int COL_THREADS = 256;  // 64 pairs x 4 blocks
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {   // exact uses only (x +-1)
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+template <bool BF16_IN>
+__device__ __forceinline__ void stage_tile(const CastParams &p, uint8_t *buf, int64_t r0, int64_t c0) {
+    using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
+    constexpr int EPC = 16 / sizeof(TIn);                   // elements per 16-byte chunk
+    constexpr int CPR = COL_TILE_C / EPC;                   // chunks per tile row
+    const TIn *x = static_cast<const TIn *>(p.x);
+    const uint32_t sbuf = static_cast<uint32_t>(__cvta_generic_to_shared(buf));
+    for (int ch = threadIdx.x; ch < COL_TILE_R * CPR; ch += COL_THREADS) {
+        const int rr = ch / CPR, cc = (ch % CPR) * EPC;
+        const int64_t gr = r0 + rr, gc = c0 + cc;
+        int64_t valid = (gr < p.rows) ? (p.cols - gc) : 0;
+        valid = valid < 0 ? 0 : (valid > EPC ? EPC : valid);
+        const TIn *src = valid > 0 ? x + gr * p.ldx + gc : x;
+        cp_async16(sbuf + (rr * COL_TILE_C + cc) * sizeof(TIn), src, static_cast<uint32_t>(valid * sizeof(TIn)));
+    }
+}
 
 template <int FMT, bool SR, bool BF16_IN, bool HAD>
-__global__ void __launch_bounds__(256) cast_cols_kernel(CastParams p) {
+__global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p) {
     using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
-    __shared__ __align__(16) TIn tile[COL_TILE_R][COL_TILE_C];
     constexpr int BITS = Fmt<FMT>::bits;
-    constexpr int ELEMS_PER_CHUNK = 16 / sizeof(TIn);
-    constexpr int CHUNKS_PER_ROW = COL_TILE_C / ELEMS_PER_CHUNK;
+    constexpr int TILE_BYTES = COL_TILE_R * COL_TILE_C * sizeof(TIn);
+    extern __shared__ __align__(16) uint8_t col_smem[];
 
     const int64_t R = p.rows, C = p.cols;
     const int64_t tiles_r = (R + COL_TILE_R - 1) / COL_TILE_R;
     const int64_t tiles_c = (C + COL_TILE_C - 1) / COL_TILE_C;
     const int64_t n_tiles = tiles_r * tiles_c;
-    const TIn *x = static_cast<const TIn *>(p.x);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int blk = warp & 3;                       // 32-row block inside the tile
+    const int pair = (warp >> 2) * 32 + lane;       // column pair inside the tile
 
-    for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t r0 = tr * COL_TILE_R, c0 = tc * COL_TILE_C;
-
-        // stage the tile with 16-byte row loads (ragged edges element-wise)
-        for (int ch = threadIdx.x; ch < COL_TILE_R * CHUNKS_PER_ROW; ch += blockDim.x) {
-            const int rr = ch / CHUNKS_PER_ROW, cc = (ch % CHUNKS_PER_ROW) * ELEMS_PER_CHUNK;
-            const int64_t gr = r0 + rr, gc = c0 + cc;
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (gr < R) {
-                const TIn *src = x + gr * p.ldx + gc;
-                if (gc + ELEMS_PER_CHUNK <= C) {
-                    w = __ldcs(reinterpret_cast<const uint4 *>(src));
-                } else {
-                    TIn tmp[ELEMS_PER_CHUNK];
-#pragma unroll
-                    for (int i = 0; i < ELEMS_PER_CHUNK; ++i) tmp[i] = (gc + i < C) ? src[i] : TIn(0);
-                    w = *reinterpret_cast<uint4 *>(tmp);
-                }
-            }
-            *reinterpret_cast<uint4 *>(&tile[rr][cc]) = w;
-        }
+    int64_t t = blockIdx.x;
+    if (t < n_tiles) stage_tile<BF16_IN>(p, col_smem, (t / tiles_c) * COL_TILE_R, (t % tiles_c) * COL_TILE_C);
+    cp_async_commit();
+    for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1) {
+        const int64_t tn = t + gridDim.x;
+        if (tn < n_tiles)
+            stage_tile<BF16_IN>(p, col_smem + (buf ^ 1) * TILE_BYTES, (tn / tiles_c) * COL_TILE_R,
+                                (tn % tiles_c) * COL_TILE_C);
+        cp_async_commit();
+        cp_async_wait_prev();        // this tile's copies (the older group) have landed
         __syncthreads();
 
-        // one column block of 32 values per thread
-        const int blk = warp & 3;
-        const int col = (warp >> 2) * 32 + lane;
-        const int64_t gc = c0 + col, gr0 = r0 + blk * 32;
+        const int64_t r0 = (t / tiles_c) * COL_TILE_R, c0 = (t % tiles_c) * COL_TILE_C;
+        const int64_t gc = c0 + 2 * pair, gr0 = r0 + blk * 32;
         if (gc < C && gr0 < R) {
-            float v[32];
+            const TIn *tile = reinterpret_cast<const TIn *>(col_smem + buf * TILE_BYTES);
+            // x[j] = (column gc, column gc + 1) at row gr0 + j, as packed f32x2
+            uint64_t x[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (BF16_IN) v[i] = __uint_as_float(static_cast<uint32_t>(tile[blk * 32 + i][col]) << 16);
-                else v[i] = tile[blk * 32 + i][col];
+            for (int j = 0; j < 32; ++j) {
+                const int off = (blk * 32 + j) * COL_TILE_C + 2 * pair;
+                if (BF16_IN) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(tile + off);
+                    x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                } else {
+                    x[j] = *reinterpret_cast<const uint64_t *>(tile + off);
+                }
             }
             if (HAD) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (!((p.sign_mask >> j) & 1u)) v[j] = -v[j];
+                for (int j = 0; j < 32; ++j) {
+                    const float sg = ((p.sign_mask >> j) & 1u) ? 1.0f : -1.0f;
+                    x[j] = f2_mul(x[j], f2_pack(sg, sg));
+                }
 #pragma unroll
                 for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         if (i & h) continue;
-                        const float a = v[i], b = v[i + h];
-                        v[i] = __fadd_rn(a, b);
-                        v[i + h] = __fsub_rn(a, b);
+                        const uint64_t a = x[i], b = x[i + h];
+                        x[i] = f2_add(a, b);
+                        x[i + h] = f2_sub(a, b);
                     }
                 }
             }
-            uint32_t amax_bits = 0;
+            const bool has_second = gc + 1 < C;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) amax_bits = max(amax_bits, __float_as_uint(v[i]) & 0x7fffffffu);
-            const bool nan_block = amax_bits >= 0x7f800000u;
-            const int e = block_exponent<FMT>(amax_bits);
+            for (int col = 0; col < 2; ++col) {
+                if (col == 1 && !has_second) break;
+                float v[32];
+                uint32_t amax_bits = 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = scale_down<FMT>(v[i], e);
-
-            uint32_t rw[8];
-            if (SR) {
-                const uint64_t idx0 = static_cast<uint64_t>(gc * R + gr0);
-                const uint32_t g = static_cast<uint32_t>(idx0 >> 2);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) rw[i] = fmix32((g + i) ^ p.key);
-            }
-            uint32_t c[16];
-            encode_values<FMT, SR>(v, 32, rw, c);
-            if (nan_block) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) c[i] = 0u;
-            }
-            if (BITS == 8) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.codes + gc * R + gr0);
-                dst[0] = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
-                dst[1] = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16), c[14] | (c[15] << 16));
-            } else if (BITS == 4) {
-                uint32_t w[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    w[i] = c[4 * i] | (c[4 * i + 1] << 8) | (c[4 * i + 2] << 16) | (c[4 * i + 3] << 24);
-                *reinterpret_cast<uint4 *>(p.codes + gc * (R >> 1) + (gr0 >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
-            } else {
-                uint64_t *dst = reinterpret_cast<uint64_t *>(p.codes + gc * (R / 4 * 3) + gr0 / 4 * 3);
-#pragma unroll
-                for (int q = 0; q < 3; ++q) {     // 3 words of 64 bits = 32 codes of 6 bits
-                    uint64_t w = 0;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int bit = 6 * j - 64 * q;
-                        const uint64_t code = (c[j >> 1] >> (8 * (j & 1))) & 0x3fu;
-                        if (bit >= 0 && bit < 64) w |= code << bit;
-                        else if (bit < 0 && bit > -6) w |= code >> (-bit);
-                    }
-                    dst[q] = w;
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t b = static_cast<uint32_t>(x[j] >> (32 * col));
+                    v[j] = __uint_as_float(b);
+                    amax_bits = max(amax_bits, b & 0x7fffffffu);
                 }
+                const bool nan_block = amax_bits >= 0x7f800000u;
+                const int e = block_exponent<FMT>(amax_bits);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = scale_down<FMT>(v[j], e);
+                const int64_t oc = gc + col;                 // output row
+                uint32_t c[16];
+                if (SR) {
+                    const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(oc * R + gr0) >> 2);
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        const uint32_t rw = fmix32((g + w) ^ p.key);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int j = 4 * w + k;
+                            const float m = sr_magnitude_int<FMT>(fabsf(v[j]), (rw >> (8 * k)) & 255u);
+                            v[j] = copysignf(m, v[j]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(v[j], v[j + 1]);
+                if (nan_block) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) c[i] = 0u;
+                }
+                if (BITS == 8) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.codes + oc * R + gr0);
+                    dst[0] = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+                    dst[1] = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16),
+                                        c[14] | (c[15] << 16));
+                } else if (BITS == 4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        w[i] = c[4 * i] | (c[4 * i + 1] << 8) | (c[4 * i + 2] << 16) | (c[4 * i + 3] << 24);
+                    *reinterpret_cast<uint4 *>(p.codes + oc * (R >> 1) + (gr0 >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
+                } else {
+                    uint64_t *dst = reinterpret_cast<uint64_t *>(p.codes + oc * (R / 4 * 3) + gr0 / 4 * 3);
+#pragma unroll
+                    for (int q = 0; q < 3; ++q) {     // 3 words of 64 bits = 32 codes of 6 bits
+                        uint64_t w = 0;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int bit = 6 * j - 64 * q;
+                            const uint64_t code = (c[j >> 1] >> (8 * (j & 1))) & 0x3fu;
+                            if (bit >= 0 && bit < 64) w |= code << bit;
+                            else if (bit < 0 && bit > -6) w |= code >> (-bit);
+                        }
+                        dst[q] = w;
+                    }
+                }
+                store_scale(p, oc, gr0 >> 5, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
             }
-            store_scale(p, gc, gr0 >> 5, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
         }
-        __syncthreads();
+        __syncthreads();             // everyone is done with `buf` before it is refilled
     }
+    cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -432,25 +524,55 @@ static int grid_for(int64_t work_items, int per_block, int max_blocks) {
     return static_cast<int>(b < 1 ? 1 : b);
 }
 
+// Blocks of `Kernel` that fit on one SM at once (queried once per kernel;
+// the cache is per template instance, i.e. per kernel): grid-stride kernels
+// are launched with exactly the resident number of blocks.
+template <auto Kernel>
+static int resident_blocks_per_sm(int threads, int smem) {
+    static int cached = 0;
+    if (cached == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess || n < 1) n = 1;
+        cached = n;
+    }
+    return cached;
+}
+
+// Column cast: two tile buffers of dynamic shared memory, a resident grid.
+template <auto Kernel>
+static cudaError_t launch_cols(int in_bytes, const CastParams &p, int64_t tiles, int sms, cudaStream_t st) {
+    const int smem = 2 * COL_TILE_R * COL_TILE_C * in_bytes;
+    static bool configured = false;    // per template instance, i.e. per kernel
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    Kernel<<<grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)), COL_THREADS, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
 template <int FMT, bool SR>
 static cudaError_t launch_cast_fmt(const CastParams &p, int xdt, int block_axis, bool had, int sms,
                                    cudaStream_t st) {
     const bool bf = xdt == MX_BF16;
     if (block_axis == 1) {
-        const int64_t segs = p.rows * (((p.cols >> 3) + 31) >> 5);
-        const int grid = grid_for(segs, 8, sms * 8);
-        if (bf) cast_rows_kernel<FMT, SR, true><<<grid, 256, 0, st>>>(p);
-        else cast_rows_kernel<FMT, SR, false><<<grid, 256, 0, st>>>(p);
+        const int64_t chunks = p.rows * (((p.cols >> 5) + 31) >> 5);    // 32-block chunks, one per warp
+        if (bf) {
+            constexpr auto k = cast_rows_kernel<FMT, SR, true>;
+            k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+        } else {
+            constexpr auto k = cast_rows_kernel<FMT, SR, false>;
+            k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+        }
     } else {
         const int64_t tiles = ((p.rows + COL_TILE_R - 1) / COL_TILE_R) * ((p.cols + COL_TILE_C - 1) / COL_TILE_C);
-        const int grid = grid_for(tiles, 1, sms * 8);
         if (had) {
-            if (bf) cast_cols_kernel<FMT, SR, true, true><<<grid, 256, 0, st>>>(p);
-            else cast_cols_kernel<FMT, SR, false, true><<<grid, 256, 0, st>>>(p);
-        } else {
-            if (bf) cast_cols_kernel<FMT, SR, true, false><<<grid, 256, 0, st>>>(p);
-            else cast_cols_kernel<FMT, SR, false, false><<<grid, 256, 0, st>>>(p);
+            if (bf) return launch_cols<cast_cols_kernel<FMT, SR, true, true>>(2, p, tiles, sms, st);
+            return launch_cols<cast_cols_kernel<FMT, SR, false, true>>(4, p, tiles, sms, st);
         }
+        if (bf) return launch_cols<cast_cols_kernel<FMT, SR, true, false>>(2, p, tiles, sms, st);
+        return launch_cols<cast_cols_kernel<FMT, SR, false, false>>(4, p, tiles, sms, st);
     }
     return cudaGetLastError();
 }

@@ -126,6 +126,25 @@ __device__ __forceinline__ float sr_magnitude(float a, uint32_t r) {
     return t * step;
 }
 
+// The same stochastic rounding in integer arithmetic, as used by the strided
+// (weight-gradient) cast.  For a >= 2^emin the grid step of a's binade is one
+// unit of fp32 mantissa bit (23 - mbits): adding r at the eight bits below that
+// unit carries into it exactly when F + r >= 256, and truncation then gives
+// lo or lo + step.  For a < 2^emin (the element's subnormal range, uniform
+// step 2^(emin - mbits)) a is first shifted to a + 2^emin with a
+// round-toward-zero add, which keeps every bit that F depends on, rounded
+// the same way, and shifted back exactly.  Returns the rounded magnitude.
+template <int FMT>
+__device__ __forceinline__ float sr_magnitude_int(float a, uint32_t r) {
+    using F = Fmt<FMT>;
+    const float t = a < pow2f(F::emin) ? pow2f(F::emin) : 0.0f;
+    const float w = __fadd_rz(a, t);
+    constexpr int UNIT = 23 - F::mbits;
+    uint32_t wb = __float_as_uint(w) + (r << (UNIT - 8));
+    wb &= ~((1u << UNIT) - 1u);
+    return fminf(__fsub_rn(__uint_as_float(wb), t), F::maxv);
+}
+
 // MurmurHash3 32-bit finaliser (public domain, A. Appleby).
 __device__ __forceinline__ uint32_t fmix32(uint32_t h) {
     h ^= h >> 16;

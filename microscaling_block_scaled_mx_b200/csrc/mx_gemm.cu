@@ -3,8 +3,8 @@
 // Formats for Deep Learning" (summary page, section 4), which take MX inputs
 // and return scalar floats.
 //
-// Design (one persistent CTA per SM, 192 threads, warp-specialized):
-//   warp 0      TMA producer: 128 x 128-byte A tile and 256 x 128-byte B tile
+// Design (one persistent CTA per SM, 320 threads, warp-specialized):
+//   warp 0      TMA producer: 128 x 128-byte A tile and 192 x 128-byte B tile
 //               per stage (128-byte swizzle), plus the 512-byte E8M0 scale
 //               atoms of both operands (bulk copies; the MMA layout written by
 //               mx_quantize is already the tensor-core layout).
@@ -12,9 +12,13 @@
 //               scale atom smem -> TMEM (32x128b, replicated to the four lane
 //               quarters), then four tcgen05.mma.block_scale per stage
 //               (kind::mxf8f6f4 K=32 for MXFP8, kind::mxf4 K=64 for MXFP4)
-//               accumulate into a 128 x 256 fp32 TMEM accumulator.
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, times alpha,
-//               rounded to fp32 / bf16, stored to C with bounds checks.
+//               accumulate into one of two 128 x 192 fp32 TMEM accumulators,
+//               so the epilogue of a tile overlaps the mainloop of the next.
+//   warps 2-9   epilogue: two warps per TMEM lane quarter, 96 columns each,
+//               three tcgen05.ld of 32 columns per wait, times alpha, rounded
+//               to fp32 / bf16, stored to C with bounds checks.
+// A 192-column tile starts 64 rows into a 128-row scale atom on odd tiles;
+// the B scale-factor TMEM address then starts two columns later.
 // Every mbarrier wait is bounded; on expiry the kernel records MX_ERR_TIMEOUT
 // in the device status word, drains what it issued (bounded again), frees
 // its TMEM and returns.
@@ -38,23 +42,24 @@ __device__ int g_mx_status;
 namespace mxg {
 
 constexpr int BM = 128;            // tile rows (A rows, TMEM lanes)
-constexpr int BN = 256;            // tile columns (B rows, accumulator columns)
+constexpr int BN = 192;            // tile columns (B rows, accumulator columns)
 constexpr int BK_BYTES = 128;      // K bytes per stage: 128 fp8 or 256 fp4 elements
-constexpr int STAGES = 4;
-constexpr int NUM_THREADS = 192;
+constexpr int STAGES = 5;
+constexpr int EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr int A_STAGE_BYTES = BM * BK_BYTES;   // 16 KiB
-constexpr int B_STAGE_BYTES = BN * BK_BYTES;   // 32 KiB
+constexpr int B_STAGE_BYTES = BN * BK_BYTES;   // 24 KiB
 constexpr int ATOM = 512;                      // scale atom: 128 rows x 4 k-blocks
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0;                // accumulator columns [0, 256)
-constexpr uint32_t SF_COL = 256;               // scale-factor columns from 256
+constexpr uint32_t ACC_COLS = BN;              // accumulator b at columns [b * 192, (b + 1) * 192)
+constexpr uint32_t SF_COL = 2 * ACC_COLS;      // scale-factor columns from 384
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;   // 0.2 s when draining
 
 template <bool FP4> struct Cfg {
     static constexpr int G = FP4 ? 2 : 1;             // scale atoms along K per stage
     static constexpr int SFA_BYTES = ATOM * G;        // per stage
-    static constexpr int SFB_BYTES = 2 * ATOM * G;    // two 128-row halves of B
+    static constexpr int SFB_BYTES = 2 * ATOM * G;    // the two 128-row scale blocks a tile touches
     static constexpr int SFA_COLS = 4 * G;            // TMEM columns per stage
     static constexpr int SFB_COLS = 8 * G;
     static constexpr int SF_STAGE_COLS = SFA_COLS + SFB_COLS;
@@ -67,8 +72,8 @@ struct Smem {
     static constexpr int SFA = B + STAGES * B_STAGE_BYTES;
     static constexpr int SFB = SFA + STAGES * 2 * ATOM;       // sized for the FP4 case
     static constexpr int BAR = SFB + STAGES * 4 * ATOM;
-    // full[STAGES], empty[STAGES], acc_full, acc_empty, drain
-    static constexpr int NUM_BARS = 2 * STAGES + 3;
+    // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
+    static constexpr int NUM_BARS = 2 * STAGES + 5;
     static constexpr int TMEM_SLOT = BAR + NUM_BARS * 8;
     static constexpr int ABORT = TMEM_SLOT + 4;
     static constexpr int TOTAL = ABORT + 4;
@@ -204,7 +209,10 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
     }
 }
 
-__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+// ------------------------------------------------------------------------
+// The kernel
+// ------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_ld_x32_nowait(uint32_t taddr, uint32_t *r) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -214,12 +222,48 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive accumulator values of one row -> C (bounds-checked).
+template <bool BF16_OUT>
+__device__ __forceinline__ void store_row_chunk(const Params &p, int m, int n0, const uint32_t *r) {
+    if (m >= p.M || n0 >= p.N) return;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), p.alpha);
+    if (BF16_OUT) {
+        __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
+        if (n0 + 32 <= p.N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * t], v[i + 2 * t + 1]);
+                    w[t] = *reinterpret_cast<uint32_t *>(&b2);
+                }
+                *reinterpret_cast<uint4 *>(row + i) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) row[i] = __float2bfloat16_rn(v[i]);
+        }
+    } else {
+        float *row = static_cast<float *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
+        if (n0 + 32 <= p.N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) row[i] = v[i];
+        }
+    }
 }
 
-// ------------------------------------------------------------------------
-// The kernel
-// ------------------------------------------------------------------------
 template <bool FP4, bool BF16_OUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, Params p) {
@@ -233,9 +277,9 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
 
     auto full_bar = [&](int s) { return sbase + Smem::BAR + 8u * s; };
     auto empty_bar = [&](int s) { return sbase + Smem::BAR + 8u * (STAGES + s); };
-    const uint32_t acc_full = sbase + Smem::BAR + 8u * (2 * STAGES);
-    const uint32_t acc_empty = acc_full + 8u;
-    const uint32_t drain_bar = acc_full + 16u;
+    auto acc_full = [&](int b) { return sbase + Smem::BAR + 8u * (2 * STAGES + b); };
+    auto acc_empty = [&](int b) { return sbase + Smem::BAR + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t drain_bar = sbase + Smem::BAR + 8u * (2 * STAGES + 4);
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -243,8 +287,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full(b), 1);
+            mbar_init(acc_empty(b), EPI_WARPS);
+        }
         mbar_init(drain_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -270,8 +316,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
                 const int m0 = tm * BM, n0 = tn * BN;
-                const int rb_a = m0 / 128, rb_b = n0 / 128;
-                const bool b_hi = (n0 + 128) < p.N;   // second 128-row half of B exists
+                const int rb_a = m0 / 128, rb_b = n0 / 128;   // 128-row scale blocks
+                const bool b_second = (rb_b + 1) * 128 < p.N;
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
                     if (kt == p.skip_k_tile && tile == static_cast<int>(blockIdx.x) && blockIdx.x == 0) {
@@ -279,7 +325,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                         break;
                     }
                     const uint32_t bytes = A_STAGE_BYTES + B_STAGE_BYTES + C::SFA_BYTES +
-                                           (b_hi ? 2 : 1) * (C::SFB_BYTES / 2);
+                                           (b_second ? 2 : 1) * (C::SFB_BYTES / 2);
                     const uint32_t fb = full_bar(s);
                     mbar_expect_tx(fb, bytes);
                     tma_load_2d(sbase + Smem::A + s * A_STAGE_BYTES, &tma_a, kt * BK_BYTES, m0, fb);
@@ -289,7 +335,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                               p.a_scales + (static_cast<int64_t>(rb_a) * p.k_groups + kg) * ATOM, C::SFA_BYTES, fb);
                     bulk_load(sbase + Smem::SFB + s * 4 * ATOM,
                               p.b_scales + (static_cast<int64_t>(rb_b) * p.k_groups + kg) * ATOM, C::SFB_BYTES / 2, fb);
-                    if (b_hi)
+                    if (b_second)
                         bulk_load(sbase + Smem::SFB + s * 4 * ATOM + C::SFB_BYTES / 2,
                                   p.b_scales + (static_cast<int64_t>(rb_b + 1) * p.k_groups + kg) * ATOM,
                                   C::SFB_BYTES / 2, fb);
@@ -316,12 +362,18 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         // ------------------------------ MMA issuer ----------------------------
         if (lane == 0) {
             int s = 0;
-            uint32_t ph = 0, acc_ph = 0;
+            uint32_t ph = 0;
             bool ok = true;
             bool issued = false;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                if (!wait_bounded(acc_empty, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
+            int local = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                const int b = local & 1;
+                const uint32_t acc_ph = (local >> 1) & 1;
+                if (!wait_bounded(acc_empty(b), acc_ph ^ 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
+                const int tn = tile / p.tiles_m;
+                const uint32_t d_tmem = tmem + b * ACC_COLS;
+                const uint32_t sfb_shift = (tn & 1) ? 2u : 0u;   // odd 192-column tiles
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!wait_bounded(full_bar(s), ph, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -345,16 +397,15 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                         const uint32_t g = FP4 ? (k >> 1) : 0u;
                         const uint32_t sf_id = FP4 ? ((2u * k) & 3u) : static_cast<uint32_t>(k);
                         const uint32_t idesc = p.idesc | (sf_id << 4) | (sf_id << 29);
-                        tc_mma<FP4>(tmem + ACC_COL, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k), idesc,
-                                    sfa_t + 4 * g, sfb_t + 8 * g, (kt > 0 || k > 0) ? 1u : 0u);
+                        tc_mma<FP4>(d_tmem, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k), idesc,
+                                    sfa_t + 4 * g, sfb_t + 8 * g + sfb_shift, (kt > 0 || k > 0) ? 1u : 0u);
                     }
                     issued = true;
                     tc_commit(empty_bar(s));
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit(acc_full);
-                acc_ph ^= 1u;
+                tc_commit(acc_full(b));
             }
             if (issued) {
                 // all issued MMAs must finish before TMEM is released
@@ -365,64 +416,35 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         }
     } else {
         // ------------------------------ epilogue ------------------------------
-        const int q = warp & 3;                 // TMEM lane quarter this warp may access
-        uint32_t acc_ph = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int q = warp & 3;                  // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;        // which 96 columns of the tile
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int b = local & 1;
+            const uint32_t acc_ph = (local >> 1) & 1;
             // one lane waits, the warp follows its verdict: tcgen05.ld below
             // must be executed by all 32 lanes together
             int ok = 1;
-            if (lane == 0) ok = wait_bounded(acc_full, acc_ph, abort_flag) ? 1 : 0;
+            if (lane == 0) ok = wait_bounded(acc_full(b), acc_ph, abort_flag) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
             const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
             const int m = tm * BM + q * 32 + lane;
-            const int n_base = tn * BN;
-#pragma unroll 1
-            for (int j = 0; j < BN / 32; ++j) {
-                uint32_t r[32];
-                tmem_ld_32cols(tmem + ACC_COL + (static_cast<uint32_t>(q * 32) << 16) + j * 32, r);
-                const int n0 = n_base + j * 32;
-                if (m < p.M && n0 < p.N) {
-                    float v[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), p.alpha);
-                    if (BF16_OUT) {
-                        __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
-                        if (n0 + 32 <= p.N) {
-#pragma unroll
-                            for (int i = 0; i < 32; i += 8) {
-                                uint32_t w[4];
-#pragma unroll
-                                for (int t = 0; t < 4; ++t) {
-                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * t], v[i + 2 * t + 1]);
-                                    w[t] = *reinterpret_cast<uint32_t *>(&b2);
-                                }
-                                *reinterpret_cast<uint4 *>(row + i) = make_uint4(w[0], w[1], w[2], w[3]);
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (n0 + i < p.N) row[i] = __float2bfloat16_rn(v[i]);
-                        }
-                    } else {
-                        float *row = static_cast<float *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
-                        if (n0 + 32 <= p.N) {
-#pragma unroll
-                            for (int i = 0; i < 32; i += 4)
-                                *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (n0 + i < p.N) row[i] = v[i];
-                        }
-                    }
-                }
-            }
+            const int c0 = half * (BN / 2);
+            const uint32_t taddr = tmem + b * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + c0;
+            uint32_t r[96];
+            tmem_ld_x32_nowait(taddr, r);
+            tmem_ld_x32_nowait(taddr + 32, r + 32);
+            tmem_ld_x32_nowait(taddr + 64, r + 64);
+            tmem_wait_ld();
+            // the accumulator buffer can be refilled as soon as it is in registers
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-            acc_ph ^= 1u;
+            if (lane == 0) mbar_arrive(acc_empty(b));
+            const int n_base = tn * BN + c0;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) store_row_chunk<BF16_OUT>(p, m, n_base + 32 * j, r + 32 * j);
         }
     }
 
