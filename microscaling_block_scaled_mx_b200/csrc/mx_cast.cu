@@ -75,7 +75,16 @@ struct ChunkPos {
     int64_t row, chunk;   // chunk = 32 consecutive blocks of one row
 };
 
-template <bool BF16_IN>
+// 32-byte global load (two uint4), streaming: no L1 allocation
+__device__ __forceinline__ void ld32_stream(const void *src, uint4 &a, uint4 &b) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(src));
+}
+
+// V32: the input rows are 32-byte aligned, so each lane fetches its block with
+// 32-byte loads (every sector a load touches is used in full).
+template <bool BF16_IN, bool V32>
 __device__ __forceinline__ void load_block(const CastParams &p, const ChunkPos &cp, int64_t blocks_per_row, int lane,
                                            BlockLoad<BF16_IN> &o) {
     constexpr int NW = BF16_IN ? 4 : 8;
@@ -84,8 +93,13 @@ __device__ __forceinline__ void load_block(const CastParams &p, const ChunkPos &
         constexpr int EB = BF16_IN ? 2 : 4;
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.x) +
                                                            (cp.row * p.ldx + kb * 32) * EB);
+        if (V32) {
 #pragma unroll
-        for (int i = 0; i < NW; ++i) o.w[i] = __ldcs(src + i);
+            for (int i = 0; i < NW; i += 2) ld32_stream(src + i, o.w[i], o.w[i + 1]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < NW; ++i) o.w[i] = __ldcs(src + i);
+        }
     } else {
 #pragma unroll
         for (int i = 0; i < NW; ++i) o.w[i] = make_uint4(0, 0, 0, 0);
@@ -191,7 +205,7 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
     store_scale(p, cp.row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
 }
 
-template <int FMT, bool SR, bool BF16_IN>
+template <int FMT, bool SR, bool BF16_IN, bool V32>
 __global__ void __launch_bounds__(256, 2) cast_rows_kernel(CastParams p) {
     const int lane = threadIdx.x & 31;
     const int64_t blocks_per_row = p.cols >> 5;
@@ -208,12 +222,12 @@ __global__ void __launch_bounds__(256, 2) cast_rows_kernel(CastParams p) {
     cur.row = warp0 / cpr;
     cur.chunk = warp0 - cur.row * cpr;
     BlockLoad<BF16_IN> cur_ld;
-    load_block<BF16_IN>(p, cur, blocks_per_row, lane, cur_ld);
+    load_block<BF16_IN, V32>(p, cur, blocks_per_row, lane, cur_ld);
     while (cur.row < p.rows) {
         ChunkPos nxt = cur;
         advance(nxt);
         BlockLoad<BF16_IN> nxt_ld;
-        load_block<BF16_IN>(p, nxt, blocks_per_row, lane, nxt_ld);
+        load_block<BF16_IN, V32>(p, nxt, blocks_per_row, lane, nxt_ld);
         cast_block<FMT, SR, BF16_IN>(p, cur, blocks_per_row, cur_ld, lane);
         cur = nxt;
         cur_ld = nxt_ld;
@@ -558,12 +572,23 @@ static cudaError_t launch_cast_fmt(const CastParams &p, int xdt, int block_axis,
     const bool bf = xdt == MX_BF16;
     if (block_axis == 1) {
         const int64_t chunks = p.rows * (((p.cols >> 5) + 31) >> 5);    // 32-block chunks, one per warp
+        const bool v32 = (reinterpret_cast<uintptr_t>(p.x) & 31u) == 0 && ((p.ldx * (bf ? 2 : 4)) & 31) == 0;
         if (bf) {
-            constexpr auto k = cast_rows_kernel<FMT, SR, true>;
-            k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+            if (v32) {
+                constexpr auto k = cast_rows_kernel<FMT, SR, true, true>;
+                k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+            } else {
+                constexpr auto k = cast_rows_kernel<FMT, SR, true, false>;
+                k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+            }
         } else {
-            constexpr auto k = cast_rows_kernel<FMT, SR, false>;
-            k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+            if (v32) {
+                constexpr auto k = cast_rows_kernel<FMT, SR, false, true>;
+                k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+            } else {
+                constexpr auto k = cast_rows_kernel<FMT, SR, false, false>;
+                k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+            }
         }
     } else {
         const int64_t tiles = ((p.rows + COL_TILE_R - 1) / COL_TILE_R) * ((p.cols + COL_TILE_C - 1) / COL_TILE_C);

@@ -457,6 +457,290 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
 }
 
 // ------------------------------------------------------------------------
+// Two-SM kernel (cta_group::2): a cluster of two CTAs computes a 256 x 192
+// tile.  CTA r of the pair holds rows [128 r, 128 r + 128) of A and B rows
+// [96 r, 96 r + 96) in its shared memory; one tcgen05.mma.cta_group::2 issued
+// by CTA 0 consumes both halves and writes each CTA's 128 accumulator rows
+// into that CTA's tensor memory.  Every tensor-memory copy and MMA therefore
+// covers twice the work of the one-SM kernel, and each SM loads only half of
+// the B tile.  Each CTA keeps its own A scales and the full B scales (the
+// pair-wide tcgen05.cp copies each CTA's shared memory into its own tensor
+// memory).  All loads of both CTAs complete on CTA 0's stage barrier (the
+// two-SM form of the TMA load); CTA 0's commit frees the stage in both CTAs.
+// ------------------------------------------------------------------------
+constexpr int PAIR_BM = 256;
+constexpr int PAIR_BN = 192;
+constexpr int PAIR_B_ROWS = PAIR_BN / 2;                 // B rows per CTA
+constexpr int PAIR_A_BYTES = 128 * BK_BYTES;             // 16 KiB per CTA per stage
+constexpr int PAIR_B_BYTES = PAIR_B_ROWS * BK_BYTES;     // 12 KiB per CTA per stage
+
+template <bool FP4> struct PairCfg {
+    static constexpr int G = FP4 ? 2 : 1;                // scale atoms along K per stage
+    static constexpr int STAGES = FP4 ? 5 : 6;           // bounded by tensor-memory columns
+    static constexpr int SFA_BYTES = ATOM * G;
+    static constexpr int SFB_BYTES = 2 * ATOM * G;       // both 128-row scale blocks the tile touches
+    static constexpr int SFA_COLS = 4 * G;
+    static constexpr int SFB_COLS = 8 * G;
+    static constexpr int SF_STAGE_COLS = SFA_COLS + SFB_COLS;
+    static constexpr int STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES;
+    // shared-memory layout
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * PAIR_A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * PAIR_B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 5;      // full, empty, acc_full[2], acc_empty[2], drain
+    static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM + 4;
+    static constexpr int SMEM = OFF_ABORT + 4 + 1024;    // + alignment slack
+    static_assert(2 * PAIR_BN + STAGES * SF_STAGE_COLS <= 512, "tensor memory columns");
+    static_assert(SMEM <= 232448, "shared memory per block");
+};
+
+struct PairParams {
+    void *c;
+    int64_t ldc;
+    int M, N, K;
+    int k_tiles;
+    int k_groups;
+    int tiles_m, tiles_n;      // 256 x 192 pair tiles
+    float alpha;
+    uint32_t idesc;
+    int skip_k_tile;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// address of the same shared-memory location in cluster CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// two-SM TMA load: data to this CTA's shared memory, bytes counted on the
+// barrier at `bar_cluster_addr` (CTA 0's)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                                 uint32_t bar_cluster_addr) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(bar), "h"(static_cast<uint16_t>(3)) : "memory");
+}
+__device__ __forceinline__ void tc_cp_scale_atom_pair(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+template <bool FP4>
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    if (FP4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+            : "memory");
+    }
+}
+
+template <bool FP4, bool BF16_OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                    const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
+                    PairParams p) {
+    using C = PairCfg<FP4>;
+    constexpr int STAGES_P = C::STAGES;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEM);
+
+    auto full_bar = [&](int s) { return sbase + C::OFF_BAR + 8u * s; };
+    auto empty_bar = [&](int s) { return sbase + C::OFF_BAR + 8u * (STAGES_P + s); };
+    auto acc_full = [&](int b) { return sbase + C::OFF_BAR + 8u * (2 * STAGES_P + b); };
+    auto acc_empty = [&](int b) { return sbase + C::OFF_BAR + 8u * (2 * STAGES_P + 2 + b); };
+    const uint32_t drain_bar = sbase + C::OFF_BAR + 8u * (2 * STAGES_P + 4);
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < STAGES_P; ++s) {
+            mbar_init(full_bar(s), 1);          // CTA 0's producer; bytes from both CTAs
+            mbar_init(empty_bar(s), 1);         // CTA 0's commit, multicast to both CTAs
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full(b), 1);
+            mbar_init(acc_empty(b), 2 * EPI_WARPS);   // epilogue warps of both CTAs (on CTA 0)
+        }
+        mbar_init(drain_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();                  // barriers of both CTAs initialised, tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+    const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+
+    if (warp == 0) {
+        // ------------------------------ producer (both CTAs) -------------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            const uint32_t stage_bytes = 2 * (C::STAGE_BYTES + C::SFA_BYTES + C::SFB_BYTES);
+            for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
+                const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+                // this CTA's A rows and B rows; a half that lies wholly past M (or N)
+                // only feeds discarded outputs, so its loads are clamped to rows
+                // that exist and no TMA box is ever entirely outside its tensor
+                const int m0 = min(tm * PAIR_BM + 128 * static_cast<int>(rank), p.M - 1);
+                const int nb0 = min(tn * PAIR_BN + PAIR_B_ROWS * static_cast<int>(rank), p.N - 1);
+                const int rb_a = m0 / 128, rb_b = (tn * PAIR_BN) / 128;
+                const int rb_b1 = min(rb_b + 1, (p.N - 1) / 128);
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
+                    if (rank == 0 && kt == p.skip_k_tile && tile == cluster_id && cluster_id == 0) {
+                        ok = false;          // injected stall: CTA 0 never arms this stage
+                        break;
+                    }
+                    const uint32_t fb = map_to_rank(full_bar(s), 0);
+                    if (rank == 0) mbar_expect_tx(full_bar(s), stage_bytes);
+                    tma_load_2d_pair(sbase + C::OFF_A + s * PAIR_A_BYTES, &tma_a, kt * BK_BYTES, m0, fb);
+                    tma_load_2d_pair(sbase + C::OFF_B + s * PAIR_B_BYTES, &tma_b, kt * BK_BYTES, nb0, fb);
+                    // scale atoms: a scale buffer is viewed as rows of 256 bytes, two per atom
+                    const int kg = kt * C::G;
+                    tma_load_2d_pair(sbase + C::OFF_SFA + s * C::SFA_BYTES, &tma_sfa, 0,
+                                     2 * (rb_a * p.k_groups + kg), fb);
+                    tma_load_2d_pair(sbase + C::OFF_SFB + s * C::SFB_BYTES, &tma_sfb, 0,
+                                     2 * (rb_b * p.k_groups + kg), fb);
+                    tma_load_2d_pair(sbase + C::OFF_SFB + s * C::SFB_BYTES + C::SFB_BYTES / 2, &tma_sfb, 0,
+                                     2 * (rb_b1 * p.k_groups + kg), fb);
+                    if (++s == STAGES_P) { s = 0; ph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer (CTA 0) ---------------------
+        if (lane == 0 && rank == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            bool issued = false;
+            int local = 0;
+            for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters, ++local) {
+                const int b = local & 1;
+                const uint32_t acc_ph = (local >> 1) & 1;
+                if (!wait_bounded(acc_empty(b), acc_ph ^ 1u, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const int tn = tile / p.tiles_m;
+                const uint32_t d_tmem = tmem + b * ACC_COLS;
+                const uint32_t sfb_shift = (tn & 1) ? 2u : 0u;   // odd 192-column tiles
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!wait_bounded(full_bar(s), ph, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sfa_t = tmem + SF_COL + s * C::SF_STAGE_COLS;
+                    const uint32_t sfb_t = sfa_t + C::SFA_COLS;
+                    const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
+                    const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
+#pragma unroll
+                    for (int g = 0; g < C::G; ++g) {
+                        tc_cp_scale_atom_pair(sfa_t + 4 * g, scale_atom_desc(sfa_s + g * ATOM));
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tc_cp_scale_atom_pair(sfb_t + 8 * g + 4 * h,
+                                                  scale_atom_desc(sfb_s + h * (C::SFB_BYTES / 2) + g * ATOM));
+                    }
+                    const uint32_t a_s = sbase + C::OFF_A + s * PAIR_A_BYTES;
+                    const uint32_t b_s = sbase + C::OFF_B + s * PAIR_B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t g = FP4 ? (k >> 1) : 0u;
+                        const uint32_t sf_id = FP4 ? ((2u * k) & 3u) : static_cast<uint32_t>(k);
+                        const uint32_t idesc = p.idesc | (sf_id << 4) | (sf_id << 29);
+                        tc_mma_pair<FP4>(d_tmem, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k), idesc,
+                                         sfa_t + 4 * g, sfb_t + 8 * g + sfb_shift, (kt > 0 || k > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit_pair(empty_bar(s));
+                    if (++s == STAGES_P) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit_pair(acc_full(b));
+            }
+            if (issued) {
+                tc_commit_pair(drain_bar);   // same cta_group as every other tcgen05 op here
+                volatile int no_abort = 0;
+                (void)wait_bounded(drain_bar, 0, &no_abort, ok ? WAIT_LIMIT_NS : DRAIN_LIMIT_NS);
+            }
+        }
+    } else {
+        // ------------------------------ epilogue (both CTAs) -------------------
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        int local = 0;
+        for (int tile = cluster_id; tile < num_tiles; tile += n_clusters, ++local) {
+            const int b = local & 1;
+            const uint32_t acc_ph = (local >> 1) & 1;
+            int ok = 1;
+            if (lane == 0) ok = wait_bounded(acc_full(b), acc_ph, abort_flag) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+            const int m = tm * PAIR_BM + 128 * static_cast<int>(rank) + q * 32 + lane;
+            const int c0 = half * (PAIR_BN / 2);
+            const uint32_t taddr = tmem + b * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + c0;
+            uint32_t r[96];
+            tmem_ld_x32_nowait(taddr, r);
+            tmem_ld_x32_nowait(taddr + 32, r + 32);
+            tmem_ld_x32_nowait(taddr + 64, r + 64);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(map_to_rank(acc_empty(b), 0));
+            const int n_base = tn * PAIR_BN + c0;
+            Params pp;
+            pp.c = p.c; pp.ldc = p.ldc; pp.M = p.M; pp.N = p.N; pp.alpha = p.alpha;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) store_row_chunk<BF16_OUT>(pp, m, n_base + 32 * j, r + 32 * j);
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();                  // all MMAs drained and all epilogue reads done in both CTAs
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -487,7 +771,22 @@ bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t 
     return r == CUDA_SUCCESS;
 }
 
-uint32_t make_idesc(int fa, int fb, bool fp4) {
+// 2-D uint8 view of an MMA-layout scale buffer as rows of 256 bytes (two rows
+// per 512-byte atom); a box of 2 * atoms rows x 256 bytes, no swizzle.
+bool make_scale_map(CUtensorMap *map, const void *base, int64_t bytes, int atoms_per_box) {
+    auto encode = get_encode();
+    if (!encode || bytes % 256 != 0) return false;
+    cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(bytes / 256)};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {256, static_cast<cuuint32_t>(2 * atoms_per_box)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN) {
     auto code = [&](int f) -> uint32_t {
         if (fp4) return 1u;               // kind::mxf4: E2M1
         return f == MX_E5M2 ? 1u : 0u;    // kind::mxf8f6f4: E4M3 = 0, E5M2 = 1
@@ -495,10 +794,24 @@ uint32_t make_idesc(int fa, int fb, bool fp4) {
     uint32_t d = 0;
     d |= code(fa) << 7;
     d |= code(fb) << 10;
-    d |= static_cast<uint32_t>(BN >> 3) << 17;
+    d |= static_cast<uint32_t>(n >> 3) << 17;
     d |= 1u << 23;                         // scale factors are UE8M0
-    d |= static_cast<uint32_t>(BM >> 4) << 24;
+    d |= static_cast<uint32_t>(m >> 4) << 24;
     return d;
+}
+
+template <bool FP4, bool BF16_OUT>
+cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
+                        const CUtensorMap &tsb, const PairParams &p, int grid, cudaStream_t st) {
+    auto kern = mx_gemm_pair_kernel<FP4, BF16_OUT>;
+    static bool configured = false;   // per instantiation
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg<FP4>::SMEM);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    kern<<<grid, NUM_THREADS, PairCfg<FP4>::SMEM, st>>>(ta, tb, tsa, tsb, p);
+    return cudaGetLastError();
 }
 
 template <bool FP4, bool BF16_OUT>
@@ -525,8 +838,50 @@ extern "C" int mx_debug_gemm_skip_stage(int k_tile) {
     return MX_OK;
 }
 
+namespace {
+
+// M > 128: the two-SM kernel (256 x 192 tiles over CTA pairs).
+int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
+    using namespace mxg;
+    const bool fp4 = a.fa == MX_E2M1;
+    const int64_t k_bytes = fp4 ? a.K / 2 : a.K;
+    const int G = fp4 ? 2 : 1;
+    const int64_t k_groups = a.K / 128;
+    CUtensorMap ta, tb, tsa, tsb;
+    if (!make_operand_map(&ta, a.a_codes, a.M, k_bytes, 128)) return MX_ERR_CUDA;
+    if (!make_operand_map(&tb, a.b_codes, a.N, k_bytes, PAIR_B_ROWS)) return MX_ERR_CUDA;
+    const int64_t sa_bytes = (a.M + 127) / 128 * 128 * k_groups * 4;
+    const int64_t sb_bytes = (a.N + 127) / 128 * 128 * k_groups * 4;
+    if (!make_scale_map(&tsa, a.a_scales, sa_bytes, G)) return MX_ERR_CUDA;
+    if (!make_scale_map(&tsb, a.b_scales, sb_bytes, G)) return MX_ERR_CUDA;
+    PairParams p;
+    p.c = a.c;
+    p.ldc = a.ldc;
+    p.M = static_cast<int>(a.M);
+    p.N = static_cast<int>(a.N);
+    p.K = static_cast<int>(a.K);
+    p.k_tiles = static_cast<int>(k_bytes / BK_BYTES);
+    p.k_groups = static_cast<int>(k_groups);
+    p.tiles_m = static_cast<int>((a.M + PAIR_BM - 1) / PAIR_BM);
+    p.tiles_n = static_cast<int>((a.N + PAIR_BN - 1) / PAIR_BN);
+    p.alpha = a.alpha;
+    p.idesc = make_idesc(a.fa, a.fb, fp4, PAIR_BM, PAIR_BN);
+    p.skip_k_tile = g_skip_k_tile.exchange(-1);
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int clusters = tiles < a.num_sms / 2 ? tiles : a.num_sms / 2;
+    const int grid = 2 * (clusters < 1 ? 1 : clusters);
+    cudaError_t e;
+    const bool bf = a.cdt == MX_BF16;
+    if (fp4) e = bf ? launch_pair<true, true>(ta, tb, tsa, tsb, p, grid, st) : launch_pair<true, false>(ta, tb, tsa, tsb, p, grid, st);
+    else e = bf ? launch_pair<false, true>(ta, tb, tsa, tsb, p, grid, st) : launch_pair<false, false>(ta, tb, tsa, tsb, p, grid, st);
+    return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+}  // namespace
+
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     using namespace mxg;
+    if (a.M > 128) return launch_gemm_pair(a, st);
     const bool fp4 = a.fa == MX_E2M1;
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;
     CUtensorMap ta, tb;

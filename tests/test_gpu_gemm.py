@@ -89,6 +89,22 @@ def test_gemm_single_tile_bit_exact(oracle, fmt, K):
     assert np.array_equal(got, exact), np.argwhere(got != exact)[:5]
 
 
+@pytest.mark.parametrize("fmt,K", [("e4m3", 256), ("e2m1", 512), ("e5m2", 128)])
+@pytest.mark.parametrize("M,N", [(256, 192), (256, 384), (512, 576)])
+def test_gemm_two_sm_tiles_bit_exact(oracle, fmt, K, M, N):
+    """M > 128 runs on CTA pairs (256 x 192 tiles); N = 384 and 576 include
+    odd 192-column tiles, whose B scales start 64 rows into a scale block."""
+    rng = np.random.default_rng(M + N + K)
+    a = small_int_operand(rng, M, K)
+    b = small_int_operand(rng, N, K)
+    if fmt == "e2m1":
+        a = np.clip(a, -3, 3)
+        b = np.clip(b, -3, 3)
+    got, ref, bound = run_gemm(oracle, a, b, fmt, M, N, K)
+    exact = oracle.round_f32(ref).astype(np.float64)
+    assert np.array_equal(got, exact), np.argwhere(got != exact)[:5]
+
+
 @pytest.mark.parametrize("fmt", ["e4m3", "e5m2", "e2m1"])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_gemm_multi_tile_tolerance(oracle, fmt, out_dtype):
@@ -103,7 +119,7 @@ def test_gemm_multi_tile_tolerance(oracle, fmt, out_dtype):
 @pytest.mark.parametrize("fmt,K", [("e4m3", 384), ("e2m1", 512)])
 def test_gemm_ragged_m_n_and_pitched_c(oracle, fmt, K):
     rng = np.random.default_rng(11)
-    for (M, N) in [(200, 300), (1, 1), (129, 257), (130, 100)]:
+    for (M, N) in [(200, 300), (1, 1), (129, 257), (130, 100), (300, 200), (520, 97)]:
         a = rng.standard_normal((M, K)).astype(np.float32)
         b = rng.standard_normal((N, K)).astype(np.float32)
         for out_dtype in (torch.float32, torch.bfloat16):
