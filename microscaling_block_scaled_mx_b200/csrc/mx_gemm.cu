@@ -457,26 +457,30 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
 }
 
 // ------------------------------------------------------------------------
-// Two-SM kernel (cta_group::2): a cluster of two CTAs computes a 256 x 192
+// Two-SM kernel (cta_group::2): a cluster of two CTAs computes a 256 x 256
 // tile.  CTA r of the pair holds rows [128 r, 128 r + 128) of A and B rows
-// [96 r, 96 r + 96) in its shared memory; one tcgen05.mma.cta_group::2 issued
-// by CTA 0 consumes both halves and writes each CTA's 128 accumulator rows
-// into that CTA's tensor memory.  Every tensor-memory copy and MMA therefore
-// covers twice the work of the one-SM kernel, and each SM loads only half of
-// the B tile.  Each CTA keeps its own A scales and the full B scales (the
-// pair-wide tcgen05.cp copies each CTA's shared memory into its own tensor
-// memory).  All loads of both CTAs complete on CTA 0's stage barrier (the
-// two-SM form of the TMA load); CTA 0's commit frees the stage in both CTAs.
+// [128 r, 128 r + 128) in its shared memory; one tcgen05.mma.cta_group::2
+// issued by CTA 0 consumes both halves and writes each CTA's 128 accumulator
+// rows into that CTA's tensor memory.  Every tensor-memory copy and MMA
+// therefore covers twice the work of the one-SM kernel, and each SM loads only
+// half of the B tile.  Each CTA keeps its own A scales and the full B scales
+// (the pair-wide tcgen05.cp copies each CTA's shared memory into its own
+// tensor memory).  All loads of both CTAs complete on CTA 0's stage barrier
+// (the two-SM form of the TMA load); CTA 0's commit frees the stage in both
+// CTAs.  A 256-column fp32 accumulator leaves no room for a second one next to
+// the scale factors, so the epilogue first drains the accumulator into
+// registers, releases it to the MMA issuer, and only then stores to C.
 // ------------------------------------------------------------------------
 constexpr int PAIR_BM = 256;
-constexpr int PAIR_BN = 192;
+constexpr int PAIR_BN = 256;
 constexpr int PAIR_B_ROWS = PAIR_BN / 2;                 // B rows per CTA
 constexpr int PAIR_A_BYTES = 128 * BK_BYTES;             // 16 KiB per CTA per stage
-constexpr int PAIR_B_BYTES = PAIR_B_ROWS * BK_BYTES;     // 12 KiB per CTA per stage
+constexpr int PAIR_B_BYTES = PAIR_B_ROWS * BK_BYTES;     // 16 KiB per CTA per stage
+constexpr uint32_t PAIR_SF_COL = PAIR_BN;                // scale factors after the accumulator
 
 template <bool FP4> struct PairCfg {
     static constexpr int G = FP4 ? 2 : 1;                // scale atoms along K per stage
-    static constexpr int STAGES = FP4 ? 5 : 6;           // bounded by tensor-memory columns
+    static constexpr int STAGES = 6;
     static constexpr int SFA_BYTES = ATOM * G;
     static constexpr int SFB_BYTES = 2 * ATOM * G;       // both 128-row scale blocks the tile touches
     static constexpr int SFA_COLS = 4 * G;
@@ -489,11 +493,11 @@ template <bool FP4> struct PairCfg {
     static constexpr int OFF_SFA = OFF_B + STAGES * PAIR_B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 5;      // full, empty, acc_full[2], acc_empty[2], drain
+    static constexpr int NUM_BARS = 2 * STAGES + 5;      // full, empty, acc_full, acc_empty, drain (+2 spare)
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
     static constexpr int SMEM = OFF_ABORT + 4 + 1024;    // + alignment slack
-    static_assert(2 * PAIR_BN + STAGES * SF_STAGE_COLS <= 512, "tensor memory columns");
+    static_assert(PAIR_BN + STAGES * SF_STAGE_COLS <= 512, "tensor memory columns");
     static_assert(SMEM <= 232448, "shared memory per block");
 };
 
@@ -654,17 +658,16 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             bool issued = false;
             int local = 0;
             for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters, ++local) {
-                const int b = local & 1;
-                const uint32_t acc_ph = (local >> 1) & 1;
+                const int b = 0;
+                const uint32_t acc_ph = local & 1;
                 if (!wait_bounded(acc_empty(b), acc_ph ^ 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const int tn = tile / p.tiles_m;
-                const uint32_t d_tmem = tmem + b * ACC_COLS;
-                const uint32_t sfb_shift = (tn & 1) ? 2u : 0u;   // odd 192-column tiles
+                const uint32_t d_tmem = tmem;
+                const uint32_t sfb_shift = 0u;
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!wait_bounded(full_bar(s), ph, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t sfa_t = tmem + SF_COL + s * C::SF_STAGE_COLS;
+                    const uint32_t sfa_t = tmem + PAIR_SF_COL + s * C::SF_STAGE_COLS;
                     const uint32_t sfb_t = sfa_t + C::SFA_COLS;
                     const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
@@ -704,9 +707,10 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
         int local = 0;
+        constexpr int NCH = PAIR_BN / 2 / 32;    // 32-column chunks per warp
         for (int tile = cluster_id; tile < num_tiles; tile += n_clusters, ++local) {
-            const int b = local & 1;
-            const uint32_t acc_ph = (local >> 1) & 1;
+            const int b = 0;
+            const uint32_t acc_ph = local & 1;
             int ok = 1;
             if (lane == 0) ok = wait_bounded(acc_full(b), acc_ph, abort_flag) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -715,12 +719,12 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
             const int m = tm * PAIR_BM + 128 * static_cast<int>(rank) + q * 32 + lane;
             const int c0 = half * (PAIR_BN / 2);
-            const uint32_t taddr = tmem + b * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + c0;
-            uint32_t r[96];
-            tmem_ld_x32_nowait(taddr, r);
-            tmem_ld_x32_nowait(taddr + 32, r + 32);
-            tmem_ld_x32_nowait(taddr + 64, r + 64);
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + c0;
+            uint32_t r[32 * NCH];
+#pragma unroll
+            for (int j = 0; j < NCH; ++j) tmem_ld_x32_nowait(taddr + 32 * j, r + 32 * j);
             tmem_wait_ld();
+            // the accumulator is in registers: hand it back to the MMA issuer
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(map_to_rank(acc_empty(b), 0));
@@ -728,7 +732,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             Params pp;
             pp.c = p.c; pp.ldc = p.ldc; pp.M = p.M; pp.N = p.N; pp.alpha = p.alpha;
 #pragma unroll
-            for (int j = 0; j < 3; ++j) store_row_chunk<BF16_OUT>(pp, m, n_base + 32 * j, r + 32 * j);
+            for (int j = 0; j < NCH; ++j) store_row_chunk<BF16_OUT>(pp, m, n_base + 32 * j, r + 32 * j);
         }
     }
 
