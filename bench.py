@@ -303,6 +303,9 @@ def run_mx(args):
         launches_gemm = gemm.pop("_launches")
     else:
         launches_gemm = 0
+    gemm8 = run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world, fmt="e4m3")
+    if gemm8 is not None:
+        launches_gemm += gemm8.pop("_launches")
     wgrad = None if args.no_wgrad else run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier,
                                                         max_over_ranks, world)
 
@@ -331,6 +334,8 @@ def run_mx(args):
                 "clocks": clocks.summary()}
         if gemm is not None:
             line["gemm"] = gemm
+        if gemm8 is not None:
+            line["gemm_fp8"] = gemm8
         if wgrad is not None:
             line["wgrad"] = wgrad
         print(json.dumps(line), flush=True)
@@ -339,29 +344,32 @@ def run_mx(args):
     return 0
 
 
-def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world):
-    """Llama-3-8B-shaped MXFP4 GEMMs on operands cast in advance; None if the
-    GEMM is not available in this build."""
+def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world, fmt="e2m1"):
+    """Block-scaled GEMMs on operands cast in advance: the Llama-3-8B-shaped
+    MXFP4 set (fmt e2m1) or the GPT-2-small-shaped MXFP8 set (fmt e4m3); None
+    if the GEMM is not available in this build."""
     import torch
     from microscaling_block_scaled_mx_b200 import inputs as I
     from microscaling_block_scaled_mx_b200 import mx
     if args.no_gemm:
         return None
+    shapes = I.LLAMA3_GEMMS if fmt == "e2m1" else I.GPT2_GEMMS
+    cfg_index = 3 if fmt == "e2m1" else 2
     ops = []
-    for idx, (M, N, K) in enumerate(I.LLAMA3_GEMMS):
-        if str(idx) not in args.gemm_shapes.split(","):
+    for idx, (M, N, K) in enumerate(shapes):
+        if fmt == "e2m1" and str(idx) not in args.gemm_shapes.split(","):
             continue
-        xb, wb = I.linear_operands(M, K, N, 3, stream=idx)
+        xb, wb = I.linear_operands(M, K, N, cfg_index, stream=idx)
         x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
         w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
-        ac, as_ = mx.quantize(x, 1, "e2m1")
-        bc, bs = mx.quantize(w, 1, "e2m1")
+        ac, as_ = mx.quantize(x, 1, fmt)
+        bc, bs = mx.quantize(w, 1, fmt)
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ops.append((M, N, K, ac, as_, bc, bs, c))
         del x, w
     try:
         M, N, K, ac, as_, bc, bs, c = ops[0]
-        mx.gemm(ac, as_, bc, bs, M, N, K, fa="e2m1", out=c)
+        mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
     except mx.MxError as e:
         if e.status == -4:
             return None
@@ -369,7 +377,7 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
     flops_step = sum(2.0 * M * N * K for (M, N, K, *_r) in ops)
     for _ in range(args.warmup):
         for (M, N, K, ac, as_, bc, bs, c) in ops:
-            mx.gemm(ac, as_, bc, bs, M, N, K, fa="e2m1", out=c)
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
     torch.cuda.synchronize()
     barrier()
     evs = []
@@ -380,7 +388,7 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         for (M, N, K, ac, as_, bc, bs, c) in ops:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            mx.gemm(ac, as_, bc, bs, M, N, K, fa="e2m1", out=c)
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
             e1.record(stream)
             evs.append(((M, N, K), e0, e1))
             launches += 1
@@ -396,14 +404,20 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
                                      "tflops": round(2.0 * M * N * K / (statistics.mean(d) * 1e-3) / 1e12, 1)}
     kern_ms = sum(a.elapsed_time(b) for (_, a, b) in evs)
     achieved = flops_step * args.steps / (kern_ms * 1e-3) / 1e12
-    fp4_peak = 4.0 * float(peaks["bf16_tflops"])      # nominal fp4 : bf16 = 9 : 2.25
+    ratio = 4.0 if fmt == "e2m1" else 2.0             # nominal fp4 : fp8 : bf16 = 9 : 4.5 : 2.25
+    peak = ratio * float(peaks["bf16_tflops"])
+    if fmt == "e2m1":
+        workload = "llama3_8b_mxfp4_gemms_m8192 (4096->6144, 4096->14336, 14336->4096), bf16 out"
+        kernel = "mx_gemm_pair_kernel (cta_group::2, kind::mxf4)"
+    else:
+        workload = "gpt2_small_mxfp8_gemms_m8192 (768->3072, 3072->768), bf16 out"
+        kernel = "mx_gemm_pair_kernel (cta_group::2, kind::mxf8f6f4)"
     return {"metric": "MX GEMM TFLOP/s", "value": round(value, 1), "unit": "TFLOP/s",
-            "workload": "llama3_8b_mxfp4_gemms_m8192 (4096->6144, 4096->14336, 14336->4096), bf16 out",
-            "ms_per_step": round(ms / args.steps, 4),
-            "roofline": {"bound": "tensor", "kernel": "mx_gemm_kernel (kind::mxf4)",
-                         "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                         "frac": round(achieved / fp4_peak, 4),
-                         "peak_kind": f"{peak_kind} bf16 burst x 4 (nominal MXFP4:bf16 ratio)",
+            "workload": workload, "ms_per_step": round(ms / args.steps, 4),
+            "roofline": {"bound": "tensor", "kernel": kernel,
+                         "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4),
+                         "peak_kind": f"{peak_kind} bf16 burst x {ratio:g} (nominal ratio for the operand type)",
                          "traffic": None, "per_shape": per_shape},
             "_launches": launches}
 

@@ -145,6 +145,32 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
 
     // V * 2^-e with the subnormal flush (mul.ftz), two values per instruction
     float u[32];
+    if (FMT == MX_INT8 && !SR && e >= -120 && e <= 120) {
+        // INT8 codes are round(V * 2^(6 - e)) clamped to +-127: fold the 2^6 into
+        // the (exact) power-of-two scale, clamp, round half to even
+        const uint32_t f = __float_as_uint(pow2f(6 - e));
+        const uint64_t ff = static_cast<uint64_t>(f) | (static_cast<uint64_t>(f) << 32);
+        uint32_t c[8];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const uint64_t r = f2_mul_ftz(static_cast<uint64_t>(b[i]) | (static_cast<uint64_t>(b[i + 1]) << 32), ff);
+            const float x0 = fminf(fmaxf(__uint_as_float(static_cast<uint32_t>(r)), -127.0f), 127.0f);
+            const float x1 = fminf(fmaxf(__uint_as_float(static_cast<uint32_t>(r >> 32)), -127.0f), 127.0f);
+            const uint32_t q0 = static_cast<uint32_t>(__float2int_rn(x0)) & 0xffu;
+            const uint32_t q1 = static_cast<uint32_t>(__float2int_rn(x1)) & 0xffu;
+            if ((i & 2) == 0) c[i >> 2] = q0 | (q1 << 8);
+            else c[i >> 2] |= (q0 << 16) | (q1 << 24);
+        }
+        if (nan_block) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) c[i] = 0u;
+        }
+        uint4 *d = reinterpret_cast<uint4 *>(p.codes + cp.row * p.cols + kb * 32);
+        d[0] = make_uint4(c[0], c[1], c[2], c[3]);
+        d[1] = make_uint4(c[4], c[5], c[6], c[7]);
+        store_scale(p, cp.row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+        return;
+    }
     if (Fmt<FMT>::emax == 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) u[i] = scale_down<FMT>(__uint_as_float(b[i]), e);
@@ -218,19 +244,25 @@ __global__ void __launch_bounds__(256, 2) cast_rows_kernel(CastParams p) {
         q.row += step_rows;
         if (q.chunk >= cpr) { q.chunk -= cpr; ++q.row; }
     };
+    // two chunks in flight while a third is converted
     ChunkPos cur;
     cur.row = warp0 / cpr;
     cur.chunk = warp0 - cur.row * cpr;
-    BlockLoad<BF16_IN> cur_ld;
+    ChunkPos nx1 = cur;
+    advance(nx1);
+    BlockLoad<BF16_IN> cur_ld, nx1_ld;
     load_block<BF16_IN, V32>(p, cur, blocks_per_row, lane, cur_ld);
+    load_block<BF16_IN, V32>(p, nx1, blocks_per_row, lane, nx1_ld);
     while (cur.row < p.rows) {
-        ChunkPos nxt = cur;
-        advance(nxt);
-        BlockLoad<BF16_IN> nxt_ld;
-        load_block<BF16_IN, V32>(p, nxt, blocks_per_row, lane, nxt_ld);
+        ChunkPos nx2 = nx1;
+        advance(nx2);
+        BlockLoad<BF16_IN> nx2_ld;
+        load_block<BF16_IN, V32>(p, nx2, blocks_per_row, lane, nx2_ld);
         cast_block<FMT, SR, BF16_IN>(p, cur, blocks_per_row, cur_ld, lane);
-        cur = nxt;
-        cur_ld = nxt_ld;
+        cur = nx1;
+        cur_ld = nx1_ld;
+        nx1 = nx2;
+        nx1_ld = nx2_ld;
     }
 }
 

@@ -883,9 +883,20 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
 
 }  // namespace
 
+// Kernel choice.  CTA pairs on 256 x 256 tiles have the higher steady-state
+// rate (each MMA and scale copy covers two SMs, each SM loads half of B), but
+// a shape with few such tiles or few K steps per tile is dominated by wave
+// quantisation and per-tile start-up, where the one-SM kernel's smaller tiles
+// and overlapped epilogue win (measured on the GPT-2-shaped GEMMs).
+bool use_pair_kernel(const MxGemmArgs &a) {
+    if (a.M <= 128 || a.K < 2048) return false;
+    const int64_t pair_tiles = ((a.M + 255) / 256) * ((a.N + 255) / 256);
+    return pair_tiles >= a.num_sms;
+}
+
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     using namespace mxg;
-    if (a.M > 128) return launch_gemm_pair(a, st);
+    if (use_pair_kernel(a)) return launch_gemm_pair(a, st);
     const bool fp4 = a.fa == MX_E2M1;
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;
     CUtensorMap ta, tb;

@@ -91,9 +91,10 @@ def test_gemm_single_tile_bit_exact(oracle, fmt, K):
 
 @pytest.mark.parametrize("fmt,K", [("e4m3", 256), ("e2m1", 512), ("e5m2", 128)])
 @pytest.mark.parametrize("M,N", [(256, 192), (256, 384), (512, 576)])
-def test_gemm_two_sm_tiles_bit_exact(oracle, fmt, K, M, N):
-    """M > 128 runs on CTA pairs (256 x 192 tiles); N = 384 and 576 include
-    odd 192-column tiles, whose B scales start 64 rows into a scale block."""
+def test_gemm_one_sm_multi_tile_bit_exact(oracle, fmt, K, M, N):
+    """Short-K shapes run on the one-SM kernel (128 x 192 tiles); N = 384 and
+    576 include odd 192-column tiles, whose B scales start 64 rows into a
+    scale block."""
     rng = np.random.default_rng(M + N + K)
     a = small_int_operand(rng, M, K)
     b = small_int_operand(rng, N, K)
@@ -103,6 +104,24 @@ def test_gemm_two_sm_tiles_bit_exact(oracle, fmt, K, M, N):
     got, ref, bound = run_gemm(oracle, a, b, fmt, M, N, K)
     exact = oracle.round_f32(ref).astype(np.float64)
     assert np.array_equal(got, exact), np.argwhere(got != exact)[:5]
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e2m1"])
+def test_gemm_two_sm_tiles_bit_exact(oracle, fmt):
+    """K >= 2048 with at least one 256 x 256 tile per SM runs on CTA pairs
+    (cta_group::2); ragged M and N exercise the clamped loads of a pair half
+    that lies wholly past the edge."""
+    K = 2048 if fmt == "e4m3" else 4096
+    for (M, N) in [(4096, 2560), (4000, 2600)]:
+        rng = np.random.default_rng(M + N)
+        a = small_int_operand(rng, M, K)
+        b = small_int_operand(rng, N, K)
+        if fmt == "e2m1":
+            a = np.clip(a, -3, 3)
+            b = np.clip(b, -3, 3)
+        got, ref, bound = run_gemm(oracle, a, b, fmt, M, N, K)
+        exact = oracle.round_f32(ref).astype(np.float64)
+        assert np.array_equal(got, exact), (M, N, np.argwhere(got != exact)[:5])
 
 
 @pytest.mark.parametrize("fmt", ["e4m3", "e5m2", "e2m1"])
@@ -216,19 +235,22 @@ def test_gemm_wgrad_config(oracle):
     check(to_f64(dw)[rows], ref, bound, torch.float32, "wgrad")
 
 
-def test_gemm_bounded_wait_reports_timeout():
+@pytest.mark.parametrize("M,N,K", [(256, 256, 1024), (4096, 2560, 2048)])
+def test_gemm_bounded_wait_reports_timeout(M, N, K):
     """A stage that is never filled: the MMA issuer's bounded wait runs out, the
-    kernel records MX_ERR_TIMEOUT and returns; the context stays usable."""
+    kernel records MX_ERR_TIMEOUT and returns; the context stays usable.  The
+    first shape runs on the one-SM kernel, the second on CTA pairs."""
     rng = np.random.default_rng(1)
-    M, N, K = 256, 256, 1024
     a = to_device(rng.standard_normal((M, K)).astype(np.float32))
+    b = to_device(rng.standard_normal((N, K)).astype(np.float32))
     ac, as_ = mx.quantize(a, 1, "e4m3")
+    bc, bs = mx.quantize(b, 1, "e4m3")
     assert mx.last_device_status() == 0
     mx.lib().mx_debug_gemm_skip_stage(3)
-    mx.gemm(ac, as_, ac, as_, M, N, K, fa="e4m3", out_dtype=torch.float32)
+    mx.gemm(ac, as_, bc, bs, M, N, K, fa="e4m3", out_dtype=torch.float32)
     assert mx.last_device_status() == -7
     assert mx.last_device_status() == 0          # read-and-clear
-    c = mx.gemm(ac, as_, ac, as_, M, N, K, fa="e4m3", out_dtype=torch.float32)
+    c = mx.gemm(ac, as_, bc, bs, M, N, K, fa="e4m3", out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert mx.last_device_status() == 0
     assert torch.isfinite(c).all()
