@@ -112,7 +112,21 @@ __device__ __forceinline__ uint64_t f2_mul_ftz(uint64_t a, uint64_t b) {
     return r;
 }
 
-template <int FMT, bool SR, bool BF16_IN>
+// 32 code bytes of one block: one 32-byte store when the buffers are 32-byte
+// aligned (V32), else two 16-byte stores
+template <bool V32>
+__device__ __forceinline__ void store_code32(uint8_t *dst, const uint4 &a, const uint4 &b) {
+    if (V32) {
+        asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                     ::"l"(dst), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                     : "memory");
+    } else {
+        reinterpret_cast<uint4 *>(dst)[0] = a;
+        reinterpret_cast<uint4 *>(dst)[1] = b;
+    }
+}
+
+template <int FMT, bool SR, bool BF16_IN, bool V32>
 __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &cp, int64_t blocks_per_row,
                                            const BlockLoad<BF16_IN> &o, int lane) {
     constexpr int BITS = Fmt<FMT>::bits;
@@ -165,9 +179,8 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
 #pragma unroll
             for (int i = 0; i < 8; ++i) c[i] = 0u;
         }
-        uint4 *d = reinterpret_cast<uint4 *>(p.codes + cp.row * p.cols + kb * 32);
-        d[0] = make_uint4(c[0], c[1], c[2], c[3]);
-        d[1] = make_uint4(c[4], c[5], c[6], c[7]);
+        store_code32<V32>(p.codes + cp.row * p.cols + kb * 32, make_uint4(c[0], c[1], c[2], c[3]),
+                          make_uint4(c[4], c[5], c[6], c[7]));
         store_scale(p, cp.row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
         return;
     }
@@ -205,9 +218,10 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
     }
     uint8_t *dst = p.codes + cp.row * (p.cols * BITS / 8) + kb * (32 * BITS / 8);
     if (BITS == 8) {
-        uint4 *d = reinterpret_cast<uint4 *>(dst);
-        d[0] = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
-        d[1] = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16), c[14] | (c[15] << 16));
+        const uint4 lo = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+        const uint4 hi = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16),
+                                    c[14] | (c[15] << 16));
+        store_code32<V32>(dst, lo, hi);
     } else if (BITS == 4) {
         uint32_t w[4];
 #pragma unroll
@@ -258,7 +272,7 @@ __global__ void __launch_bounds__(256, 2) cast_rows_kernel(CastParams p) {
         advance(nx2);
         BlockLoad<BF16_IN> nx2_ld;
         load_block<BF16_IN, V32>(p, nx2, blocks_per_row, lane, nx2_ld);
-        cast_block<FMT, SR, BF16_IN>(p, cur, blocks_per_row, cur_ld, lane);
+        cast_block<FMT, SR, BF16_IN, V32>(p, cur, blocks_per_row, cur_ld, lane);
         cur = nx1;
         cur_ld = nx1_ld;
         nx1 = nx2;
@@ -383,21 +397,36 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
                 }
             }
             const bool has_second = gc + 1 < C;
+            // block amax and exponent of both columns
+            uint32_t am0 = 0, am1 = 0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                am0 = __vimax3_u32(am0, static_cast<uint32_t>(x[j]) & 0x7fffffffu,
+                                   static_cast<uint32_t>(x[j + 1]) & 0x7fffffffu);
+                am1 = __vimax3_u32(am1, static_cast<uint32_t>(x[j] >> 32) & 0x7fffffffu,
+                                   static_cast<uint32_t>(x[j + 1] >> 32) & 0x7fffffffu);
+            }
+            const int e0 = block_exponent<FMT>(am0), e1 = block_exponent<FMT>(am1);
+            // V * 2^-e for both columns with one packed multiply (flushing
+            // FP32 subnormals); INT8's e = 127 case takes the two-step path
+            const bool packed = Fmt<FMT>::emax != 0 || (e0 <= 126 && e1 <= 126);
+            if (packed) {
+                const uint64_t ff = f2_pack(pow2f(-e0), pow2f(-e1));
+#pragma unroll
+                for (int j = 0; j < 32; ++j) x[j] = f2_mul_ftz(x[j], ff);
+            }
 #pragma unroll
             for (int col = 0; col < 2; ++col) {
                 if (col == 1 && !has_second) break;
+                const uint32_t amax_bits = col ? am1 : am0;
+                const int e = col ? e1 : e0;
+                const bool nan_block = amax_bits >= 0x7f800000u;
                 float v[32];
-                uint32_t amax_bits = 0;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const uint32_t b = static_cast<uint32_t>(x[j] >> (32 * col));
-                    v[j] = __uint_as_float(b);
-                    amax_bits = max(amax_bits, b & 0x7fffffffu);
+                    v[j] = __uint_as_float(static_cast<uint32_t>(x[j] >> (32 * col)));
+                    if (!packed) v[j] = scale_down<FMT>(v[j], e);
                 }
-                const bool nan_block = amax_bits >= 0x7f800000u;
-                const int e = block_exponent<FMT>(amax_bits);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = scale_down<FMT>(v[j], e);
                 const int64_t oc = gc + col;                 // output row
                 uint32_t c[16];
                 if (SR) {
@@ -604,7 +633,10 @@ static cudaError_t launch_cast_fmt(const CastParams &p, int xdt, int block_axis,
     const bool bf = xdt == MX_BF16;
     if (block_axis == 1) {
         const int64_t chunks = p.rows * (((p.cols >> 5) + 31) >> 5);    // 32-block chunks, one per warp
-        const bool v32 = (reinterpret_cast<uintptr_t>(p.x) & 31u) == 0 && ((p.ldx * (bf ? 2 : 4)) & 31) == 0;
+        // 32-byte accesses need 32-byte aligned input rows and code rows (a code
+        // row is cols * bits / 8 bytes, a multiple of 32 for 8-bit formats)
+        const bool v32 = (reinterpret_cast<uintptr_t>(p.x) & 31u) == 0 && ((p.ldx * (bf ? 2 : 4)) & 31) == 0 &&
+                         (reinterpret_cast<uintptr_t>(p.codes) & 31u) == 0;
         if (bf) {
             if (v32) {
                 constexpr auto k = cast_rows_kernel<FMT, SR, true, true>;

@@ -133,7 +133,8 @@ __device__ __forceinline__ float sr_magnitude(float a, uint32_t r) {
 // lo or lo + step.  For a < 2^emin (the element's subnormal range, uniform
 // step 2^(emin - mbits)) a is first shifted to a + 2^emin with a
 // round-toward-zero add, which keeps every bit that F depends on, rounded
-// the same way, and shifted back exactly.  Returns the rounded magnitude.
+// the same way, and shifted back exactly.  Returns the rounded magnitude
+// (callers convert it with a saturating conversion).
 template <int FMT>
 __device__ __forceinline__ float sr_magnitude_int(float a, uint32_t r) {
     using F = Fmt<FMT>;
@@ -142,7 +143,9 @@ __device__ __forceinline__ float sr_magnitude_int(float a, uint32_t r) {
     constexpr int UNIT = 23 - F::mbits;
     uint32_t wb = __float_as_uint(w) + (r << (UNIT - 8));
     wb &= ~((1u << UNIT) - 1u);
-    return fminf(__fsub_rn(__uint_as_float(wb), t), F::maxv);
+    // may exceed max by one grid step when |a| >= max: the saturating
+    // conversions that follow clamp it to max, which is the rule for |a| >= max
+    return __fsub_rn(__uint_as_float(wb), t);
 }
 
 // MurmurHash3 32-bit finaliser (public domain, A. Appleby).
