@@ -21,6 +21,7 @@ sample of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -39,6 +40,42 @@ BITS = {"e4m3": 8, "e5m2": 8, "e2m3": 6, "e3m2": 6, "e2m1": 4, "int8": 8}
 ROWS = COLS = 8192
 N_ROTATE = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+# the roofline kernels, from one ncu capture of this benchmark's own launches
+# (summaries in profiles/dram_traffic_bench.md).  Each entry holds the kernel
+# sources, the sha256 of their contents at capture time and bytes per launch
+# by workload.  A figure is reported only while the sources still hash to that
+# value; after any change to them it reads null until captured again.
+_CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
+MEASURED_TRAFFIC = {
+    "cast_rows": (("mx_cast.cu", "mx_device.cuh"),
+                  "2945c1c69bfdd1d635ce3c858285c2e7ce575a4cf32893e82efaa70c3b62b1ee",
+                  {"e4m3_bf16_8192x8192": 173593856, "e5m2_bf16_8192x8192": 169520640,
+                   "e2m3_bf16_8192x8192": 158908160, "e3m2_bf16_8192x8192": 158370304,
+                   "e2m1_bf16_8192x8192": 148999168, "int8_bf16_8192x8192": 168584448}),
+    "gemm": (("mx_gemm.cu",),
+             "a1e2301352c6b982eeed9652400e2fd06a30fb8561f62a85ebfd3c3cd250c045",
+             {"e2m1_8192x6144x4096": 80179456, "e2m1_8192x14336x4096": 227883264,
+              "e2m1_8192x4096x14336": 302555392, "e4m3_8192x3072x768": 9484800,
+              "e4m3_8192x768x3072": 28418560}),
+}
+
+
+def sources_sha256(names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(_CSRC, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel: str, workload: str):
+    names, sha, table = MEASURED_TRAFFIC[kernel]
+    if sha is None or workload not in table or sources_sha256(names) != sha:
+        return None
+    return table[workload]
 
 
 def cast_alg_bytes(fmt: str, rows: int = ROWS, cols: int = COLS, in_bytes: int = 2) -> int:
@@ -261,25 +298,59 @@ def run_mx(args):
     all_durs_ms = sum(a.elapsed_time(b) for (_, a, b) in events)
     achieved = alg_bytes_step * args.steps / (all_durs_ms * 1e-3) / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
+    traffic = None
+    t_fmt = {f: measured_traffic("cast_rows", f"{f}_bf16_{ROWS}x{COLS}") for f in FMTS}
+    if all(v is not None for v in t_fmt.values()):
+        traffic = round(statistics.mean(t_fmt.values()))
+        for f in FMTS:
+            per_fmt[f]["traffic"] = t_fmt[f]
+            per_fmt[f]["alg_bytes"] = cast_alg_bytes(f)
     roofline = {"bound": "hbm", "kernel": "cast_rows_kernel (six format instantiations)",
                 "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "peak_kind": f"{peak_kind} copy bandwidth (burst)",
-                "traffic": None, "per_format": per_fmt}
+                "traffic": traffic, "alg_bytes_per_launch": round(alg_bytes_step / len(FMTS)),
+                "per_format": per_fmt}
 
     # ---- end to end through the C ABI with host buffers ----
+    # The tensor streams through in row chunks on three streams: the host->device
+    # copy of chunk i+1 and the device->host copy of chunk i-1 overlap the six
+    # casts of chunk i (the two copy directions use separate engines).  Codes
+    # and scales land in pinned host buffers; plain scale layout, so each
+    # chunk's scales are one contiguous slice.
     pinned = host.pin_memory()
-    host_out = {f: (torch.empty(outs[f][0][0].shape, dtype=torch.uint8).pin_memory(),
-                    torch.empty(outs[f][0][1].shape, dtype=torch.uint8).pin_memory()) for f in FMTS}
+    E2E_CHUNKS = 8
+    rows_c = ROWS // E2E_CHUNKS
+    host_out = {f: (torch.empty((ROWS, mx.codes_row_bytes(f, COLS)), dtype=torch.uint8).pin_memory(),
+                    torch.empty(mx.scales_bytes("plain", ROWS, COLS), dtype=torch.uint8).pin_memory())
+                for f in FMTS}
+    dev_sc = {f: torch.empty(mx.scales_bytes("plain", ROWS, COLS), dtype=torch.uint8, device=dev) for f in FMTS}
     d2h = sum(host_out[f][0].numel() + host_out[f][1].numel() for f in FMTS)
     h2d = pinned.numel() * 2
+    s_in, s_cast, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_step():
-        xs[0].copy_(pinned, non_blocking=True)
-        for f in FMTS:
-            c, s = outs[f][0]
-            mx.quantize(xs[0], 1, f, codes=c, scales=s, scale_layout="mma")
-            host_out[f][0].copy_(c, non_blocking=True)
-            host_out[f][1].copy_(s, non_blocking=True)
+        s_in.wait_stream(stream)      # each step starts after the previous one ended
+        for i in range(E2E_CHUNKS):
+            r0, r1 = i * rows_c, (i + 1) * rows_c
+            with torch.cuda.stream(s_in):
+                xs[0][r0:r1].copy_(pinned[r0:r1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(s_in)
+            with torch.cuda.stream(s_cast):
+                s_cast.wait_event(ev)
+                for f in FMTS:
+                    c = outs[f][0][0][r0:r1]
+                    sc = dev_sc[f][r0 * (COLS // 32):r1 * (COLS // 32)]
+                    mx.quantize(xs[0][r0:r1], 1, f, codes=c, scales=sc, scale_layout="plain", stream=s_cast)
+                evc = torch.cuda.Event()
+                evc.record(s_cast)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(evc)
+                for f in FMTS:
+                    host_out[f][0][r0:r1].copy_(outs[f][0][0][r0:r1], non_blocking=True)
+                    a, b = r0 * (COLS // 32), r1 * (COLS // 32)
+                    host_out[f][1][a:b].copy_(dev_sc[f][a:b], non_blocking=True)
+        stream.wait_stream(s_out)
 
     e2e_steps = min(args.steps, 50)
     e2e_val = None
@@ -329,7 +400,8 @@ def run_mx(args):
                 "e2e": None if e2e_val is None else
                        {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                        "path": "pinned host bf16 -> H2D -> mx_quantize (6 formats) -> D2H codes+scales"},
+                        "path": "pinned host bf16 -> H2D -> mx_quantize (6 formats) -> D2H codes+scales, "
+                                "8 row chunks pipelined over 3 streams"},
                 "gpu_launches": launches + launches_gemm,
                 "clocks": clocks.summary()}
         if gemm is not None:
@@ -402,6 +474,12 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         d = [a.elapsed_time(b) for (s, a, b) in evs if s == (M, N, K)]
         per_shape[f"{M}x{N}x{K}"] = {"us": round(1e3 * statistics.mean(d), 1),
                                      "tflops": round(2.0 * M * N * K / (statistics.mean(d) * 1e-3) / 1e12, 1)}
+    traffic = None
+    t_shape = {k: measured_traffic("gemm", f"{fmt}_{k}") for k in per_shape}
+    if all(v is not None for v in t_shape.values()):
+        traffic = round(statistics.mean(t_shape.values()))
+        for k in per_shape:
+            per_shape[k]["traffic"] = t_shape[k]
     kern_ms = sum(a.elapsed_time(b) for (_, a, b) in evs)
     achieved = flops_step * args.steps / (kern_ms * 1e-3) / 1e12
     ratio = 4.0 if fmt == "e2m1" else 2.0             # nominal fp4 : fp8 : bf16 = 9 : 4.5 : 2.25
@@ -411,14 +489,14 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         kernel = "mx_gemm_pair_kernel (cta_group::2, kind::mxf4)"
     else:
         workload = "gpt2_small_mxfp8_gemms_m8192 (768->3072, 3072->768), bf16 out"
-        kernel = "mx_gemm_pair_kernel (cta_group::2, kind::mxf8f6f4)"
+        kernel = "mx_gemm_kernel (cta_group::1, kind::mxf8f6f4; short K / few tiles)"
     return {"metric": "MX GEMM TFLOP/s", "value": round(value, 1), "unit": "TFLOP/s",
             "workload": workload, "ms_per_step": round(ms / args.steps, 4),
             "roofline": {"bound": "tensor", "kernel": kernel,
                          "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peak_kind} bf16 burst x {ratio:g} (nominal ratio for the operand type)",
-                         "traffic": None, "per_shape": per_shape},
+                         "traffic": traffic, "per_shape": per_shape},
             "_launches": launches}
 
 
