@@ -379,6 +379,9 @@ def run_mx(args):
         launches_gemm += gemm8.pop("_launches")
     wgrad = None if args.no_wgrad else run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier,
                                                         max_over_ranks, world)
+    dual = None if args.no_dual else run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world)
+    if dual is not None:
+        launches_gemm += dual.pop("_launches")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -410,6 +413,8 @@ def run_mx(args):
             line["gemm_fp8"] = gemm8
         if wgrad is not None:
             line["wgrad"] = wgrad
+        if dual is not None:
+            line["dual_cast"] = dual
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -565,6 +570,75 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
     return out
 
 
+def run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world):
+    """Dual cast of the weight-gradient operands (dY 16384x4096, X 16384x14336,
+    bf16): E2M1 codes along rows (RNE, for the forward and data-gradient GEMMs)
+    and along tokens (Hadamard + SR, for the weight-gradient GEMM) from one
+    read, timed against the two single-axis casts that produce the same bytes."""
+    import torch
+    from microscaling_block_scaled_mx_b200 import inputs as I
+    from microscaling_block_scaled_mx_b200 import mx
+    dyb, xb = I.wgrad_operands()
+    ops = []
+    for name, bits in (("dY", dyb), ("X", xb)):
+        t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        R, C = t.shape
+        out = mx.quantize_dual(t, "e2m1", rnd_rows="rne", rnd_cols="sr", seed_cols=42, hadamard=True)
+        ops.append((name, t, out))
+    del dyb, xb
+    launches = 0
+
+    def dual(record, evs):
+        nonlocal launches
+        for name, t, out in ops:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mx.quantize_dual(t, "e2m1", rnd_rows="rne", rnd_cols="sr", seed_cols=42, hadamard=True, out=out)
+            e1.record(stream)
+            if record:
+                evs.setdefault(name, []).append((e0, e1))
+                launches += 1
+
+    def single(record, evs):
+        nonlocal launches
+        for name, t, out in ops:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mx.quantize(t, 1, "e2m1", codes=out[0], scales=out[1])
+            mx.quantize(t, 0, "e2m1", rnd="sr", seed=42, hadamard=True, codes=out[2], scales=out[3])
+            e1.record(stream)
+            if record:
+                evs.setdefault(name, []).append((e0, e1))
+                launches += 2
+
+    steps = max(3, min(args.steps, 20))
+    res = {}
+    for label, fn in (("dual", dual), ("two_casts", single)):
+        for _ in range(args.warmup):
+            fn(False, {})
+        torch.cuda.synchronize()
+        barrier()
+        evs = {}
+        for _ in range(steps):
+            fn(True, evs)
+        torch.cuda.synchronize()
+        barrier()
+        res[label] = {k: max_over_ranks(1e3 * statistics.mean(a.elapsed_time(b) for a, b in v))
+                      for k, v in evs.items()}
+    hbm = float(peaks["hbm_gbs"])
+    out = {"workload": "dual_cast_e2m1 dY 16384x4096, X 16384x14336 bf16: rows RNE + tokens Hadamard+SR",
+           "steps": steps}
+    for name, t, _ in ops:
+        n = t.numel()
+        alg = n * 2 + 2 * (n // 2 + n // 32)        # one read, two sets of codes and scales
+        d, s2 = res["dual"][name], res["two_casts"][name]
+        out[name] = {"dual_us": round(d, 1), "two_casts_us": round(s2, 1), "speedup": round(s2 / d, 3),
+                     "dual_gbs": round(alg / (d * 1e-6) / 1e9, 1),
+                     "frac_hbm": round(alg / (d * 1e-6) / 1e9 / hbm, 4)}
+    out["_launches"] = launches
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -576,6 +650,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phase")
     ap.add_argument("--no-cast", action="store_true", help="GEMM phase only (profiling)")
     ap.add_argument("--no-wgrad", action="store_true", help="skip the weight-gradient phase")
+    ap.add_argument("--no-dual", action="store_true", help="skip the dual-cast phase")
     ap.add_argument("--fmts", default=",".join(FMTS), help="comma-separated cast formats (profiling)")
     ap.add_argument("--gemm-shapes", default="0,1,2", help="indices of the Llama-3 GEMM shapes to time")
     args = ap.parse_args()

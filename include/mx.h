@@ -152,6 +152,34 @@ MX_API int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, 
                 void *stream);
 
 /*
+ * mx_quantize_dual -- both quantizations of one rows x cols tensor from a
+ * single read of it: the codes and scales of mx_quantize along rows
+ * (block_axis 1, for a GEMM contracting over cols) and of mx_quantize along
+ * columns (block_axis 0, transposed output, for a GEMM contracting over rows).
+ * The MX summary page's section 3 observes that these two quantizations of a
+ * tensor differ, and a training step needs both (forward and weight
+ * gradient); the FP4-pretraining abstract's fused producers motivate reading
+ * the tensor once.
+ *
+ *  x, xdt, rows, cols, ldx, fmt, sl   as for mx_quantize; rows and cols must
+ *           both be multiples of 32 (MX_ERR_SHAPE otherwise).
+ *  rnd_rows, seed_rows   rounding of the along-rows output.
+ *  rnd_cols, seed_cols, pre_cols   rounding and the optional fixed-sign
+ *           Hadamard of the along-columns output (pre_cols may be NULL).
+ *  codes_rows  device, rows x (cols * bits / 8) bytes, 16-byte aligned.
+ *  scales_rows device, mx_scales_bytes(sl, rows, cols) bytes.
+ *  codes_cols  device, cols x (rows * bits / 8) bytes, 16-byte aligned.
+ *  scales_cols device, mx_scales_bytes(sl, cols, rows) bytes.
+ * Each output is bit-identical to the corresponding mx_quantize call with the
+ * same arguments.  All four buffers are owned by the caller and must not
+ * overlap x or each other.  Errors as for mx_quantize.
+ */
+MX_API int mx_quantize_dual(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, mx_fmt fmt,
+                            mx_round rnd_rows, uint64_t seed_rows, mx_round rnd_cols, uint64_t seed_cols,
+                            const mx_precond *pre_cols, void *codes_rows, void *scales_rows,
+                            void *codes_cols, void *scales_cols, mx_scale_layout sl, void *stream);
+
+/*
  * mx_dequantize -- v = X * P (section 2), exact, rounded once to ydt.
  *
  *  codes, scales  device, as written by mx_quantize for (outer, inner).
@@ -170,7 +198,8 @@ MX_API int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_s
  * compute flow on the fifth-generation tensor cores.
  *
  *  a_codes  device, M x K codes of format fa, quantized along K
- *           (block_axis 1 of an M x K tensor), 16-byte aligned.
+ *           (block_axis 1 of an M x K tensor), 16-byte aligned; 32-byte
+ *           aligned when fa is FP6, or FP4 outside the kind::mxf4 case.
  *  a_scales device, MX_SCALES_MMA layout for (M, K).
  *  b_codes  device, N x K codes of format fb, quantized along K.
  *  b_scales device, MX_SCALES_MMA layout for (N, K).
@@ -178,8 +207,14 @@ MX_API int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_s
  *           rounded to nearest even from the fp32 accumulator).
  *  workspace / ws_bytes  reserved; pass NULL / 0 (mx_gemm_workspace_bytes
  *           returns 0 in this build).
- * Supported: fa == fb in {MX_E4M3, MX_E5M2} (kind::mxf8f6f4, K % 128 == 0)
- * and fa == fb == MX_E2M1 (kind::mxf4, K % 256 == 0); any M, N >= 1.
+ *  b_codes has the same alignment rule for fb.
+ * Supported: fa, fb each any of MX_E4M3, MX_E5M2, MX_E2M3, MX_E3M2, MX_E2M1
+ * (mixed pairs included, e.g. MXFP4 weights x MXFP6 activations), with
+ * K % 128 == 0 and any M, N >= 1.  fa == fb == MX_E2M1 with K % 256 == 0 runs
+ * kind::mxf4 on the packed codes; every other pair runs kind::mxf8f6f4, whose
+ * operands the copy engine expands to one code per byte in shared memory.
+ * MX_INT8 operands give MX_ERR_UNSUPPORTED (sm_100a has no block-scaled
+ * integer MMA).
  * Accumulation is fp32 on the tensor cores; |C - C_exact| stays within
  * 1e-5 * |alpha| * sum_k |a_mk b_nk| in the tested configurations.
  * Errors: MX_ERR_ARG, MX_ERR_ALIGN, MX_ERR_SHAPE, MX_ERR_UNSUPPORTED,

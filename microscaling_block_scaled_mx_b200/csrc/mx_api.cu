@@ -28,6 +28,7 @@ int sm_count(int *device_out) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 int elem_bits(int fmt) {
     switch (fmt) {
@@ -107,6 +108,37 @@ int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t
     return mx_launch_quantize(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
+int mx_quantize_dual(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, mx_fmt fmt,
+                     mx_round rnd_rows, uint64_t seed_rows, mx_round rnd_cols, uint64_t seed_cols,
+                     const mx_precond *pre_cols, void *codes_rows, void *scales_rows, void *codes_cols,
+                     void *scales_cols, mx_scale_layout sl, void *stream) {
+    if ((xdt != MX_F32 && xdt != MX_BF16) || elem_bits(fmt) == 0) return MX_ERR_ARG;
+    if ((rnd_rows != MX_RNE && rnd_rows != MX_SR) || (rnd_cols != MX_RNE && rnd_cols != MX_SR)) return MX_ERR_ARG;
+    if (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA) return MX_ERR_ARG;
+    if (rows < 0 || cols < 0) return MX_ERR_ARG;
+    if (rows % 32 != 0 || cols % 32 != 0) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;            // empty: pointers may be NULL
+    if (!x || !codes_rows || !scales_rows || !codes_cols || !scales_cols) return MX_ERR_ARG;
+    if (ldx < cols) return MX_ERR_ARG;
+    if (!aligned16(x) || (ldx * dtype_bytes(xdt)) % 16 != 0 || !aligned16(codes_rows) || !aligned16(codes_cols))
+        return MX_ERR_ALIGN;
+    if ((rnd_rows == MX_SR || rnd_cols == MX_SR) &&
+        static_cast<uint64_t>(rows) * static_cast<uint64_t>(cols) > (1ull << 34))
+        return MX_ERR_SR_RANGE;
+    if (mx_scales_bytes(sl, rows, cols) >= (1ull << 32) || mx_scales_bytes(sl, cols, rows) >= (1ull << 32))
+        return MX_ERR_UNSUPPORTED;
+    const bool had = pre_cols && pre_cols->hadamard;
+    MxQuantizeDualArgs a;
+    a.x = x; a.xdt = xdt; a.rows = rows; a.cols = cols; a.ldx = ldx; a.fmt = fmt;
+    a.rnd_rows = rnd_rows; a.rnd_cols = rnd_cols; a.seed_rows = seed_rows; a.seed_cols = seed_cols;
+    a.hadamard = had; a.sign_mask = had ? pre_cols->sign_mask : 0u;
+    a.codes_rows = codes_rows; a.scales_rows = scales_rows; a.codes_cols = codes_cols; a.scales_cols = scales_cols;
+    a.sl = sl;
+    a.num_sms = sm_count(nullptr);
+    if (a.num_sms <= 0) return MX_ERR_CUDA;
+    return mx_launch_quantize_dual(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
 int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_scale_layout sl,
                   int64_t outer, int64_t inner, void *y, mx_dtype ydt, int64_t ldy, void *stream) {
     if (elem_bits(fmt) == 0 || (ydt != MX_F32 && ydt != MX_BF16)) return MX_ERR_ARG;
@@ -136,12 +168,15 @@ int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
     if (M == 0 || N == 0) return MX_OK;                  // empty: pointers may be NULL
     if (!c || ldc < N) return MX_ERR_ARG;
     if (K > 0 && (!a_codes || !a_scales || !b_codes || !b_scales)) return MX_ERR_ARG;
-    const bool fp8 = (fa == MX_E4M3 || fa == MX_E5M2) && (fb == MX_E4M3 || fb == MX_E5M2);
-    const bool fp4 = fa == MX_E2M1 && fb == MX_E2M1;
-    if (!fp8 && !fp4) return MX_ERR_UNSUPPORTED;
-    if ((fp8 && K % 128 != 0) || (fp4 && K % 256 != 0)) return MX_ERR_UNSUPPORTED;
+    if (fa == MX_INT8 || fb == MX_INT8) return MX_ERR_UNSUPPORTED;   // no block-scaled INT8 MMA
+    if (K % 128 != 0) return MX_ERR_UNSUPPORTED;
     if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
         !aligned16(c) || (ldc * dtype_bytes(cdt)) % 16 != 0)
+        return MX_ERR_ALIGN;
+    // FP6 codes, and FP4 codes outside the E2M1 x E2M1 (K % 256 == 0) case, are
+    // read through packed tensor maps, which need 32-byte aligned bases
+    const bool mxf4 = fa == MX_E2M1 && fb == MX_E2M1 && K % 256 == 0;
+    if (!mxf4 && ((elem_bits(fa) < 8 && !aligned32(a_codes)) || (elem_bits(fb) < 8 && !aligned32(b_codes))))
         return MX_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (K == 0) {

@@ -126,30 +126,14 @@ __device__ __forceinline__ void store_code32(uint8_t *dst, const uint4 &a, const
     }
 }
 
-template <int FMT, bool SR, bool BF16_IN, bool V32>
-__device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &cp, int64_t blocks_per_row,
-                                           const BlockLoad<BF16_IN> &o, int lane) {
+// Encode one 32-block along a row from its values as FP32 bit patterns:
+// block amax -> E8M0 exponent, V * 2^-e (flushing FP32 subnormals), RNE or
+// stochastic rounding, and the packed codes and scale byte of (row, kb).
+// `codes_row` is the start of the row's codes.  SR's index is the element's
+// position row * cols + kb * 32 + j in the output.
+template <int FMT, bool SR, bool V32>
+__device__ __forceinline__ void encode_row_block(const CastParams &p, int64_t row, int64_t kb, uint32_t (&b)[32]) {
     constexpr int BITS = Fmt<FMT>::bits;
-    const int64_t kb = cp.chunk * 32 + lane;
-    if (cp.row >= p.rows || kb >= blocks_per_row) return;
-    // the 32 values as fp32 bit patterns
-    uint32_t b[32];
-    if (BF16_IN) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t ws[4] = {o.w[i].x, o.w[i].y, o.w[i].z, o.w[i].w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                b[8 * i + 2 * k] = ws[k] << 16;
-                b[8 * i + 2 * k + 1] = ws[k] & 0xffff0000u;
-            }
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            b[4 * i] = o.w[i].x; b[4 * i + 1] = o.w[i].y; b[4 * i + 2] = o.w[i].z; b[4 * i + 3] = o.w[i].w;
-        }
-    }
     uint32_t amax_bits = 0;
 #pragma unroll
     for (int i = 0; i < 32; i += 2)
@@ -179,9 +163,9 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
 #pragma unroll
             for (int i = 0; i < 8; ++i) c[i] = 0u;
         }
-        store_code32<V32>(p.codes + cp.row * p.cols + kb * 32, make_uint4(c[0], c[1], c[2], c[3]),
+        store_code32<V32>(p.codes + row * p.cols + kb * 32, make_uint4(c[0], c[1], c[2], c[3]),
                           make_uint4(c[4], c[5], c[6], c[7]));
-        store_scale(p, cp.row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+        store_scale(p, row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
         return;
     }
     if (Fmt<FMT>::emax == 0) {
@@ -198,7 +182,7 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
         }
     }
     if (SR) {
-        const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(cp.row * p.cols + kb * 32) >> 2);
+        const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(row * p.cols + kb * 32) >> 2);
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
             const uint32_t rw = fmix32((g + w) ^ p.key);
@@ -216,7 +200,7 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
 #pragma unroll
         for (int i = 0; i < 16; ++i) c[i] = 0u;
     }
-    uint8_t *dst = p.codes + cp.row * (p.cols * BITS / 8) + kb * (32 * BITS / 8);
+    uint8_t *dst = p.codes + row * (p.cols * BITS / 8) + kb * (32 * BITS / 8);
     if (BITS == 8) {
         const uint4 lo = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
         const uint4 hi = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16),
@@ -242,7 +226,34 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
             d[q] = w;
         }
     }
-    store_scale(p, cp.row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+    store_scale(p, row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+}
+
+
+template <int FMT, bool SR, bool BF16_IN, bool V32>
+__device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &cp, int64_t blocks_per_row,
+                                           const BlockLoad<BF16_IN> &o, int lane) {
+    const int64_t kb = cp.chunk * 32 + lane;
+    if (cp.row >= p.rows || kb >= blocks_per_row) return;
+    // the 32 values as fp32 bit patterns
+    uint32_t b[32];
+    if (BF16_IN) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t ws[4] = {o.w[i].x, o.w[i].y, o.w[i].z, o.w[i].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                b[8 * i + 2 * k] = ws[k] << 16;
+                b[8 * i + 2 * k + 1] = ws[k] & 0xffff0000u;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            b[4 * i] = o.w[i].x; b[4 * i + 1] = o.w[i].y; b[4 * i + 2] = o.w[i].z; b[4 * i + 3] = o.w[i].w;
+        }
+    }
+    encode_row_block<FMT, SR, V32>(p, cp.row, kb, b);
 }
 
 template <int FMT, bool SR, bool BF16_IN, bool V32>
@@ -319,7 +330,20 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-template <bool BF16_IN>
+// Shared-memory position of 16-byte chunk q of tile row rr.  Unswizzled for
+// the column cast.  The dual cast, which also reads 32-element row segments,
+// XORs the chunk's index inside its 128-byte span with the span index and the
+// row's parity, so both its column reads (a warp reads 128 contiguous bytes of
+// one row) and its row reads (eight lanes read the same chunk of 2 rows x 4
+// row blocks) touch distinct banks.
+template <bool BF16_IN, bool SWZ>
+__device__ __forceinline__ int tile_chunk(int rr, int q) {
+    if (!SWZ) return q;
+    constexpr int SH = BF16_IN ? 1 : 2;                      // spans per row: 2 (bf16), 4 (fp32)
+    return q ^ (((rr & 1) << SH) | (q >> 3));
+}
+
+template <bool BF16_IN, bool SWZ = false>
 __device__ __forceinline__ void stage_tile(const CastParams &p, uint8_t *buf, int64_t r0, int64_t c0) {
     using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
     constexpr int EPC = 16 / sizeof(TIn);                   // elements per 16-byte chunk
@@ -327,19 +351,128 @@ __device__ __forceinline__ void stage_tile(const CastParams &p, uint8_t *buf, in
     const TIn *x = static_cast<const TIn *>(p.x);
     const uint32_t sbuf = static_cast<uint32_t>(__cvta_generic_to_shared(buf));
     for (int ch = threadIdx.x; ch < COL_TILE_R * CPR; ch += COL_THREADS) {
-        const int rr = ch / CPR, cc = (ch % CPR) * EPC;
+        const int rr = ch / CPR, q = ch % CPR, cc = q * EPC;
         const int64_t gr = r0 + rr, gc = c0 + cc;
         int64_t valid = (gr < p.rows) ? (p.cols - gc) : 0;
         valid = valid < 0 ? 0 : (valid > EPC ? EPC : valid);
         const TIn *src = valid > 0 ? x + gr * p.ldx + gc : x;
-        cp_async16(sbuf + (rr * COL_TILE_C + cc) * sizeof(TIn), src, static_cast<uint32_t>(valid * sizeof(TIn)));
+        cp_async16(sbuf + rr * COL_TILE_C * sizeof(TIn) + tile_chunk<BF16_IN, SWZ>(rr, q) * 16, src,
+                   static_cast<uint32_t>(valid * sizeof(TIn)));
+    }
+}
+
+// Encode the two column blocks (columns gc, gc + 1; rows gr0 .. gr0 + 31) held
+// as packed f32x2 values x[j] = (column gc, column gc + 1) at row gr0 + j:
+// optional fixed-sign Hadamard, amax -> E8M0, exact scaling with the FP32
+// subnormal flush, RNE or stochastic rounding, and the codes as rows gc and
+// gc + 1 of the transposed output.  SR's index is the element's position
+// (gc + col) * rows + gr0 + j in that output.
+template <int FMT, bool SR, bool HAD>
+__device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&x)[32], int64_t gc, int64_t gr0) {
+    constexpr int BITS = Fmt<FMT>::bits;
+    const int64_t R = p.rows, C = p.cols;
+    if (HAD) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float sg = ((p.sign_mask >> j) & 1u) ? 1.0f : -1.0f;
+            x[j] = f2_mul(x[j], f2_pack(sg, sg));
+        }
+#pragma unroll
+        for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (i & h) continue;
+                const uint64_t a = x[i], b = x[i + h];
+                x[i] = f2_add(a, b);
+                x[i + h] = f2_sub(a, b);
+            }
+        }
+    }
+    const bool has_second = gc + 1 < C;
+    // block amax and exponent of both columns
+    uint32_t am0 = 0, am1 = 0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+        am0 = __vimax3_u32(am0, static_cast<uint32_t>(x[j]) & 0x7fffffffu,
+                           static_cast<uint32_t>(x[j + 1]) & 0x7fffffffu);
+        am1 = __vimax3_u32(am1, static_cast<uint32_t>(x[j] >> 32) & 0x7fffffffu,
+                           static_cast<uint32_t>(x[j + 1] >> 32) & 0x7fffffffu);
+    }
+    const int e0 = block_exponent<FMT>(am0), e1 = block_exponent<FMT>(am1);
+    // V * 2^-e for both columns with one packed multiply (flushing
+    // FP32 subnormals); INT8's e = 127 case takes the two-step path
+    const bool packed = Fmt<FMT>::emax != 0 || (e0 <= 126 && e1 <= 126);
+    if (packed) {
+        const uint64_t ff = f2_pack(pow2f(-e0), pow2f(-e1));
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = f2_mul_ftz(x[j], ff);
+    }
+#pragma unroll
+    for (int col = 0; col < 2; ++col) {
+        if (col == 1 && !has_second) break;
+        const uint32_t amax_bits = col ? am1 : am0;
+        const int e = col ? e1 : e0;
+        const bool nan_block = amax_bits >= 0x7f800000u;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            v[j] = __uint_as_float(static_cast<uint32_t>(x[j] >> (32 * col)));
+            if (!packed) v[j] = scale_down<FMT>(v[j], e);
+        }
+        const int64_t oc = gc + col;                 // output row
+        uint32_t c[16];
+        if (SR) {
+            const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(oc * R + gr0) >> 2);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const uint32_t rw = fmix32((g + w) ^ p.key);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int j = 4 * w + k;
+                    const float m = sr_magnitude_int<FMT>(fabsf(v[j]), (rw >> (8 * k)) & 255u);
+                    v[j] = copysignf(m, v[j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(v[j], v[j + 1]);
+        if (nan_block) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) c[i] = 0u;
+        }
+        if (BITS == 8) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.codes + oc * R + gr0);
+            dst[0] = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+            dst[1] = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16),
+                                c[14] | (c[15] << 16));
+        } else if (BITS == 4) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w[i] = c[4 * i] | (c[4 * i + 1] << 8) | (c[4 * i + 2] << 16) | (c[4 * i + 3] << 24);
+            *reinterpret_cast<uint4 *>(p.codes + oc * (R >> 1) + (gr0 >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+            uint64_t *dst = reinterpret_cast<uint64_t *>(p.codes + oc * (R / 4 * 3) + gr0 / 4 * 3);
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {     // 3 words of 64 bits = 32 codes of 6 bits
+                uint64_t w = 0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int bit = 6 * j - 64 * q;
+                    const uint64_t code = (c[j >> 1] >> (8 * (j & 1))) & 0x3fu;
+                    if (bit >= 0 && bit < 64) w |= code << bit;
+                    else if (bit < 0 && bit > -6) w |= code >> (-bit);
+                }
+                dst[q] = w;
+            }
+        }
+        store_scale(p, oc, gr0 >> 5, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
     }
 }
 
 template <int FMT, bool SR, bool BF16_IN, bool HAD>
 __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p) {
     using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
-    constexpr int BITS = Fmt<FMT>::bits;
     constexpr int TILE_BYTES = COL_TILE_R * COL_TILE_C * sizeof(TIn);
     extern __shared__ __align__(16) uint8_t col_smem[];
 
@@ -379,103 +512,103 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
                     x[j] = *reinterpret_cast<const uint64_t *>(tile + off);
                 }
             }
-            if (HAD) {
+            encode_col_pair<FMT, SR, HAD>(p, x, gc, gr0);
+        }
+        __syncthreads();             // everyone is done with `buf` before it is refilled
+    }
+    cp_async_wait_all();
+}
+
+// ---------------------------------------------------------------------------
+// Dual cast: one read of the input, codes along both axes.
+// ---------------------------------------------------------------------------
+// The forward GEMM contracts an activation over its columns (blocks along
+// rows) and the weight-gradient GEMM over its rows (blocks down columns,
+// transposed output); section 3 of the MX summary notes that the two
+// quantizations of one tensor differ, so both are needed.  This kernel stages
+// each 128 x 128 tile once (swizzled, see tile_chunk) and writes both: every
+// thread encodes one column pair of one 32-row block (as cast_cols) and two
+// 32-element row blocks (as cast_rows, RNE or SR with its own seed).  The
+// result equals mx_quantize along rows plus mx_quantize along columns.
+template <int FMT, bool BF16_IN, bool HAD>
+__global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr, CastParams pc, int sr_rows,
+                                                                   int sr_cols) {
+    using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
+    constexpr int TILE_BYTES = COL_TILE_R * COL_TILE_C * sizeof(TIn);
+    constexpr int ROW_BYTES = COL_TILE_C * sizeof(TIn);
+    constexpr int CPB = 32 * sizeof(TIn) / 16;              // 16-byte chunks per 32-element row block
+    extern __shared__ __align__(16) uint8_t col_smem[];
+
+    const int64_t R = pc.rows, C = pc.cols;
+    const int64_t tiles_r = (R + COL_TILE_R - 1) / COL_TILE_R;
+    const int64_t tiles_c = (C + COL_TILE_C - 1) / COL_TILE_C;
+    const int64_t n_tiles = tiles_r * tiles_c;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int blk = warp & 3;                       // column part: 32-row block inside the tile
+    const int pair = (warp >> 2) * 32 + lane;       // column part: column pair inside the tile
+    const int rb = threadIdx.x & 3;                 // row part: 32-column block inside the tile
+    const int rrow = threadIdx.x >> 2;              // row part: tile rows rrow and rrow + 64
+
+    // the column pair's byte offset inside even and odd tile rows
+    const int cbyte = 2 * pair * static_cast<int>(sizeof(TIn));
+    const int col_off[2] = {tile_chunk<BF16_IN, true>(0, cbyte >> 4) * 16 + (cbyte & 15),
+                            tile_chunk<BF16_IN, true>(1, cbyte >> 4) * 16 + (cbyte & 15)};
+
+    int64_t t = blockIdx.x;
+    if (t < n_tiles) stage_tile<BF16_IN, true>(pc, col_smem, (t / tiles_c) * COL_TILE_R, (t % tiles_c) * COL_TILE_C);
+    cp_async_commit();
+    for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1) {
+        const int64_t tn = t + gridDim.x;
+        if (tn < n_tiles)
+            stage_tile<BF16_IN, true>(pc, col_smem + (buf ^ 1) * TILE_BYTES, (tn / tiles_c) * COL_TILE_R,
+                                      (tn % tiles_c) * COL_TILE_C);
+        cp_async_commit();
+        cp_async_wait_prev();        // this tile's copies (the older group) have landed
+        __syncthreads();
+
+        const uint8_t *tile = col_smem + buf * TILE_BYTES;
+        const int64_t r0 = (t / tiles_c) * COL_TILE_R, c0 = (t % tiles_c) * COL_TILE_C;
+        // ---- column blocks ----
+        const int64_t gc = c0 + 2 * pair, gr0 = r0 + blk * 32;
+        if (gc < C && gr0 < R) {
+            uint64_t x[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float sg = ((p.sign_mask >> j) & 1u) ? 1.0f : -1.0f;
-                    x[j] = f2_mul(x[j], f2_pack(sg, sg));
-                }
-#pragma unroll
-                for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        if (i & h) continue;
-                        const uint64_t a = x[i], b = x[i + h];
-                        x[i] = f2_add(a, b);
-                        x[i + h] = f2_sub(a, b);
-                    }
-                }
-            }
-            const bool has_second = gc + 1 < C;
-            // block amax and exponent of both columns
-            uint32_t am0 = 0, am1 = 0;
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                am0 = __vimax3_u32(am0, static_cast<uint32_t>(x[j]) & 0x7fffffffu,
-                                   static_cast<uint32_t>(x[j + 1]) & 0x7fffffffu);
-                am1 = __vimax3_u32(am1, static_cast<uint32_t>(x[j] >> 32) & 0x7fffffffu,
-                                   static_cast<uint32_t>(x[j + 1] >> 32) & 0x7fffffffu);
-            }
-            const int e0 = block_exponent<FMT>(am0), e1 = block_exponent<FMT>(am1);
-            // V * 2^-e for both columns with one packed multiply (flushing
-            // FP32 subnormals); INT8's e = 127 case takes the two-step path
-            const bool packed = Fmt<FMT>::emax != 0 || (e0 <= 126 && e1 <= 126);
-            if (packed) {
-                const uint64_t ff = f2_pack(pow2f(-e0), pow2f(-e1));
-#pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] = f2_mul_ftz(x[j], ff);
-            }
-#pragma unroll
-            for (int col = 0; col < 2; ++col) {
-                if (col == 1 && !has_second) break;
-                const uint32_t amax_bits = col ? am1 : am0;
-                const int e = col ? e1 : e0;
-                const bool nan_block = amax_bits >= 0x7f800000u;
-                float v[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    v[j] = __uint_as_float(static_cast<uint32_t>(x[j] >> (32 * col)));
-                    if (!packed) v[j] = scale_down<FMT>(v[j], e);
-                }
-                const int64_t oc = gc + col;                 // output row
-                uint32_t c[16];
-                if (SR) {
-                    const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(oc * R + gr0) >> 2);
-#pragma unroll
-                    for (int w = 0; w < 8; ++w) {
-                        const uint32_t rw = fmix32((g + w) ^ p.key);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int j = 4 * w + k;
-                            const float m = sr_magnitude_int<FMT>(fabsf(v[j]), (rw >> (8 * k)) & 255u);
-                            v[j] = copysignf(m, v[j]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(v[j], v[j + 1]);
-                if (nan_block) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) c[i] = 0u;
-                }
-                if (BITS == 8) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.codes + oc * R + gr0);
-                    dst[0] = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
-                    dst[1] = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16),
-                                        c[14] | (c[15] << 16));
-                } else if (BITS == 4) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        w[i] = c[4 * i] | (c[4 * i + 1] << 8) | (c[4 * i + 2] << 16) | (c[4 * i + 3] << 24);
-                    *reinterpret_cast<uint4 *>(p.codes + oc * (R >> 1) + (gr0 >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int j = 0; j < 32; ++j) {
+                const uint8_t *src = tile + (blk * 32 + j) * ROW_BYTES + col_off[j & 1];
+                if (BF16_IN) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(src);
+                    x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
                 } else {
-                    uint64_t *dst = reinterpret_cast<uint64_t *>(p.codes + oc * (R / 4 * 3) + gr0 / 4 * 3);
-#pragma unroll
-                    for (int q = 0; q < 3; ++q) {     // 3 words of 64 bits = 32 codes of 6 bits
-                        uint64_t w = 0;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int bit = 6 * j - 64 * q;
-                            const uint64_t code = (c[j >> 1] >> (8 * (j & 1))) & 0x3fu;
-                            if (bit >= 0 && bit < 64) w |= code << bit;
-                            else if (bit < 0 && bit > -6) w |= code >> (-bit);
-                        }
-                        dst[q] = w;
-                    }
+                    x[j] = *reinterpret_cast<const uint64_t *>(src);
                 }
-                store_scale(p, oc, gr0 >> 5, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
             }
+            if (sr_cols) encode_col_pair<FMT, true, HAD>(pc, x, gc, gr0);
+            else encode_col_pair<FMT, false, HAD>(pc, x, gc, gr0);
+        }
+        // ---- row blocks ----
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            const int rr = rrow + 64 * h;
+            const int64_t row = r0 + rr, kb = (c0 >> 5) + rb;
+            if (row >= R || 32 * kb >= C) continue;
+            uint32_t b[32];
+#pragma unroll
+            for (int i = 0; i < CPB; ++i) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(
+                    tile + rr * ROW_BYTES + tile_chunk<BF16_IN, true>(rr, rb * CPB + i) * 16);
+                if (BF16_IN) {
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        b[8 * i + 2 * k] = ws[k] << 16;
+                        b[8 * i + 2 * k + 1] = ws[k] & 0xffff0000u;
+                    }
+                } else {
+                    b[4 * i] = w.x; b[4 * i + 1] = w.y; b[4 * i + 2] = w.z; b[4 * i + 3] = w.w;
+                }
+            }
+            if (sr_rows) encode_row_block<FMT, true, false>(pr, row, kb, b);
+            else encode_row_block<FMT, false, false>(pr, row, kb, b);
         }
         __syncthreads();             // everyone is done with `buf` before it is refilled
     }
@@ -673,6 +806,35 @@ static cudaError_t launch_cast_rnd(const CastParams &p, int xdt, int block_axis,
               : launch_cast_fmt<FMT, false>(p, xdt, block_axis, had, sms, st);
 }
 
+// Dual cast: the column cast's tile buffers and resident grid.
+template <auto Kernel>
+static cudaError_t launch_dual(int in_bytes, const CastParams &pr, const CastParams &pc, int sr_rows, int sr_cols,
+                               int64_t tiles, int sms, cudaStream_t st) {
+    const int smem = 2 * COL_TILE_R * COL_TILE_C * in_bytes;
+    static bool configured = false;    // per template instance, i.e. per kernel
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    Kernel<<<grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)), COL_THREADS, smem, st>>>(
+        pr, pc, sr_rows, sr_cols);
+    return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t launch_dual_fmt(const CastParams &pr, const CastParams &pc, int xdt, bool had, int sr_rows,
+                                   int sr_cols, int sms, cudaStream_t st) {
+    const int64_t tiles = ((pc.rows + COL_TILE_R - 1) / COL_TILE_R) * ((pc.cols + COL_TILE_C - 1) / COL_TILE_C);
+    const bool bf = xdt == MX_BF16;
+    if (had) {
+        if (bf) return launch_dual<cast_dual_kernel<FMT, true, true>>(2, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+        return launch_dual<cast_dual_kernel<FMT, false, true>>(4, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+    }
+    if (bf) return launch_dual<cast_dual_kernel<FMT, true, false>>(2, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+    return launch_dual<cast_dual_kernel<FMT, false, false>>(4, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+}
+
 }  // namespace mxk
 
 cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st) {
@@ -732,4 +894,39 @@ cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st) {
     }
 #undef MX_DQ
     return cudaGetLastError();
+}
+
+cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st) {
+    using namespace mxk;
+    auto key = [](uint64_t seed) {
+        return fmix32_host(static_cast<uint32_t>(seed)) ^ static_cast<uint32_t>(seed >> 32);
+    };
+    CastParams pr, pc;
+    pr.x = pc.x = a.x;
+    pr.rows = pc.rows = a.rows;
+    pr.cols = pc.cols = a.cols;
+    pr.ldx = pc.ldx = a.ldx;
+    pr.mma_scales = pc.mma_scales = a.sl == MX_SCALES_MMA;
+    pr.codes = static_cast<uint8_t *>(a.codes_rows);
+    pr.scales = static_cast<uint8_t *>(a.scales_rows);
+    pr.k_blocks = a.cols / 32;
+    pr.k_groups = (pr.k_blocks + 3) / 4;
+    pr.key = key(a.seed_rows);
+    pr.sign_mask = 0;
+    pc.codes = static_cast<uint8_t *>(a.codes_cols);
+    pc.scales = static_cast<uint8_t *>(a.scales_cols);
+    pc.k_blocks = a.rows / 32;
+    pc.k_groups = (pc.k_blocks + 3) / 4;
+    pc.key = key(a.seed_cols);
+    pc.sign_mask = a.sign_mask;
+    const int sr_r = a.rnd_rows == MX_SR, sr_c = a.rnd_cols == MX_SR;
+    switch (a.fmt) {
+        case MX_E4M3: return launch_dual_fmt<MX_E4M3>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);
+        case MX_E5M2: return launch_dual_fmt<MX_E5M2>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);
+        case MX_E2M3: return launch_dual_fmt<MX_E2M3>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);
+        case MX_E3M2: return launch_dual_fmt<MX_E3M2>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);
+        case MX_E2M1: return launch_dual_fmt<MX_E2M1>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);
+        case MX_INT8: return launch_dual_fmt<MX_INT8>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);
+    }
+    return cudaErrorInvalidValue;
 }

@@ -91,6 +91,7 @@ struct Params {
     int tiles_m, tiles_n;
     float alpha;
     uint32_t idesc;  // instruction descriptor without the scale-factor ids
+    uint32_t ab_tx;  // bytes the A and B loads of one stage deliver (packed size in global)
     int skip_k_tile; // testing hook: CTA 0 withholds this k-tile of its first tile (-1: off)
 };
 
@@ -324,8 +325,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                         ok = false;          // injected stall: this stage is never filled
                         break;
                     }
-                    const uint32_t bytes = A_STAGE_BYTES + B_STAGE_BYTES + C::SFA_BYTES +
-                                           (b_second ? 2 : 1) * (C::SFB_BYTES / 2);
+                    const uint32_t bytes = p.ab_tx + C::SFA_BYTES + (b_second ? 2 : 1) * (C::SFB_BYTES / 2);
                     const uint32_t fb = full_bar(s);
                     mbar_expect_tx(fb, bytes);
                     tma_load_2d(sbase + Smem::A + s * A_STAGE_BYTES, &tma_a, kt * BK_BYTES, m0, fb);
@@ -510,6 +510,7 @@ struct PairParams {
     int tiles_m, tiles_n;      // 256 x 192 pair tiles
     float alpha;
     uint32_t idesc;
+    uint32_t ab_tx;            // bytes one CTA's A and B loads of a stage deliver
     int skip_k_tile;
 };
 
@@ -617,7 +618,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            const uint32_t stage_bytes = 2 * (C::STAGE_BYTES + C::SFA_BYTES + C::SFB_BYTES);
+            const uint32_t stage_bytes = 2 * (p.ab_tx + C::SFA_BYTES + C::SFB_BYTES);
             for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
                 const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
                 // this CTA's A rows and B rows; a half that lies wholly past M (or N)
@@ -760,19 +761,42 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 2-D uint8 tensor map over a rows x row_bytes matrix, box of box_rows x 128
-// bytes, 128-byte swizzle; out-of-range rows read as zero.
-bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t row_bytes, int box_rows) {
+int elem_bits(int f) { return f == MX_E2M1 ? 4 : (f == MX_E2M3 || f == MX_E3M2) ? 6 : 8; }
+
+// Tensor map over one operand's codes (rows x K, K contiguous), a box of
+// box_rows x one stage of K, 128-byte swizzle; rows past the end read as zero.
+// kind::mxf4 takes E2M1 codes packed two to a byte, so its stage is 128 bytes
+// = 256 codes of a uint8 view.  kind::mxf8f6f4 takes one code per byte in
+// shared memory: FP8 codes are bytes already, and the copy engine expands
+// FP6 (16 codes in 12 bytes) and FP4 (16 codes in 8 bytes) to 16 bytes each
+// on the way in (the 16U6 / 16U4 packed tensor-map types), so a stage is 128
+// codes in 128 bytes of shared memory for every element format.
+bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int fmt, bool mxf4,
+                      int box_rows) {
     auto encode = get_encode();
     if (!encode) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const int bits = elem_bits(fmt);
+    CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    cuuint64_t inner = static_cast<cuuint64_t>(K);            // elements along K
+    if (mxf4) inner = static_cast<cuuint64_t>(K / 2);           // bytes of packed pairs
+    else if (bits == 6) dt = CU_TENSOR_MAP_DATA_TYPE_16U6_ALIGN16B;
+    else if (bits == 4) dt = CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+    cuuint64_t dims[2] = {inner, static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * bits / 8)};
     cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+    CUresult r = encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Bytes one stage's load of box_rows rows delivers: the packed size in global
+// memory (128 bytes per row for FP8 and packed FP4, 96 for FP6, 64 for FP4
+// expanded to bytes).
+uint32_t stage_tx_bytes(int fmt, bool mxf4, int box_rows) {
+    const int per_row = mxf4 ? BK_BYTES : BK_BYTES * elem_bits(fmt) / 8;
+    return static_cast<uint32_t>(per_row * box_rows);
 }
 
 // 2-D uint8 view of an MMA-layout scale buffer as rows of 256 bytes (two rows
@@ -793,7 +817,13 @@ bool make_scale_map(CUtensorMap *map, const void *base, int64_t bytes, int atoms
 uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN) {
     auto code = [&](int f) -> uint32_t {
         if (fp4) return 1u;               // kind::mxf4: E2M1
-        return f == MX_E5M2 ? 1u : 0u;    // kind::mxf8f6f4: E4M3 = 0, E5M2 = 1
+        switch (f) {                      // kind::mxf8f6f4 operand type codes
+            case MX_E5M2: return 1u;
+            case MX_E2M3: return 3u;
+            case MX_E3M2: return 4u;
+            case MX_E2M1: return 5u;
+            default: return 0u;           // E4M3
+        }
     };
     uint32_t d = 0;
     d |= code(fa) << 7;
@@ -844,16 +874,23 @@ extern "C" int mx_debug_gemm_skip_stage(int k_tile) {
 
 namespace {
 
-// M > 128: the two-SM kernel (256 x 192 tiles over CTA pairs).
+// E2M1 x E2M1 with K a multiple of 256 runs kind::mxf4 on packed codes (256
+// per stage); every other pair, and FP4 x FP4 with K = 128 (mod 256), runs
+// kind::mxf8f6f4 with 128 codes per stage.
+bool use_mxf4(const MxGemmArgs &a) {
+    return a.fa == MX_E2M1 && a.fb == MX_E2M1 && a.K % 256 == 0;
+}
+
+// M > 128: the two-SM kernel (256 x 256 tiles over CTA pairs).
 int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     using namespace mxg;
-    const bool fp4 = a.fa == MX_E2M1;
-    const int64_t k_bytes = fp4 ? a.K / 2 : a.K;
+    const bool fp4 = use_mxf4(a);
+    const int64_t k_bytes = fp4 ? a.K / 2 : a.K;     // K bytes of a uint8 stage view
     const int G = fp4 ? 2 : 1;
     const int64_t k_groups = a.K / 128;
     CUtensorMap ta, tb, tsa, tsb;
-    if (!make_operand_map(&ta, a.a_codes, a.M, k_bytes, 128)) return MX_ERR_CUDA;
-    if (!make_operand_map(&tb, a.b_codes, a.N, k_bytes, PAIR_B_ROWS)) return MX_ERR_CUDA;
+    if (!make_operand_map(&ta, a.a_codes, a.M, a.K, a.fa, fp4, 128)) return MX_ERR_CUDA;
+    if (!make_operand_map(&tb, a.b_codes, a.N, a.K, a.fb, fp4, PAIR_B_ROWS)) return MX_ERR_CUDA;
     const int64_t sa_bytes = (a.M + 127) / 128 * 128 * k_groups * 4;
     const int64_t sb_bytes = (a.N + 127) / 128 * 128 * k_groups * 4;
     if (!make_scale_map(&tsa, a.a_scales, sa_bytes, G)) return MX_ERR_CUDA;
@@ -870,6 +907,7 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     p.tiles_n = static_cast<int>((a.N + PAIR_BN - 1) / PAIR_BN);
     p.alpha = a.alpha;
     p.idesc = make_idesc(a.fa, a.fb, fp4, PAIR_BM, PAIR_BN);
+    p.ab_tx = stage_tx_bytes(a.fa, fp4, 128) + stage_tx_bytes(a.fb, fp4, PAIR_B_ROWS);
     p.skip_k_tile = g_skip_k_tile.exchange(-1);
     const int tiles = p.tiles_m * p.tiles_n;
     const int clusters = tiles < a.num_sms / 2 ? tiles : a.num_sms / 2;
@@ -897,11 +935,11 @@ bool use_pair_kernel(const MxGemmArgs &a) {
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     using namespace mxg;
     if (use_pair_kernel(a)) return launch_gemm_pair(a, st);
-    const bool fp4 = a.fa == MX_E2M1;
+    const bool fp4 = use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;
     CUtensorMap ta, tb;
-    if (!make_operand_map(&ta, a.a_codes, a.M, k_bytes, BM)) return MX_ERR_CUDA;
-    if (!make_operand_map(&tb, a.b_codes, a.N, k_bytes, BN)) return MX_ERR_CUDA;
+    if (!make_operand_map(&ta, a.a_codes, a.M, a.K, a.fa, fp4, BM)) return MX_ERR_CUDA;
+    if (!make_operand_map(&tb, a.b_codes, a.N, a.K, a.fb, fp4, BN)) return MX_ERR_CUDA;
     Params p;
     p.a_scales = static_cast<const uint8_t *>(a.a_scales);
     p.b_scales = static_cast<const uint8_t *>(a.b_scales);
@@ -916,6 +954,7 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     p.tiles_n = static_cast<int>((a.N + BN - 1) / BN);
     p.alpha = a.alpha;
     p.idesc = make_idesc(a.fa, a.fb, fp4);
+    p.ab_tx = stage_tx_bytes(a.fa, fp4, BM) + stage_tx_bytes(a.fb, fp4, BN);
     p.skip_k_tile = g_skip_k_tile.exchange(-1);
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < a.num_sms ? tiles : a.num_sms;

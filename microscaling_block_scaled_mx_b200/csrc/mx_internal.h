@@ -24,6 +24,20 @@ struct MxQuantizeArgs {
     int num_sms;
 };
 
+struct MxQuantizeDualArgs {
+    const void *x;
+    int xdt;
+    int64_t rows, cols, ldx;
+    int fmt;
+    int rnd_rows, rnd_cols;
+    uint64_t seed_rows, seed_cols;
+    bool hadamard;            // column (block_axis 0) output only
+    uint32_t sign_mask;
+    void *codes_rows, *scales_rows, *codes_cols, *scales_cols;
+    int sl;
+    int num_sms;
+};
+
 struct MxDequantArgs {
     const void *codes;
     const void *scales;
@@ -59,6 +73,7 @@ inline uint32_t fmix32_host(uint32_t h) {
 }
 
 cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st);
+cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st);
 cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st);
 // returns an mx_status (MX_OK, MX_ERR_CUDA, MX_ERR_UNSUPPORTED)
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st);

@@ -61,6 +61,9 @@ def lib() -> ctypes.CDLL:
             L.mx_quantize.restype = i32
             L.mx_quantize.argtypes = [vp, i32, i64, i64, i64, i32, i32, i32, u64,
                                       ctypes.POINTER(_Precond), vp, vp, i32, vp]
+            L.mx_quantize_dual.restype = i32
+            L.mx_quantize_dual.argtypes = [vp, i32, i64, i64, i64, i32, i32, u64, i32, u64,
+                                           ctypes.POINTER(_Precond), vp, vp, vp, vp, i32, vp]
             L.mx_dequantize.restype = i32
             L.mx_dequantize.argtypes = [vp, vp, i32, i32, i64, i64, vp, i32, i64, vp]
             L.mx_gemm.restype = i32
@@ -145,6 +148,39 @@ def quantize(x: torch.Tensor, block_axis: int = 1, fmt="e4m3", rnd="rne", seed: 
                            ctypes.byref(pre), codes.data_ptr(), scales.data_ptr(), sl, _stream(stream))
     _check(rc, "mx_quantize")
     return codes, scales
+
+
+def quantize_dual(x: torch.Tensor, fmt="e4m3", rnd_rows="rne", seed_rows: int = 0, rnd_cols="rne",
+                  seed_cols: int = 0, hadamard: bool = False, sign_mask: int = DEFAULT_SIGN_MASK,
+                  scale_layout="mma", out=None, stream=None):
+    """Both MX casts of a 2-D CUDA tensor from one read of it.
+
+    Returns (codes_rows, scales_rows, codes_cols, scales_cols): the results of
+    quantize(x, 1, ...) with (rnd_rows, seed_rows) and of quantize(x, 0, ...)
+    with (rnd_cols, seed_cols, hadamard); `out` may supply the four buffers.
+    """
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    if x.dtype not in DTYPE:
+        raise TypeError("x must be float32 or bfloat16")
+    f = _fmt(fmt)
+    sl = _layout(scale_layout)
+    rows, cols = x.shape
+    if out is None:
+        u8 = dict(dtype=torch.uint8, device=x.device)
+        out = (torch.empty((rows, codes_row_bytes(f, cols)), **u8),
+               torch.empty(max(scales_bytes(sl, rows, cols), 1), **u8),
+               torch.empty((cols, codes_row_bytes(f, rows)), **u8),
+               torch.empty(max(scales_bytes(sl, cols, rows), 1), **u8))
+    cr, sr_, cc, sc = out
+    pre = _Precond(1 if hadamard else 0, sign_mask & 0xFFFFFFFF)
+    rnd = lambda r: ROUND[r] if isinstance(r, str) else int(r)
+    rc = lib().mx_quantize_dual(x.data_ptr(), DTYPE[x.dtype], rows, cols, x.stride(0), f,
+                                rnd(rnd_rows), seed_rows & (2**64 - 1), rnd(rnd_cols), seed_cols & (2**64 - 1),
+                                ctypes.byref(pre), cr.data_ptr(), sr_.data_ptr(), cc.data_ptr(), sc.data_ptr(),
+                                sl, _stream(stream))
+    _check(rc, "mx_quantize_dual")
+    return cr, sr_, cc, sc
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, fmt, outer: int, inner: int,

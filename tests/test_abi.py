@@ -95,9 +95,35 @@ def test_dequantize_validation(mx):
     assert L.mx_dequantize(16, 16, 0, 1, 4, 32, 16, 1, 36, None) == -2
 
 
+def _d(mx, rows=64, cols=64, x=16, ldx=64, xdt=1, fmt=0, rr=0, rc=0, cr=16, sr=16, cc=16, sc=16, sl=1):
+    L = mx.lib()
+    return L.mx_quantize_dual(x, xdt, rows, cols, ldx, fmt, rr, 0, rc, 0, None, cr, sr, cc, sc, sl, None)
+
+
+def test_quantize_dual_validation(mx):
+    assert _d(mx, fmt=9) == -1
+    assert _d(mx, rr=2) == -1
+    assert _d(mx, sl=3) == -1
+    assert _d(mx, rows=-32) == -1
+    assert _d(mx, rows=48) == -3                  # both axes are block axes
+    assert _d(mx, cols=80, ldx=80) == -3
+    assert _d(mx, rows=0) == 0                    # empty: no-op, pointers unused
+    assert _d(mx, cols=0, x=None, cr=None) == 0
+    assert _d(mx, cc=None) == -1
+    assert _d(mx, ldx=32) == -1
+    assert _d(mx, x=8) == -2
+    assert _d(mx, ldx=68) == -2                   # 136-byte bf16 row pitch
+    assert _d(mx, cr=24) == -2
+    assert _d(mx, rows=2 ** 20, cols=2 ** 15, ldx=2 ** 15, rc=1) == -5   # 2^35 elements with SR
+
+
 def _g(mx, fa=0, fb=0, M=128, N=128, K=256, c=16, cdt=1, ldc=128, a=16):
     L = mx.lib()
     return L.mx_gemm(a, 16, fa, 16, 16, fb, M, N, K, 1.0, c, cdt, ldc, None, 0, None)
+
+
+def L_gemm_b_misaligned(mx, fa, fb):
+    return mx.lib().mx_gemm(32, 16, fa, 48, 16, fb, 128, 128, 256, 1.0, 16, 1, 128, None, 0, None)
 
 
 def test_gemm_validation(mx):
@@ -107,10 +133,15 @@ def test_gemm_validation(mx):
     assert _g(mx, ldc=64) == -1
     assert _g(mx, K=48) == -3
     assert _g(mx, fa=5, fb=5) == -4               # no block-scaled INT8 MMA
-    assert _g(mx, fa=0, fb=4) == -4               # mixed FP8 x FP4 not built
-    assert _g(mx, fa=2, fb=2) == -4               # FP6 not built
-    assert _g(mx, K=160) == -4                    # FP8 needs K % 128
-    assert _g(mx, fa=4, fb=4, K=384) == -4        # FP4 needs K % 256
+    assert _g(mx, fa=0, fb=5) == -4               # INT8 in either operand
+    assert _g(mx, K=160) == -4                    # K % 128
+    assert _g(mx, fa=2, fb=3, K=160) == -4
+    assert _g(mx, fa=4, fb=4, K=192) == -4
+    # FP6 codes, and FP4 codes fed to kind::mxf8f6f4, need 32-byte aligned bases
+    assert _g(mx, fa=2, fb=2, a=48) == -2
+    assert _g(mx, fa=0, fb=1, a=48) != -2         # FP8 codes at 16 bytes are fine ...
+    assert L_gemm_b_misaligned(mx, fa=0, fb=3) == -2   # ... FP6 B at 16 bytes is not
+    assert _g(mx, fa=4, fb=4, K=384, a=48) == -2  # FP4 x FP4, K = 128 (mod 256)
     assert _g(mx, c=8) == -2
     assert _g(mx, ldc=129, cdt=1) == -2
 

@@ -44,22 +44,24 @@ def to_f64(t):
     return host(t.float()).astype(np.float64) if t.dtype == torch.bfloat16 else host(t).astype(np.float64)
 
 
-def run_gemm(oracle, a, b, fmt, M, N, K, alpha=1.0, out_dtype=torch.float32, ldc=None, rows=None):
+def run_gemm(oracle, a, b, fmt, M, N, K, alpha=1.0, out_dtype=torch.float32, ldc=None, rows=None, fb=None):
     """a: M x K, b: N x K host arrays (float32 or bf16 bits); both cast along K
-    by the GPU (verified bit-exact elsewhere) and by the oracle."""
+    by the GPU (verified bit-exact elsewhere) and by the oracle.  A is cast to
+    fmt, B to fb (default fmt)."""
+    fb = fmt if fb is None else fb
     ac, as_ = mx.quantize(to_device(a), 1, fmt)
-    bc, bs = mx.quantize(to_device(b), 1, fmt)
+    bc, bs = mx.quantize(to_device(b), 1, fb)
     if ldc is None:
         out = torch.empty((M, N), dtype=out_dtype, device=dev())
     else:
         out = torch.empty((M, ldc), dtype=out_dtype, device=dev())[:, :N]
     out.fill_(float("nan"))
-    mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, alpha=alpha, out=out)
+    mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, fb=fb, alpha=alpha, out=out)
     torch.cuda.synchronize()
-    f = oracle.FORMATS[fmt]
+    f, g = oracle.FORMATS[fmt], oracle.FORMATS[fb]
     oac, oas = oracle.quantize(a, 1, f, scale_layout=oracle.MMA)
-    obc, obs = oracle.quantize(b, 1, f, scale_layout=oracle.MMA)
-    ref, bound = oracle.gemm_decoded(oac, oas, f, obc, obs, f, M, N, K, alpha=alpha, rows=rows)
+    obc, obs = oracle.quantize(b, 1, g, scale_layout=oracle.MMA)
+    ref, bound = oracle.gemm_decoded(oac, oas, f, obc, obs, g, M, N, K, alpha=alpha, rows=rows)
     got = to_f64(out)
     if rows is not None:
         got = got[np.asarray(rows)]
@@ -122,6 +124,55 @@ def test_gemm_two_sm_tiles_bit_exact(oracle, fmt):
         got, ref, bound = run_gemm(oracle, a, b, fmt, M, N, K)
         exact = oracle.round_f32(ref).astype(np.float64)
         assert np.array_equal(got, exact), (M, N, np.argwhere(got != exact)[:5])
+
+
+# Mixed and FP6 pairs run kind::mxf8f6f4 with FP6 and FP4 codes expanded to
+# one per byte by the copy engine; E2M1 x E2M1 with K = 128 (mod 256) takes
+# the same route instead of kind::mxf4.
+MIXED_PAIRS = [("e2m1", "e3m2"), ("e3m2", "e2m1"), ("e2m3", "e2m3"), ("e3m2", "e3m2"),
+               ("e4m3", "e2m1"), ("e2m1", "e5m2"), ("e5m2", "e2m3"), ("e2m3", "e4m3")]
+
+
+@pytest.mark.parametrize("fa,fb", MIXED_PAIRS + [("e2m1", "e2m1")])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (256, 384, 384), (512, 576, 256)])
+def test_gemm_mixed_one_sm_bit_exact(oracle, fa, fb, M, N, K):
+    rng = np.random.default_rng(M + N + K + len(fa + fb))
+    # values clipped to [-3, 3] times the block's power of two sit on every element grid
+    a = np.clip(small_int_operand(rng, M, K), -3, 3)
+    b = np.clip(small_int_operand(rng, N, K), -3, 3)
+    if fa == fb == "e2m1" and K % 256 == 0:
+        K = K + 128          # the FP4 x FP4 case of interest here is K = 128 (mod 256)
+        a = np.concatenate([a, a[:, :128]], axis=1)
+        b = np.concatenate([b, b[:, :128]], axis=1)
+    got, ref, bound = run_gemm(oracle, a, b, fa, M, N, K, fb=fb)
+    exact = oracle.round_f32(ref).astype(np.float64)
+    assert np.array_equal(got, exact), (fa, fb, np.argwhere(got != exact)[:5])
+
+
+@pytest.mark.parametrize("fa,fb", [("e2m1", "e3m2"), ("e3m2", "e3m2"), ("e4m3", "e2m3")])
+def test_gemm_mixed_two_sm_bit_exact(oracle, fa, fb):
+    """Pair-kernel shapes (K >= 2048, >= one 256 x 256 tile per SM), ragged
+    second shape."""
+    K = 2048
+    for (M, N) in [(4096, 2560), (4000, 2600)]:
+        rng = np.random.default_rng(M + N + 1)
+        a, b = small_int_operand(rng, M, K), small_int_operand(rng, N, K)
+        a, b = np.clip(a, -3, 3), np.clip(b, -3, 3)
+        got, ref, bound = run_gemm(oracle, a, b, fa, M, N, K, fb=fb)
+        exact = oracle.round_f32(ref).astype(np.float64)
+        assert np.array_equal(got, exact), (fa, fb, M, N, np.argwhere(got != exact)[:5])
+
+
+@pytest.mark.parametrize("fa,fb", MIXED_PAIRS)
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_mixed_tolerance(oracle, fa, fb, out_dtype):
+    rng = np.random.default_rng(17)
+    for (M, N, K) in [(384, 768, 1024), (200, 300, 384)]:
+        a = (rng.standard_normal((M, K)) * np.exp2(rng.uniform(-4, 4, (M, 1)))).astype(np.float32)
+        b = rng.standard_t(3, size=(N, K)).astype(np.float32)
+        ldc = (N + 7) // 8 * 8 + 8          # padded pitch, a multiple of 16 bytes
+        got, ref, bound = run_gemm(oracle, a, b, fa, M, N, K, alpha=0.75, out_dtype=out_dtype, fb=fb, ldc=ldc)
+        check(got, ref, bound, out_dtype, (fa, fb, M, N, K))
 
 
 @pytest.mark.parametrize("fmt", ["e4m3", "e5m2", "e2m1"])
