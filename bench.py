@@ -50,12 +50,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # value; after any change to them it reads null until captured again.
 _CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
 MEASURED_TRAFFIC = {
-    "cast_rows": (("mx_cast.cu", "mx_device.cuh"),
+    "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
                   "2945c1c69bfdd1d635ce3c858285c2e7ce575a4cf32893e82efaa70c3b62b1ee",
                   {"e4m3_bf16_8192x8192": 173593856, "e5m2_bf16_8192x8192": 169520640,
                    "e2m3_bf16_8192x8192": 158908160, "e3m2_bf16_8192x8192": 158370304,
                    "e2m1_bf16_8192x8192": 148999168, "int8_bf16_8192x8192": 168584448}),
-    "gemm": (("mx_gemm.cu",),
+    "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
              "a1e2301352c6b982eeed9652400e2fd06a30fb8561f62a85ebfd3c3cd250c045",
              {"e2m1_8192x6144x4096": 80179456, "e2m1_8192x14336x4096": 227883264,
               "e2m1_8192x4096x14336": 302555392, "e4m3_8192x3072x768": 9484800,
@@ -487,6 +487,37 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
             per_shape[k]["traffic"] = t_shape[k]
     kern_ms = sum(a.elapsed_time(b) for (_, a, b) in evs)
     achieved = flops_step * args.steps / (kern_ms * 1e-3) / 1e12
+    # the same GEMMs with C quantized in the epilogue (to the operand format, along
+    # N: the next layer's A operand) against the GEMM followed by a row cast of C
+    fused = {}
+    q_steps = max(3, min(args.steps, 20))
+    for (M, N, K, ac, as_, bc, bs, c) in ops:
+        qc = torch.empty((M, mx.codes_row_bytes(fmt, N)), dtype=torch.uint8, device=dev)
+        qs = torch.empty(mx.scales_bytes("mma", M, N), dtype=torch.uint8, device=dev)
+        res = {}
+        for label in ("gemm_then_cast", "fused"):
+            def once():
+                if label == "fused":
+                    mx.gemm_quantize(ac, as_, bc, bs, M, N, K, fa=fmt, out_fmt=fmt, out=(qc, qs))
+                else:
+                    mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
+                    mx.quantize(c, 1, fmt, codes=qc, scales=qs)
+            for _ in range(args.warmup):
+                once()
+            torch.cuda.synchronize()
+            barrier()
+            q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            q0.record(stream)
+            for _ in range(q_steps):
+                once()
+            q1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            res[label] = max_over_ranks(1e3 * q0.elapsed_time(q1) / q_steps)
+            launches += q_steps * (1 if label == "fused" else 2)
+        fused[f"{M}x{N}x{K}"] = {"gemm_then_cast_us": round(res["gemm_then_cast"], 1),
+                                 "fused_us": round(res["fused"], 1),
+                                 "speedup": round(res["gemm_then_cast"] / res["fused"], 3)}
     ratio = 4.0 if fmt == "e2m1" else 2.0             # nominal fp4 : fp8 : bf16 = 9 : 4.5 : 2.25
     peak = ratio * float(peaks["bf16_tflops"])
     if fmt == "e2m1":
@@ -502,6 +533,7 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
                          "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peak_kind} bf16 burst x {ratio:g} (nominal ratio for the operand type)",
                          "traffic": traffic, "per_shape": per_shape},
+            "quantizing_epilogue": fused,
             "_launches": launches}
 
 

@@ -227,6 +227,32 @@ MX_API int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
             void *c, mx_dtype cdt, int64_t ldc, void *workspace, size_t ws_bytes,
             void *stream);
 
+/*
+ * mx_gemm_quantize -- C = alpha * A * B^T as mx_gemm computes it, written
+ * directly as MX codes and scales of C quantized along its rows (blocks of 32
+ * consecutive columns), the layout the next GEMM reads as its A operand.  The
+ * FP4-pretraining abstract's principle of a producer that writes the layout
+ * its consumer reads, applied to the GEMM epilogue; the quantization is
+ * Algorithm 1 (section 3) on the fp32 values fl32(alpha * acc), acc being the
+ * GEMM's fp32 accumulator, so the result is the bytes mx_quantize(block_axis
+ * 1) would write for the fp32 C that mx_gemm returns.
+ *
+ *  a_codes ... alpha   as for mx_gemm (same formats, K % 128 == 0).
+ *  out_fmt    element format of C's codes (any mx_fmt, MX_INT8 included).
+ *  out_rnd, out_seed   RNE, or SR with C's element index m * N + n.
+ *  out_codes  device, M x (N * bits / 8) bytes, 16-byte aligned.
+ *  out_scales device, mx_scales_bytes(out_sl, M, N) bytes.
+ *  N must be a multiple of 32 (MX_ERR_SHAPE).  With K == 0, C = 0: all codes
+ *  and every byte of the scale buffer (padding included) are set to zero.
+ * Errors: as mx_gemm, plus MX_ERR_SR_RANGE; a bounded-wait expiry is reported
+ * by mx_last_device_status.
+ */
+MX_API int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa,
+                            const void *b_codes, const void *b_scales, mx_fmt fb,
+                            int64_t M, int64_t N, int64_t K, float alpha,
+                            mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
+                            void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream);
+
 /* Byte sizes of the buffers above (0 for invalid arguments). */
 MX_API size_t mx_codes_bytes(mx_fmt fmt, int64_t outer, int64_t inner);
 MX_API size_t mx_scales_bytes(mx_scale_layout sl, int64_t outer, int64_t inner);

@@ -156,6 +156,41 @@ int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_scale_la
     return mx_launch_dequantize(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Checks shared by mx_gemm and mx_gemm_quantize on the operands; MX_OK to go on.
+int check_gemm_operands(const void *a_codes, const void *a_scales, mx_fmt fa, const void *b_codes,
+                        const void *b_scales, mx_fmt fb, int64_t K) {
+    if (K > 0 && (!a_codes || !a_scales || !b_codes || !b_scales)) return MX_ERR_ARG;
+    if (fa == MX_INT8 || fb == MX_INT8) return MX_ERR_UNSUPPORTED;   // no block-scaled INT8 MMA
+    if (K % 128 != 0) return MX_ERR_UNSUPPORTED;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales))
+        return MX_ERR_ALIGN;
+    // FP6 codes, and FP4 codes outside the E2M1 x E2M1 (K % 256 == 0) case, are
+    // read through packed tensor maps, which need 32-byte aligned bases
+    const bool mxf4 = fa == MX_E2M1 && fb == MX_E2M1 && K % 256 == 0;
+    if (!mxf4 && ((elem_bits(fa) < 8 && !aligned32(a_codes)) || (elem_bits(fb) < 8 && !aligned32(b_codes))))
+        return MX_ERR_ALIGN;
+    return MX_OK;
+}
+
+MxGemmArgs gemm_args(const void *a_codes, const void *a_scales, mx_fmt fa, const void *b_codes,
+                     const void *b_scales, mx_fmt fb, int64_t M, int64_t N, int64_t K, float alpha) {
+    MxGemmArgs a;
+    a.a_codes = a_codes; a.a_scales = a_scales; a.b_codes = b_codes; a.b_scales = b_scales;
+    a.fa = fa; a.fb = fb; a.M = M; a.N = N; a.K = K; a.alpha = alpha;
+    a.c = nullptr; a.cdt = MX_F32; a.ldc = 0;
+    a.q_codes = nullptr; a.q_scales = nullptr; a.q_fmt = 0; a.q_rnd = MX_RNE; a.q_sl = MX_SCALES_MMA; a.q_seed = 0;
+    a.num_sms = 0; a.device = 0;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
 int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
             const void *b_codes, const void *b_scales, mx_fmt fb,
             int64_t M, int64_t N, int64_t K, float alpha,
@@ -167,26 +202,49 @@ int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
     if (K % 32 != 0) return MX_ERR_SHAPE;
     if (M == 0 || N == 0) return MX_OK;                  // empty: pointers may be NULL
     if (!c || ldc < N) return MX_ERR_ARG;
-    if (K > 0 && (!a_codes || !a_scales || !b_codes || !b_scales)) return MX_ERR_ARG;
-    if (fa == MX_INT8 || fb == MX_INT8) return MX_ERR_UNSUPPORTED;   // no block-scaled INT8 MMA
-    if (K % 128 != 0) return MX_ERR_UNSUPPORTED;
-    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
-        !aligned16(c) || (ldc * dtype_bytes(cdt)) % 16 != 0)
-        return MX_ERR_ALIGN;
-    // FP6 codes, and FP4 codes outside the E2M1 x E2M1 (K % 256 == 0) case, are
-    // read through packed tensor maps, which need 32-byte aligned bases
-    const bool mxf4 = fa == MX_E2M1 && fb == MX_E2M1 && K % 256 == 0;
-    if (!mxf4 && ((elem_bits(fa) < 8 && !aligned32(a_codes)) || (elem_bits(fb) < 8 && !aligned32(b_codes))))
-        return MX_ERR_ALIGN;
+    const int rc = check_gemm_operands(a_codes, a_scales, fa, b_codes, b_scales, fb, K);
+    if (rc != MX_OK) return rc;
+    if (!aligned16(c) || (ldc * dtype_bytes(cdt)) % 16 != 0) return MX_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (K == 0) {
         const size_t esz = static_cast<size_t>(dtype_bytes(cdt));
         return cudaMemset2DAsync(c, ldc * esz, 0, N * esz, M, st) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
     }
-    MxGemmArgs a;
-    a.a_codes = a_codes; a.a_scales = a_scales; a.b_codes = b_codes; a.b_scales = b_scales;
-    a.fa = fa; a.fb = fb; a.M = M; a.N = N; a.K = K; a.alpha = alpha;
+    MxGemmArgs a = gemm_args(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha);
     a.c = c; a.cdt = cdt; a.ldc = ldc;
+    a.num_sms = sm_count(&a.device);
+    if (a.num_sms <= 0) return MX_ERR_CUDA;
+    return mx_launch_gemm(a, st);
+}
+
+int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa,
+                     const void *b_codes, const void *b_scales, mx_fmt fb,
+                     int64_t M, int64_t N, int64_t K, float alpha,
+                     mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
+                     void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream) {
+    if (elem_bits(fa) == 0 || elem_bits(fb) == 0 || elem_bits(out_fmt) == 0) return MX_ERR_ARG;
+    if ((out_rnd != MX_RNE && out_rnd != MX_SR) || (out_sl != MX_SCALES_PLAIN && out_sl != MX_SCALES_MMA))
+        return MX_ERR_ARG;
+    if (M < 0 || N < 0 || K < 0) return MX_ERR_ARG;
+    if (K % 32 != 0 || N % 32 != 0) return MX_ERR_SHAPE;  // C's blocks run along N
+    if (M == 0 || N == 0) return MX_OK;                   // empty: pointers may be NULL
+    if (!out_codes || !out_scales) return MX_ERR_ARG;
+    const int rc = check_gemm_operands(a_codes, a_scales, fa, b_codes, b_scales, fb, K);
+    if (rc != MX_OK) return rc;
+    if (!aligned16(out_codes)) return MX_ERR_ALIGN;
+    if (out_rnd == MX_SR && static_cast<uint64_t>(M) * static_cast<uint64_t>(N) > (1ull << 34))
+        return MX_ERR_SR_RANGE;
+    const size_t sbytes = mx_scales_bytes(out_sl, M, N);
+    if (sbytes >= (1ull << 32)) return MX_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) {
+        // C = 0: every block is all zero (code 0, scale code 0)
+        if (cudaMemsetAsync(out_codes, 0, mx_codes_bytes(out_fmt, M, N), st) != cudaSuccess) return MX_ERR_CUDA;
+        return cudaMemsetAsync(out_scales, 0, sbytes, st) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+    }
+    MxGemmArgs a = gemm_args(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha);
+    a.q_codes = out_codes; a.q_scales = out_scales; a.q_fmt = out_fmt; a.q_rnd = out_rnd; a.q_sl = out_sl;
+    a.q_seed = out_seed;
     a.num_sms = sm_count(&a.device);
     if (a.num_sms <= 0) return MX_ERR_CUDA;
     return mx_launch_gemm(a, st);

@@ -18,6 +18,7 @@
 
 #include "mx.h"
 #include "mx_device.cuh"
+#include "mx_encode.cuh"
 #include "mx_internal.h"
 
 namespace mxk {
@@ -40,22 +41,6 @@ __device__ __forceinline__ void store_scale(const CastParams &p, int64_t o, int6
     const uint32_t off = p.mma_scales ? mma_scale_offset32(oo, k, static_cast<uint32_t>(p.k_groups))
                                       : oo * static_cast<uint32_t>(p.k_blocks) + k;
     p.scales[off] = static_cast<uint8_t>(s);
-}
-
-// Encode n (even) scaled values u[] to codes; sign is carried by u.
-template <int FMT, bool SR>
-__device__ __forceinline__ void encode_values(float *u, int n, const uint32_t *rnd_words, uint32_t *pairs) {
-#pragma unroll
-    for (int j = 0; j < n; j += 2) {
-        float a = u[j], b = u[j + 1];
-        if (SR) {
-            uint32_t ra = (rnd_words[j >> 2] >> (8 * (j & 3))) & 255u;
-            uint32_t rb = (rnd_words[(j + 1) >> 2] >> (8 * ((j + 1) & 3))) & 255u;
-            a = copysignf(sr_magnitude<FMT>(fabsf(a), ra), a);
-            b = copysignf(sr_magnitude<FMT>(fabsf(b), rb), b);
-        }
-        pairs[j >> 1] = cvt_pair<FMT>(a, b);
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -106,129 +91,23 @@ __device__ __forceinline__ void load_block(const CastParams &p, const ChunkPos &
     }
 }
 
-__device__ __forceinline__ uint64_t f2_mul_ftz(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
+// The row cast's blocks go to the shared 32-block encoder (mx_encode.cuh).
+__device__ __forceinline__ BlockSink row_sink(const CastParams &p) {
+    BlockSink o;
+    o.codes = p.codes;
+    o.scales = p.scales;
+    o.inner = p.cols;
+    o.k_blocks = static_cast<uint32_t>(p.k_blocks);
+    o.k_groups = static_cast<uint32_t>(p.k_groups);
+    o.mma_scales = p.mma_scales;
+    o.key = p.key;
+    return o;
 }
 
-// 32 code bytes of one block: one 32-byte store when the buffers are 32-byte
-// aligned (V32), else two 16-byte stores
-template <bool V32>
-__device__ __forceinline__ void store_code32(uint8_t *dst, const uint4 &a, const uint4 &b) {
-    if (V32) {
-        asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-                     ::"l"(dst), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
-                     : "memory");
-    } else {
-        reinterpret_cast<uint4 *>(dst)[0] = a;
-        reinterpret_cast<uint4 *>(dst)[1] = b;
-    }
-}
-
-// Encode one 32-block along a row from its values as FP32 bit patterns:
-// block amax -> E8M0 exponent, V * 2^-e (flushing FP32 subnormals), RNE or
-// stochastic rounding, and the packed codes and scale byte of (row, kb).
-// `codes_row` is the start of the row's codes.  SR's index is the element's
-// position row * cols + kb * 32 + j in the output.
 template <int FMT, bool SR, bool V32>
 __device__ __forceinline__ void encode_row_block(const CastParams &p, int64_t row, int64_t kb, uint32_t (&b)[32]) {
-    constexpr int BITS = Fmt<FMT>::bits;
-    uint32_t amax_bits = 0;
-#pragma unroll
-    for (int i = 0; i < 32; i += 2)
-        amax_bits = __vimax3_u32(amax_bits, b[i] & 0x7fffffffu, b[i + 1] & 0x7fffffffu);
-    const bool nan_block = amax_bits >= 0x7f800000u;
-    const int e = block_exponent<FMT>(amax_bits);
-
-    // V * 2^-e with the subnormal flush (mul.ftz), two values per instruction
-    float u[32];
-    if (FMT == MX_INT8 && !SR && e >= -120 && e <= 120) {
-        // INT8 codes are round(V * 2^(6 - e)) clamped to +-127: fold the 2^6 into
-        // the (exact) power-of-two scale, clamp, round half to even
-        const uint32_t f = __float_as_uint(pow2f(6 - e));
-        const uint64_t ff = static_cast<uint64_t>(f) | (static_cast<uint64_t>(f) << 32);
-        uint32_t c[8];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-            const uint64_t r = f2_mul_ftz(static_cast<uint64_t>(b[i]) | (static_cast<uint64_t>(b[i + 1]) << 32), ff);
-            const float x0 = fminf(fmaxf(__uint_as_float(static_cast<uint32_t>(r)), -127.0f), 127.0f);
-            const float x1 = fminf(fmaxf(__uint_as_float(static_cast<uint32_t>(r >> 32)), -127.0f), 127.0f);
-            const uint32_t q0 = static_cast<uint32_t>(__float2int_rn(x0)) & 0xffu;
-            const uint32_t q1 = static_cast<uint32_t>(__float2int_rn(x1)) & 0xffu;
-            if ((i & 2) == 0) c[i >> 2] = q0 | (q1 << 8);
-            else c[i >> 2] |= (q0 << 16) | (q1 << 24);
-        }
-        if (nan_block) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) c[i] = 0u;
-        }
-        store_code32<V32>(p.codes + row * p.cols + kb * 32, make_uint4(c[0], c[1], c[2], c[3]),
-                          make_uint4(c[4], c[5], c[6], c[7]));
-        store_scale(p, row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
-        return;
-    }
-    if (Fmt<FMT>::emax == 0) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) u[i] = scale_down<FMT>(__uint_as_float(b[i]), e);
-    } else {
-        const uint32_t f = __float_as_uint(pow2f(-e));
-        const uint64_t ff = static_cast<uint64_t>(f) | (static_cast<uint64_t>(f) << 32);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-            const uint64_t r = f2_mul_ftz(static_cast<uint64_t>(b[i]) | (static_cast<uint64_t>(b[i + 1]) << 32), ff);
-            u[i] = __uint_as_float(static_cast<uint32_t>(r));
-            u[i + 1] = __uint_as_float(static_cast<uint32_t>(r >> 32));
-        }
-    }
-    if (SR) {
-        const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(row * p.cols + kb * 32) >> 2);
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            const uint32_t rw = fmix32((g + w) ^ p.key);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int j = 4 * w + k;
-                u[j] = copysignf(sr_magnitude_int<FMT>(fabsf(u[j]), (rw >> (8 * k)) & 255u), u[j]);
-            }
-        }
-    }
-    uint32_t c[16];
-#pragma unroll
-    for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(u[j], u[j + 1]);
-    if (nan_block) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) c[i] = 0u;
-    }
-    uint8_t *dst = p.codes + row * (p.cols * BITS / 8) + kb * (32 * BITS / 8);
-    if (BITS == 8) {
-        const uint4 lo = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
-        const uint4 hi = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16),
-                                    c[14] | (c[15] << 16));
-        store_code32<V32>(dst, lo, hi);
-    } else if (BITS == 4) {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) w[i] = c[4 * i] | (c[4 * i + 1] << 8) | (c[4 * i + 2] << 16) | (c[4 * i + 3] << 24);
-        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-        uint64_t *d = reinterpret_cast<uint64_t *>(dst);     // 24 bytes, 8-byte aligned
-#pragma unroll
-        for (int q = 0; q < 3; ++q) {
-            uint64_t w = 0;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int bit = 6 * j - 64 * q;
-                const uint64_t code = (c[j >> 1] >> (8 * (j & 1))) & 0x3fu;
-                if (bit >= 0 && bit < 64) w |= code << bit;
-                else if (bit < 0 && bit > -6) w |= code >> (-bit);
-            }
-            d[q] = w;
-        }
-    }
-    store_scale(p, row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+    encode_block32<FMT, SR, V32>(row_sink(p), row, kb, b);
 }
-
 
 template <int FMT, bool SR, bool BF16_IN, bool V32>
 __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &cp, int64_t blocks_per_row,

@@ -1,0 +1,156 @@
+// mx_encode.cuh -- the 32-block encoder shared by the row cast, the dual cast
+// and the quantizing GEMM epilogue.
+#pragma once
+
+#include <cstdint>
+
+#include "mx_device.cuh"
+
+namespace mxk {
+
+// Where the encoded blocks of a row-major tensor go: `inner` elements per row,
+// codes packed with no padding (row pitch inner * bits / 8 bytes), one E8M0
+// scale per block in the plain (row-major) or MMA layout.
+struct BlockSink {
+    uint8_t *codes;
+    uint8_t *scales;
+    int64_t inner;
+    uint32_t k_blocks;   // inner / 32
+    uint32_t k_groups;   // ceil(k_blocks / 4), MMA layout
+    int mma_scales;
+    uint32_t key;        // stochastic-rounding seed key
+};
+
+__device__ __forceinline__ void sink_scale(const BlockSink &o, int64_t row, int64_t kb, uint32_t s) {
+    // scale buffers are far below 4 GiB: offsets in 32-bit arithmetic
+    const uint32_t r = static_cast<uint32_t>(row), k = static_cast<uint32_t>(kb);
+    const uint32_t off = o.mma_scales ? mma_scale_offset32(r, k, o.k_groups) : r * o.k_blocks + k;
+    o.scales[off] = static_cast<uint8_t>(s);
+}
+
+__device__ __forceinline__ uint64_t f2_mul_ftz(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 32 code bytes of one block: one 32-byte store when the buffers are 32-byte
+// aligned (V32), else two 16-byte stores
+template <bool V32>
+__device__ __forceinline__ void store_code32(uint8_t *dst, const uint4 &a, const uint4 &b) {
+    if (V32) {
+        asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                     ::"l"(dst), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                     : "memory");
+    } else {
+        reinterpret_cast<uint4 *>(dst)[0] = a;
+        reinterpret_cast<uint4 *>(dst)[1] = b;
+    }
+}
+
+// Encode one 32-block along a row from its values as FP32 bit patterns
+// (Algorithm 1 of the MX summary page, section 3): block amax -> E8M0
+// exponent, V * 2^-e (flushing FP32 subnormals), RNE or stochastic rounding,
+// and the packed codes and scale byte of block (row, kb).  SR's index is the
+// element's position row * inner + kb * 32 + j in the output.
+template <int FMT, bool SR, bool V32>
+__device__ __forceinline__ void encode_block32(const BlockSink &o, int64_t row, int64_t kb, uint32_t (&b)[32]) {
+    constexpr int BITS = Fmt<FMT>::bits;
+    uint32_t amax_bits = 0;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2)
+        amax_bits = __vimax3_u32(amax_bits, b[i] & 0x7fffffffu, b[i + 1] & 0x7fffffffu);
+    const bool nan_block = amax_bits >= 0x7f800000u;
+    const int e = block_exponent<FMT>(amax_bits);
+
+    // V * 2^-e with the subnormal flush (mul.ftz), two values per instruction
+    float u[32];
+    if (FMT == MX_INT8 && !SR && e >= -120 && e <= 120) {
+        // INT8 codes are round(V * 2^(6 - e)) clamped to +-127: fold the 2^6 into
+        // the (exact) power-of-two scale, clamp, round half to even
+        const uint32_t f = __float_as_uint(pow2f(6 - e));
+        const uint64_t ff = static_cast<uint64_t>(f) | (static_cast<uint64_t>(f) << 32);
+        uint32_t c[8];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const uint64_t r = f2_mul_ftz(static_cast<uint64_t>(b[i]) | (static_cast<uint64_t>(b[i + 1]) << 32), ff);
+            const float x0 = fminf(fmaxf(__uint_as_float(static_cast<uint32_t>(r)), -127.0f), 127.0f);
+            const float x1 = fminf(fmaxf(__uint_as_float(static_cast<uint32_t>(r >> 32)), -127.0f), 127.0f);
+            const uint32_t q0 = static_cast<uint32_t>(__float2int_rn(x0)) & 0xffu;
+            const uint32_t q1 = static_cast<uint32_t>(__float2int_rn(x1)) & 0xffu;
+            if ((i & 2) == 0) c[i >> 2] = q0 | (q1 << 8);
+            else c[i >> 2] |= (q0 << 16) | (q1 << 24);
+        }
+        if (nan_block) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) c[i] = 0u;
+        }
+        store_code32<V32>(o.codes + row * o.inner + kb * 32, make_uint4(c[0], c[1], c[2], c[3]),
+                          make_uint4(c[4], c[5], c[6], c[7]));
+        sink_scale(o, row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+        return;
+    }
+    if (Fmt<FMT>::emax == 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) u[i] = scale_down<FMT>(__uint_as_float(b[i]), e);
+    } else {
+        const uint32_t f = __float_as_uint(pow2f(-e));
+        const uint64_t ff = static_cast<uint64_t>(f) | (static_cast<uint64_t>(f) << 32);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const uint64_t r = f2_mul_ftz(static_cast<uint64_t>(b[i]) | (static_cast<uint64_t>(b[i + 1]) << 32), ff);
+            u[i] = __uint_as_float(static_cast<uint32_t>(r));
+            u[i + 1] = __uint_as_float(static_cast<uint32_t>(r >> 32));
+        }
+    }
+    if (SR) {
+        const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(row * o.inner + kb * 32) >> 2);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const uint32_t rw = fmix32((g + w) ^ o.key);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = 4 * w + k;
+                u[j] = copysignf(sr_magnitude_int<FMT>(fabsf(u[j]), (rw >> (8 * k)) & 255u), u[j]);
+            }
+        }
+    }
+    uint32_t c[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(u[j], u[j + 1]);
+    if (nan_block) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) c[i] = 0u;
+    }
+    uint8_t *dst = o.codes + row * (o.inner * BITS / 8) + kb * (32 * BITS / 8);
+    if (BITS == 8) {
+        const uint4 lo = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+        const uint4 hi = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16),
+                                    c[14] | (c[15] << 16));
+        store_code32<V32>(dst, lo, hi);
+    } else if (BITS == 4) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = c[4 * i] | (c[4 * i + 1] << 8) | (c[4 * i + 2] << 16) | (c[4 * i + 3] << 24);
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+        uint64_t *d = reinterpret_cast<uint64_t *>(dst);     // 24 bytes, 8-byte aligned
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+            uint64_t w = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int bit = 6 * j - 64 * q;
+                const uint64_t code = (c[j >> 1] >> (8 * (j & 1))) & 0x3fu;
+                if (bit >= 0 && bit < 64) w |= code << bit;
+                else if (bit < 0 && bit > -6) w |= code >> (-bit);
+            }
+            d[q] = w;
+        }
+    }
+    sink_scale(o, row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+}
+
+
+
+}  // namespace mxk

@@ -34,6 +34,7 @@
 
 #include "mx.h"
 #include "mx_debug.h"
+#include "mx_encode.cuh"
 #include "mx_internal.h"
 
 // Device status word: kernels that give up a bounded wait record MX_ERR_TIMEOUT here.
@@ -80,6 +81,19 @@ struct Smem {
 };
 constexpr int SMEM_BYTES = Smem::TOTAL + 1024;   // slack for 1024-byte alignment
 
+// Output of the epilogue: C in fp32 or bf16, or C quantized along its rows
+// (blocks of 32 consecutive columns) to MX codes and E8M0 scales.
+constexpr int OUT_F32 = 0, OUT_BF16 = 1, OUT_MX = 2;
+
+struct MxOut {
+    uint8_t *codes;      // M x (N * bits / 8) bytes
+    uint8_t *scales;     // plain or MMA layout for (M, N)
+    int fmt;             // element format
+    int sr;              // stochastic rounding (else RNE)
+    int mma;             // MMA scale layout (else plain)
+    uint32_t key;        // stochastic-rounding seed key
+};
+
 struct Params {
     const uint8_t *a_scales;
     const uint8_t *b_scales;
@@ -93,6 +107,7 @@ struct Params {
     uint32_t idesc;  // instruction descriptor without the scale-factor ids
     uint32_t ab_tx;  // bytes the A and B loads of one stage deliver (packed size in global)
     int skip_k_tile; // testing hook: CTA 0 withholds this k-tile of its first tile (-1: off)
+    MxOut q;         // OUT_MX only
 };
 
 // ------------------------------------------------------------------------
@@ -226,46 +241,84 @@ __device__ __forceinline__ void tmem_ld_x32_nowait(uint32_t taddr, uint32_t *r) 
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// alpha * (32 consecutive accumulator values of row m), quantized as one MX
+// block of C's row: the block (m, n0 / 32) of mx_quantize along the rows of
+// an M x N tensor holding fl32(alpha * acc).  N is a multiple of 32, so a
+// chunk that starts inside C lies wholly inside it.
+template <int FMT>
+__device__ __forceinline__ void quantize_chunk_fmt(const mxk::BlockSink &o, int m, int kb, uint32_t (&b)[32], bool sr) {
+    if (sr) mxk::encode_block32<FMT, true, false>(o, m, kb, b);
+    else mxk::encode_block32<FMT, false, false>(o, m, kb, b);
+}
+
+__device__ __forceinline__ void quantize_chunk(const Params &p, int m, int n0, const uint32_t *r) {
+    uint32_t b[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) b[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), p.alpha));
+    mxk::BlockSink o;
+    o.codes = p.q.codes;
+    o.scales = p.q.scales;
+    o.inner = p.N;
+    o.k_blocks = static_cast<uint32_t>(p.N) >> 5;
+    o.k_groups = (o.k_blocks + 3) >> 2;
+    o.mma_scales = p.q.mma;
+    o.key = p.q.key;
+    const int kb = n0 >> 5;
+    const bool sr = p.q.sr != 0;
+    switch (p.q.fmt) {
+        case MX_E4M3: quantize_chunk_fmt<MX_E4M3>(o, m, kb, b, sr); break;
+        case MX_E5M2: quantize_chunk_fmt<MX_E5M2>(o, m, kb, b, sr); break;
+        case MX_E2M3: quantize_chunk_fmt<MX_E2M3>(o, m, kb, b, sr); break;
+        case MX_E3M2: quantize_chunk_fmt<MX_E3M2>(o, m, kb, b, sr); break;
+        case MX_E2M1: quantize_chunk_fmt<MX_E2M1>(o, m, kb, b, sr); break;
+        default: quantize_chunk_fmt<MX_INT8>(o, m, kb, b, sr); break;
+    }
+}
+
 // 32 consecutive accumulator values of one row -> C (bounds-checked).
-template <bool BF16_OUT>
-__device__ __forceinline__ void store_row_chunk(const Params &p, int m, int n0, const uint32_t *r) {
+template <int OUT>
+__device__ __forceinline__ void store_chunk(const Params &p, int m, int n0, const uint32_t *r) {
     if (m >= p.M || n0 >= p.N) return;
-    float v[32];
+    if constexpr (OUT == OUT_MX) {
+        quantize_chunk(p, m, n0, r);
+    } else {
+        float v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), p.alpha);
-    if (BF16_OUT) {
-        __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
-        if (n0 + 32 <= p.N) {
+        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), p.alpha);
+        if (OUT == OUT_BF16) {
+            __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
+            if (n0 + 32 <= p.N) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-                uint32_t w[4];
+                for (int i = 0; i < 32; i += 8) {
+                    uint32_t w[4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * t], v[i + 2 * t + 1]);
-                    w[t] = *reinterpret_cast<uint32_t *>(&b2);
+                    for (int t = 0; t < 4; ++t) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * t], v[i + 2 * t + 1]);
+                        w[t] = *reinterpret_cast<uint32_t *>(&b2);
+                    }
+                    *reinterpret_cast<uint4 *>(row + i) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
-                *reinterpret_cast<uint4 *>(row + i) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (n0 + i < p.N) row[i] = __float2bfloat16_rn(v[i]);
             }
         } else {
+            float *row = static_cast<float *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
+            if (n0 + 32 <= p.N) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (n0 + i < p.N) row[i] = __float2bfloat16_rn(v[i]);
-        }
-    } else {
-        float *row = static_cast<float *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
-        if (n0 + 32 <= p.N) {
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (n0 + i < p.N) row[i] = v[i];
+                for (int i = 0; i < 32; ++i)
+                    if (n0 + i < p.N) row[i] = v[i];
+            }
         }
     }
 }
 
-template <bool FP4, bool BF16_OUT>
+template <bool FP4, int OUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, Params p) {
     using C = Cfg<FP4>;
@@ -444,7 +497,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             if (lane == 0) mbar_arrive(acc_empty(b));
             const int n_base = tn * BN + c0;
 #pragma unroll
-            for (int j = 0; j < 3; ++j) store_row_chunk<BF16_OUT>(p, m, n_base + 32 * j, r + 32 * j);
+            for (int j = 0; j < 3; ++j) store_chunk<OUT>(p, m, n_base + 32 * j, r + 32 * j);
         }
     }
 
@@ -512,6 +565,7 @@ struct PairParams {
     uint32_t idesc;
     uint32_t ab_tx;            // bytes one CTA's A and B loads of a stage deliver
     int skip_k_tile;
+    MxOut q;                   // OUT_MX only
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -565,7 +619,7 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
     }
 }
 
-template <bool FP4, bool BF16_OUT>
+template <bool FP4, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                     const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
@@ -731,9 +785,9 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             if (lane == 0) mbar_arrive_cluster(map_to_rank(acc_empty(b), 0));
             const int n_base = tn * PAIR_BN + c0;
             Params pp;
-            pp.c = p.c; pp.ldc = p.ldc; pp.M = p.M; pp.N = p.N; pp.alpha = p.alpha;
+            pp.c = p.c; pp.ldc = p.ldc; pp.M = p.M; pp.N = p.N; pp.alpha = p.alpha; pp.q = p.q;
 #pragma unroll
-            for (int j = 0; j < NCH; ++j) store_row_chunk<BF16_OUT>(pp, m, n_base + 32 * j, r + 32 * j);
+            for (int j = 0; j < NCH; ++j) store_chunk<OUT>(pp, m, n_base + 32 * j, r + 32 * j);
         }
     }
 
@@ -834,10 +888,10 @@ uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN) {
     return d;
 }
 
-template <bool FP4, bool BF16_OUT>
+template <bool FP4, int OUT>
 cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
                         const CUtensorMap &tsb, const PairParams &p, int grid, cudaStream_t st) {
-    auto kern = mx_gemm_pair_kernel<FP4, BF16_OUT>;
+    auto kern = mx_gemm_pair_kernel<FP4, OUT>;
     static bool configured = false;   // per instantiation
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg<FP4>::SMEM);
@@ -848,9 +902,9 @@ cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
     return cudaGetLastError();
 }
 
-template <bool FP4, bool BF16_OUT>
+template <bool FP4, int OUT>
 cudaError_t launch(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int grid, cudaStream_t st) {
-    auto kern = mx_gemm_kernel<FP4, BF16_OUT>;
+    auto kern = mx_gemm_kernel<FP4, OUT>;
     static bool configured = false;   // per instantiation; attribute setting is idempotent
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -859,6 +913,37 @@ cudaError_t launch(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p
     }
     kern<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, p);
     return cudaGetLastError();
+}
+
+template <bool FP4>
+cudaError_t launch_pair_out(int out, const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
+                            const CUtensorMap &tsb, const PairParams &p, int grid, cudaStream_t st) {
+    if (out == OUT_MX) return launch_pair<FP4, OUT_MX>(ta, tb, tsa, tsb, p, grid, st);
+    if (out == OUT_BF16) return launch_pair<FP4, OUT_BF16>(ta, tb, tsa, tsb, p, grid, st);
+    return launch_pair<FP4, OUT_F32>(ta, tb, tsa, tsb, p, grid, st);
+}
+
+template <bool FP4>
+cudaError_t launch_out(int out, const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int grid,
+                       cudaStream_t st) {
+    if (out == OUT_MX) return launch<FP4, OUT_MX>(ta, tb, p, grid, st);
+    if (out == OUT_BF16) return launch<FP4, OUT_BF16>(ta, tb, p, grid, st);
+    return launch<FP4, OUT_F32>(ta, tb, p, grid, st);
+}
+
+int out_mode(const MxGemmArgs &a) {
+    return a.q_codes ? OUT_MX : (a.cdt == MX_BF16 ? OUT_BF16 : OUT_F32);
+}
+
+MxOut mx_out(const MxGemmArgs &a) {
+    MxOut q;
+    q.codes = static_cast<uint8_t *>(a.q_codes);
+    q.scales = static_cast<uint8_t *>(a.q_scales);
+    q.fmt = a.q_fmt;
+    q.sr = a.q_rnd == MX_SR;
+    q.mma = a.q_sl == MX_SCALES_MMA;
+    q.key = fmix32_host(static_cast<uint32_t>(a.q_seed)) ^ static_cast<uint32_t>(a.q_seed >> 32);
+    return q;
 }
 
 }  // namespace mxg
@@ -913,9 +998,10 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     const int clusters = tiles < a.num_sms / 2 ? tiles : a.num_sms / 2;
     const int grid = 2 * (clusters < 1 ? 1 : clusters);
     cudaError_t e;
-    const bool bf = a.cdt == MX_BF16;
-    if (fp4) e = bf ? launch_pair<true, true>(ta, tb, tsa, tsb, p, grid, st) : launch_pair<true, false>(ta, tb, tsa, tsb, p, grid, st);
-    else e = bf ? launch_pair<false, true>(ta, tb, tsa, tsb, p, grid, st) : launch_pair<false, false>(ta, tb, tsa, tsb, p, grid, st);
+    p.q = mx_out(a);
+    const int out = out_mode(a);
+    if (fp4) e = launch_pair_out<true>(out, ta, tb, tsa, tsb, p, grid, st);
+    else e = launch_pair_out<false>(out, ta, tb, tsa, tsb, p, grid, st);
     return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
@@ -959,9 +1045,10 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < a.num_sms ? tiles : a.num_sms;
     cudaError_t e;
-    const bool bf = a.cdt == MX_BF16;
-    if (fp4) e = bf ? launch<true, true>(ta, tb, p, grid, st) : launch<true, false>(ta, tb, p, grid, st);
-    else e = bf ? launch<false, true>(ta, tb, p, grid, st) : launch<false, false>(ta, tb, p, grid, st);
+    p.q = mx_out(a);
+    const int out = out_mode(a);
+    if (fp4) e = launch_out<true>(out, ta, tb, p, grid, st);
+    else e = launch_out<false>(out, ta, tb, p, grid, st);
     return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 

@@ -58,6 +58,10 @@ struct MxGemmArgs {
     void *c;
     int cdt;
     int64_t ldc;
+    // quantized output (mx_gemm_quantize): q_codes non-NULL replaces c
+    void *q_codes, *q_scales;
+    int q_fmt, q_rnd, q_sl;
+    uint64_t q_seed;
     int num_sms;
     int device;
 };

@@ -69,6 +69,9 @@ def lib() -> ctypes.CDLL:
             L.mx_gemm.restype = i32
             L.mx_gemm.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, ctypes.c_float,
                                   vp, i32, i64, vp, ctypes.c_size_t, vp]
+            L.mx_gemm_quantize.restype = i32
+            L.mx_gemm_quantize.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, ctypes.c_float,
+                                           i32, i32, u64, vp, vp, i32, vp]
             L.mx_codes_bytes.restype = ctypes.c_size_t
             L.mx_codes_bytes.argtypes = [i32, i64, i64]
             L.mx_scales_bytes.restype = ctypes.c_size_t
@@ -208,6 +211,29 @@ def gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
                        out.data_ptr(), DTYPE[out.dtype], out.stride(0), None, 0, _stream(stream))
     _check(rc, "mx_gemm")
     return out
+
+
+def gemm_quantize(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
+                  b_scales: torch.Tensor, M: int, N: int, K: int, fa="e4m3", fb=None, alpha: float = 1.0,
+                  out_fmt="e4m3", rnd="rne", seed: int = 0, scale_layout="mma", out=None, stream=None):
+    """alpha * A * B^T quantized along its rows in the GEMM epilogue.
+
+    Returns (codes, scales): M x (N * bits / 8) codes and the scales of an
+    M x N tensor in `scale_layout`; `out` may supply both buffers."""
+    fb = fa if fb is None else fb
+    of = _fmt(out_fmt)
+    sl = _layout(scale_layout)
+    if out is None:
+        dev = a_codes.device
+        out = (torch.empty((M, codes_row_bytes(of, N)), dtype=torch.uint8, device=dev),
+               torch.empty(max(scales_bytes(sl, M, N), 1), dtype=torch.uint8, device=dev))
+    codes, scales = out
+    rc = lib().mx_gemm_quantize(a_codes.data_ptr(), a_scales.data_ptr(), _fmt(fa), b_codes.data_ptr(),
+                                b_scales.data_ptr(), _fmt(fb), M, N, K, float(alpha), of,
+                                ROUND[rnd] if isinstance(rnd, str) else int(rnd), seed & (2**64 - 1),
+                                codes.data_ptr(), scales.data_ptr(), sl, _stream(stream))
+    _check(rc, "mx_gemm_quantize")
+    return codes, scales
 
 
 def last_device_status(stream=None) -> int:

@@ -146,6 +146,28 @@ def test_gemm_validation(mx):
     assert _g(mx, ldc=129, cdt=1) == -2
 
 
+def _gq(mx, M=128, N=128, K=256, fa=0, fb=0, of=0, rnd=0, codes=16, scales=16, sl=1, a=16):
+    L = mx.lib()
+    return L.mx_gemm_quantize(a, 16, fa, 16, 16, fb, M, N, K, 1.0, of, rnd, 0, codes, scales, sl, None)
+
+
+def test_gemm_quantize_validation(mx):
+    assert _gq(mx, of=6) == -1
+    assert _gq(mx, rnd=5) == -1
+    assert _gq(mx, sl=2) == -1
+    assert _gq(mx, M=-1) == -1
+    assert _gq(mx, N=48) == -3                    # C's blocks run along N
+    assert _gq(mx, K=48) == -3
+    assert _gq(mx, M=0) == 0                      # empty
+    assert _gq(mx, codes=None) == -1
+    assert _gq(mx, a=None) == -1
+    assert _gq(mx, fa=5) == -4
+    assert _gq(mx, K=160) == -4
+    assert _gq(mx, codes=24) == -2
+    assert _gq(mx, fa=2, fb=2, a=48) == -2
+    assert _gq(mx, M=2 ** 20, N=2 ** 15, rnd=1) == -5
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     from microscaling_block_scaled_mx_b200 import mx as m
     monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
