@@ -1,17 +1,18 @@
 // mx_cast.cu -- MX cast (Algorithm 1 of "Microscaling Data Formats for Deep
 // Learning", summary page, section 3) and exact decode (section 2) on sm_100a.
 //
-// Both casts are HBM-bound streaming kernels: every input byte is read once
-// with 16-byte coalesced loads, every code and scale byte written once.
-//  * cast_rows: blocks run along the contiguous axis.  Four lanes cover one
-//    32-block (8 values each, one 16-byte bf16 load); the block amax is two
-//    xor-shuffles.  A warp walks a 256-element segment of one row.
-//  * cast_cols: blocks run down columns.  A CTA stages a 128-row x 64-column
-//    tile in shared memory with coalesced row loads; each thread then owns one
-//    column block of 32 values in registers, where the optional fixed-sign
-//    32-point Hadamard ("Format-Aware Fusion for Fast FP4 Pretraining",
-//    abstract) runs as five fp32 butterfly stages, and writes its codes as
-//    one row of the transposed (block-axis-major) output.
+// The casts are streaming kernels: every input byte is read once, every code
+// and scale byte written once.
+//  * cast_rows: blocks run along the contiguous axis.  One lane owns one
+//    32-block (two 32-byte loads for bf16); a warp covers 32 consecutive
+//    blocks of a row, with the next two chunks' loads in flight.
+//  * cast_cols: blocks run down columns.  A CTA stages 128 x 128 tiles in
+//    shared memory (double-buffered cp.async); each thread owns one column
+//    pair of a 32-row block, where the optional fixed-sign 32-point Hadamard
+//    ("Format-Aware Fusion for Fast FP4 Pretraining", abstract) runs as five
+//    packed fp32 butterfly stages, and writes its codes as rows of the
+//    transposed (block-axis-major) output.
+//  * cast_dual: both of the above from one staged tile.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
