@@ -51,15 +51,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
 MEASURED_TRAFFIC = {
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "2945c1c69bfdd1d635ce3c858285c2e7ce575a4cf32893e82efaa70c3b62b1ee",
-                  {"e4m3_bf16_8192x8192": 173593856, "e5m2_bf16_8192x8192": 169520640,
-                   "e2m3_bf16_8192x8192": 158908160, "e3m2_bf16_8192x8192": 158370304,
-                   "e2m1_bf16_8192x8192": 148999168, "int8_bf16_8192x8192": 168584448}),
+                  "d3da0717c96c2f95b5d4bec3117b455374bac6fe8ae02c782bf5d65fdc40c907",
+                  {"e4m3_bf16_8192x8192": 172882176, "e5m2_bf16_8192x8192": 169610752,
+                   "e2m3_bf16_8192x8192": 158393600, "e3m2_bf16_8192x8192": 158375680,
+                   "e2m1_bf16_8192x8192": 149267200, "int8_bf16_8192x8192": 168440320}),
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "a1e2301352c6b982eeed9652400e2fd06a30fb8561f62a85ebfd3c3cd250c045",
-             {"e2m1_8192x6144x4096": 80179456, "e2m1_8192x14336x4096": 227883264,
-              "e2m1_8192x4096x14336": 302555392, "e4m3_8192x3072x768": 9484800,
-              "e4m3_8192x768x3072": 28418560}),
+             "912b56beecdb017c926e0563b82a84398e53e5c31fc082fb7ff89a9ebc59f39b",
+             {"e2m1_8192x6144x4096": 78177792, "e2m1_8192x14336x4096": 227502336,
+              "e2m1_8192x4096x14336": 295097344, "e4m3_8192x3072x768": 9265664,
+              "e4m3_8192x768x3072": 28417536}),
 }
 
 
@@ -155,11 +155,12 @@ class ClockSampler:
 # reference arm: the CPU oracle on a bounded sample
 # ---------------------------------------------------------------------------
 
-def oracle_cast_sample(rows: int):
+def oracle_cast_sample(rows: int, x=None):
     """Time the oracle casting `rows` rows of the sweep input to all six formats."""
     import oracle
     from microscaling_block_scaled_mx_b200 import inputs as I
-    x = I.cast_sweep_input(rows, COLS)
+    if x is None:
+        x = I.cast_sweep_input(rows, COLS)
     oracle.build()
     t0 = time.perf_counter()
     for f in FMTS:
@@ -177,15 +178,20 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    rows = 512
-    oracle_cast_sample(64)                     # warm the library
+    from microscaling_block_scaled_mx_b200 import inputs as I
+    # each step casts a bounded sample of rows, sized so that all steps take
+    # about a minute of oracle time (between 32 and 512 rows per step)
+    _, dt64, _ = oracle_cast_sample(64)        # also warms the library
+    rows = int(60.0 / (args.steps * dt64 / 64)) // 32 * 32
+    rows = max(32, min(512, rows))
+    x = I.cast_sweep_input(rows, COLS)
     vals = []
     for _ in range(args.warmup):
-        oracle_cast_sample(rows)
+        oracle_cast_sample(rows, x)
     t_total = 0.0
     nbytes = 0
     for _ in range(args.steps):
-        v, dt, nb = oracle_cast_sample(rows)
+        v, dt, nb = oracle_cast_sample(rows, x)
         vals.append(v)
         t_total += dt
         nbytes += nb
@@ -234,8 +240,9 @@ def run_mx(args):
     stream = torch.cuda.current_stream()
     if args.no_cast:
         gemm = run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world)
+        gemm8 = run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world, fmt="e4m3")
         if rank == 0:
-            print(json.dumps({"gemm_only": True, "gemm": gemm}), flush=True)
+            print(json.dumps({"gemm_only": True, "gemm": gemm, "gemm_fp8": gemm8}), flush=True)
         if world > 1:
             dist.destroy_process_group()
         return 0
@@ -251,22 +258,26 @@ def run_mx(args):
                    for _ in range(N_ROTATE)]
     stream = torch.cuda.current_stream()
 
-    launches = 0
-    events = []
-
-    def step(i, record=False):
-        nonlocal launches
+    def step(i):
         for j, f in enumerate(FMTS):
             r = (i * len(FMTS) + j) % N_ROTATE
             c, s = outs[f][r]
-            if record:
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
             mx.quantize(xs[r], 1, f, codes=c, scales=s, scale_layout="mma")
-            if record:
-                e1.record(stream)
-                events.append((f, e0, e1))
-            launches += 1
+
+    def timed_region(body, n):
+        """Milliseconds of n calls of body(i), events only at the two ends (an
+        event between launches costs device time and lets the host fall behind)."""
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(n):
+            body(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(t0.elapsed_time(t1))
 
     for i in range(args.warmup):
         step(i)
@@ -274,29 +285,25 @@ def run_mx(args):
 
     # timed region: K steps, barrier + synchronize on both sides
     with ClockSampler(local) as clocks:
-        barrier()
-        torch.cuda.synchronize()
-        launches = 0
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for i in range(args.steps):
-            step(i, record=True)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        ms_total = t0.elapsed_time(t1)
-    ms_total = max_over_ranks(ms_total)
+        ms_total = timed_region(step, args.steps)
+    launches = len(FMTS) * args.steps
     alg_bytes_step = sum(cast_alg_bytes(f) for f in FMTS)
     value = world * alg_bytes_step * args.steps / (ms_total * 1e-3) / 1e9
 
+    # per format: a timed region of that cast alone (same input rotation)
     per_fmt = {}
+    n_fmt = max(3 * N_ROTATE, min(args.steps, 300))
     for f in FMTS:
-        durs = [a.elapsed_time(b) for (g, a, b) in events if g == f]
-        per_fmt[f] = {"us": round(1e3 * statistics.mean(durs), 2),
-                      "gbs": round(cast_alg_bytes(f) / (statistics.mean(durs) * 1e-3) / 1e9, 1)}
-    all_durs_ms = sum(a.elapsed_time(b) for (_, a, b) in events)
-    achieved = alg_bytes_step * args.steps / (all_durs_ms * 1e-3) / 1e9
+        def one(i, f=f):
+            r = i % N_ROTATE
+            c, s = outs[f][r]
+            mx.quantize(xs[r], 1, f, codes=c, scales=s, scale_layout="mma")
+        one(0)
+        us = 1e3 * timed_region(one, n_fmt) / n_fmt
+        launches += n_fmt
+        per_fmt[f] = {"us": round(us, 2), "gbs": round(cast_alg_bytes(f) / (us * 1e-6) / 1e9, 1)}
+    # the roofline kernel's average launch duration in the timed region above
+    achieved = alg_bytes_step * args.steps / (ms_total * 1e-3) / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
     traffic = None
     t_fmt = {f: measured_traffic("cast_rows", f"{f}_bf16_{ROWS}x{COLS}") for f in FMTS}
@@ -456,47 +463,52 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         for (M, N, K, ac, as_, bc, bs, c) in ops:
             mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
     torch.cuda.synchronize()
-    barrier()
-    evs = []
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches = 0
-    t0.record(stream)
-    for _ in range(args.steps):
+
+    def timed_region(body, n):
+        barrier()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(n):
+            body(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(t0.elapsed_time(t1))
+
+    def step(i):
         for (M, N, K, ac, as_, bc, bs, c) in ops:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
             mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
-            e1.record(stream)
-            evs.append(((M, N, K), e0, e1))
-            launches += 1
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(t0.elapsed_time(t1))
+
+    ms = timed_region(step, args.steps)
+    launches = len(ops) * args.steps
     value = world * flops_step * args.steps / (ms * 1e-3) / 1e12
     per_shape = {}
-    for (M, N, K, *_r) in ops:
-        d = [a.elapsed_time(b) for (s, a, b) in evs if s == (M, N, K)]
-        per_shape[f"{M}x{N}x{K}"] = {"us": round(1e3 * statistics.mean(d), 1),
-                                     "tflops": round(2.0 * M * N * K / (statistics.mean(d) * 1e-3) / 1e12, 1)}
+    n_shape = max(3, min(args.steps, 200))
+    for (M, N, K, ac, as_, bc, bs, c) in ops:
+        def one(i, M=M, N=N, K=K, ac=ac, as_=as_, bc=bc, bs=bs, c=c):
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
+        us = 1e3 * timed_region(one, n_shape) / n_shape
+        launches += n_shape
+        per_shape[f"{M}x{N}x{K}"] = {"us": round(us, 1), "tflops": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 1)}
     traffic = None
     t_shape = {k: measured_traffic("gemm", f"{fmt}_{k}") for k in per_shape}
     if all(v is not None for v in t_shape.values()):
         traffic = round(statistics.mean(t_shape.values()))
         for k in per_shape:
             per_shape[k]["traffic"] = t_shape[k]
-    kern_ms = sum(a.elapsed_time(b) for (_, a, b) in evs)
-    achieved = flops_step * args.steps / (kern_ms * 1e-3) / 1e12
+    # all launches of the timed region are this kernel: its average launch duration
+    achieved = flops_step * args.steps / (ms * 1e-3) / 1e12
     # the same GEMMs with C quantized in the epilogue (to the operand format, along
     # N: the next layer's A operand) against the GEMM followed by a row cast of C
     fused = {}
     q_steps = max(3, min(args.steps, 20))
-    for (M, N, K, ac, as_, bc, bs, c) in ops:
+    for (M, N, K, ac, as_, bc, bs, c) in ([] if args.no_fused else ops):
         qc = torch.empty((M, mx.codes_row_bytes(fmt, N)), dtype=torch.uint8, device=dev)
         qs = torch.empty(mx.scales_bytes("mma", M, N), dtype=torch.uint8, device=dev)
         res = {}
         for label in ("gemm_then_cast", "fused"):
-            def once():
+            def once(label=label, M=M, N=N, K=K, ac=ac, as_=as_, bc=bc, bs=bs, c=c, qc=qc, qs=qs):
                 if label == "fused":
                     mx.gemm_quantize(ac, as_, bc, bs, M, N, K, fa=fmt, out_fmt=fmt, out=(qc, qs))
                 else:
@@ -674,15 +686,16 @@ def run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mx", "reference"], default="mx")
     ap.add_argument("--no-gemm", action="store_true", help="skip the GEMM phase")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phase")
-    ap.add_argument("--no-cast", action="store_true", help="GEMM phase only (profiling)")
+    ap.add_argument("--no-cast", action="store_true", help="GEMM phases only (profiling)")
     ap.add_argument("--no-wgrad", action="store_true", help="skip the weight-gradient phase")
     ap.add_argument("--no-dual", action="store_true", help="skip the dual-cast phase")
+    ap.add_argument("--no-fused", action="store_true", help="skip the quantizing-epilogue comparison")
     ap.add_argument("--fmts", default=",".join(FMTS), help="comma-separated cast formats (profiling)")
     ap.add_argument("--gemm-shapes", default="0,1,2", help="indices of the Llama-3 GEMM shapes to time")
     args = ap.parse_args()
