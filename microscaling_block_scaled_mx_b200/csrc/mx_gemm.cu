@@ -110,6 +110,21 @@ struct Params {
     MxOut q;         // OUT_MX only
 };
 
+// Tile order: tiles are taken in groups of RASTER_M row-tiles, column by
+// column inside a group, so the CTAs working at the same time share a few A
+// row panels and a few B column panels (L2 reuse) instead of sweeping every
+// row panel of A for each column of B.
+constexpr int RASTER_M = 8;
+
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &tm, int &tn) {
+    const int per_group = RASTER_M * tiles_n;
+    const int group = tile / per_group, r = tile - group * per_group;
+    const int m0 = group * RASTER_M;
+    const int rows = tiles_m - m0 < RASTER_M ? tiles_m - m0 : RASTER_M;
+    tm = m0 + r % rows;
+    tn = r / rows;
+}
+
 // ------------------------------------------------------------------------
 // PTX wrappers
 // ------------------------------------------------------------------------
@@ -368,7 +383,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             uint32_t outstanding = 0;   // bit s: stage s has loads in flight not yet observed
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+                int tm, tn;
+                tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
                 const int m0 = tm * BM, n0 = tn * BN;
                 const int rb_a = m0 / 128, rb_b = n0 / 128;   // 128-row scale blocks
                 const bool b_second = (rb_b + 1) * 128 < p.N;
@@ -424,7 +440,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                 const uint32_t acc_ph = (local >> 1) & 1;
                 if (!wait_bounded(acc_empty(b), acc_ph ^ 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const int tn = tile / p.tiles_m;
+                int tm, tn;
+                tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
                 const uint32_t d_tmem = tmem + b * ACC_COLS;
                 const uint32_t sfb_shift = (tn & 1) ? 2u : 0u;   // odd 192-column tiles
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
@@ -482,7 +499,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+            int tm, tn;
+            tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
             const int m = tm * BM + q * 32 + lane;
             const int c0 = half * (BN / 2);
             const uint32_t taddr = tmem + b * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + c0;
@@ -560,7 +578,7 @@ struct PairParams {
     int M, N, K;
     int k_tiles;
     int k_groups;
-    int tiles_m, tiles_n;      // 256 x 192 pair tiles
+    int tiles_m, tiles_n;      // 256 x 256 pair tiles
     float alpha;
     uint32_t idesc;
     uint32_t ab_tx;            // bytes one CTA's A and B loads of a stage deliver
@@ -674,7 +692,8 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             bool ok = true;
             const uint32_t stage_bytes = 2 * (p.ab_tx + C::SFA_BYTES + C::SFB_BYTES);
             for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
-                const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+                int tm, tn;
+                tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
                 // this CTA's A rows and B rows; a half that lies wholly past M (or N)
                 // only feeds discarded outputs, so its loads are clamped to rows
                 // that exist and no TMA box is ever entirely outside its tensor
@@ -771,7 +790,8 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+            int tm, tn;
+            tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
             const int m = tm * PAIR_BM + 128 * static_cast<int>(rank) + q * 32 + lane;
             const int c0 = half * (PAIR_BN / 2);
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + c0;
