@@ -56,10 +56,10 @@ MEASURED_TRAFFIC = {
                    "e2m3_bf16_8192x8192": 158393600, "e3m2_bf16_8192x8192": 158375680,
                    "e2m1_bf16_8192x8192": 149267200, "int8_bf16_8192x8192": 168440320}),
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "912b56beecdb017c926e0563b82a84398e53e5c31fc082fb7ff89a9ebc59f39b",
-             {"e2m1_8192x6144x4096": 78177792, "e2m1_8192x14336x4096": 227502336,
-              "e2m1_8192x4096x14336": 295097344, "e4m3_8192x3072x768": 9265664,
-              "e4m3_8192x768x3072": 28417536}),
+             "7e3fc2a3366087919b164dbad63ee23f0831d169cacd3f305058221d7eea9dc3",
+             {"e2m1_8192x6144x4096": 78374912, "e2m1_8192x14336x4096": 227282688,
+              "e2m1_8192x4096x14336": 141698304, "e4m3_8192x3072x768": 9384704,
+              "e4m3_8192x768x3072": 28419072}),
 }
 
 

@@ -107,22 +107,26 @@ struct Params {
     uint32_t idesc;  // instruction descriptor without the scale-factor ids
     uint32_t ab_tx;  // bytes the A and B loads of one stage deliver (packed size in global)
     int skip_k_tile; // testing hook: CTA 0 withholds this k-tile of its first tile (-1: off)
+    int raster_group, raster_n_major;   // tile order (tile_coords)
     MxOut q;         // OUT_MX only
 };
 
-// Tile order: tiles are taken in groups of RASTER_M row-tiles, column by
-// column inside a group, so the CTAs working at the same time share a few A
-// row panels and a few B column panels (L2 reuse) instead of sweeping every
-// row panel of A for each column of B.
-constexpr int RASTER_M = 8;
-
-__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &tm, int &tn) {
-    const int per_group = RASTER_M * tiles_n;
-    const int group = tile / per_group, r = tile - group * per_group;
-    const int m0 = group * RASTER_M;
-    const int rows = tiles_m - m0 < RASTER_M ? tiles_m - m0 : RASTER_M;
-    tm = m0 + r % rows;
-    tn = r / rows;
+// Tile order.  Tiles are taken in bands of `group` tiles along the major
+// axis (M, or N when n_major), the band's tiles along the minor axis one after
+// the other.  The host picks the order per shape (see raster_for): with the
+// band as wide as the whole axis, the CTAs in flight share the operand whose
+// panels all stay in L2 while the other operand streams through once; narrow
+// bands bound the working set when neither operand fits.
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int group, int n_major, int &tm,
+                                            int &tn) {
+    const int major = n_major ? tiles_n : tiles_m, minor_tiles = n_major ? tiles_m : tiles_n;
+    const int per_band = group * minor_tiles;
+    const int band = tile / per_band, r = tile - band * per_band;
+    const int j0 = band * group;
+    const int width = major - j0 < group ? major - j0 : group;
+    const int j = j0 + r % width, i = r / width;
+    tm = n_major ? i : j;
+    tn = n_major ? j : i;
 }
 
 // ------------------------------------------------------------------------
@@ -384,7 +388,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 int tm, tn;
-                tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+                tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
                 const int m0 = tm * BM, n0 = tn * BN;
                 const int rb_a = m0 / 128, rb_b = n0 / 128;   // 128-row scale blocks
                 const bool b_second = (rb_b + 1) * 128 < p.N;
@@ -441,7 +445,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                 if (!wait_bounded(acc_empty(b), acc_ph ^ 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 int tm, tn;
-                tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+                tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
                 const uint32_t d_tmem = tmem + b * ACC_COLS;
                 const uint32_t sfb_shift = (tn & 1) ? 2u : 0u;   // odd 192-column tiles
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
@@ -500,7 +504,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             if (!ok) break;
             tc_fence_after();
             int tm, tn;
-            tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+            tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
             const int m = tm * BM + q * 32 + lane;
             const int c0 = half * (BN / 2);
             const uint32_t taddr = tmem + b * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + c0;
@@ -583,6 +587,7 @@ struct PairParams {
     uint32_t idesc;
     uint32_t ab_tx;            // bytes one CTA's A and B loads of a stage deliver
     int skip_k_tile;
+    int raster_group, raster_n_major;   // tile order (tile_coords)
     MxOut q;                   // OUT_MX only
 };
 
@@ -693,7 +698,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             const uint32_t stage_bytes = 2 * (p.ab_tx + C::SFA_BYTES + C::SFB_BYTES);
             for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
                 int tm, tn;
-                tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+                tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
                 // this CTA's A rows and B rows; a half that lies wholly past M (or N)
                 // only feeds discarded outputs, so its loads are clamped to rows
                 // that exist and no TMA box is ever entirely outside its tensor
@@ -791,7 +796,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             if (!ok) break;
             tc_fence_after();
             int tm, tn;
-            tile_coords(tile, p.tiles_m, p.tiles_n, tm, tn);
+            tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
             const int m = tm * PAIR_BM + 128 * static_cast<int>(rank) + q * 32 + lane;
             const int c0 = half * (PAIR_BN / 2);
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + c0;
@@ -979,6 +984,17 @@ extern "C" int mx_debug_gemm_skip_stage(int k_tile) {
 
 namespace {
 
+// Tile order for a shape: keep the operand whose codes fit in a third of the
+// L2 resident (M fastest when A fits, N fastest when B fits) so that each
+// operand is read from HBM about once; otherwise bands of 8 row-tiles.
+void raster_for(const MxGemmArgs &a, int tiles_m, int tiles_n, int &group, int &n_major) {
+    constexpr int64_t kResident = 40ll << 20;
+    const int64_t a_bytes = a.M * a.K * mxg::elem_bits(a.fa) / 8, b_bytes = a.N * a.K * mxg::elem_bits(a.fb) / 8;
+    if (a_bytes <= kResident) { group = tiles_m; n_major = 0; }
+    else if (b_bytes <= kResident) { group = tiles_n; n_major = 1; }
+    else { group = 8; n_major = 0; }
+}
+
 // E2M1 x E2M1 with K a multiple of 256 runs kind::mxf4 on packed codes (256
 // per stage); every other pair, and FP4 x FP4 with K = 128 (mod 256), runs
 // kind::mxf8f6f4 with 128 codes per stage.
@@ -1013,6 +1029,7 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     p.alpha = a.alpha;
     p.idesc = make_idesc(a.fa, a.fb, fp4, PAIR_BM, PAIR_BN);
     p.ab_tx = stage_tx_bytes(a.fa, fp4, 128) + stage_tx_bytes(a.fb, fp4, PAIR_B_ROWS);
+    raster_for(a, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major);
     p.skip_k_tile = g_skip_k_tile.exchange(-1);
     const int tiles = p.tiles_m * p.tiles_n;
     const int clusters = tiles < a.num_sms / 2 ? tiles : a.num_sms / 2;
@@ -1061,6 +1078,7 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     p.alpha = a.alpha;
     p.idesc = make_idesc(a.fa, a.fb, fp4);
     p.ab_tx = stage_tx_bytes(a.fa, fp4, BM) + stage_tx_bytes(a.fb, fp4, BN);
+    raster_for(a, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major);
     p.skip_k_tile = g_skip_k_tile.exchange(-1);
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < a.num_sms ? tiles : a.num_sms;
