@@ -5,7 +5,8 @@
 // and scale byte written once.
 //  * cast_rows: blocks run along the contiguous axis.  One lane owns one
 //    32-block (two 32-byte loads for bf16); a warp covers 32 consecutive
-//    blocks of a row, with the next two chunks' loads in flight.
+//    blocks of a row, with the next two chunks' loads in flight in a ring of
+//    register slots.
 //  * cast_cols: blocks run down columns.  A CTA stages 128 x 128 tiles in
 //    shared memory (double-buffered cp.async); each thread owns one column
 //    pair of a 32-row block, where the optional fixed-sign 32-point Hadamard
@@ -47,11 +48,11 @@ __device__ __forceinline__ void store_scale(const CastParams &p, int64_t o, int6
 // ---------------------------------------------------------------------------
 // Row cast: block axis contiguous.
 // ---------------------------------------------------------------------------
-// One lane owns one 32-block (64 bytes of bf16, four 16-byte loads), so the
-// block's amax, exponent, scale byte and addresses are computed once per 32
-// values; a warp covers 32 consecutive blocks (1024 values) of one row.  The
-// next chunk's loads are issued before the current chunk is converted, so each
-// thread keeps up to eight 16-byte loads in flight.
+// One lane owns one 32-block (64 bytes of bf16: two 32-byte loads, or four
+// 16-byte loads when rows are not 32-byte aligned), so the block's amax,
+// exponent, scale byte and addresses are computed once per 32 values; a warp
+// covers 32 consecutive blocks (1024 values) of one row.  The loads of the
+// next two chunks are in flight while the current chunk is converted.
 template <bool BF16_IN>
 struct BlockLoad {
     uint4 w[BF16_IN ? 4 : 8];
@@ -138,6 +139,7 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
 
 template <int FMT, bool SR, bool BF16_IN, bool V32>
 __global__ void __launch_bounds__(256, 2) cast_rows_kernel(CastParams p) {
+    constexpr int DIST = 2;                               // chunks in flight while one is converted
     const int lane = threadIdx.x & 31;
     const int64_t blocks_per_row = p.cols >> 5;
     const int64_t cpr = (blocks_per_row + 31) >> 5;      // chunks per row
@@ -149,25 +151,30 @@ __global__ void __launch_bounds__(256, 2) cast_rows_kernel(CastParams p) {
         q.row += step_rows;
         if (q.chunk >= cpr) { q.chunk -= cpr; ++q.row; }
     };
-    // two chunks in flight while a third is converted
-    ChunkPos cur;
-    cur.row = warp0 / cpr;
-    cur.chunk = warp0 - cur.row * cpr;
-    ChunkPos nx1 = cur;
-    advance(nx1);
-    BlockLoad<BF16_IN> cur_ld, nx1_ld;
-    load_block<BF16_IN, V32>(p, cur, blocks_per_row, lane, cur_ld);
-    load_block<BF16_IN, V32>(p, nx1, blocks_per_row, lane, nx1_ld);
-    while (cur.row < p.rows) {
-        ChunkPos nx2 = nx1;
-        advance(nx2);
-        BlockLoad<BF16_IN> nx2_ld;
-        load_block<BF16_IN, V32>(p, nx2, blocks_per_row, lane, nx2_ld);
-        cast_block<FMT, SR, BF16_IN, V32>(p, cur, blocks_per_row, cur_ld, lane);
-        cur = nx1;
-        cur_ld = nx1_ld;
-        nx1 = nx2;
-        nx1_ld = nx2_ld;
+    // a ring of DIST + 1 load slots, indexed statically by unrolling one turn
+    // of the ring: slot u is converted while slot (u + DIST) % (DIST + 1) loads
+    ChunkPos pos[DIST + 1];
+    BlockLoad<BF16_IN> ld[DIST + 1];
+    pos[0].row = warp0 / cpr;
+    pos[0].chunk = warp0 - pos[0].row * cpr;
+#pragma unroll
+    for (int i = 1; i <= DIST; ++i) {
+        pos[i] = pos[i - 1];
+        advance(pos[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < DIST; ++i) load_block<BF16_IN, V32>(p, pos[i], blocks_per_row, lane, ld[i]);
+    for (;;) {
+#pragma unroll
+        for (int u = 0; u <= DIST; ++u) {
+            constexpr int NEXT = DIST;                    // slot offset of the chunk to load
+            const int nxt = (u + NEXT) % (DIST + 1);
+            if (pos[u].row >= p.rows) return;
+            load_block<BF16_IN, V32>(p, pos[nxt], blocks_per_row, lane, ld[nxt]);
+            cast_block<FMT, SR, BF16_IN, V32>(p, pos[u], blocks_per_row, ld[u], lane);
+            pos[u] = pos[nxt];                            // this slot's next chunk: one after pos[nxt]
+            advance(pos[u]);
+        }
     }
 }
 
