@@ -321,17 +321,25 @@ def run_mx(args):
     # ---- end to end through the C ABI with host buffers ----
     # The tensor streams through in row chunks on three streams: the host->device
     # copy of chunk i+1 and the device->host copy of chunk i-1 overlap the six
-    # casts of chunk i (the two copy directions use separate engines).  Codes
-    # and scales land in pinned host buffers; plain scale layout, so each
-    # chunk's scales are one contiguous slice.
+    # casts of chunk i (the two copy directions use separate engines).  Each
+    # chunk's outputs (codes and plain-layout scales of all six formats) sit
+    # contiguously in one device buffer, so they return to pinned host memory
+    # in one copy per chunk.
     pinned = host.pin_memory()
     E2E_CHUNKS = 8
     rows_c = ROWS // E2E_CHUNKS
-    host_out = {f: (torch.empty((ROWS, mx.codes_row_bytes(f, COLS)), dtype=torch.uint8).pin_memory(),
-                    torch.empty(mx.scales_bytes("plain", ROWS, COLS), dtype=torch.uint8).pin_memory())
-                for f in FMTS}
-    dev_sc = {f: torch.empty(mx.scales_bytes("plain", ROWS, COLS), dtype=torch.uint8, device=dev) for f in FMTS}
-    d2h = sum(host_out[f][0].numel() + host_out[f][1].numel() for f in FMTS)
+    seg = []                                   # (format, codes offset, scales offset) inside a chunk
+    off = 0
+    for f in FMTS:
+        cb = rows_c * mx.codes_row_bytes(f, COLS)
+        sb = mx.scales_bytes("plain", rows_c, COLS)
+        seg.append((f, off, off + cb, sb))
+        off += cb + sb
+        off = (off + 255) // 256 * 256         # keep every slice 256-byte aligned
+    chunk_bytes = off
+    dev_chunks = [torch.empty(chunk_bytes, dtype=torch.uint8, device=dev) for _ in range(E2E_CHUNKS)]
+    host_chunks = torch.empty((E2E_CHUNKS, chunk_bytes), dtype=torch.uint8).pin_memory()
+    d2h = E2E_CHUNKS * chunk_bytes
     h2d = pinned.numel() * 2
     s_in, s_cast, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
@@ -345,18 +353,16 @@ def run_mx(args):
                 ev.record(s_in)
             with torch.cuda.stream(s_cast):
                 s_cast.wait_event(ev)
-                for f in FMTS:
-                    c = outs[f][0][0][r0:r1]
-                    sc = dev_sc[f][r0 * (COLS // 32):r1 * (COLS // 32)]
-                    mx.quantize(xs[0][r0:r1], 1, f, codes=c, scales=sc, scale_layout="plain", stream=s_cast)
+                buf = dev_chunks[i]
+                for (f, co, so, sb) in seg:
+                    c = buf[co:so].view(rows_c, -1)
+                    mx.quantize(xs[0][r0:r1], 1, f, codes=c, scales=buf[so:so + sb], scale_layout="plain",
+                                stream=s_cast)
                 evc = torch.cuda.Event()
                 evc.record(s_cast)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(evc)
-                for f in FMTS:
-                    host_out[f][0][r0:r1].copy_(outs[f][0][0][r0:r1], non_blocking=True)
-                    a, b = r0 * (COLS // 32), r1 * (COLS // 32)
-                    host_out[f][1][a:b].copy_(dev_sc[f][a:b], non_blocking=True)
+                host_chunks[i].copy_(dev_chunks[i], non_blocking=True)
         stream.wait_stream(s_out)
 
     e2e_steps = min(args.steps, 50)
@@ -411,7 +417,7 @@ def run_mx(args):
                        {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                         "path": "pinned host bf16 -> H2D -> mx_quantize (6 formats) -> D2H codes+scales, "
-                                "8 row chunks pipelined over 3 streams"},
+                                "8 row chunks pipelined over 3 streams, one D2H copy per chunk"},
                 "gpu_launches": launches + launches_gemm,
                 "clocks": clocks.summary()}
         if gemm is not None:
@@ -567,37 +573,29 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
     bc = torch.empty((Di, T // 2), dtype=torch.uint8, device=dev)
     bs = torch.empty(mx.scales_bytes("mma", Di, T), dtype=torch.uint8, device=dev)
     dw = torch.empty((Do, Di), dtype=torch.float32, device=dev)
-    evs = {"cast_dY": [], "cast_X": [], "gemm_dW": []}
+    ops = {"cast_dY": lambda: mx.quantize(dy, 0, "e2m1", rnd="sr", seed=42, hadamard=True, codes=ac, scales=as_),
+           "cast_X": lambda: mx.quantize(x, 0, "e2m1", rnd="sr", seed=43, hadamard=True, codes=bc, scales=bs),
+           "gemm_dW": lambda: mx.gemm(ac, as_, bc, bs, Do, Di, T, fa="e2m1", alpha=1.0 / 32, out=dw)}
 
-    def step(record):
-        for name, fn in (("cast_dY", lambda: mx.quantize(dy, 0, "e2m1", rnd="sr", seed=42, hadamard=True,
-                                                         codes=ac, scales=as_)),
-                         ("cast_X", lambda: mx.quantize(x, 0, "e2m1", rnd="sr", seed=43, hadamard=True,
-                                                        codes=bc, scales=bs)),
-                         ("gemm_dW", lambda: mx.gemm(ac, as_, bc, bs, Do, Di, T, fa="e2m1", alpha=1.0 / 32,
-                                                     out=dw))):
-            if record:
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
+    def timed(fn, n):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
             fn()
-            if record:
-                e1.record(stream)
-                evs[name].append((e0, e1))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
 
     steps = max(3, min(args.steps, 20))
     for _ in range(args.warmup):
-        step(False)
+        for fn in ops.values():
+            fn()
     torch.cuda.synchronize()
-    barrier()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        step(True)
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(t0.elapsed_time(t1))
-    us = {k: 1e3 * statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in evs.items()}
+    ms = timed(lambda: [fn() for fn in ops.values()], steps)      # the whole step
+    us = {k: 1e3 * timed(fn, steps) / steps for k, fn in ops.items()}
     cast_bytes = {"cast_dY": T * Do * 2 + T * Do // 2 + T * Do // 32,
                   "cast_X": T * Di * 2 + T * Di // 2 + T * Di // 32}
     flops = 2.0 * Do * Di * T
@@ -623,59 +621,50 @@ def run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world):
     from microscaling_block_scaled_mx_b200 import inputs as I
     from microscaling_block_scaled_mx_b200 import mx
     dyb, xb = I.wgrad_operands()
+    rng = np.random.default_rng(1004)
+    act = I.to_bf16_bits(rng.standard_normal((8192, 4096)).astype(np.float32))
+    # (name, tensor, format, column rounding, Hadamard on the column output)
+    cases = [("dY", dyb, "e2m1", "sr", True), ("X", xb, "e2m1", "sr", True),
+             ("act_e4m3", act, "e4m3", "rne", False)]
     ops = []
-    for name, bits in (("dY", dyb), ("X", xb)):
+    for name, bits, f, rc, had in cases:
         t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
-        R, C = t.shape
-        out = mx.quantize_dual(t, "e2m1", rnd_rows="rne", rnd_cols="sr", seed_cols=42, hadamard=True)
-        ops.append((name, t, out))
-    del dyb, xb
+        out = mx.quantize_dual(t, f, rnd_rows="rne", rnd_cols=rc, seed_cols=42, hadamard=had)
+        ops.append((name, t, f, rc, had, out))
+    del dyb, xb, act
     launches = 0
 
-    def dual(record, evs):
-        nonlocal launches
-        for name, t, out in ops:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            mx.quantize_dual(t, "e2m1", rnd_rows="rne", rnd_cols="sr", seed_cols=42, hadamard=True, out=out)
-            e1.record(stream)
-            if record:
-                evs.setdefault(name, []).append((e0, e1))
-                launches += 1
-
-    def single(record, evs):
-        nonlocal launches
-        for name, t, out in ops:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            mx.quantize(t, 1, "e2m1", codes=out[0], scales=out[1])
-            mx.quantize(t, 0, "e2m1", rnd="sr", seed=42, hadamard=True, codes=out[2], scales=out[3])
-            e1.record(stream)
-            if record:
-                evs.setdefault(name, []).append((e0, e1))
-                launches += 2
+    def timed(fn, n):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(1e3 * e0.elapsed_time(e1) / n)
 
     steps = max(3, min(args.steps, 20))
-    res = {}
-    for label, fn in (("dual", dual), ("two_casts", single)):
-        for _ in range(args.warmup):
-            fn(False, {})
-        torch.cuda.synchronize()
-        barrier()
-        evs = {}
-        for _ in range(steps):
-            fn(True, evs)
-        torch.cuda.synchronize()
-        barrier()
-        res[label] = {k: max_over_ranks(1e3 * statistics.mean(a.elapsed_time(b) for a, b in v))
-                      for k, v in evs.items()}
     hbm = float(peaks["hbm_gbs"])
-    out = {"workload": "dual_cast_e2m1 dY 16384x4096, X 16384x14336 bf16: rows RNE + tokens Hadamard+SR",
-           "steps": steps}
-    for name, t, _ in ops:
+    out = {"workload": "dual cast: dY 16384x4096 and X 16384x14336 bf16 to E2M1 (rows RNE, tokens Hadamard+SR); "
+                       "Llama-3 activation 8192x4096 bf16 to E4M3 (RNE both axes)", "steps": steps}
+    for name, t, f, rc, had, o in ops:
+        def dual(t=t, f=f, rc=rc, had=had, o=o):
+            mx.quantize_dual(t, f, rnd_rows="rne", rnd_cols=rc, seed_cols=42, hadamard=had, out=o)
+
+        def two(t=t, f=f, rc=rc, had=had, o=o):
+            mx.quantize(t, 1, f, codes=o[0], scales=o[1])
+            mx.quantize(t, 0, f, rnd=rc, seed=42, hadamard=had, codes=o[2], scales=o[3])
+        for _ in range(args.warmup):
+            dual()
+            two()
+        d, s2 = timed(dual, steps), timed(two, steps)
+        launches += 3 * steps
         n = t.numel()
-        alg = n * 2 + 2 * (n // 2 + n // 32)        # one read, two sets of codes and scales
-        d, s2 = res["dual"][name], res["two_casts"][name]
+        bits = mx.FMT_BITS[mx.FMT[f]]
+        alg = n * 2 + 2 * (n * bits // 8 + n // 32)        # one read, two sets of codes and scales
         out[name] = {"dual_us": round(d, 1), "two_casts_us": round(s2, 1), "speedup": round(s2 / d, 3),
                      "dual_gbs": round(alg / (d * 1e-6) / 1e9, 1),
                      "frac_hbm": round(alg / (d * 1e-6) / 1e9 / hbm, 4)}
