@@ -110,6 +110,11 @@ template <int FMT, bool SR, bool V32>
 __device__ __forceinline__ void encode_row_block(const CastParams &p, int64_t row, int64_t kb, uint32_t (&b)[32]) {
     encode_block32<FMT, SR, V32>(row_sink(p), row, kb, b);
 }
+template <int FMT, bool SR, bool V32>
+__device__ __forceinline__ void encode_row_block(const CastParams &p, int64_t row, int64_t kb, uint32_t (&b)[32],
+                                                 uint32_t amax_bits) {
+    encode_block32_amax<FMT, SR, V32>(row_sink(p), row, kb, b, amax_bits);
+}
 
 template <int FMT, bool SR, bool BF16_IN, bool V32>
 __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &cp, int64_t blocks_per_row,
@@ -119,15 +124,19 @@ __device__ __forceinline__ void cast_block(const CastParams &p, const ChunkPos &
     // the 32 values as fp32 bit patterns
     uint32_t b[32];
     if (BF16_IN) {
+        uint32_t words[16];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t ws[4] = {o.w[i].x, o.w[i].y, o.w[i].z, o.w[i].w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
+                words[4 * i + k] = ws[k];
                 b[8 * i + 2 * k] = ws[k] << 16;
                 b[8 * i + 2 * k + 1] = ws[k] & 0xffff0000u;
             }
         }
+        encode_row_block<FMT, SR, V32>(p, cp.row, kb, b, bf16_max_bits(bf16_pair_max<16>(words)));
+        return;
     } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -254,8 +263,12 @@ __device__ __forceinline__ void stage_tile(const CastParams &p, uint8_t *buf, in
 // subnormal flush, RNE or stochastic rounding, and the codes as rows gc and
 // gc + 1 of the transposed output.  SR's index is the element's position
 // (gc + col) * rows + gr0 + j in that output.
-template <int FMT, bool SR, bool HAD>
-__device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&x)[32], int64_t gc, int64_t gr0) {
+// KEYED: the caller passes the packed 16-bit maxima of |bf16| of the two
+// columns (bf16_pair_max over the raw words), valid without the Hadamard.
+template <int FMT, bool SR, bool HAD, bool KEYED = false>
+__device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&x)[32], int64_t gc, int64_t gr0,
+                                                uint32_t pair_max16 = 0) {
+    static_assert(!(KEYED && HAD), "the bf16 maxima describe the values before the Hadamard");
     constexpr int BITS = Fmt<FMT>::bits;
     const int64_t R = p.rows, C = p.cols;
     if (HAD) {
@@ -278,12 +291,17 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
     const bool has_second = gc + 1 < C;
     // block amax and exponent of both columns
     uint32_t am0 = 0, am1 = 0;
+    if (KEYED) {
+        am0 = pair_max16 << 16;
+        am1 = pair_max16 & 0xffff0000u;
+    } else {
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-        am0 = __vimax3_u32(am0, static_cast<uint32_t>(x[j]) & 0x7fffffffu,
-                           static_cast<uint32_t>(x[j + 1]) & 0x7fffffffu);
-        am1 = __vimax3_u32(am1, static_cast<uint32_t>(x[j] >> 32) & 0x7fffffffu,
-                           static_cast<uint32_t>(x[j + 1] >> 32) & 0x7fffffffu);
+        for (int j = 0; j < 32; j += 2) {
+            am0 = __vimax3_u32(am0, static_cast<uint32_t>(x[j]) & 0x7fffffffu,
+                               static_cast<uint32_t>(x[j + 1]) & 0x7fffffffu);
+            am1 = __vimax3_u32(am1, static_cast<uint32_t>(x[j] >> 32) & 0x7fffffffu,
+                               static_cast<uint32_t>(x[j + 1] >> 32) & 0x7fffffffu);
+        }
     }
     const int e0 = block_exponent<FMT>(am0), e1 = block_exponent<FMT>(am1);
     // V * 2^-e for both columns with one packed multiply (flushing
@@ -389,17 +407,20 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
             const TIn *tile = reinterpret_cast<const TIn *>(col_smem + buf * TILE_BYTES);
             // x[j] = (column gc, column gc + 1) at row gr0 + j, as packed f32x2
             uint64_t x[32];
+            uint32_t words[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int off = (blk * 32 + j) * COL_TILE_C + 2 * pair;
                 if (BF16_IN) {
                     const uint32_t w = *reinterpret_cast<const uint32_t *>(tile + off);
+                    words[j] = w;
                     x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
                 } else {
                     x[j] = *reinterpret_cast<const uint64_t *>(tile + off);
                 }
             }
-            encode_col_pair<FMT, SR, HAD>(p, x, gc, gr0);
+            if (BF16_IN && !HAD) encode_col_pair<FMT, SR, false, true>(p, x, gc, gr0, bf16_pair_max<32>(words));
+            else encode_col_pair<FMT, SR, HAD>(p, x, gc, gr0);
         }
         __syncthreads();             // everyone is done with `buf` before it is refilled
     }
@@ -459,18 +480,26 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
         const int64_t gc = c0 + 2 * pair, gr0 = r0 + blk * 32;
         if (gc < C && gr0 < R) {
             uint64_t x[32];
+            uint32_t words[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const uint8_t *src = tile + (blk * 32 + j) * ROW_BYTES + col_off[j & 1];
                 if (BF16_IN) {
                     const uint32_t w = *reinterpret_cast<const uint32_t *>(src);
+                    words[j] = w;
                     x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
                 } else {
                     x[j] = *reinterpret_cast<const uint64_t *>(src);
                 }
             }
-            if (sr_cols) encode_col_pair<FMT, true, HAD>(pc, x, gc, gr0);
-            else encode_col_pair<FMT, false, HAD>(pc, x, gc, gr0);
+            if (BF16_IN && !HAD) {
+                const uint32_t m16 = bf16_pair_max<32>(words);
+                if (sr_cols) encode_col_pair<FMT, true, false, true>(pc, x, gc, gr0, m16);
+                else encode_col_pair<FMT, false, false, true>(pc, x, gc, gr0, m16);
+            } else {
+                if (sr_cols) encode_col_pair<FMT, true, HAD>(pc, x, gc, gr0);
+                else encode_col_pair<FMT, false, HAD>(pc, x, gc, gr0);
+            }
         }
         // ---- row blocks ----
 #pragma unroll 1
@@ -479,6 +508,7 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
             const int64_t row = r0 + rr, kb = (c0 >> 5) + rb;
             if (row >= R || 32 * kb >= C) continue;
             uint32_t b[32];
+            uint32_t words[16];
 #pragma unroll
             for (int i = 0; i < CPB; ++i) {
                 const uint4 w = *reinterpret_cast<const uint4 *>(
@@ -487,6 +517,7 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
                     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
+                        words[4 * i + k] = ws[k];
                         b[8 * i + 2 * k] = ws[k] << 16;
                         b[8 * i + 2 * k + 1] = ws[k] & 0xffff0000u;
                     }
@@ -494,8 +525,14 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
                     b[4 * i] = w.x; b[4 * i + 1] = w.y; b[4 * i + 2] = w.z; b[4 * i + 3] = w.w;
                 }
             }
-            if (sr_rows) encode_row_block<FMT, true, false>(pr, row, kb, b);
-            else encode_row_block<FMT, false, false>(pr, row, kb, b);
+            if (BF16_IN) {
+                const uint32_t amax = bf16_max_bits(bf16_pair_max<16>(words));
+                if (sr_rows) encode_row_block<FMT, true, false>(pr, row, kb, b, amax);
+                else encode_row_block<FMT, false, false>(pr, row, kb, b, amax);
+            } else {
+                if (sr_rows) encode_row_block<FMT, true, false>(pr, row, kb, b);
+                else encode_row_block<FMT, false, false>(pr, row, kb, b);
+            }
         }
         __syncthreads();             // everyone is done with `buf` before it is refilled
     }

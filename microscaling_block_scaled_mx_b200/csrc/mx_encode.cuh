@@ -53,13 +53,12 @@ __device__ __forceinline__ void store_code32(uint8_t *dst, const uint4 &a, const
 // exponent, V * 2^-e (flushing FP32 subnormals), RNE or stochastic rounding,
 // and the packed codes and scale byte of block (row, kb).  SR's index is the
 // element's position row * inner + kb * 32 + j in the output.
+// amax_bits: the largest |b[i]| as FP32 bits (sign cleared), computed by the
+// caller (encode_block32 below, or bf16_amax_bits from the packed input).
 template <int FMT, bool SR, bool V32>
-__device__ __forceinline__ void encode_block32(const BlockSink &o, int64_t row, int64_t kb, uint32_t (&b)[32]) {
+__device__ __forceinline__ void encode_block32_amax(const BlockSink &o, int64_t row, int64_t kb, uint32_t (&b)[32],
+                                                    uint32_t amax_bits) {
     constexpr int BITS = Fmt<FMT>::bits;
-    uint32_t amax_bits = 0;
-#pragma unroll
-    for (int i = 0; i < 32; i += 2)
-        amax_bits = __vimax3_u32(amax_bits, b[i] & 0x7fffffffu, b[i + 1] & 0x7fffffffu);
     const bool nan_block = amax_bits >= 0x7f800000u;
     const int e = block_exponent<FMT>(amax_bits);
 
@@ -152,5 +151,30 @@ __device__ __forceinline__ void encode_block32(const BlockSink &o, int64_t row, 
 }
 
 
+
+template <int FMT, bool SR, bool V32>
+__device__ __forceinline__ void encode_block32(const BlockSink &o, int64_t row, int64_t kb, uint32_t (&b)[32]) {
+    uint32_t amax_bits = 0;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2)
+        amax_bits = __vimax3_u32(amax_bits, b[i] & 0x7fffffffu, b[i + 1] & 0x7fffffffu);
+    encode_block32_amax<FMT, SR, V32>(o, row, kb, b, amax_bits);
+}
+
+// Packed 16-bit maximum of |bf16| over NW words of two bf16 values each (one
+// 3-input max per two words): the low and high halves hold the maxima of the
+// even and odd elements.  Widening bf16 to FP32 appends 16 zero bits, so a
+// half shifted left by 16 is the FP32 magnitude bits of that maximum.
+template <int NW>
+__device__ __forceinline__ uint32_t bf16_pair_max(const uint32_t *w) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < NW; i += 2) m = __vimax3_u16x2(m, w[i] & 0x7fff7fffu, w[i + 1] & 0x7fff7fffu);
+    return m;
+}
+__device__ __forceinline__ uint32_t bf16_max_bits(uint32_t m) {
+    const uint32_t lo = m << 16, hi = m & 0xffff0000u;
+    return lo > hi ? lo : hi;
+}
 
 }  // namespace mxk
