@@ -45,18 +45,23 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp_dir = os.path.join(PKG, "_build")
     os.makedirs(tmp_dir, exist_ok=True)
-    objs = []
+    jobs = []
     for src in SOURCES:
         obj = os.path.join(tmp_dir, src.replace(".cu", ".o"))
         cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        jobs.append((obj, cmd))
+    # the translation units are independent: compile them concurrently
+    procs = [(obj, cmd, subprocess.Popen(cmd)) for obj, cmd in jobs]
+    failed = [cmd for _, cmd, proc in procs if proc.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
+    objs = [obj for obj, _ in jobs]
     tmp_lib = LIB + f".tmp{os.getpid()}"
     subprocess.run([nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp_lib, *objs,
-                    "-lcudart_static" if False else "-lcudart"], check=True)
+                    "-lcudart"], check=True)
     os.replace(tmp_lib, LIB)
     return LIB
 
