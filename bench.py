@@ -51,10 +51,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
 MEASURED_TRAFFIC = {
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "86dfba1976e21fa1b36d4de9ee8e6210a200eba30d6f2f3cac20e9f962921b7c",
-                  {"e4m3_bf16_8192x8192": 170583296, "e5m2_bf16_8192x8192": 167645952,
-                   "e2m3_bf16_8192x8192": 157669632, "e3m2_bf16_8192x8192": 157880320,
-                   "e2m1_bf16_8192x8192": 148873472, "int8_bf16_8192x8192": 168344064}),
+                  "b03c7b7bbe97f5a80f5bc2dbba4ed1caa7efe47131ad5106e8f74f46fc5ed74d",
+                  {"e4m3_bf16_8192x8192": 170230528, "e5m2_bf16_8192x8192": 166918144,
+                   "e2m3_bf16_8192x8192": 157719296, "e3m2_bf16_8192x8192": 158026496,
+                   "e2m1_bf16_8192x8192": 149246720, "int8_bf16_8192x8192": 168035328}),
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
              "7e3fc2a3366087919b164dbad63ee23f0831d169cacd3f305058221d7eea9dc3",
              {"e2m1_8192x6144x4096": 78374912, "e2m1_8192x14336x4096": 227282688,
