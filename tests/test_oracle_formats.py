@@ -143,6 +143,58 @@ def test_rne_agrees_with_significand_encoder(oracle, name):
     assert bad.size == 0, [(u[i], hex(got[i]), hex(want[i])) for i in bad[:10]]
 
 
+def _rounding_classes(name):
+    """fp32 inputs covering every case RNE to `name` distinguishes: every fp32
+    exponent field 0..254 (zero, subnormals, normals up to the largest), both
+    signs, every pattern of the top mbits + 2 mantissa bits (the bits a value
+    of that binade keeps plus the next two, which decide the rounding of
+    binades down to two below) and the sticky patterns below them (none, only
+    the lowest bit, all bits, the top sticky bit alone)."""
+    mb = ind.FIELDS[name][1]
+    top = mb + 2
+    low_bits = 23 - top
+    lows = np.array([0, 1, (1 << low_bits) - 1, 1 << (low_bits - 1)], dtype=np.uint32)
+    exp = np.arange(0, 255, dtype=np.uint32)
+    hi = np.arange(1 << top, dtype=np.uint32) << low_bits
+    sign = np.array([0, 1], dtype=np.uint32) << 31
+    bits = (sign[:, None, None, None] | (exp[None, :, None, None] << 23) | hi[None, None, :, None]
+            | lows[None, None, None, :]).reshape(-1)
+    return np.unique(bits).view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("name", [n for n in NAMES if n != "int8"])
+def test_rne_rounding_classes_exhaustive(oracle, name):
+    """Oracle vs the significand-arithmetic encoder on every rounding class of
+    fp32 inputs (all exponents, all kept + guard + round bit patterns, the
+    sticky cases).  The classes at the grid's smallest binade cover the
+    element-subnormal range; those above the largest cover saturation."""
+    f = fmt_id(name)
+    u = _rounding_classes(name)
+    want = ind.encode_rne(name, u)
+    lib = oracle.lib()
+    got = np.fromiter((lib.mxref_encode_rne(f, float(x)) for x in u), dtype=np.int64, count=u.size)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, [(u[i], hex(got[i]), hex(want[i])) for i in bad[:10]]
+
+
+def test_rne_int8_rounding_classes_exhaustive(oracle):
+    """INT8 (x 2^-6): every integer step 0..128 with fractions 0, just above 0,
+    just below, at and just above one half, just below one, both signs, and
+    values far beyond the clamp."""
+    eps = 2.0 ** -30
+    k = np.arange(0, 129, dtype=np.float64)
+    fr = np.array([0.0, eps, 0.5 - eps, 0.5, 0.5 + eps, 1.0 - eps])
+    mag = ((k[:, None] + fr[None, :]) / 64.0).reshape(-1)
+    mag = np.concatenate([mag, [3.0, 1e10, 2.0 ** -40]])
+    u = np.concatenate([mag, -mag])
+    want = ind.encode_rne("int8", u)
+    lib = oracle.lib()
+    f = fmt_id("int8")
+    got = np.fromiter((lib.mxref_encode_rne(f, float(x)) for x in u), dtype=np.int64, count=u.size)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, [(u[i], hex(got[i]), hex(want[i])) for i in bad[:10]]
+
+
 @pytest.mark.parametrize("name,dtype,lim", [("e4m3", torch.float8_e4m3fn, 448.0),
                                             ("e5m2", torch.float8_e5m2, 57344.0)])
 def test_rne_agrees_with_torch_float8(oracle, name, dtype, lim):
