@@ -191,3 +191,21 @@ def unpack_codes(name: str, packed: np.ndarray, inner: int) -> np.ndarray:
     w = t[..., 0] | (t[..., 1] << 8) | (t[..., 2] << 16)
     out = np.stack([(w >> (6 * j)) & 0x3F for j in range(4)], axis=-1)
     return out.reshape(outer, inner).astype(np.int64)
+
+
+def rounding_class_bits(mbits: int) -> np.ndarray:
+    """fp32 bit patterns covering every case round-to-nearest-even onto a grid
+    with `mbits` mantissa bits distinguishes: every fp32 exponent field 0..254,
+    both signs, every pattern of the top mbits + 2 mantissa bits (kept bits of
+    a binade plus the next two, which decide the rounding of binades down to
+    two below) and the sticky patterns below them (none, only the lowest bit,
+    all bits, the top sticky bit alone).  Sorted, unique, uint32."""
+    top = mbits + 2
+    low_bits = 23 - top
+    lows = np.array([0, 1, (1 << low_bits) - 1, 1 << (low_bits - 1)], dtype=np.uint32)
+    exp = np.arange(0, 255, dtype=np.uint32)
+    hi = np.arange(1 << top, dtype=np.uint32) << low_bits
+    sign = np.array([0, 1], dtype=np.uint32) << 31
+    bits = (sign[:, None, None, None] | (exp[None, :, None, None] << 23) | hi[None, None, :, None]
+            | lows[None, None, None, :]).reshape(-1)
+    return np.unique(bits)

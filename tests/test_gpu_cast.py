@@ -7,6 +7,7 @@ import numpy as np
 import pytest
 import torch
 
+import mx_independent as ind
 from gpu_helpers import FMTS, dev, first_mismatch, host, to_device
 from microscaling_block_scaled_mx_b200 import inputs as I
 from microscaling_block_scaled_mx_b200 import mx
@@ -225,6 +226,32 @@ def test_roundtrip_config(oracle):
                           "e4m3", outer, inner, "mma", torch.float32)
         w = oracle.round_f32(oracle.dequantize(want[0], want[1], 0, outer, inner, 1))
         assert np.array_equal(host(y).view(np.uint32), w.view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt", [f for f in FMTS if f != "int8"])
+@pytest.mark.parametrize("rnd", ["rne", "sr"])
+def test_rounding_classes_at_unit_scale(oracle, fmt, rnd):
+    """Every RNE rounding class of fp32 inputs (all exponents up to the block's
+    top binade, both signs, every kept + guard + round bit pattern, the sticky
+    cases; see mx_independent.rounding_class_bits), 31 per block after a
+    leading 2^emax that fixes the block scale at 2^0: every code against the
+    oracle, including the exact ties and the saturation band."""
+    emax = {"e4m3": 8, "e5m2": 15, "e2m3": 2, "e3m2": 4, "e2m1": 2}[fmt]
+    mbits = {"e4m3": 3, "e5m2": 2, "e2m3": 3, "e3m2": 2, "e2m1": 1}[fmt]
+    cls = ind.rounding_class_bits(mbits)
+    cls = cls[((cls >> 23) & 0xff) <= 127 + emax]            # inside the scale-2^0 block
+    nb = -(-cls.size // 31)
+    nb = -(-nb // 8) * 8                                     # whole rows of 8 blocks
+    body = np.zeros(nb * 31, dtype=np.uint32)
+    body[:cls.size] = cls
+    bits = np.empty((nb, 32), dtype=np.uint32)
+    bits[:, 0] = (127 + emax) << 23
+    bits[:, 1:] = body.reshape(nb, 31)
+    x = bits.view(np.float32).reshape(nb // 8, 256)
+    got = gpu_cast(x, 1, fmt, rnd, seed=17)
+    want = oracle_cast(oracle, x, 1, fmt, rnd, seed=17)
+    assert_same(got, want, (fmt, rnd))
+    assert np.count_nonzero(got[1] == 127) == nb             # every block at scale 2^0 (the rest is padding)
 
 
 @pytest.mark.parametrize("fmt", FMTS)

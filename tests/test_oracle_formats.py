@@ -144,22 +144,7 @@ def test_rne_agrees_with_significand_encoder(oracle, name):
 
 
 def _rounding_classes(name):
-    """fp32 inputs covering every case RNE to `name` distinguishes: every fp32
-    exponent field 0..254 (zero, subnormals, normals up to the largest), both
-    signs, every pattern of the top mbits + 2 mantissa bits (the bits a value
-    of that binade keeps plus the next two, which decide the rounding of
-    binades down to two below) and the sticky patterns below them (none, only
-    the lowest bit, all bits, the top sticky bit alone)."""
-    mb = ind.FIELDS[name][1]
-    top = mb + 2
-    low_bits = 23 - top
-    lows = np.array([0, 1, (1 << low_bits) - 1, 1 << (low_bits - 1)], dtype=np.uint32)
-    exp = np.arange(0, 255, dtype=np.uint32)
-    hi = np.arange(1 << top, dtype=np.uint32) << low_bits
-    sign = np.array([0, 1], dtype=np.uint32) << 31
-    bits = (sign[:, None, None, None] | (exp[None, :, None, None] << 23) | hi[None, None, :, None]
-            | lows[None, None, None, :]).reshape(-1)
-    return np.unique(bits).view(np.float32).astype(np.float64)
+    return ind.rounding_class_bits(ind.FIELDS[name][1]).view(np.float32).astype(np.float64)
 
 
 @pytest.mark.parametrize("name", [n for n in NAMES if n != "int8"])
