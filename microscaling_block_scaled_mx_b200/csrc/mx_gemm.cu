@@ -56,6 +56,7 @@ constexpr uint32_t ACC_COLS = BN;              // accumulator b at columns [b * 
 constexpr uint32_t SF_COL = 2 * ACC_COLS;      // scale-factor columns from 384
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;   // 0.2 s when draining
+constexpr unsigned long long DRAIN_SETTLE_NS = 1000000ull;    // 1 ms for loads in flight after an abort
 
 template <bool FP4> struct Cfg {
     static constexpr int G = FP4 ? 2 : 1;             // scale atoms along K per stage
@@ -725,6 +726,14 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                     tma_load_2d_pair(sbase + C::OFF_SFB + s * C::SFB_BYTES + C::SFB_BYTES / 2, &tma_sfb, 0,
                                      2 * (rb_b1 * p.k_groups + kg), fb);
                     if (++s == STAGES_P) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (!ok) {
+                // this CTA's loads complete on CTA 0's barriers, which it cannot
+                // wait on: after an abort, give any load still in flight far more
+                // than its latency (microseconds) to land before the CTA may exit
+                const unsigned long long t0 = globaltimer();
+                while (globaltimer() - t0 < DRAIN_SETTLE_NS) {
                 }
             }
         }
