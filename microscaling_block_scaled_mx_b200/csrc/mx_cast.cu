@@ -160,6 +160,11 @@ __global__ void __launch_bounds__(256, 2) cast_rows_kernel(CastParams p) {
         q.row += step_rows;
         if (q.chunk >= cpr) { q.chunk -= cpr; ++q.row; }
     };
+    // Programmatic dependent launch: let the next kernel in the stream start
+    // placing its CTAs as this grid's CTAs finish, and touch no global memory
+    // before the grid this one depends on has completed and flushed.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // a ring of DIST + 1 load slots, indexed statically by unrolling one turn
     // of the ring: slot u is converted while slot (u + DIST) % (DIST + 1) loads
     ChunkPos pos[DIST + 1];
@@ -389,6 +394,8 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
     const int blk = warp & 3;                       // 32-row block inside the tile
     const int pair = (warp >> 2) * 32 + lane;       // column pair inside the tile
 
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");     // inputs of the previous kernel are visible
     int64_t t = blockIdx.x;
     if (t < n_tiles) stage_tile<BF16_IN>(p, col_smem, (t / tiles_c) * COL_TILE_R, (t % tiles_c) * COL_TILE_C);
     cp_async_commit();
@@ -462,6 +469,8 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
     const int col_off[2] = {tile_chunk<BF16_IN, true>(0, cbyte >> 4) * 16 + (cbyte & 15),
                             tile_chunk<BF16_IN, true>(1, cbyte >> 4) * 16 + (cbyte & 15)};
 
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");     // inputs of the previous kernel are visible
     int64_t t = blockIdx.x;
     if (t < n_tiles) stage_tile<BF16_IN, true>(pc, col_smem, (t / tiles_c) * COL_TILE_R, (t % tiles_c) * COL_TILE_C);
     cp_async_commit();
@@ -599,6 +608,9 @@ struct DequantParams {
 template <int FMT, bool BF16_OUT>
 __global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
     constexpr int BITS = Fmt<FMT>::bits;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");     // inputs of the previous kernel are visible
+
     const int64_t octs_per_row = p.inner >> 3;
     const int64_t n = p.outer * octs_per_row;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -670,6 +682,23 @@ static int resident_blocks_per_sm(int threads, int smem) {
     return cached;
 }
 
+// Launch allowed to overlap the previous kernel in the stream (programmatic
+// dependent launch); the kernel waits for that kernel's results itself.
+template <auto Kernel, typename... Args>
+static cudaError_t launch_overlapped(int grid, int block, int smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, Kernel, args...);
+}
+
 // Column cast: two tile buffers of dynamic shared memory, a resident grid.
 template <auto Kernel>
 static cudaError_t launch_cols(int in_bytes, const CastParams &p, int64_t tiles, int sms, cudaStream_t st) {
@@ -680,8 +709,8 @@ static cudaError_t launch_cols(int in_bytes, const CastParams &p, int64_t tiles,
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    Kernel<<<grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)), COL_THREADS, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_overlapped<Kernel>(grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)),
+                                     COL_THREADS, smem, st, p);
 }
 
 template <int FMT, bool SR>
@@ -697,18 +726,18 @@ static cudaError_t launch_cast_fmt(const CastParams &p, int xdt, int block_axis,
         if (bf) {
             if (v32) {
                 constexpr auto k = cast_rows_kernel<FMT, SR, true, true>;
-                k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+                return launch_overlapped<k>(grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st, p);
             } else {
                 constexpr auto k = cast_rows_kernel<FMT, SR, true, false>;
-                k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+                return launch_overlapped<k>(grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st, p);
             }
         } else {
             if (v32) {
                 constexpr auto k = cast_rows_kernel<FMT, SR, false, true>;
-                k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+                return launch_overlapped<k>(grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st, p);
             } else {
                 constexpr auto k = cast_rows_kernel<FMT, SR, false, false>;
-                k<<<grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st>>>(p);
+                return launch_overlapped<k>(grid_for(chunks, 8, sms * resident_blocks_per_sm<k>(256, 0)), 256, 0, st, p);
             }
         }
     } else {
@@ -741,9 +770,8 @@ static cudaError_t launch_dual(int in_bytes, const CastParams &pr, const CastPar
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    Kernel<<<grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)), COL_THREADS, smem, st>>>(
-        pr, pc, sr_rows, sr_cols);
-    return cudaGetLastError();
+    return launch_overlapped<Kernel>(grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)),
+                                     COL_THREADS, smem, st, pr, pc, sr_rows, sr_cols);
 }
 
 template <int FMT>
@@ -802,11 +830,10 @@ cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st) {
     p.ldy = a.ldy;
     const int grid = grid_for(a.outer * (a.inner / 8), 256, a.num_sms * 8);
     const bool bf = a.ydt == MX_BF16;
-#define MX_DQ(F)                                                        \
-    case F:                                                             \
-        if (bf) dequant_kernel<F, true><<<grid, 256, 0, st>>>(p);       \
-        else dequant_kernel<F, false><<<grid, 256, 0, st>>>(p);         \
-        break;
+#define MX_DQ(F)                                                                                      \
+    case F:                                                                                           \
+        return bf ? launch_overlapped<dequant_kernel<F, true>>(grid, 256, 0, st, p)                   \
+                  : launch_overlapped<dequant_kernel<F, false>>(grid, 256, 0, st, p);
     switch (a.fmt) {
         MX_DQ(MX_E4M3)
         MX_DQ(MX_E5M2)
@@ -817,7 +844,6 @@ cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st) {
         default: return cudaErrorInvalidValue;
     }
 #undef MX_DQ
-    return cudaGetLastError();
 }
 
 cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st) {

@@ -379,6 +379,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int num_tiles = p.tiles_m * p.tiles_n;
+    // programmatic dependent launch: barriers and tensor memory are set up
+    // above; no global memory is touched before the previous kernel is done
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == 0) {
         // ------------------------------ producer ------------------------------
@@ -688,6 +692,10 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int num_tiles = p.tiles_m * p.tiles_n;
+    // programmatic dependent launch: barriers and tensor memory are set up
+    // above; no global memory is touched before the previous kernel is done
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
 
     if (warp == 0) {
@@ -922,6 +930,23 @@ uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN) {
     return d;
 }
 
+// Launch allowed to overlap the previous kernel in the stream (programmatic
+// dependent launch); the kernel waits for that kernel's results itself.
+template <typename Kern, typename... Args>
+cudaError_t launch_overlapped(Kern kern, int grid, int smem, cudaStream_t st, const Args &...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <bool FP4, int OUT>
 cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
                         const CUtensorMap &tsb, const PairParams &p, int grid, cudaStream_t st) {
@@ -932,8 +957,7 @@ cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    kern<<<grid, NUM_THREADS, PairCfg<FP4>::SMEM, st>>>(ta, tb, tsa, tsb, p);
-    return cudaGetLastError();
+    return launch_overlapped(kern, grid, PairCfg<FP4>::SMEM, st, ta, tb, tsa, tsb, p);
 }
 
 template <bool FP4, int OUT>
@@ -945,8 +969,7 @@ cudaError_t launch(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    kern<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, p);
-    return cudaGetLastError();
+    return launch_overlapped(kern, grid, SMEM_BYTES, st, ta, tb, p);
 }
 
 template <bool FP4>
