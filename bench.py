@@ -51,15 +51,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
 MEASURED_TRAFFIC = {
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "b03c7b7bbe97f5a80f5bc2dbba4ed1caa7efe47131ad5106e8f74f46fc5ed74d",
-                  {"e4m3_bf16_8192x8192": 170230528, "e5m2_bf16_8192x8192": 166918144,
-                   "e2m3_bf16_8192x8192": 157719296, "e3m2_bf16_8192x8192": 158026496,
-                   "e2m1_bf16_8192x8192": 149246720, "int8_bf16_8192x8192": 168035328}),
+                  "419fde90cd8982daee4fc01f94633e4126b0573faff07a4579a07c76ebe83b0f",
+                  {"e4m3_bf16_8192x8192": 169978112, "e5m2_bf16_8192x8192": 167048704,
+                   "e2m3_bf16_8192x8192": 157626880, "e3m2_bf16_8192x8192": 157469952,
+                   "e2m1_bf16_8192x8192": 148634368, "int8_bf16_8192x8192": 168653568}),
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "7e3fc2a3366087919b164dbad63ee23f0831d169cacd3f305058221d7eea9dc3",
-             {"e2m1_8192x6144x4096": 78374912, "e2m1_8192x14336x4096": 227282688,
-              "e2m1_8192x4096x14336": 141698304, "e4m3_8192x3072x768": 9384704,
-              "e4m3_8192x768x3072": 28419072}),
+             "91659eff0f3eee6bbb04d9c6f09b641a5a8bcba35ff835a8a28fa362d388ab76",
+             {"e2m1_8192x6144x4096": 78150144, "e2m1_8192x14336x4096": 227906560,
+              "e2m1_8192x4096x14336": 140676096, "e4m3_8192x3072x768": 9297920,
+              "e4m3_8192x768x3072": 28422912}),
 }
 
 
