@@ -330,22 +330,20 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
             if (!packed) v[j] = scale_down<FMT>(v[j], e);
         }
         const int64_t oc = gc + col;                 // output row
-        uint32_t c[16];
+        uint32_t c[16];     // c[i]: the codes of values 2i, 2i + 1 as cvt_pair packs them
         if (SR) {
+            constexpr int PAIR_BITS = 2 * (BITS == 4 ? 4 : 8);
             const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(oc * R + gr0) >> 2);
 #pragma unroll
             for (int w = 0; w < 8; ++w) {
-                const uint32_t rw = fmix32((g + w) ^ p.key);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int j = 4 * w + k;
-                    const float m = sr_magnitude_int<FMT>(fabsf(v[j]), (rw >> (8 * k)) & 255u);
-                    v[j] = copysignf(m, v[j]);
-                }
+                const uint32_t q = sr_quad<FMT>(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3], fmix32((g + w) ^ p.key));
+                c[2 * w] = q & ((1u << PAIR_BITS) - 1u);
+                c[2 * w + 1] = q >> PAIR_BITS;
             }
-        }
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(v[j], v[j + 1]);
+            for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(v[j], v[j + 1]);
+        }
         if (nan_block) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) c[i] = 0u;

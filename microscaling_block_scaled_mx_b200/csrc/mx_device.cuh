@@ -148,6 +148,63 @@ __device__ __forceinline__ float sr_magnitude_int(float a, uint32_t r) {
     return __fsub_rn(__uint_as_float(wb), t);
 }
 
+// The same stochastic rounding for four scaled values, v_k taking byte k of
+// rw, done by the sm_100a conversion cvt.rs.satfinite.<fmt>x4.f32 d, {p0, p1,
+// p2, p3}, rbits.  Measured on B200 (every operand, every random bit, every
+// element format): d holds p0 in its top code slot down to p3 in slot 0, and
+// each operand rounds up iff the 16 bits of its value below the kept mantissa
+// plus a 16-bit random number R carry out, with R = rbits[31:16] for p1 and
+// rbits[15:0] for p3 (E2M1: bytes 3:1 and 2:0), while p0 and p2 read the same
+// bits reversed.  So only p1 and p3 carry values here, each with its byte in
+// the top half of R and zeros below: frac16 + r * 2^8 carries out exactly when
+// frac8 + r does, the rule of sr_magnitude_int (saturation and signs agree
+// too; 2^20 values per format matched it bit for bit).  p0 = p2 = 0 stay 0.
+// Returns the codes packed as cvt_pair(v0, v1) | cvt_pair(v2, v3) << (16, or 8
+// for E2M1).  INT8 has no such conversion and keeps the integer path.
+template <int FMT> __device__ __forceinline__ uint32_t cvt_rs_x4(float p1, float p3, uint32_t rbits);
+template <> __device__ __forceinline__ uint32_t cvt_rs_x4<MX_E4M3>(float p1, float p3, uint32_t rbits) {
+    uint32_t d;
+    asm("cvt.rs.satfinite.e4m3x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=r"(d) : "f"(0.0f), "f"(p1), "f"(0.0f), "f"(p3), "r"(rbits));
+    return d;
+}
+template <> __device__ __forceinline__ uint32_t cvt_rs_x4<MX_E5M2>(float p1, float p3, uint32_t rbits) {
+    uint32_t d;
+    asm("cvt.rs.satfinite.e5m2x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=r"(d) : "f"(0.0f), "f"(p1), "f"(0.0f), "f"(p3), "r"(rbits));
+    return d;
+}
+template <> __device__ __forceinline__ uint32_t cvt_rs_x4<MX_E2M3>(float p1, float p3, uint32_t rbits) {
+    uint32_t d;
+    asm("cvt.rs.satfinite.e2m3x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=r"(d) : "f"(0.0f), "f"(p1), "f"(0.0f), "f"(p3), "r"(rbits));
+    return d;
+}
+template <> __device__ __forceinline__ uint32_t cvt_rs_x4<MX_E3M2>(float p1, float p3, uint32_t rbits) {
+    uint32_t d;
+    asm("cvt.rs.satfinite.e3m2x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=r"(d) : "f"(0.0f), "f"(p1), "f"(0.0f), "f"(p3), "r"(rbits));
+    return d;
+}
+template <> __device__ __forceinline__ uint32_t cvt_rs_x4<MX_E2M1>(float p1, float p3, uint32_t rbits) {
+    uint16_t d;
+    asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=h"(d) : "f"(0.0f), "f"(p1), "f"(0.0f), "f"(p3), "r"(rbits));
+    return d;
+}
+
+template <int FMT>
+__device__ __forceinline__ uint32_t sr_quad(float v0, float v1, float v2, float v3, uint32_t rw) {
+    if constexpr (FMT == MX_INT8) {
+        auto m = [](float v, uint32_t r) { return copysignf(sr_magnitude_int<FMT>(fabsf(v), r), v); };
+        return cvt_pair<FMT>(m(v0, rw & 255u), m(v1, (rw >> 8) & 255u)) |
+               (cvt_pair<FMT>(m(v2, (rw >> 16) & 255u), m(v3, rw >> 24)) << 16);
+    } else {
+        constexpr bool FP4 = FMT == MX_E2M1;
+        // rbits: byte 2 of rw as v2's top byte, byte 0 as v0's (and 3, 1 for v3, v1)
+        const uint32_t ra = __byte_perm(rw, 0u, FP4 ? 0x2044u : 0x2404u);
+        const uint32_t rb = __byte_perm(rw, 0u, FP4 ? 0x3144u : 0x3414u);
+        const uint32_t a = cvt_rs_x4<FMT>(v2, v0, ra);   // v0 in slot 0, v2 in slot 2
+        const uint32_t b = cvt_rs_x4<FMT>(v3, v1, rb);   // v1 in slot 0, v3 in slot 2
+        return a | (b << (FP4 ? 4 : 8));
+    }
+}
+
 // MurmurHash3 32-bit finaliser (public domain, A. Appleby).
 __device__ __forceinline__ uint32_t fmix32(uint32_t h) {
     h ^= h >> 16;

@@ -102,21 +102,21 @@ __device__ __forceinline__ void encode_block32_amax(const BlockSink &o, int64_t 
             u[i + 1] = __uint_as_float(static_cast<uint32_t>(r >> 32));
         }
     }
+    // c[i]: the codes of values 2i, 2i + 1 as cvt_pair packs them
+    uint32_t c[16];
     if (SR) {
+        constexpr int PAIR_BITS = 2 * (BITS == 4 ? 4 : 8);
         const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(row * o.inner + kb * 32) >> 2);
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-            const uint32_t rw = fmix32((g + w) ^ o.key);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int j = 4 * w + k;
-                u[j] = copysignf(sr_magnitude_int<FMT>(fabsf(u[j]), (rw >> (8 * k)) & 255u), u[j]);
-            }
+            const uint32_t q = sr_quad<FMT>(u[4 * w], u[4 * w + 1], u[4 * w + 2], u[4 * w + 3], fmix32((g + w) ^ o.key));
+            c[2 * w] = q & ((1u << PAIR_BITS) - 1u);
+            c[2 * w + 1] = q >> PAIR_BITS;
         }
-    }
-    uint32_t c[16];
+    } else {
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(u[j], u[j + 1]);
+        for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(u[j], u[j + 1]);
+    }
     if (nan_block) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) c[i] = 0u;

@@ -254,6 +254,39 @@ def test_rounding_classes_at_unit_scale(oracle, fmt, rnd):
     assert np.count_nonzero(got[1] == 127) == nb             # every block at scale 2^0 (the rest is padding)
 
 
+@pytest.mark.parametrize("fmt", [f for f in FMTS if f != "int8"])
+@pytest.mark.parametrize("axis", [1, 0])
+def test_sr_carry_boundary(oracle, fmt, axis):
+    """Stochastic rounding where only the 8 bits below the grid may decide:
+    values whose fraction of a grid step is f8 / 256 plus 255, 128, 1 or 0
+    65536ths, on the subnormal grid and in every binade of a scale-2^0 block,
+    both signs.  A rounding that looked at more than 8 bits of the fraction,
+    or at more random bits than the element's byte, would round up the
+    f8 + r = 255 cases (about 1 in 256) that must round down."""
+    emax = {"e4m3": 8, "e5m2": 15, "e2m3": 2, "e3m2": 4, "e2m1": 2}[fmt]
+    mbits = {"e4m3": 3, "e5m2": 2, "e2m3": 3, "e3m2": 2, "e2m1": 1}[fmt]
+    emin = {"e4m3": -6, "e5m2": -14, "e2m3": 0, "e3m2": -2, "e2m1": 0}[fmt]
+    rng = np.random.default_rng(31)
+    nb = 8 * 512
+    n = nb * 31
+    binade = rng.integers(emin - 1, emax + 1, n)              # emin - 1: the subnormal grid
+    k = rng.integers(0, 1 << mbits, n)
+    f = rng.integers(0, 256, n) / 256.0 + rng.choice([255, 128, 1, 0], n) / 65536.0
+    base = np.where(binade < emin, 0.0, float(1 << mbits))
+    step = np.exp2(np.maximum(binade, emin) - mbits)
+    v = (base + k + f) * step * rng.choice([-1.0, 1.0], n)
+    assert np.all(v.astype(np.float32).astype(np.float64) == v)   # exact in fp32
+    x = np.empty((nb, 32), dtype=np.float32)
+    x[:, 0] = 2.0 ** emax
+    x[:, 1:] = v.reshape(nb, 31)
+    x = x.reshape(nb // 8, 256)
+    if axis == 0:
+        x = np.ascontiguousarray(x.T)
+    got = gpu_cast(x, axis, fmt, "sr", seed=23)
+    want = oracle_cast(oracle, x, axis, fmt, "sr", seed=23)
+    assert_same(got, want, (fmt, axis))
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_cast_sweep_full_size(oracle, fmt):
     """bf16 8192 x 8192 with outliers, blocks along rows, RNE: every byte."""
