@@ -300,13 +300,15 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
         am0 = pair_max16 << 16;
         am1 = pair_max16 & 0xffff0000u;
     } else {
+        float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-            am0 = __vimax3_u32(am0, static_cast<uint32_t>(x[j]) & 0x7fffffffu,
-                               static_cast<uint32_t>(x[j + 1]) & 0x7fffffffu);
-            am1 = __vimax3_u32(am1, static_cast<uint32_t>(x[j] >> 32) & 0x7fffffffu,
-                               static_cast<uint32_t>(x[j + 1] >> 32) & 0x7fffffffu);
+            m0 = max_abs3(m0, __uint_as_float(static_cast<uint32_t>(x[j])), __uint_as_float(static_cast<uint32_t>(x[j + 1])));
+            m1 = max_abs3(m1, __uint_as_float(static_cast<uint32_t>(x[j] >> 32)),
+                          __uint_as_float(static_cast<uint32_t>(x[j + 1] >> 32)));
         }
+        am0 = __float_as_uint(m0);
+        am1 = __float_as_uint(m1);
     }
     const int e0 = block_exponent<FMT>(am0), e1 = block_exponent<FMT>(am1);
     // V * 2^-e for both columns with one packed multiply (flushing

@@ -205,6 +205,18 @@ __device__ __forceinline__ uint32_t sr_quad(float v0, float v1, float v2, float 
     }
 }
 
+// Running block amax: max(m, |a|, |b|) for m >= 0 with one 3-input max.  A
+// NaN input gives the canonical NaN 0x7fffffff (like any NaN, at or above
+// the Inf pattern 0x7f800000 that marks a NaN/Inf block); subnormal inputs are
+// kept (no .ftz), so the result's bits equal the integer maximum of the
+// magnitude bits for every non-NaN input.
+__device__ __forceinline__ float max_abs3(float m, float a, float b) {
+    float r;
+    asm("{\n\t.reg .f32 ta, tb;\n\tabs.f32 ta, %2;\n\tabs.f32 tb, %3;\n\tmax.NaN.f32 %0, %1, ta, tb;\n\t}"
+        : "=f"(r) : "f"(m), "f"(a), "f"(b));
+    return r;
+}
+
 // MurmurHash3 32-bit finaliser (public domain, A. Appleby).
 __device__ __forceinline__ uint32_t fmix32(uint32_t h) {
     h ^= h >> 16;

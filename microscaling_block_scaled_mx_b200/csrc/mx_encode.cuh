@@ -54,7 +54,8 @@ __device__ __forceinline__ void store_code32(uint8_t *dst, const uint4 &a, const
 // and the packed codes and scale byte of block (row, kb).  SR's index is the
 // element's position row * inner + kb * 32 + j in the output.
 // amax_bits: the largest |b[i]| as FP32 bits (sign cleared), computed by the
-// caller (encode_block32 below, or bf16_amax_bits from the packed input).
+// caller (encode_block32 below, or bf16_max_bits of the packed input); for a
+// block holding a NaN it may be any pattern at or above 0x7f800000.
 template <int FMT, bool SR, bool V32>
 __device__ __forceinline__ void encode_block32_amax(const BlockSink &o, int64_t row, int64_t kb, uint32_t (&b)[32],
                                                     uint32_t amax_bits) {
@@ -154,11 +155,10 @@ __device__ __forceinline__ void encode_block32_amax(const BlockSink &o, int64_t 
 
 template <int FMT, bool SR, bool V32>
 __device__ __forceinline__ void encode_block32(const BlockSink &o, int64_t row, int64_t kb, uint32_t (&b)[32]) {
-    uint32_t amax_bits = 0;
+    float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; i += 2)
-        amax_bits = __vimax3_u32(amax_bits, b[i] & 0x7fffffffu, b[i + 1] & 0x7fffffffu);
-    encode_block32_amax<FMT, SR, V32>(o, row, kb, b, amax_bits);
+    for (int i = 0; i < 32; i += 2) m = max_abs3(m, __uint_as_float(b[i]), __uint_as_float(b[i + 1]));
+    encode_block32_amax<FMT, SR, V32>(o, row, kb, b, __float_as_uint(m));
 }
 
 // Packed 16-bit maximum of |bf16| over NW words of two bf16 values each (one
