@@ -51,15 +51,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
 MEASURED_TRAFFIC = {
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "419fde90cd8982daee4fc01f94633e4126b0573faff07a4579a07c76ebe83b0f",
-                  {"e4m3_bf16_8192x8192": 169978112, "e5m2_bf16_8192x8192": 167048704,
-                   "e2m3_bf16_8192x8192": 157626880, "e3m2_bf16_8192x8192": 157469952,
-                   "e2m1_bf16_8192x8192": 148634368, "int8_bf16_8192x8192": 168653568}),
+                  "cdc494636913d3e605f5eb6465ccfd08358112037dacf17a084e390dcde06110",
+                  {"e4m3_bf16_8192x8192": 169413120, "e5m2_bf16_8192x8192": 166688000,
+                   "e2m3_bf16_8192x8192": 158004736, "e3m2_bf16_8192x8192": 157851392,
+                   "e2m1_bf16_8192x8192": 148614912, "int8_bf16_8192x8192": 168644352}),
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "91659eff0f3eee6bbb04d9c6f09b641a5a8bcba35ff835a8a28fa362d388ab76",
-             {"e2m1_8192x6144x4096": 78150144, "e2m1_8192x14336x4096": 227906560,
-              "e2m1_8192x4096x14336": 140676096, "e4m3_8192x3072x768": 9297920,
-              "e4m3_8192x768x3072": 28422912}),
+             "db828a7e6e32df7df86765366ef57954ea60eaa4be4d59e8de98cf141f45f56c",
+             {"e2m1_8192x6144x4096": 78426624, "e2m1_8192x14336x4096": 227905024,
+              "e2m1_8192x4096x14336": 141267200, "e4m3_8192x3072x768": 9491968,
+              "e4m3_8192x768x3072": 28422656}),
 }
 
 
