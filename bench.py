@@ -51,7 +51,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
 MEASURED_TRAFFIC = {
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "cdc494636913d3e605f5eb6465ccfd08358112037dacf17a084e390dcde06110",
+                  "f5802bd3bf270f24c9b8a84decb2665d2ea13f86d92f074446bf7655a343793d",
                   {"e4m3_bf16_8192x8192": 169413120, "e5m2_bf16_8192x8192": 166688000,
                    "e2m3_bf16_8192x8192": 158004736, "e3m2_bf16_8192x8192": 157851392,
                    "e2m1_bf16_8192x8192": 148614912, "int8_bf16_8192x8192": 168644352}),

@@ -106,35 +106,19 @@ template <> __device__ __forceinline__ uint32_t cvt_pair<MX_INT8>(float a, float
     return one(a) | (one(b) << 8);
 }
 
-// Stochastic rounding of a non-negative FP32 value onto the element grid: with
-// lo the grid point at or below a and s the grid step there, take the 8 bits
-// of (a - lo) / s just below the step, F; the result is lo + s when
-// F + r >= 256, else lo; a >= max gives max.  Every step is exact in FP32.
-template <int FMT>
-__device__ __forceinline__ float sr_magnitude(float a, uint32_t r) {
-    using F = Fmt<FMT>;
-    if (a >= F::maxv) return F::maxv;
-    int ea = static_cast<int>(__float_as_uint(a) >> 23) - 127;   // -127 for 0 / subnormal
-    int E = ea < F::emin ? F::emin : ea;
-    if (FMT == MX_INT8) E = 0;
-    float inv_step = pow2f(F::mbits - E);
-    float step = pow2f(E - F::mbits);
-    float q = a * inv_step;
-    float lo = floorf(q);
-    uint32_t frac8 = static_cast<uint32_t>((q - lo) * 256.0f);
-    float t = (frac8 + r >= 256u) ? lo + 1.0f : lo;
-    return t * step;
-}
-
-// The same stochastic rounding in integer arithmetic, as used by the strided
-// (weight-gradient) cast.  For a >= 2^emin the grid step of a's binade is one
-// unit of fp32 mantissa bit (23 - mbits): adding r at the eight bits below that
-// unit carries into it exactly when F + r >= 256, and truncation then gives
-// lo or lo + step.  For a < 2^emin (the element's subnormal range, uniform
-// step 2^(emin - mbits)) a is first shifted to a + 2^emin with a
-// round-toward-zero add, which keeps every bit that F depends on, rounded
-// the same way, and shifted back exactly.  Returns the rounded magnitude
-// (callers convert it with a saturating conversion).
+// Stochastic rounding of a non-negative FP32 value a onto the element grid:
+// with lo the grid point at or below a and s the grid step there, F = the 8
+// bits of (a - lo) / s just below the step; the result is lo + s when F + r >=
+// 256, else lo (r the random byte).  In integer arithmetic: for a >= 2^emin the
+// grid step of a's binade is one unit of fp32 mantissa bit (23 - mbits), so
+// adding r at the eight bits below that unit carries into it exactly when
+// F + r >= 256, and truncation then gives lo or lo + step.  For a < 2^emin
+// (the element's subnormal range, uniform step 2^(emin - mbits)) a is first
+// shifted to a + 2^emin with a round-toward-zero add, which keeps every bit
+// that F depends on, rounded the same way, and shifted back exactly.  Returns
+// the rounded magnitude (callers convert it with a saturating conversion).
+// INT8 uses it directly; the other formats round the same way in hardware
+// (sr_quad below).
 template <int FMT>
 __device__ __forceinline__ float sr_magnitude_int(float a, uint32_t r) {
     using F = Fmt<FMT>;
