@@ -51,15 +51,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
 MEASURED_TRAFFIC = {
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "f5802bd3bf270f24c9b8a84decb2665d2ea13f86d92f074446bf7655a343793d",
-                  {"e4m3_bf16_8192x8192": 169413120, "e5m2_bf16_8192x8192": 166688000,
-                   "e2m3_bf16_8192x8192": 158004736, "e3m2_bf16_8192x8192": 157851392,
-                   "e2m1_bf16_8192x8192": 148614912, "int8_bf16_8192x8192": 168644352}),
+                  "21c13cd4e7a3657226ce260915a58d45276e77cba8f53b8744192be6197a113e",
+                  {"e4m3_bf16_8192x8192": 169430272, "e5m2_bf16_8192x8192": 166759168,
+                   "e2m3_bf16_8192x8192": 158376192, "e3m2_bf16_8192x8192": 157790976,
+                   "e2m1_bf16_8192x8192": 148557312, "int8_bf16_8192x8192": 169712384}),
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "db828a7e6e32df7df86765366ef57954ea60eaa4be4d59e8de98cf141f45f56c",
-             {"e2m1_8192x6144x4096": 78426624, "e2m1_8192x14336x4096": 227905024,
-              "e2m1_8192x4096x14336": 141267200, "e4m3_8192x3072x768": 9491968,
-              "e4m3_8192x768x3072": 28422656}),
+             "c0792af6b749f96e1b6170749458bf04f9760c61c60696dc34860212860cebd0",
+             {"e2m1_8192x6144x4096": 78123264, "e2m1_8192x14336x4096": 227853056,
+              "e2m1_8192x4096x14336": 138795520, "e4m3_8192x3072x768": 9282304,
+              "e4m3_8192x768x3072": 28421120}),
 }
 
 

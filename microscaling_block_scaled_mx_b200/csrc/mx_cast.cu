@@ -332,34 +332,28 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
             if (!packed) v[j] = scale_down<FMT>(v[j], e);
         }
         const int64_t oc = gc + col;                 // output row
-        uint32_t c[16];     // c[i]: the codes of values 2i, 2i + 1 as cvt_pair packs them
+        // pw[w]: the codes of values 4w .. 4w + 3, one per byte (per nibble for E2M1)
+        constexpr int SLOT = BITS == 4 ? 4 : 8;
+        uint32_t pw[8];
         if (SR) {
-            constexpr int PAIR_BITS = 2 * (BITS == 4 ? 4 : 8);
             const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(oc * R + gr0) >> 2);
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                const uint32_t q = sr_quad<FMT>(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3], fmix32((g + w) ^ p.key));
-                c[2 * w] = q & ((1u << PAIR_BITS) - 1u);
-                c[2 * w + 1] = q >> PAIR_BITS;
-            }
+            for (int w = 0; w < 8; ++w)
+                pw[w] = sr_quad<FMT>(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3], fmix32((g + w) ^ p.key));
         } else {
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) c[j >> 1] = cvt_pair<FMT>(v[j], v[j + 1]);
+            for (int w = 0; w < 8; ++w)
+                pw[w] = cvt_pair<FMT>(v[4 * w], v[4 * w + 1]) | (cvt_pair<FMT>(v[4 * w + 2], v[4 * w + 3]) << (2 * SLOT));
         }
-        if (nan_block) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) c[i] = 0u;
-        }
+        const uint32_t keep = nan_block ? 0u : 0xffffffffu;     // a NaN/Inf block stores zero codes
         if (BITS == 8) {
             uint4 *dst = reinterpret_cast<uint4 *>(p.codes + oc * R + gr0);
-            dst[0] = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
-            dst[1] = make_uint4(c[8] | (c[9] << 16), c[10] | (c[11] << 16), c[12] | (c[13] << 16),
-                                c[14] | (c[15] << 16));
+            dst[0] = make_uint4(pw[0] & keep, pw[1] & keep, pw[2] & keep, pw[3] & keep);
+            dst[1] = make_uint4(pw[4] & keep, pw[5] & keep, pw[6] & keep, pw[7] & keep);
         } else if (BITS == 4) {
             uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                w[i] = c[4 * i] | (c[4 * i + 1] << 8) | (c[4 * i + 2] << 16) | (c[4 * i + 3] << 24);
+            for (int i = 0; i < 4; ++i) w[i] = (pw[2 * i] | (pw[2 * i + 1] << 16)) & keep;
             *reinterpret_cast<uint4 *>(p.codes + oc * (R >> 1) + (gr0 >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
         } else {
             uint64_t *dst = reinterpret_cast<uint64_t *>(p.codes + oc * (R / 4 * 3) + gr0 / 4 * 3);
@@ -369,11 +363,11 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int bit = 6 * j - 64 * q;
-                    const uint64_t code = (c[j >> 1] >> (8 * (j & 1))) & 0x3fu;
+                    const uint64_t code = (pw[j >> 2] >> (8 * (j & 3))) & 0x3fu;
                     if (bit >= 0 && bit < 64) w |= code << bit;
                     else if (bit < 0 && bit > -6) w |= code >> (-bit);
                 }
-                dst[q] = w;
+                dst[q] = w & (static_cast<uint64_t>(keep) << 32 | keep);
             }
         }
         store_scale(p, oc, gr0 >> 5, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
