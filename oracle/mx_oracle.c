@@ -29,7 +29,10 @@
  * OCP MX v1.0 definition the summary page refers to.  Readings taken where the
  * pages are silent (all-zero block scale, signed zero, INT8 -128, the
  * stochastic-rounding width and hash, the Hadamard normalisation and sign mask)
- * are marked "reading:" below.
+ * are marked "reading:" below.  Parity unpinned: nothing outside the oracle
+ * fixes which of those readings the pages' authors used, so the functions
+ * that apply them are pinned only on their arithmetic (round-up counts,
+ * published hash vectors, the Sylvester matrix product), not on the choice.
  *
  * Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -fPIC -shared.
  * No fast-math, no FMA contraction: every float operation is a single IEEE
