@@ -209,3 +209,152 @@ def rounding_class_bits(mbits: int) -> np.ndarray:
     bits = (sign[:, None, None, None] | (exp[None, :, None, None] << 23) | hi[None, None, :, None]
             | lows[None, None, None, :]).reshape(-1)
     return np.unique(bits)
+
+
+# --------------------------------------------------------------------------
+# Stochastic rounding and the whole block cast, restated independently.
+#
+# The oracle's stochastic rounding (C, table search, one scalar element at a
+# time) is pinned here by a vectorised numpy restatement of the definition:
+#   * the random byte of the element at linear position i of the
+#     block-axis-major OUTPUT (i = outer_index * inner_length + inner_index)
+#     is byte (i mod 4) of fmix32(floor(i / 4) xor key), where
+#     key = fmix32(low 32 bits of the seed) xor (high 32 bits of the seed) and
+#     fmix32 is the MurmurHash3 32-bit finaliser;
+#   * with lo <= |u| < hi the two grid points around |u|, the magnitude rounds
+#     up iff floor(256 (|u| - lo) / (hi - lo)) + r >= 256; |u| >= max gives max;
+#     the sign is put back afterwards (FP formats keep the sign of zero).
+# The hash below is checked on its own against the published MurmurHash3
+# vectors (tests/golden/murmur3_x86_32.txt), so nothing here is taken from the
+# oracle.
+# --------------------------------------------------------------------------
+
+_M32 = np.uint64(0xFFFFFFFF)
+
+
+def fmix32(h) -> np.ndarray:
+    """MurmurHash3's 32-bit finaliser, vectorised (uint32 in, uint32 out)."""
+    h = np.asarray(h, dtype=np.uint64) & _M32
+    h ^= h >> np.uint64(16)
+    h = (h * np.uint64(0x85EBCA6B)) & _M32
+    h ^= h >> np.uint64(13)
+    h = (h * np.uint64(0xC2B2AE35)) & _M32
+    h ^= h >> np.uint64(16)
+    return h.astype(np.uint32)
+
+
+def murmur3_x86_32(data: bytes, seed: int) -> int:
+    """The whole MurmurHash3_x86_32 around this module's fmix32."""
+    c1, c2 = 0xCC9E2D51, 0x1B873593
+
+    def rotl(x, r):
+        return ((x << r) | (x >> (32 - r))) & 0xFFFFFFFF
+
+    h = seed & 0xFFFFFFFF
+    n = len(data) // 4
+    for i in range(n):
+        k = int.from_bytes(data[4 * i:4 * i + 4], "little")
+        h ^= (rotl((k * c1) & 0xFFFFFFFF, 15) * c2) & 0xFFFFFFFF
+        h = (rotl(h, 13) * 5 + 0xE6546B64) & 0xFFFFFFFF
+    if len(data) % 4:
+        k = int.from_bytes(data[4 * n:], "little")
+        h ^= (rotl((k * c1) & 0xFFFFFFFF, 15) * c2) & 0xFFFFFFFF
+    return int(fmix32(h ^ len(data)))
+
+
+def sr_key(seed: int) -> int:
+    seed &= (1 << 64) - 1
+    return int(fmix32(seed & 0xFFFFFFFF)) ^ (seed >> 32)
+
+
+def sr_bytes(seed: int, idx) -> np.ndarray:
+    """Random byte of each linear output position idx (any integer array)."""
+    idx = np.asarray(idx, dtype=np.uint64)
+    words = fmix32(((idx >> np.uint64(2)) & _M32) ^ np.uint64(sr_key(seed)))
+    shift = (np.uint64(8) * (idx & np.uint64(3))).astype(np.uint32)
+    return ((words >> shift) & np.uint32(0xFF)).astype(np.int64)
+
+
+def encode_sr(name: str, u: np.ndarray, r: np.ndarray) -> np.ndarray:
+    """Stochastic rounding onto the element grid by significand arithmetic.
+
+    u: finite float64 values already divided by the block scale; r: one
+    random byte (0..255) per value."""
+    u = np.asarray(u, dtype=np.float64)
+    r = np.asarray(r, dtype=np.int64)
+    a = np.abs(u)
+    neg = np.signbit(u)
+    vmax = FORMATS[name]["max"]
+    q = grid_spacing(name, a)                  # spacing of the grid at |u|
+    lo = np.floor(a / q) * q                   # exact: q is a power of two
+    f = np.floor((a - lo) / q * 256.0).astype(np.int64)
+    mag = np.where(f + r >= 256, lo + q, lo)
+    mag = np.where(a >= vmax, vmax, mag)
+    # the magnitude is on the grid: its RNE code is its code
+    code = encode_rne(name, mag)
+    if name == "int8":
+        return np.where(neg & (code != 0), (256 - code) % 256, code).astype(np.int64)
+    bits = 8 if name == "e5m2" or name == "e4m3" else (6 if name in ("e2m3", "e3m2") else 4)
+    return np.where(neg, code | (1 << (bits - 1)), code).astype(np.int64)
+
+
+def hadamard_blocks(v: np.ndarray, sign_mask: int) -> np.ndarray:
+    """Fixed-sign 32-point Hadamard on the last axis (length 32), in float32.
+
+    Position j is negated unless bit j of sign_mask is set; then five butterfly
+    stages with distance 1, 2, 4, 8, 16, each replacing the pair (x_i, x_{i+h})
+    (i with bit h clear) by (x_i + x_{i+h}, x_i - x_{i+h}), every operation an
+    IEEE float32 add or subtract."""
+    x = np.array(v, dtype=np.float32, copy=True)
+    keep = ((np.uint64(sign_mask) >> np.arange(32, dtype=np.uint64)) & np.uint64(1)).astype(bool)
+    x[..., ~keep] = -x[..., ~keep]
+    pos = np.arange(32)
+    for h in (1, 2, 4, 8, 16):
+        i = pos[(pos & h) == 0]
+        a, b = x[..., i].copy(), x[..., i + h].copy()
+        x[..., i] = a + b
+        x[..., i + h] = a - b
+    return x
+
+
+def quantize(x: np.ndarray, block_axis: int, name: str, sr: bool = False, seed: int = 0,
+             hadamard: bool = False, sign_mask: int = 0, mma_layout: bool = False):
+    """The whole MX cast of a 2-D tensor: float32 values, or bf16 bits as uint16.
+
+    Returns (packed codes, scales) in the library's storage layout: codes one
+    row per line along the block axis (transposed for block_axis 0), scales
+    plain (outer x inner/32) or in the tensor-core layout (padding bytes 0)."""
+    v = bf16_bits_to_f32(x) if x.dtype == np.uint16 else np.asarray(x, dtype=np.float32)
+    if block_axis == 0:
+        v = v.T
+    outer, inner = v.shape
+    assert inner % 32 == 0
+    blocks = np.ascontiguousarray(v).reshape(outer, inner // 32, 32)
+    if hadamard:
+        blocks = hadamard_blocks(blocks, sign_mask)
+    # FP32 subnormal -> signed zero, before anything else looks at the values
+    tiny = np.abs(blocks) < np.float32(2.0 ** -126)
+    blocks = np.where(tiny, np.copysign(np.float32(0.0), blocks), blocks).astype(np.float32)
+    w = blocks.astype(np.float64)
+    bad = ~np.all(np.isfinite(w), axis=-1)
+    amax = np.max(np.abs(np.where(np.isfinite(w), w, 0.0)), axis=-1)
+    _, ex = np.frexp(amax)
+    emax = {"e4m3": 8, "e5m2": 15, "e2m3": 2, "e3m2": 4, "e2m1": 2, "int8": 0}[name]
+    e = np.clip(np.where(amax > 0, ex - 1 - emax, -127), -127, 127)
+    u = np.where(np.isfinite(w), w, 0.0) * np.exp2(-e.astype(np.float64))[..., None]
+    if sr:
+        idx = (np.arange(outer, dtype=np.uint64)[:, None] * np.uint64(inner)
+               + np.arange(inner, dtype=np.uint64)[None, :]).reshape(outer, inner // 32, 32)
+        codes = encode_sr(name, u, sr_bytes(seed, idx))
+    else:
+        codes = encode_rne(name, u)
+    codes = np.where(bad[..., None], 0, codes)
+    scale = np.where(bad, 255, e + 127).astype(np.uint8)
+    packed = pack_codes(name, codes.reshape(outer, inner))
+    if not mma_layout:
+        return packed, scale.reshape(-1)
+    perm = mma_scale_permutation(outer, inner // 32)
+    rp, kp = (outer + 127) // 128 * 128, (inner // 32 + 3) // 4 * 4
+    out = np.zeros(rp * kp, dtype=np.uint8)
+    out[perm.reshape(-1)] = scale.reshape(-1)
+    return packed, out

@@ -303,11 +303,10 @@ def _sweep_input():
     return _SWEEP["x"]
 
 
-def test_wgrad_casts_full_size(oracle):
+def test_wgrad_casts_full_size(oracle, wgrad_oracle_operands):
     """dY 16384 x 4096 and X 16384 x 14336 (bf16, Student-t), cast along tokens
     with the fixed-sign Hadamard and stochastic rounding to E2M1: every byte."""
-    dy, xx = I.wgrad_operands()
-    for name, t, seed in (("dY", dy, 42), ("X", xx, 43)):
+    d = wgrad_oracle_operands
+    for name, t, seed, want in (("dY", d["dy"], 42, d["dy_q"]), ("X", d["xx"], 43, d["xx_q"])):
         got = gpu_cast(t, 0, "e2m1", "sr", seed=seed, hadamard=True)
-        want = oracle_cast(oracle, t, 0, "e2m1", "sr", seed=seed, hadamard=True)
         assert_same(got, want, name)

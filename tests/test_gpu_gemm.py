@@ -236,13 +236,23 @@ def test_gemm_gpt2_config(oracle, idx):
 
 @pytest.mark.parametrize("idx", [0, 1, 2])
 def test_gemm_llama3_config(oracle, idx):
-    """Llama-3-8B-shaped MXFP4 GEMMs along K, bf16 out: 384 sampled rows of C
-    (every column)."""
+    """Llama-3-8B-shaped MXFP4 GEMMs along K, bf16 out: 512 sampled rows of C
+    (every column) and four whole 128 x 128 output tiles."""
     M, N, K = I.LLAMA3_GEMMS[idx]
     x, w = I.linear_operands(M, K, N, 3, stream=idx)
-    rows = np.sort(np.random.default_rng(idx).choice(M, 384, replace=False))
-    got, ref, bound = run_gemm(oracle, x, w, "e2m1", M, N, K, out_dtype=torch.bfloat16, rows=rows)
-    check(got, ref, bound, torch.bfloat16, (M, N, K))
+    rng = np.random.default_rng(idx)
+    rows = np.sort(rng.choice(M, 512, replace=False))
+    tiles = [(int(rng.integers(M // 128)) * 128, int(rng.integers(N // 128)) * 128) for _ in range(4)]
+    tile_rows = np.unique(np.concatenate([np.arange(m0, m0 + 128) for m0, _ in tiles]))
+    all_rows = np.union1d(rows, tile_rows)
+    got, ref, bound = run_gemm(oracle, x, w, "e2m1", M, N, K, out_dtype=torch.bfloat16, rows=all_rows)
+    pos = {int(r): i for i, r in enumerate(all_rows)}
+    sel = np.array([pos[int(r)] for r in rows])
+    check(got[sel], ref[sel], bound[sel], torch.bfloat16, (M, N, K, "rows"))
+    for m0, n0 in tiles:
+        ti = np.array([pos[r] for r in range(m0, m0 + 128)])
+        check(got[ti, n0:n0 + 128], ref[ti, n0:n0 + 128], bound[ti, n0:n0 + 128], torch.bfloat16,
+              (M, N, K, "tile", m0, n0))
 
 
 def test_gemm_llama3_along_m(oracle):
@@ -268,22 +278,36 @@ def test_gemm_llama3_along_m(oracle):
     check(to_f64(dw)[rows], ref, bound, torch.float32, "along M")
 
 
-def test_gemm_wgrad_config(oracle):
+def test_gemm_wgrad_config(oracle, wgrad_oracle_operands):
     """dW = alpha * dY^T X with tokens K=16384: dY 16384x4096 and X 16384x14336
     (Student-t), both cast along tokens with the fixed-sign Hadamard and
-    stochastic rounding to E2M1, alpha = 1/32, fp32 out; 256 sampled rows."""
-    dy, xx = I.wgrad_operands()
+    stochastic rounding to E2M1, alpha = 1/32, fp32 out; 512 sampled rows and
+    four whole 128 x 128 tiles.  The reference is computed from the oracle's
+    own casts of dY and X; the GPU's casts must equal them byte for byte."""
+    d = wgrad_oracle_operands
+    dy, xx = d["dy"], d["xx"]
     T, Do = dy.shape
     Di = xx.shape[1]
-    ac, as_ = mx.quantize(to_device(dy), 0, "e2m1", rnd="sr", seed=42, hadamard=True)
-    bc, bs = mx.quantize(to_device(xx), 0, "e2m1", rnd="sr", seed=43, hadamard=True)
+    (oac, oas), (obc, obs) = d["dy_q"], d["xx_q"]
+    ac, as_ = mx.quantize(to_device(dy), 0, "e2m1", rnd="sr", seed=42, hadamard=True, sign_mask=d["mask"])
+    bc, bs = mx.quantize(to_device(xx), 0, "e2m1", rnd="sr", seed=43, hadamard=True, sign_mask=d["mask"])
     dw = mx.gemm(ac, as_, bc, bs, Do, Di, T, fa="e2m1", alpha=1.0 / 32, out_dtype=torch.float32)
     torch.cuda.synchronize()
-    rows = np.sort(np.random.default_rng(9).choice(Do, 256, replace=False))
-    # the operands are bit-identical to the oracle's (checked by the cast tests)
-    ref, bound = oracle.gemm_decoded(host(ac), host(as_), oracle.E2M1, host(bc), host(bs), oracle.E2M1,
-                                     Do, Di, T, alpha=1.0 / 32, rows=rows)
-    check(to_f64(dw)[rows], ref, bound, torch.float32, "wgrad")
+    assert np.array_equal(host(ac), oac) and np.array_equal(host(as_)[:oas.size], oas)
+    assert np.array_equal(host(bc), obc) and np.array_equal(host(bs)[:obs.size], obs)
+    rng = np.random.default_rng(9)
+    rows = np.sort(rng.choice(Do, 512, replace=False))
+    tiles = [(int(rng.integers(Do // 128)) * 128, int(rng.integers(Di // 128)) * 128) for _ in range(4)]
+    all_rows = np.union1d(rows, np.concatenate([np.arange(m0, m0 + 128) for m0, _ in tiles]))
+    ref, bound = oracle.gemm_decoded(oac, oas, oracle.E2M1, obc, obs, oracle.E2M1, Do, Di, T,
+                                     alpha=1.0 / 32, rows=all_rows)
+    got = to_f64(dw)[all_rows]
+    check(got, ref, bound, torch.float32, "wgrad")
+    pos = {int(r): i for i, r in enumerate(all_rows)}
+    for m0, n0 in tiles:
+        ti = np.array([pos[r] for r in range(m0, m0 + 128)])
+        check(got[ti, n0:n0 + 128], ref[ti, n0:n0 + 128], bound[ti, n0:n0 + 128], torch.float32,
+              ("wgrad tile", m0, n0))
 
 
 @pytest.mark.parametrize("M,N,K", [(256, 256, 1024), (4096, 2560, 2048)])
