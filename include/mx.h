@@ -210,7 +210,10 @@ MX_API int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_s
  *  b_codes has the same alignment rule for fb.
  * Supported: fa, fb each any of MX_E4M3, MX_E5M2, MX_E2M3, MX_E3M2, MX_E2M1
  * (mixed pairs included, e.g. MXFP4 weights x MXFP6 activations), with
- * K % 128 == 0 and any M, N >= 1.  fa == fb == MX_E2M1 with K % 256 == 0 runs
+ * K % 128 == 0 and any M, N >= 1.  Size limit: M, N and K at most 2^31 - 1 and
+ * ceil(M / 128) * ceil(N / 128) at most 2^31 - 1 (the kernels index with
+ * 32-bit integers); larger sizes give MX_ERR_UNSUPPORTED before anything is
+ * launched.  fa == fb == MX_E2M1 with K % 256 == 0 runs
  * kind::mxf4 on the packed codes; every other pair runs kind::mxf8f6f4, whose
  * operands the copy engine expands to one code per byte in shared memory.
  * MX_INT8 operands give MX_ERR_UNSUPPORTED (sm_100a has no block-scaled
@@ -237,7 +240,8 @@ MX_API int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
  * GEMM's fp32 accumulator, so the result is the bytes mx_quantize(block_axis
  * 1) would write for the fp32 C that mx_gemm returns.
  *
- *  a_codes ... alpha   as for mx_gemm (same formats, K % 128 == 0).
+ *  a_codes ... alpha   as for mx_gemm (same formats, K % 128 == 0, same
+ *             size limit).
  *  out_fmt    element format of C's codes (any mx_fmt, MX_INT8 included).
  *  out_rnd, out_seed   RNE, or SR with C's element index m * N + n.
  *  out_codes  device, M x (N * bits / 8) bytes, 16-byte aligned.

@@ -14,10 +14,11 @@ extern "C" {
 
 /*
  * mx_debug_gemm_skip_stage -- arm (k_tile >= 0) or disarm (k_tile < 0) a
- * one-shot injected stall for the next mx_gemm call on this host thread's
- * process: the producer of the first CTA does not issue the loads of its first
- * tile's k-tile `k_tile`, so the MMA issuer's bounded wait on that stage runs
- * out (after about 2 s).  The kernel then records MX_ERR_TIMEOUT in the device
+ * one-shot injected stall for the next mx_gemm or mx_gemm_quantize call made
+ * by the calling host thread (calls from other threads are not affected):
+ * the producer of the first CTA does not issue the loads of its first tile's
+ * k-tile `k_tile`, so the MMA issuer's bounded wait on that stage runs out
+ * (after about 2 s).  The kernel then records MX_ERR_TIMEOUT in the device
  * status word (read with mx_last_device_status), waits for the copies it did
  * issue, frees its tensor memory and returns; the CUDA context stays usable.
  * C is left partly unwritten.  Returns MX_OK.

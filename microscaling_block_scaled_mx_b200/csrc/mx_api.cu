@@ -176,6 +176,13 @@ int check_gemm_operands(const void *a_codes, const void *a_scales, mx_fmt fa, co
     return MX_OK;
 }
 
+// The GEMM kernels index rows, columns, K and tiles with 32-bit integers.
+bool gemm_dims_fit(int64_t M, int64_t N, int64_t K) {
+    constexpr int64_t kMax = 2147483647;
+    if (M > kMax || N > kMax || K > kMax) return false;
+    return ((M + 127) / 128) * ((N + 127) / 128) <= kMax;
+}
+
 MxGemmArgs gemm_args(const void *a_codes, const void *a_scales, mx_fmt fa, const void *b_codes,
                      const void *b_scales, mx_fmt fb, int64_t M, int64_t N, int64_t K, float alpha) {
     MxGemmArgs a;
@@ -199,6 +206,7 @@ int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
     (void)ws_bytes;
     if (elem_bits(fa) == 0 || elem_bits(fb) == 0 || (cdt != MX_F32 && cdt != MX_BF16)) return MX_ERR_ARG;
     if (M < 0 || N < 0 || K < 0) return MX_ERR_ARG;
+    if (!gemm_dims_fit(M, N, K)) return MX_ERR_UNSUPPORTED;
     if (K % 32 != 0) return MX_ERR_SHAPE;
     if (M == 0 || N == 0) return MX_OK;                  // empty: pointers may be NULL
     if (!c || ldc < N) return MX_ERR_ARG;
@@ -226,6 +234,7 @@ int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa,
     if ((out_rnd != MX_RNE && out_rnd != MX_SR) || (out_sl != MX_SCALES_PLAIN && out_sl != MX_SCALES_MMA))
         return MX_ERR_ARG;
     if (M < 0 || N < 0 || K < 0) return MX_ERR_ARG;
+    if (!gemm_dims_fit(M, N, K)) return MX_ERR_UNSUPPORTED;
     if (K % 32 != 0 || N % 32 != 0) return MX_ERR_SHAPE;  // C's blocks run along N
     if (M == 0 || N == 0) return MX_OK;                   // empty: pointers may be NULL
     if (!out_codes || !out_scales) return MX_ERR_ARG;

@@ -697,12 +697,8 @@ static cudaError_t launch_overlapped(int grid, int block, int smem, cudaStream_t
 template <auto Kernel>
 static cudaError_t launch_cols(int in_bytes, const CastParams &p, int64_t tiles, int sms, cudaStream_t st) {
     const int smem = 2 * COL_TILE_R * COL_TILE_C * in_bytes;
-    static bool configured = false;    // per template instance, i.e. per kernel
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};    // per kernel, one bit per device
+    if (cudaError_t e = ensure_smem_limit(Kernel, smem, configured); e != cudaSuccess) return e;
     return launch_overlapped<Kernel>(grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)),
                                      COL_THREADS, smem, st, p);
 }
@@ -758,12 +754,8 @@ template <auto Kernel>
 static cudaError_t launch_dual(int in_bytes, const CastParams &pr, const CastParams &pc, int sr_rows, int sr_cols,
                                int64_t tiles, int sms, cudaStream_t st) {
     const int smem = 2 * COL_TILE_R * COL_TILE_C * in_bytes;
-    static bool configured = false;    // per template instance, i.e. per kernel
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};    // per kernel, one bit per device
+    if (cudaError_t e = ensure_smem_limit(Kernel, smem, configured); e != cudaSuccess) return e;
     return launch_overlapped<Kernel>(grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)),
                                      COL_THREADS, smem, st, pr, pc, sr_rows, sr_cols);
 }

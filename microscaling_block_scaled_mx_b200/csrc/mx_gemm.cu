@@ -859,6 +859,61 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 
 int elem_bits(int f) { return f == MX_E2M1 ? 4 : (f == MX_E2M3 || f == MX_E3M2) ? 6 : 8; }
 
+// Encoded 2-D tensor maps, reused across calls.  A map is a pure function of
+// the arguments of its encoding (address, element type, sizes, row stride,
+// box, swizzle), so a cached map stays valid whatever buffer lives at that
+// address later.  Direct-mapped, 256 entries, one lock.
+struct MapKey {
+    const void *base;
+    uint64_t d0, d1, stride;
+    uint32_t b0, b1;
+    int dt, swz;
+    bool operator==(const MapKey &o) const {
+        return base == o.base && d0 == o.d0 && d1 == o.d1 && stride == o.stride && b0 == o.b0 && b1 == o.b1 &&
+               dt == o.dt && swz == o.swz;
+    }
+};
+struct MapSlot {
+    bool used = false;
+    MapKey key{};
+    CUtensorMap map{};
+};
+constexpr int kMapSlots = 256;
+MapSlot g_map_cache[kMapSlots];
+std::mutex g_map_lock;
+
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t d0, uint64_t d1,
+               uint64_t stride, uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz) {
+    const MapKey key{base, d0, d1, stride, b0, b1, static_cast<int>(dt), static_cast<int>(swz)};
+    uint64_t h = reinterpret_cast<uintptr_t>(base) >> 4;
+    for (uint64_t v : {d0, d1, stride, static_cast<uint64_t>(b0) << 32 | b1,
+                       static_cast<uint64_t>(key.dt) << 8 | static_cast<uint64_t>(key.swz)})
+        h = (h ^ v) * 0x100000001b3ull;
+    MapSlot &slot = g_map_cache[(h ^ (h >> 29)) % kMapSlots];
+    {
+        std::lock_guard<std::mutex> g(g_map_lock);
+        if (slot.used && slot.key == key) {
+            *map = slot.map;
+            return true;
+        }
+    }
+    auto encode = get_encode();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {d0, d1};
+    cuuint64_t strides[1] = {stride};
+    cuuint32_t box[2] = {b0, b1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    std::lock_guard<std::mutex> g(g_map_lock);
+    slot.used = true;
+    slot.key = key;
+    slot.map = *map;
+    return true;
+}
+
 // Tensor map over one operand's codes (rows x K, K contiguous), a box of
 // box_rows x one stage of K, 128-byte swizzle; rows past the end read as zero.
 // kind::mxf4 takes E2M1 codes packed two to a byte, so its stage is 128 bytes
@@ -869,22 +924,14 @@ int elem_bits(int f) { return f == MX_E2M1 ? 4 : (f == MX_E2M3 || f == MX_E3M2) 
 // codes in 128 bytes of shared memory for every element format.
 bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int fmt, bool mxf4,
                       int box_rows) {
-    auto encode = get_encode();
-    if (!encode) return false;
     const int bits = elem_bits(fmt);
     CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    cuuint64_t inner = static_cast<cuuint64_t>(K);            // elements along K
-    if (mxf4) inner = static_cast<cuuint64_t>(K / 2);           // bytes of packed pairs
+    uint64_t inner = static_cast<uint64_t>(K);                 // elements along K
+    if (mxf4) inner = static_cast<uint64_t>(K / 2);            // bytes of packed pairs
     else if (bits == 6) dt = CU_TENSOR_MAP_DATA_TYPE_16U6_ALIGN16B;
     else if (bits == 4) dt = CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
-    cuuint64_t dims[2] = {inner, static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * bits / 8)};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return encode_2d(map, dt, base, inner, static_cast<uint64_t>(rows), static_cast<uint64_t>(K * bits / 8),
+                     BK_BYTES, static_cast<uint32_t>(box_rows), CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Bytes one stage's load of box_rows rows delivers: the packed size in global
@@ -898,16 +945,9 @@ uint32_t stage_tx_bytes(int fmt, bool mxf4, int box_rows) {
 // 2-D uint8 view of an MMA-layout scale buffer as rows of 256 bytes (two rows
 // per 512-byte atom); a box of 2 * atoms rows x 256 bytes, no swizzle.
 bool make_scale_map(CUtensorMap *map, const void *base, int64_t bytes, int atoms_per_box) {
-    auto encode = get_encode();
-    if (!encode || bytes % 256 != 0) return false;
-    cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(bytes / 256)};
-    cuuint64_t strides[1] = {256};
-    cuuint32_t box[2] = {256, static_cast<cuuint32_t>(2 * atoms_per_box)};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (bytes % 256 != 0) return false;
+    return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 256, static_cast<uint64_t>(bytes / 256), 256, 256,
+                     static_cast<uint32_t>(2 * atoms_per_box), CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN) {
@@ -951,24 +991,16 @@ template <bool FP4, int OUT>
 cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
                         const CUtensorMap &tsb, const PairParams &p, int grid, cudaStream_t st) {
     auto kern = mx_gemm_pair_kernel<FP4, OUT>;
-    static bool configured = false;   // per instantiation
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg<FP4>::SMEM);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};   // per instantiation, one bit per device
+    if (cudaError_t e = ensure_smem_limit(kern, PairCfg<FP4>::SMEM, configured); e != cudaSuccess) return e;
     return launch_overlapped(kern, grid, PairCfg<FP4>::SMEM, st, ta, tb, tsa, tsb, p);
 }
 
 template <bool FP4, int OUT>
 cudaError_t launch(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int grid, cudaStream_t st) {
     auto kern = mx_gemm_kernel<FP4, OUT>;
-    static bool configured = false;   // per instantiation; attribute setting is idempotent
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};   // per instantiation, one bit per device
+    if (cudaError_t e = ensure_smem_limit(kern, SMEM_BYTES, configured); e != cudaSuccess) return e;
     return launch_overlapped(kern, grid, SMEM_BYTES, st, ta, tb, p);
 }
 
@@ -1006,11 +1038,12 @@ MxOut mx_out(const MxGemmArgs &a) {
 }  // namespace mxg
 
 namespace {
-std::atomic<int> g_skip_k_tile{-1};
+// armed by mx_debug_gemm_skip_stage; consumed by the next GEMM call of the same host thread
+thread_local int g_skip_k_tile = -1;
 }
 
 extern "C" int mx_debug_gemm_skip_stage(int k_tile) {
-    g_skip_k_tile.store(k_tile < 0 ? -1 : k_tile);
+    g_skip_k_tile = k_tile < 0 ? -1 : k_tile;
     return MX_OK;
 }
 
@@ -1062,7 +1095,8 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     p.idesc = make_idesc(a.fa, a.fb, fp4, PAIR_BM, PAIR_BN);
     p.ab_tx = stage_tx_bytes(a.fa, fp4, 128) + stage_tx_bytes(a.fb, fp4, PAIR_B_ROWS);
     raster_for(a, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major);
-    p.skip_k_tile = g_skip_k_tile.exchange(-1);
+    p.skip_k_tile = g_skip_k_tile;
+    g_skip_k_tile = -1;
     const int tiles = p.tiles_m * p.tiles_n;
     const int clusters = tiles < a.num_sms / 2 ? tiles : a.num_sms / 2;
     const int grid = 2 * (clusters < 1 ? 1 : clusters);
@@ -1111,7 +1145,8 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     p.idesc = make_idesc(a.fa, a.fb, fp4);
     p.ab_tx = stage_tx_bytes(a.fa, fp4, BM) + stage_tx_bytes(a.fb, fp4, BN);
     raster_for(a, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major);
-    p.skip_k_tile = g_skip_k_tile.exchange(-1);
+    p.skip_k_tile = g_skip_k_tile;
+    g_skip_k_tile = -1;
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < a.num_sms ? tiles : a.num_sms;
     cudaError_t e;

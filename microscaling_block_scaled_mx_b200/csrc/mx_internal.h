@@ -3,6 +3,7 @@
 // validated.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -83,3 +84,20 @@ cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st);
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st);
 // reads and clears the device status word of the current device (after a sync)
 int mx_read_device_status(cudaStream_t st);
+
+// Raises a kernel's dynamic shared-memory limit on the current device the
+// first time that device launches it.  The attribute belongs to the device's
+// context, so `done` keeps one bit per device (devices 64 and up set it on
+// every launch).  Setting it twice is harmless, so two threads that race on a
+// first launch need no lock.
+template <typename Kern>
+cudaError_t ensure_smem_limit(Kern kern, int bytes, std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}

@@ -146,6 +146,19 @@ def test_gemm_validation(mx):
     assert _g(mx, ldc=129, cdt=1) == -2
 
 
+def test_gemm_rejects_sizes_past_32_bit_indexing(mx):
+    """M, N, K up to 2^31 - 1 and at most 2^31 - 1 tiles of 128 x 128: larger
+    sizes are refused on the host (MX_ERR_UNSUPPORTED) instead of wrapping."""
+    big = 2 ** 31
+    assert _g(mx, M=big, ldc=128) == -4
+    assert _g(mx, N=big, ldc=big) == -4
+    assert _g(mx, K=big) == -4
+    assert _g(mx, M=2 ** 30, N=2 ** 24, ldc=2 ** 24) == -4       # 2^23 x 2^17 tiles
+    assert _gq(mx, M=big) == -4
+    assert _gq(mx, K=big) == -4
+    assert _gq(mx, M=2 ** 30, N=2 ** 24) == -4
+
+
 def _gq(mx, M=128, N=128, K=256, fa=0, fb=0, of=0, rnd=0, codes=16, scales=16, sl=1, a=16):
     L = mx.lib()
     return L.mx_gemm_quantize(a, 16, fa, 16, 16, fb, M, N, K, 1.0, of, rnd, 0, codes, scales, sl, None)
