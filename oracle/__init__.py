@@ -87,6 +87,11 @@ def lib() -> ctypes.CDLL:
             L.mxref_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i64, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
                                          ctypes.c_int, ctypes.c_uint32, _vp, _vp, ctypes.c_int]
+            L.mxref_quantize_shard.restype = ctypes.c_int
+            L.mxref_quantize_shard.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i64, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
+                                               ctypes.c_int, ctypes.c_uint32, _i64, _i64, _i64, _i64,
+                                               _vp, _vp, ctypes.c_int]
             L.mxref_dequantize.restype = ctypes.c_int
             L.mxref_dequantize.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _i64, _i64, _vp]
             L.mxref_round_f32.restype = None
@@ -172,11 +177,14 @@ def scales_bytes(sl: int, outer: int, inner: int) -> int:
 
 def quantize(x: np.ndarray, block_axis: int, fmt: int, rnd: int = RNE, seed: int = 0,
              hadamard: bool = False, sign_mask: int = 0, scale_layout: int = PLAIN,
-             ldx: int | None = None, cols: int | None = None, fill: int = 0):
+             ldx: int | None = None, cols: int | None = None, fill: int = 0, shard=None):
     """Cast a 2-D float32 array, or bf16 given as a uint16 bit array, to MX.
 
     With ``cols``/``ldx`` given, x is a pitched buffer: the logical tensor is
     its first ``cols`` columns and rows are ``ldx`` elements apart.
+    ``shard`` = (row0, col0, total_rows, total_cols) places x at (row0, col0)
+    of a larger tensor: stochastic rounding then uses the whole tensor's
+    element positions (mxref_quantize_shard).
 
     Returns (codes, scales) as uint8 arrays: codes has one row per block-axis
     line (transposed for block_axis=0); scales is flat in the chosen layout.
@@ -196,9 +204,16 @@ def quantize(x: np.ndarray, block_axis: int, fmt: int, rnd: int = RNE, seed: int
     row_bytes = codes_bytes(fmt, 1, inner) if inner % 32 == 0 else 0
     codes = np.full((outer, row_bytes), fill, dtype=np.uint8)
     scales = np.full(max(scales_bytes(scale_layout, outer, inner), 0), fill, dtype=np.uint8)
-    rc = lib().mxref_quantize(_ptr(x), xdt, rows, cols, ld, block_axis, fmt, rnd, seed,
-                              1 if hadamard else 0, sign_mask & 0xFFFFFFFF,
-                              _ptr(codes), _ptr(scales), scale_layout)
+    if shard is None:
+        rc = lib().mxref_quantize(_ptr(x), xdt, rows, cols, ld, block_axis, fmt, rnd, seed,
+                                  1 if hadamard else 0, sign_mask & 0xFFFFFFFF,
+                                  _ptr(codes), _ptr(scales), scale_layout)
+    else:
+        row0, col0, total_rows, total_cols = shard
+        rc = lib().mxref_quantize_shard(_ptr(x), xdt, rows, cols, ld, block_axis, fmt, rnd, seed,
+                                        1 if hadamard else 0, sign_mask & 0xFFFFFFFF,
+                                        row0, col0, total_rows, total_cols,
+                                        _ptr(codes), _ptr(scales), scale_layout)
     _check(rc, "mxref_quantize")
     return codes, scales
 

@@ -397,22 +397,38 @@ static unsigned quantize_block(int fmt, int rnd, uint64_t seed, const float *vin
  * hadamard != 0 applies the fixed-sign 32-point transform to each block.
  * codes / scales are written in full (packing bytes are overwritten); padding
  * entries of the MMA scale layout are left untouched.
+ *
+ * Shards (reading: stochastic rounding draws its random byte from the
+ * element's position in the block-axis-major output of the WHOLE tensor, so
+ * a tensor cut into pieces casts to the same bytes as the whole).  The tensor
+ * given is the piece whose element (0, 0) is element (row0, col0) of a
+ * total_rows x total_cols tensor; the element at (r, c) of the piece then has
+ * stochastic-rounding index (row0 + r) * total_cols + col0 + c along rows
+ * (block_axis 1) and (col0 + c) * total_rows + row0 + r along columns
+ * (block_axis 0).  Blocks stay those of the whole tensor, so the offset along
+ * the block axis is a multiple of 32.  Codes and scales are the piece's own
+ * (its block-axis-major output, in local coordinates).
  */
-int mxref_quantize(const void *x, int xdt, int64_t rows, int64_t cols, int64_t ldx,
-                   int block_axis, int fmt, int rnd, uint64_t seed,
-                   int hadamard, uint32_t sign_mask,
-                   uint8_t *codes, uint8_t *scales, int sl)
+int mxref_quantize_shard(const void *x, int xdt, int64_t rows, int64_t cols, int64_t ldx,
+                         int block_axis, int fmt, int rnd, uint64_t seed,
+                         int hadamard, uint32_t sign_mask,
+                         int64_t row0, int64_t col0, int64_t total_rows, int64_t total_cols,
+                         uint8_t *codes, uint8_t *scales, int sl)
 {
     build_tables();
     if (!x || !codes || !scales) return MXO_ERR_ARG;
     if (fmt < 0 || fmt >= FMT_COUNT || (xdt != DT_F32 && xdt != DT_BF16)) return MXO_ERR_ARG;
     if (block_axis != 0 && block_axis != 1) return MXO_ERR_ARG;
     if (rows < 0 || cols < 0 || ldx < cols) return MXO_ERR_ARG;
+    if (row0 < 0 || col0 < 0 || row0 + rows > total_rows || col0 + cols > total_cols) return MXO_ERR_ARG;
     int64_t outer = block_axis == 1 ? rows : cols;
     int64_t inner = block_axis == 1 ? cols : rows;
-    if (inner % BLOCK != 0) return MXO_ERR_SHAPE;
+    int64_t inner_total = block_axis == 1 ? total_cols : total_rows;
+    int64_t inner_off = block_axis == 1 ? col0 : row0;
+    int64_t outer_off = block_axis == 1 ? row0 : col0;
+    if (inner % BLOCK != 0 || inner_total % BLOCK != 0 || inner_off % BLOCK != 0) return MXO_ERR_SHAPE;
     /* the random-word counter floor(i / 4) must fit 32 bits: at most 2^34 elements */
-    if (rnd == RND_SR && (uint64_t)(outer * inner) > (1ull << 34)) return MXO_ERR_SR_RANGE;
+    if (rnd == RND_SR && (uint64_t)total_rows * (uint64_t)total_cols > (1ull << 34)) return MXO_ERR_SR_RANGE;
     int64_t kb_total = inner / BLOCK;
     int64_t row_bytes = mxref_codes_bytes(fmt, 1, inner);
 
@@ -429,13 +445,24 @@ int mxref_quantize(const void *x, int xdt, int64_t rows, int64_t cols, int64_t l
                 v[j] = load_elem(x, xdt, r * ldx + cc);
             }
             if (hadamard) mxref_hadamard32(v, sign_mask);
-            uint64_t idx0 = (uint64_t)(o * inner + kb * BLOCK);
+            /* position of the block's first element in the whole tensor's output */
+            uint64_t idx0 = (uint64_t)((outer_off + o) * inner_total + inner_off + kb * BLOCK);
             unsigned s = quantize_block(fmt, rnd, seed, v, idx0, c);
             for (int j = 0; j < BLOCK; ++j) put_code(fmt, crow, kb * BLOCK + j, c[j]);
             scales[scale_offset(sl, o, kb, kb_total)] = (uint8_t)s;
         }
     }
     return MXO_OK;
+}
+
+/* The whole tensor: a piece at (0, 0) of itself. */
+int mxref_quantize(const void *x, int xdt, int64_t rows, int64_t cols, int64_t ldx,
+                   int block_axis, int fmt, int rnd, uint64_t seed,
+                   int hadamard, uint32_t sign_mask,
+                   uint8_t *codes, uint8_t *scales, int sl)
+{
+    return mxref_quantize_shard(x, xdt, rows, cols, ldx, block_axis, fmt, rnd, seed, hadamard, sign_mask,
+                                0, 0, rows, cols, codes, scales, sl);
 }
 
 /* Exact decode v = 2^(scale - 127) * P (section 2); a 0xFF scale gives NaN. */
