@@ -180,6 +180,54 @@ MX_API int mx_quantize_dual(const void *x, mx_dtype xdt, int64_t rows, int64_t c
                             void *codes_cols, void *scales_cols, mx_scale_layout sl, void *stream);
 
 /*
+ * Placement of a tensor inside a larger one, for casts of shards.  The tensor
+ * passed to mx_quantize_shard / mx_quantize_dual_shard is the piece whose
+ * element (0, 0) is element (row0, col0) of a total_rows x total_cols tensor.
+ */
+typedef struct {
+    int64_t row0, col0;               /* offset of the piece in the whole tensor  */
+    int64_t total_rows, total_cols;   /* shape of the whole tensor                */
+} mx_shard;
+
+/*
+ * mx_quantize_shard -- mx_quantize of one piece of a larger tensor, giving
+ * exactly the bytes of the matching slice of the whole tensor's cast.  Only
+ * stochastic rounding depends on the placement: its index i is the element's
+ * position in the block-axis-major output of the WHOLE tensor, (row0 + r) *
+ * total_cols + col0 + c along rows (block_axis 1) and (col0 + c) * total_rows
+ * + row0 + r along columns (block_axis 0); blocks are the whole tensor's, so
+ * the offset along the block axis (col0, resp. row0) and the whole tensor's
+ * length along it must be multiples of 32.  This is the data-parallel split
+ * of the stochastic-rounding cast ("Format-Aware Fusion for Fast FP4
+ * Pretraining", abstract: row-gradient stochastic rounding, here for token
+ * shards of the weight-gradient operands held by different ranks).
+ *
+ *  shard   host pointer, required (NULL gives MX_ERR_ARG).  The piece must
+ *          lie inside the whole tensor (MX_ERR_ARG otherwise).
+ *  other arguments, outputs (the piece's own codes and scales, in its local
+ *  coordinates) and errors as for mx_quantize; MX_ERR_SR_RANGE applies to the
+ *  whole tensor's element count.
+ */
+MX_API int mx_quantize_shard(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                             int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
+                             const mx_precond *pre, const mx_shard *shard, void *codes, void *scales,
+                             mx_scale_layout sl, void *stream);
+
+/*
+ * mx_quantize_dual_shard -- mx_quantize_dual of one piece of a larger tensor,
+ * each output equal to the matching slice of the whole tensor's output (the
+ * stochastic-rounding positions of mx_quantize_shard).  Both axes are block
+ * axes here, so row0, col0, total_rows and total_cols must all be multiples
+ * of 32.  shard is required; arguments and errors otherwise as for
+ * mx_quantize_dual.
+ */
+MX_API int mx_quantize_dual_shard(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                  mx_fmt fmt, mx_round rnd_rows, uint64_t seed_rows, mx_round rnd_cols,
+                                  uint64_t seed_cols, const mx_precond *pre_cols, const mx_shard *shard,
+                                  void *codes_rows, void *scales_rows, void *codes_cols, void *scales_cols,
+                                  mx_scale_layout sl, void *stream);
+
+/*
  * mx_dequantize -- v = X * P (section 2), exact, rounded once to ydt.
  *
  *  codes, scales  device, as written by mx_quantize for (outer, inner).

@@ -77,24 +77,65 @@ size_t mx_scales_bytes(mx_scale_layout sl, int64_t outer, int64_t inner) {
 
 size_t mx_gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
 
-int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
-                int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
-                const mx_precond *pre, void *codes, void *scales, mx_scale_layout sl,
-                void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Where a tensor sits in the whole tensor its stochastic-rounding positions
+// refer to; NULL means the tensor is the whole.  Returns MX_OK or an error.
+struct Placement {
+    int64_t row0 = 0, col0 = 0, total_rows = 0, total_cols = 0;
+};
+
+int place(const mx_shard *shard, int64_t rows, int64_t cols, Placement &pl) {
+    if (!shard) {
+        pl.total_rows = rows;
+        pl.total_cols = cols;
+        return MX_OK;
+    }
+    pl.row0 = shard->row0;
+    pl.col0 = shard->col0;
+    pl.total_rows = shard->total_rows;
+    pl.total_cols = shard->total_cols;
+    if (pl.row0 < 0 || pl.col0 < 0 || pl.total_rows < 0 || pl.total_cols < 0) return MX_ERR_ARG;
+    if (rows > pl.total_rows - pl.row0 || cols > pl.total_cols - pl.col0) return MX_ERR_ARG;
+    return MX_OK;
+}
+
+// SR position of output element (o, i) = base + o * stride + i, for the output
+// along `block_axis` of a tensor placed by pl.
+void sr_position(const Placement &pl, int block_axis, uint64_t &base, uint64_t &stride) {
+    if (block_axis == 1) {
+        stride = static_cast<uint64_t>(pl.total_cols);
+        base = static_cast<uint64_t>(pl.row0) * stride + static_cast<uint64_t>(pl.col0);
+    } else {
+        stride = static_cast<uint64_t>(pl.total_rows);
+        base = static_cast<uint64_t>(pl.col0) * stride + static_cast<uint64_t>(pl.row0);
+    }
+}
+
+int quantize_impl(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, int block_axis,
+                  mx_fmt fmt, mx_round rnd, uint64_t seed, const mx_precond *pre, const mx_shard *shard,
+                  void *codes, void *scales, mx_scale_layout sl, void *stream) {
     if ((xdt != MX_F32 && xdt != MX_BF16) || elem_bits(fmt) == 0) return MX_ERR_ARG;
     if ((rnd != MX_RNE && rnd != MX_SR) || (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA)) return MX_ERR_ARG;
     if (block_axis != 0 && block_axis != 1) return MX_ERR_ARG;
     if (rows < 0 || cols < 0) return MX_ERR_ARG;
+    Placement pl;
+    if (int rc = place(shard, rows, cols, pl); rc != MX_OK) return rc;
     const int64_t outer = block_axis == 1 ? rows : cols;
     const int64_t inner = block_axis == 1 ? cols : rows;
-    if (inner % 32 != 0) return MX_ERR_SHAPE;
+    const int64_t inner_off = block_axis == 1 ? pl.col0 : pl.row0;
+    const int64_t inner_total = block_axis == 1 ? pl.total_cols : pl.total_rows;
+    if (inner % 32 != 0 || inner_off % 32 != 0 || inner_total % 32 != 0) return MX_ERR_SHAPE;
     if (outer == 0 || inner == 0) return MX_OK;          // empty: pointers may be NULL
     if (!x || !codes || !scales) return MX_ERR_ARG;
     if (ldx < cols) return MX_ERR_ARG;
     if (!aligned16(x) || (ldx * dtype_bytes(xdt)) % 16 != 0 || !aligned16(codes)) return MX_ERR_ALIGN;
     const bool had = pre && pre->hadamard;
     if (had && block_axis != 0) return MX_ERR_UNSUPPORTED;
-    if (rnd == MX_SR && static_cast<uint64_t>(outer) * static_cast<uint64_t>(inner) > (1ull << 34))
+    if (rnd == MX_SR &&
+        static_cast<uint64_t>(pl.total_rows) * static_cast<uint64_t>(pl.total_cols) > (1ull << 34))
         return MX_ERR_SR_RANGE;
     if (mx_scales_bytes(sl, outer, inner) >= (1ull << 32)) return MX_ERR_UNSUPPORTED;  // 32-bit scale offsets
 
@@ -103,27 +144,32 @@ int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t
     a.block_axis = block_axis; a.fmt = fmt; a.rnd = rnd; a.seed = seed;
     a.hadamard = had; a.sign_mask = had ? pre->sign_mask : 0u;
     a.codes = codes; a.scales = scales; a.sl = sl;
+    sr_position(pl, block_axis, a.sr_base, a.sr_stride);
     a.num_sms = sm_count(nullptr);
     if (a.num_sms <= 0) return MX_ERR_CUDA;
     return mx_launch_quantize(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
-int mx_quantize_dual(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, mx_fmt fmt,
-                     mx_round rnd_rows, uint64_t seed_rows, mx_round rnd_cols, uint64_t seed_cols,
-                     const mx_precond *pre_cols, void *codes_rows, void *scales_rows, void *codes_cols,
-                     void *scales_cols, mx_scale_layout sl, void *stream) {
+int quantize_dual_impl(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, mx_fmt fmt,
+                       mx_round rnd_rows, uint64_t seed_rows, mx_round rnd_cols, uint64_t seed_cols,
+                       const mx_precond *pre_cols, const mx_shard *shard, void *codes_rows, void *scales_rows,
+                       void *codes_cols, void *scales_cols, mx_scale_layout sl, void *stream) {
     if ((xdt != MX_F32 && xdt != MX_BF16) || elem_bits(fmt) == 0) return MX_ERR_ARG;
     if ((rnd_rows != MX_RNE && rnd_rows != MX_SR) || (rnd_cols != MX_RNE && rnd_cols != MX_SR)) return MX_ERR_ARG;
     if (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA) return MX_ERR_ARG;
     if (rows < 0 || cols < 0) return MX_ERR_ARG;
+    Placement pl;
+    if (int rc = place(shard, rows, cols, pl); rc != MX_OK) return rc;
     if (rows % 32 != 0 || cols % 32 != 0) return MX_ERR_SHAPE;
+    if (pl.row0 % 32 != 0 || pl.col0 % 32 != 0 || pl.total_rows % 32 != 0 || pl.total_cols % 32 != 0)
+        return MX_ERR_SHAPE;
     if (rows == 0 || cols == 0) return MX_OK;            // empty: pointers may be NULL
     if (!x || !codes_rows || !scales_rows || !codes_cols || !scales_cols) return MX_ERR_ARG;
     if (ldx < cols) return MX_ERR_ARG;
     if (!aligned16(x) || (ldx * dtype_bytes(xdt)) % 16 != 0 || !aligned16(codes_rows) || !aligned16(codes_cols))
         return MX_ERR_ALIGN;
     if ((rnd_rows == MX_SR || rnd_cols == MX_SR) &&
-        static_cast<uint64_t>(rows) * static_cast<uint64_t>(cols) > (1ull << 34))
+        static_cast<uint64_t>(pl.total_rows) * static_cast<uint64_t>(pl.total_cols) > (1ull << 34))
         return MX_ERR_SR_RANGE;
     if (mx_scales_bytes(sl, rows, cols) >= (1ull << 32) || mx_scales_bytes(sl, cols, rows) >= (1ull << 32))
         return MX_ERR_UNSUPPORTED;
@@ -134,9 +180,50 @@ int mx_quantize_dual(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, in
     a.hadamard = had; a.sign_mask = had ? pre_cols->sign_mask : 0u;
     a.codes_rows = codes_rows; a.scales_rows = scales_rows; a.codes_cols = codes_cols; a.scales_cols = scales_cols;
     a.sl = sl;
+    sr_position(pl, 1, a.sr_base_rows, a.sr_stride_rows);
+    sr_position(pl, 0, a.sr_base_cols, a.sr_stride_cols);
     a.num_sms = sm_count(nullptr);
     if (a.num_sms <= 0) return MX_ERR_CUDA;
     return mx_launch_quantize_dual(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
+                const mx_precond *pre, void *codes, void *scales, mx_scale_layout sl,
+                void *stream) {
+    return quantize_impl(x, xdt, rows, cols, ldx, block_axis, fmt, rnd, seed, pre, nullptr, codes, scales, sl,
+                         stream);
+}
+
+int mx_quantize_shard(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                      int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
+                      const mx_precond *pre, const mx_shard *shard, void *codes, void *scales,
+                      mx_scale_layout sl, void *stream) {
+    if (!shard) return MX_ERR_ARG;
+    return quantize_impl(x, xdt, rows, cols, ldx, block_axis, fmt, rnd, seed, pre, shard, codes, scales, sl,
+                         stream);
+}
+
+int mx_quantize_dual(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, mx_fmt fmt,
+                     mx_round rnd_rows, uint64_t seed_rows, mx_round rnd_cols, uint64_t seed_cols,
+                     const mx_precond *pre_cols, void *codes_rows, void *scales_rows, void *codes_cols,
+                     void *scales_cols, mx_scale_layout sl, void *stream) {
+    return quantize_dual_impl(x, xdt, rows, cols, ldx, fmt, rnd_rows, seed_rows, rnd_cols, seed_cols, pre_cols,
+                              nullptr, codes_rows, scales_rows, codes_cols, scales_cols, sl, stream);
+}
+
+int mx_quantize_dual_shard(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, mx_fmt fmt,
+                           mx_round rnd_rows, uint64_t seed_rows, mx_round rnd_cols, uint64_t seed_cols,
+                           const mx_precond *pre_cols, const mx_shard *shard, void *codes_rows,
+                           void *scales_rows, void *codes_cols, void *scales_cols, mx_scale_layout sl,
+                           void *stream) {
+    if (!shard) return MX_ERR_ARG;
+    return quantize_dual_impl(x, xdt, rows, cols, ldx, fmt, rnd_rows, seed_rows, rnd_cols, seed_cols, pre_cols,
+                              shard, codes_rows, scales_rows, codes_cols, scales_cols, sl, stream);
 }
 
 int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_scale_layout sl,

@@ -35,6 +35,8 @@ struct CastParams {
     int64_t k_groups;    // ceil(k_blocks / 4), MMA layout
     uint32_t key;        // stochastic-rounding seed key
     uint32_t sign_mask;  // Hadamard signs
+    // stochastic-rounding position of output element (o, i): sr_base + o * sr_stride + i
+    uint64_t sr_base, sr_stride;
 };
 
 __device__ __forceinline__ void store_scale(const CastParams &p, int64_t o, int64_t kb, uint32_t s) {
@@ -103,6 +105,8 @@ __device__ __forceinline__ BlockSink row_sink(const CastParams &p) {
     o.k_groups = static_cast<uint32_t>(p.k_groups);
     o.mma_scales = p.mma_scales;
     o.key = p.key;
+    o.sr_base = p.sr_base;
+    o.sr_stride = p.sr_stride;
     return o;
 }
 
@@ -267,7 +271,8 @@ __device__ __forceinline__ void stage_tile(const CastParams &p, uint8_t *buf, in
 // optional fixed-sign Hadamard, amax -> E8M0, exact scaling with the FP32
 // subnormal flush, RNE or stochastic rounding, and the codes as rows gc and
 // gc + 1 of the transposed output.  SR's index is the element's position
-// (gc + col) * rows + gr0 + j in that output.
+// sr_base + (gc + col) * sr_stride + gr0 + j in the whole tensor's output
+// (sr_base 0 and sr_stride = rows for a whole tensor).
 // KEYED: the caller passes the packed 16-bit maxima of |bf16| of the two
 // columns (bf16_pair_max over the raw words), valid without the Hadamard.
 template <int FMT, bool SR, bool HAD, bool KEYED = false>
@@ -336,7 +341,8 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
         constexpr int SLOT = BITS == 4 ? 4 : 8;
         uint32_t pw[8];
         if (SR) {
-            const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(oc * R + gr0) >> 2);
+            const uint32_t g = static_cast<uint32_t>(
+                (p.sr_base + static_cast<uint64_t>(oc) * p.sr_stride + static_cast<uint64_t>(gr0)) >> 2);
 #pragma unroll
             for (int w = 0; w < 8; ++w)
                 pw[w] = sr_quad<FMT>(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3], fmix32((g + w) ^ p.key));
@@ -790,6 +796,8 @@ cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st) {
     p.k_groups = (p.k_blocks + 3) / 4;
     p.key = fmix32_host(static_cast<uint32_t>(a.seed)) ^ static_cast<uint32_t>(a.seed >> 32);
     p.sign_mask = a.sign_mask;
+    p.sr_base = a.sr_base;
+    p.sr_stride = a.sr_stride;
     const bool sr = a.rnd == MX_SR;
     switch (a.fmt) {
         case MX_E4M3: return launch_cast_rnd<MX_E4M3>(p, a.xdt, a.block_axis, sr, a.hadamard, a.num_sms, st);
@@ -849,12 +857,16 @@ cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st
     pr.k_groups = (pr.k_blocks + 3) / 4;
     pr.key = key(a.seed_rows);
     pr.sign_mask = 0;
+    pr.sr_base = a.sr_base_rows;
+    pr.sr_stride = a.sr_stride_rows;
     pc.codes = static_cast<uint8_t *>(a.codes_cols);
     pc.scales = static_cast<uint8_t *>(a.scales_cols);
     pc.k_blocks = a.rows / 32;
     pc.k_groups = (pc.k_blocks + 3) / 4;
     pc.key = key(a.seed_cols);
     pc.sign_mask = a.sign_mask;
+    pc.sr_base = a.sr_base_cols;
+    pc.sr_stride = a.sr_stride_cols;
     const int sr_r = a.rnd_rows == MX_SR, sr_c = a.rnd_cols == MX_SR;
     switch (a.fmt) {
         case MX_E4M3: return launch_dual_fmt<MX_E4M3>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);

@@ -19,6 +19,9 @@ struct BlockSink {
     uint32_t k_groups;   // ceil(k_blocks / 4), MMA layout
     int mma_scales;
     uint32_t key;        // stochastic-rounding seed key
+    // stochastic-rounding position of element (row, i): sr_base + row * sr_stride + i
+    // (a whole tensor: 0 and inner; a shard: its place in the whole tensor's output)
+    uint64_t sr_base, sr_stride;
 };
 
 __device__ __forceinline__ void sink_scale(const BlockSink &o, int64_t row, int64_t kb, uint32_t s) {
@@ -52,7 +55,8 @@ __device__ __forceinline__ void store_code32(uint8_t *dst, const uint4 &a, const
 // (Algorithm 1 of the MX summary page, section 3): block amax -> E8M0
 // exponent, V * 2^-e (flushing FP32 subnormals), RNE or stochastic rounding,
 // and the packed codes and scale byte of block (row, kb).  SR's index is the
-// element's position row * inner + kb * 32 + j in the output.
+// element's position sr_base + row * sr_stride + kb * 32 + j in the output of
+// the whole tensor.
 // amax_bits: the largest |b[i]| as FP32 bits (sign cleared), computed by the
 // caller (encode_block32 below, or bf16_max_bits of the packed input); for a
 // block holding a NaN it may be any pattern at or above 0x7f800000.
@@ -107,7 +111,8 @@ __device__ __forceinline__ void encode_block32_amax(const BlockSink &o, int64_t 
     constexpr int SLOT = BITS == 4 ? 4 : 8;
     uint32_t pw[8];
     if (SR) {
-        const uint32_t g = static_cast<uint32_t>(static_cast<uint64_t>(row * o.inner + kb * 32) >> 2);
+        const uint32_t g = static_cast<uint32_t>(
+            (o.sr_base + static_cast<uint64_t>(row) * o.sr_stride + static_cast<uint64_t>(kb * 32)) >> 2);
 #pragma unroll
         for (int w = 0; w < 8; ++w)
             pw[w] = sr_quad<FMT>(u[4 * w], u[4 * w + 1], u[4 * w + 2], u[4 * w + 3], fmix32((g + w) ^ o.key));

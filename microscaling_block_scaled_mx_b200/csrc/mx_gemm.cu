@@ -16,7 +16,9 @@
 //               so the epilogue of a tile overlaps the mainloop of the next.
 //   warps 2-9   epilogue: two warps per TMEM lane quarter, 96 columns each,
 //               three tcgen05.ld of 32 columns per wait, times alpha, rounded
-//               to fp32 / bf16, stored to C with bounds checks.
+//               to fp32 / bf16, written to a per-warp shared-memory piece of
+//               32 rows x 64 bytes and stored to C by one TMA store per piece
+//               (the copy engine clips the ragged edges of C).
 // A 192-column tile starts 64 rows into a 128-row scale atom on odd tiles;
 // the B scale-factor TMEM address then starts two columns later.
 // Every mbarrier wait is bounded; on expiry the kernel records MX_ERR_TIMEOUT
@@ -45,7 +47,7 @@ namespace mxg {
 constexpr int BM = 128;            // tile rows (A rows, TMEM lanes)
 constexpr int BN = 192;            // tile columns (B rows, accumulator columns)
 constexpr int BK_BYTES = 128;      // K bytes per stage: 128 fp8 or 256 fp4 elements
-constexpr int STAGES = 5;
+constexpr int STAGES = 4;
 constexpr int EPI_WARPS = 8;
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr int A_STAGE_BYTES = BM * BK_BYTES;   // 16 KiB
@@ -54,6 +56,8 @@ constexpr int ATOM = 512;                      // scale atom: 128 rows x 4 k-blo
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = BN;              // accumulator b at columns [b * 192, (b + 1) * 192)
 constexpr uint32_t SF_COL = 2 * ACC_COLS;      // scale-factor columns from 384
+constexpr int EPI_PIECE = 2048;                // one staged piece of C: 32 rows x 64 bytes
+constexpr int EPI_WARP_BYTES = 2 * EPI_PIECE;  // two pieces per epilogue warp (double buffer)
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;   // 0.2 s when draining
 constexpr unsigned long long DRAIN_SETTLE_NS = 1000000ull;    // 1 ms for loads in flight after an abort
@@ -73,7 +77,8 @@ struct Smem {
     static constexpr int B = A + STAGES * A_STAGE_BYTES;
     static constexpr int SFA = B + STAGES * B_STAGE_BYTES;
     static constexpr int SFB = SFA + STAGES * 2 * ATOM;       // sized for the FP4 case
-    static constexpr int BAR = SFB + STAGES * 4 * ATOM;
+    static constexpr int EPI = (SFB + STAGES * 4 * ATOM + 1023) / 1024 * 1024;
+    static constexpr int BAR = EPI + EPI_WARPS * EPI_WARP_BYTES;
     // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
     static constexpr int NUM_BARS = 2 * STAGES + 5;
     static constexpr int TMEM_SLOT = BAR + NUM_BARS * 8;
@@ -81,6 +86,7 @@ struct Smem {
     static constexpr int TOTAL = ABORT + 4;
 };
 constexpr int SMEM_BYTES = Smem::TOTAL + 1024;   // slack for 1024-byte alignment
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 
 // Output of the epilogue: C in fp32 or bf16, or C quantized along its rows
 // (blocks of 32 consecutive columns) to MX codes and E8M0 scales.
@@ -191,6 +197,23 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
+// TMA store of a shared-memory box to global memory, tracked by bulk groups
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(src) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most N committed bulk groups may still be reading their shared-memory source
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+// every committed bulk group has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// generic-proxy shared-memory writes become visible to the copy engine
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -283,6 +306,8 @@ __device__ __forceinline__ void quantize_chunk(const Params &p, int m, int n0, c
     o.k_groups = (o.k_blocks + 3) >> 2;
     o.mma_scales = p.q.mma;
     o.key = p.q.key;
+    o.sr_base = 0;
+    o.sr_stride = static_cast<uint64_t>(p.N);
     const int kb = n0 >> 5;
     const bool sr = p.q.sr != 0;
     switch (p.q.fmt) {
@@ -295,52 +320,62 @@ __device__ __forceinline__ void quantize_chunk(const Params &p, int m, int n0, c
     }
 }
 
-// 32 consecutive accumulator values of one row -> C (bounds-checked).
+// Epilogue through shared memory: an epilogue warp owns 32 rows of C; a piece
+// is those 32 rows x 64 bytes (32 bf16 or 16 fp32 columns), written by each
+// lane for its own row into one of the warp's two 2 KB buffers and stored to
+// C with one TMA store.  The buffers use the copy engine's 64-byte swizzle
+// (16-byte granule g of row r sits at granule g ^ ((r >> 1) & 3)), so the
+// lanes' 16-byte writes spread over all banks.  The tensor map clips rows
+// >= M and columns >= N.
+struct EpiWriter {
+    const CUtensorMap *map;
+    uint32_t buf;      // this warp's two pieces (1024-byte aligned)
+    int count;         // pieces issued so far (selects the buffer)
+    int lane;
+};
+// vals: 32 accumulator words (bf16 output) or 16 (fp32 output) of this lane's row
 template <int OUT>
-__device__ __forceinline__ void store_chunk(const Params &p, int m, int n0, const uint32_t *r) {
-    if (m >= p.M || n0 >= p.N) return;
-    if constexpr (OUT == OUT_MX) {
-        quantize_chunk(p, m, n0, r);
-    } else {
-        float v[32];
+__device__ __forceinline__ void epi_piece(EpiWriter &w, const uint32_t *vals, float alpha, int x, int y) {
+    const uint32_t b = w.buf + static_cast<uint32_t>(w.count & 1) * EPI_PIECE;
+    if (w.lane == 0) bulk_wait_read<1>();       // this buffer's previous store has read it
+    __syncwarp();
+    uint32_t q[16];
+    if constexpr (OUT == OUT_BF16) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), p.alpha);
-        if (OUT == OUT_BF16) {
-            __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
-            if (n0 + 32 <= p.N) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 8) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * t], v[i + 2 * t + 1]);
-                        w[t] = *reinterpret_cast<uint32_t *>(&b2);
-                    }
-                    *reinterpret_cast<uint4 *>(row + i) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (n0 + i < p.N) row[i] = __float2bfloat16_rn(v[i]);
-            }
-        } else {
-            float *row = static_cast<float *>(p.c) + static_cast<int64_t>(m) * p.ldc + n0;
-            if (n0 + 32 <= p.N) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (n0 + i < p.N) row[i] = v[i];
-            }
+        for (int i = 0; i < 16; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(vals[2 * i]), alpha),
+                                                     __fmul_rn(__uint_as_float(vals[2 * i + 1]), alpha));
+            q[i] = *reinterpret_cast<uint32_t *>(&h);
         }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[i] = __float_as_uint(__fmul_rn(__uint_as_float(vals[i]), alpha));
     }
+    const uint32_t row = b + static_cast<uint32_t>(w.lane) * 64u;
+    const uint32_t sw = (static_cast<uint32_t>(w.lane) >> 1) & 3u;
+#pragma unroll
+    for (uint32_t g = 0; g < 4; ++g)
+        st_shared_v4(row + ((g ^ sw) << 4), q[4 * g], q[4 * g + 1], q[4 * g + 2], q[4 * g + 3]);
+    fence_async_smem();
+    __syncwarp();
+    if (w.lane == 0) {
+        tma_store_2d(w.map, b, x, y);
+        bulk_commit();
+    }
+    ++w.count;
+}
+
+// 32 consecutive accumulator values of one row -> one MX block of C's row
+// (quantizing epilogue; rows >= M and blocks past N are skipped).
+__device__ __forceinline__ void store_chunk_mx(const Params &p, int m, int n0, const uint32_t *r) {
+    if (m >= p.M || n0 >= p.N) return;
+    quantize_chunk(p, m, n0, r);
 }
 
 template <bool FP4, int OUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, Params p) {
+mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+               const __grid_constant__ CUtensorMap tma_c, Params p) {
     using C = Cfg<FP4>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -497,6 +532,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         // ------------------------------ epilogue ------------------------------
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
         const int half = (warp - 2) >> 2;        // which 96 columns of the tile
+        EpiWriter ew{&tma_c, sbase + Smem::EPI + static_cast<uint32_t>(warp - 2) * EPI_WARP_BYTES, 0, lane};
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int b = local & 1;
@@ -523,9 +559,20 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty(b));
             const int n_base = tn * BN + c0;
+            if constexpr (OUT == OUT_MX) {
 #pragma unroll
-            for (int j = 0; j < 3; ++j) store_chunk<OUT>(p, m, n_base + 32 * j, r + 32 * j);
+                for (int j = 0; j < 3; ++j) store_chunk_mx(p, m, n_base + 32 * j, r + 32 * j);
+            } else {
+                const int m_warp = tm * BM + q * 32;
+                constexpr int PC = OUT == OUT_BF16 ? 32 : 16;   // columns per piece
+                if (m_warp < p.M) {
+#pragma unroll
+                    for (int j = 0; j < (BN / 2) / PC; ++j)
+                        if (n_base + PC * j < p.N) epi_piece<OUT>(ew, r + PC * j, p.alpha, n_base + PC * j, m_warp);
+                }
+            }
         }
+        if (lane == 0) bulk_wait_all();          // stores done reading shared memory and written
     }
 
     tc_fence_before();
@@ -560,7 +607,7 @@ constexpr uint32_t PAIR_SF_COL = PAIR_BN;                // scale factors after 
 
 template <bool FP4> struct PairCfg {
     static constexpr int G = FP4 ? 2 : 1;                // scale atoms along K per stage
-    static constexpr int STAGES = 6;
+    static constexpr int STAGES = 5;
     static constexpr int SFA_BYTES = ATOM * G;
     static constexpr int SFB_BYTES = 2 * ATOM * G;       // both 128-row scale blocks the tile touches
     static constexpr int SFA_COLS = 4 * G;
@@ -572,7 +619,8 @@ template <bool FP4> struct PairCfg {
     static constexpr int OFF_B = OFF_A + STAGES * PAIR_A_BYTES;
     static constexpr int OFF_SFA = OFF_B + STAGES * PAIR_B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr int OFF_EPI = (OFF_SFB + STAGES * SFB_BYTES + 1023) / 1024 * 1024;
+    static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_WARP_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 5;      // full, empty, acc_full, acc_empty, drain (+2 spare)
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
@@ -651,7 +699,7 @@ template <bool FP4, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                     const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
-                    PairParams p) {
+                    const __grid_constant__ CUtensorMap tma_c, PairParams p) {
     using C = PairCfg<FP4>;
     constexpr int STAGES_P = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -802,6 +850,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
         // ------------------------------ epilogue (both CTAs) -------------------
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
+        EpiWriter ew{&tma_c, sbase + C::OFF_EPI + static_cast<uint32_t>(warp - 2) * EPI_WARP_BYTES, 0, lane};
         int local = 0;
         constexpr int NCH = PAIR_BN / 2 / 32;    // 32-column chunks per warp
         for (int tile = cluster_id; tile < num_tiles; tile += n_clusters, ++local) {
@@ -826,11 +875,22 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(map_to_rank(acc_empty(b), 0));
             const int n_base = tn * PAIR_BN + c0;
-            Params pp;
-            pp.c = p.c; pp.ldc = p.ldc; pp.M = p.M; pp.N = p.N; pp.alpha = p.alpha; pp.q = p.q;
+            if constexpr (OUT == OUT_MX) {
+                Params pp;
+                pp.c = p.c; pp.ldc = p.ldc; pp.M = p.M; pp.N = p.N; pp.alpha = p.alpha; pp.q = p.q;
 #pragma unroll
-            for (int j = 0; j < NCH; ++j) store_chunk<OUT>(pp, m, n_base + 32 * j, r + 32 * j);
+                for (int j = 0; j < NCH; ++j) store_chunk_mx(pp, m, n_base + 32 * j, r + 32 * j);
+            } else {
+                const int m_warp = tm * PAIR_BM + 128 * static_cast<int>(rank) + q * 32;
+                constexpr int PC = OUT == OUT_BF16 ? 32 : 16;   // columns per piece
+                if (m_warp < p.M) {
+#pragma unroll
+                    for (int j = 0; j < (PAIR_BN / 2) / PC; ++j)
+                        if (n_base + PC * j < p.N) epi_piece<OUT>(ew, r + PC * j, p.alpha, n_base + PC * j, m_warp);
+                }
+            }
         }
+        if (lane == 0) bulk_wait_all();          // stores done reading shared memory and written
     }
 
     tc_fence_before();
@@ -950,6 +1010,22 @@ bool make_scale_map(CUtensorMap *map, const void *base, int64_t bytes, int atoms
                      static_cast<uint32_t>(2 * atoms_per_box), CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// Tensor map over C (M x N, leading dimension ldc) for the epilogue's TMA
+// stores: boxes of 32 rows x 64 bytes (32 bf16 or 16 fp32 columns), 64-byte
+// swizzle, matching the staged pieces.  Without a C (quantizing epilogue) the
+// map is zeroed and never used.
+bool make_c_map(CUtensorMap *map, const MxGemmArgs &a) {
+    if (a.q_codes) {
+        std::memset(map, 0, sizeof(*map));
+        return true;
+    }
+    const bool bf16 = a.cdt == MX_BF16;
+    const uint64_t esz = bf16 ? 2 : 4;
+    return encode_2d(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.c,
+                     static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.ldc) * esz,
+                     bf16 ? 32u : 16u, 32u, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN) {
     auto code = [&](int f) -> uint32_t {
         if (fp4) return 1u;               // kind::mxf4: E2M1
@@ -989,35 +1065,38 @@ cudaError_t launch_overlapped(Kern kern, int grid, int smem, cudaStream_t st, co
 
 template <bool FP4, int OUT>
 cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
-                        const CUtensorMap &tsb, const PairParams &p, int grid, cudaStream_t st) {
+                        const CUtensorMap &tsb, const CUtensorMap &tc, const PairParams &p, int grid,
+                        cudaStream_t st) {
     auto kern = mx_gemm_pair_kernel<FP4, OUT>;
     static std::atomic<uint64_t> configured{0};   // per instantiation, one bit per device
     if (cudaError_t e = ensure_smem_limit(kern, PairCfg<FP4>::SMEM, configured); e != cudaSuccess) return e;
-    return launch_overlapped(kern, grid, PairCfg<FP4>::SMEM, st, ta, tb, tsa, tsb, p);
+    return launch_overlapped(kern, grid, PairCfg<FP4>::SMEM, st, ta, tb, tsa, tsb, tc, p);
 }
 
 template <bool FP4, int OUT>
-cudaError_t launch(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int grid, cudaStream_t st) {
+cudaError_t launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const Params &p, int grid,
+                   cudaStream_t st) {
     auto kern = mx_gemm_kernel<FP4, OUT>;
     static std::atomic<uint64_t> configured{0};   // per instantiation, one bit per device
     if (cudaError_t e = ensure_smem_limit(kern, SMEM_BYTES, configured); e != cudaSuccess) return e;
-    return launch_overlapped(kern, grid, SMEM_BYTES, st, ta, tb, p);
+    return launch_overlapped(kern, grid, SMEM_BYTES, st, ta, tb, tc, p);
 }
 
 template <bool FP4>
 cudaError_t launch_pair_out(int out, const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
-                            const CUtensorMap &tsb, const PairParams &p, int grid, cudaStream_t st) {
-    if (out == OUT_MX) return launch_pair<FP4, OUT_MX>(ta, tb, tsa, tsb, p, grid, st);
-    if (out == OUT_BF16) return launch_pair<FP4, OUT_BF16>(ta, tb, tsa, tsb, p, grid, st);
-    return launch_pair<FP4, OUT_F32>(ta, tb, tsa, tsb, p, grid, st);
+                            const CUtensorMap &tsb, const CUtensorMap &tc, const PairParams &p, int grid,
+                            cudaStream_t st) {
+    if (out == OUT_MX) return launch_pair<FP4, OUT_MX>(ta, tb, tsa, tsb, tc, p, grid, st);
+    if (out == OUT_BF16) return launch_pair<FP4, OUT_BF16>(ta, tb, tsa, tsb, tc, p, grid, st);
+    return launch_pair<FP4, OUT_F32>(ta, tb, tsa, tsb, tc, p, grid, st);
 }
 
 template <bool FP4>
-cudaError_t launch_out(int out, const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int grid,
-                       cudaStream_t st) {
-    if (out == OUT_MX) return launch<FP4, OUT_MX>(ta, tb, p, grid, st);
-    if (out == OUT_BF16) return launch<FP4, OUT_BF16>(ta, tb, p, grid, st);
-    return launch<FP4, OUT_F32>(ta, tb, p, grid, st);
+cudaError_t launch_out(int out, const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
+                       const Params &p, int grid, cudaStream_t st) {
+    if (out == OUT_MX) return launch<FP4, OUT_MX>(ta, tb, tc, p, grid, st);
+    if (out == OUT_BF16) return launch<FP4, OUT_BF16>(ta, tb, tc, p, grid, st);
+    return launch<FP4, OUT_F32>(ta, tb, tc, p, grid, st);
 }
 
 int out_mode(const MxGemmArgs &a) {
@@ -1074,7 +1153,8 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;     // K bytes of a uint8 stage view
     const int G = fp4 ? 2 : 1;
     const int64_t k_groups = a.K / 128;
-    CUtensorMap ta, tb, tsa, tsb;
+    CUtensorMap ta, tb, tsa, tsb, tc;
+    if (!make_c_map(&tc, a)) return MX_ERR_CUDA;
     if (!make_operand_map(&ta, a.a_codes, a.M, a.K, a.fa, fp4, 128)) return MX_ERR_CUDA;
     if (!make_operand_map(&tb, a.b_codes, a.N, a.K, a.fb, fp4, PAIR_B_ROWS)) return MX_ERR_CUDA;
     const int64_t sa_bytes = (a.M + 127) / 128 * 128 * k_groups * 4;
@@ -1103,8 +1183,8 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     cudaError_t e;
     p.q = mx_out(a);
     const int out = out_mode(a);
-    if (fp4) e = launch_pair_out<true>(out, ta, tb, tsa, tsb, p, grid, st);
-    else e = launch_pair_out<false>(out, ta, tb, tsa, tsb, p, grid, st);
+    if (fp4) e = launch_pair_out<true>(out, ta, tb, tsa, tsb, tc, p, grid, st);
+    else e = launch_pair_out<false>(out, ta, tb, tsa, tsb, tc, p, grid, st);
     return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
@@ -1126,7 +1206,8 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     if (use_pair_kernel(a)) return launch_gemm_pair(a, st);
     const bool fp4 = use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tc;
+    if (!make_c_map(&tc, a)) return MX_ERR_CUDA;
     if (!make_operand_map(&ta, a.a_codes, a.M, a.K, a.fa, fp4, BM)) return MX_ERR_CUDA;
     if (!make_operand_map(&tb, a.b_codes, a.N, a.K, a.fb, fp4, BN)) return MX_ERR_CUDA;
     Params p;
@@ -1152,8 +1233,8 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     cudaError_t e;
     p.q = mx_out(a);
     const int out = out_mode(a);
-    if (fp4) e = launch_out<true>(out, ta, tb, p, grid, st);
-    else e = launch_out<false>(out, ta, tb, p, grid, st);
+    if (fp4) e = launch_out<true>(out, ta, tb, tc, p, grid, st);
+    else e = launch_out<false>(out, ta, tb, tc, p, grid, st);
     return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 

@@ -23,6 +23,8 @@ struct MxQuantizeArgs {
     void *scales;
     int sl;
     int num_sms;
+    // stochastic-rounding position of output element (o, i): sr_base + o * sr_stride + i
+    uint64_t sr_base, sr_stride;
 };
 
 struct MxQuantizeDualArgs {
@@ -37,6 +39,7 @@ struct MxQuantizeDualArgs {
     void *codes_rows, *scales_rows, *codes_cols, *scales_cols;
     int sl;
     int num_sms;
+    uint64_t sr_base_rows, sr_stride_rows, sr_base_cols, sr_stride_cols;
 };
 
 struct MxDequantArgs {

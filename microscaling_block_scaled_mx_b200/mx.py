@@ -42,6 +42,11 @@ class _Precond(ctypes.Structure):
     _fields_ = [("hadamard", ctypes.c_int32), ("sign_mask", ctypes.c_uint32)]
 
 
+class _Shard(ctypes.Structure):
+    _fields_ = [("row0", ctypes.c_int64), ("col0", ctypes.c_int64),
+                ("total_rows", ctypes.c_int64), ("total_cols", ctypes.c_int64)]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -61,6 +66,13 @@ def lib() -> ctypes.CDLL:
             L.mx_quantize.restype = i32
             L.mx_quantize.argtypes = [vp, i32, i64, i64, i64, i32, i32, i32, u64,
                                       ctypes.POINTER(_Precond), vp, vp, i32, vp]
+            L.mx_quantize_shard.restype = i32
+            L.mx_quantize_shard.argtypes = [vp, i32, i64, i64, i64, i32, i32, i32, u64,
+                                            ctypes.POINTER(_Precond), ctypes.POINTER(_Shard), vp, vp, i32, vp]
+            L.mx_quantize_dual_shard.restype = i32
+            L.mx_quantize_dual_shard.argtypes = [vp, i32, i64, i64, i64, i32, i32, u64, i32, u64,
+                                                 ctypes.POINTER(_Precond), ctypes.POINTER(_Shard),
+                                                 vp, vp, vp, vp, i32, vp]
             L.mx_quantize_dual.restype = i32
             L.mx_quantize_dual.argtypes = [vp, i32, i64, i64, i64, i32, i32, u64, i32, u64,
                                            ctypes.POINTER(_Precond), vp, vp, vp, vp, i32, vp]
@@ -127,11 +139,13 @@ def codes_row_bytes(fmt, inner: int) -> int:
 def quantize(x: torch.Tensor, block_axis: int = 1, fmt="e4m3", rnd="rne", seed: int = 0,
              hadamard: bool = False, sign_mask: int = DEFAULT_SIGN_MASK, scale_layout="mma",
              codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
-             stream=None):
+             stream=None, shard=None):
     """MX cast of a 2-D CUDA tensor (rows x cols, row pitch x.stride(0)).
 
     Returns (codes, scales): codes is (outer, packed_inner_bytes) uint8 with
     outer = rows for block_axis=1 and cols for block_axis=0; scales is flat.
+    shard = (row0, col0, total_rows, total_cols) casts x as the piece at
+    (row0, col0) of a larger tensor (mx_quantize_shard).
     """
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit column stride")
@@ -146,21 +160,31 @@ def quantize(x: torch.Tensor, block_axis: int = 1, fmt="e4m3", rnd="rne", seed: 
     if scales is None:
         scales = torch.empty(max(scales_bytes(sl, outer, inner), 1), dtype=torch.uint8, device=x.device)
     pre = _Precond(1 if hadamard else 0, sign_mask & 0xFFFFFFFF)
-    rc = lib().mx_quantize(x.data_ptr(), DTYPE[x.dtype], rows, cols, x.stride(0), block_axis, f,
-                           ROUND[rnd] if isinstance(rnd, str) else int(rnd), seed & (2**64 - 1),
-                           ctypes.byref(pre), codes.data_ptr(), scales.data_ptr(), sl, _stream(stream))
-    _check(rc, "mx_quantize")
+    r = ROUND[rnd] if isinstance(rnd, str) else int(rnd)
+    if shard is None:
+        rc = lib().mx_quantize(x.data_ptr(), DTYPE[x.dtype], rows, cols, x.stride(0), block_axis, f,
+                               r, seed & (2**64 - 1), ctypes.byref(pre), codes.data_ptr(), scales.data_ptr(),
+                               sl, _stream(stream))
+        _check(rc, "mx_quantize")
+    else:
+        sh = _Shard(*shard)
+        rc = lib().mx_quantize_shard(x.data_ptr(), DTYPE[x.dtype], rows, cols, x.stride(0), block_axis, f,
+                                     r, seed & (2**64 - 1), ctypes.byref(pre), ctypes.byref(sh),
+                                     codes.data_ptr(), scales.data_ptr(), sl, _stream(stream))
+        _check(rc, "mx_quantize_shard")
     return codes, scales
 
 
 def quantize_dual(x: torch.Tensor, fmt="e4m3", rnd_rows="rne", seed_rows: int = 0, rnd_cols="rne",
                   seed_cols: int = 0, hadamard: bool = False, sign_mask: int = DEFAULT_SIGN_MASK,
-                  scale_layout="mma", out=None, stream=None):
+                  scale_layout="mma", out=None, stream=None, shard=None):
     """Both MX casts of a 2-D CUDA tensor from one read of it.
 
     Returns (codes_rows, scales_rows, codes_cols, scales_cols): the results of
     quantize(x, 1, ...) with (rnd_rows, seed_rows) and of quantize(x, 0, ...)
     with (rnd_cols, seed_cols, hadamard); `out` may supply the four buffers.
+    shard = (row0, col0, total_rows, total_cols) casts x as that piece of a
+    larger tensor (mx_quantize_dual_shard).
     """
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit column stride")
@@ -178,11 +202,20 @@ def quantize_dual(x: torch.Tensor, fmt="e4m3", rnd_rows="rne", seed_rows: int = 
     cr, sr_, cc, sc = out
     pre = _Precond(1 if hadamard else 0, sign_mask & 0xFFFFFFFF)
     rnd = lambda r: ROUND[r] if isinstance(r, str) else int(r)
-    rc = lib().mx_quantize_dual(x.data_ptr(), DTYPE[x.dtype], rows, cols, x.stride(0), f,
-                                rnd(rnd_rows), seed_rows & (2**64 - 1), rnd(rnd_cols), seed_cols & (2**64 - 1),
-                                ctypes.byref(pre), cr.data_ptr(), sr_.data_ptr(), cc.data_ptr(), sc.data_ptr(),
-                                sl, _stream(stream))
-    _check(rc, "mx_quantize_dual")
+    if shard is None:
+        rc = lib().mx_quantize_dual(x.data_ptr(), DTYPE[x.dtype], rows, cols, x.stride(0), f,
+                                    rnd(rnd_rows), seed_rows & (2**64 - 1), rnd(rnd_cols), seed_cols & (2**64 - 1),
+                                    ctypes.byref(pre), cr.data_ptr(), sr_.data_ptr(), cc.data_ptr(), sc.data_ptr(),
+                                    sl, _stream(stream))
+        _check(rc, "mx_quantize_dual")
+    else:
+        sh = _Shard(*shard)
+        rc = lib().mx_quantize_dual_shard(x.data_ptr(), DTYPE[x.dtype], rows, cols, x.stride(0), f,
+                                          rnd(rnd_rows), seed_rows & (2**64 - 1), rnd(rnd_cols),
+                                          seed_cols & (2**64 - 1), ctypes.byref(pre), ctypes.byref(sh),
+                                          cr.data_ptr(), sr_.data_ptr(), cc.data_ptr(), sc.data_ptr(),
+                                          sl, _stream(stream))
+        _check(rc, "mx_quantize_dual_shard")
     return cr, sr_, cc, sc
 
 

@@ -187,3 +187,33 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(m, "_lib", None)
     with pytest.raises(RuntimeError, match="libmx.so not found"):
         m.lib()
+
+
+def test_shard_validation(mx):
+    """Host-side checks of the sharded casts (nothing is launched)."""
+    import ctypes as C
+    L = mx.lib()
+    pre = mx._Precond(0, 0)
+
+    def q(axis, shard, rows=64, cols=64, rnd=1):
+        sh = mx._Shard(*shard) if shard is not None else None
+        return L.mx_quantize_shard(16, 1, rows, cols, cols, axis, 4, rnd, 0, C.byref(pre),
+                                   C.byref(sh) if sh is not None else None, 16, 16, 1, None)
+
+    def d(shard, rows=64, cols=64):
+        sh = mx._Shard(*shard)
+        return L.mx_quantize_dual_shard(16, 1, rows, cols, cols, 4, 1, 0, 1, 0, C.byref(pre), C.byref(sh),
+                                        16, 16, 16, 16, 1, None)
+
+    assert q(0, None) == -1                             # shard is required
+    assert q(0, (16, 0, 128, 64)) == -3                 # block-axis offset off a block boundary
+    assert q(1, (0, 16, 64, 128)) == -3
+    assert q(0, (0, 0, 112, 64), rows=64) == -3         # whole length along the block axis % 32
+    assert q(0, (96, 0, 128, 64)) == -1                 # piece past the end of the whole tensor
+    assert q(1, (-1, 0, 128, 64)) == -1
+    assert q(0, (0, 0, 2 ** 20, 2 ** 15)) == -5         # SR range counts the whole tensor
+    assert q(0, (0, 0, 2 ** 20, 2 ** 15), rnd=0) != -5
+    assert q(1, (0, 0, 64, 64), rows=0) == 0            # empty piece
+    assert d((16, 0, 128, 64)) == -3                    # both axes are block axes in the dual cast
+    assert d((0, 16, 64, 128)) == -3
+    assert d((96, 0, 128, 64)) == -1

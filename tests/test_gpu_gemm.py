@@ -329,3 +329,27 @@ def test_gemm_bounded_wait_reports_timeout(M, N, K):
     torch.cuda.synchronize()
     assert mx.last_device_status() == 0
     assert torch.isfinite(c).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 300, 384), (520, 97, 512), (4000, 2600, 2048)])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_writes_only_inside_c(oracle, M, N, K, out_dtype):
+    """The epilogue's stores stay inside the M x N window of a pitched C: the
+    columns between N and the leading dimension and the rows after M keep
+    their contents (one-SM and CTA-pair kernels, both output types)."""
+    rng = np.random.default_rng(M * 7 + N)
+    a = rng.standard_normal((M, K)).astype(np.float32)
+    b = rng.standard_normal((N, K)).astype(np.float32)
+    ac, as_ = mx.quantize(to_device(a), 1, "e4m3")
+    bc, bs = mx.quantize(to_device(b), 1, "e4m3")
+    ldc = (N + 7) // 8 * 8 + 40
+    buf = torch.full((M + 3, ldc), 123.0, dtype=out_dtype, device=dev())
+    out = buf[:M, :N]
+    mx.gemm(ac, as_, bc, bs, M, N, K, fa="e4m3", out=out)
+    torch.cuda.synchronize()
+    h = to_f64(buf)
+    assert np.all(h[:M, N:] == 123.0) and np.all(h[M:, :] == 123.0)
+    oac, oas = oracle.quantize(a, 1, oracle.E4M3, scale_layout=oracle.MMA)
+    obc, obs = oracle.quantize(b, 1, oracle.E4M3, scale_layout=oracle.MMA)
+    ref, bound = oracle.gemm_decoded(oac, oas, oracle.E4M3, obc, obs, oracle.E4M3, M, N, K)
+    check(h[:M, :N], ref, bound, out_dtype, (M, N, K))
