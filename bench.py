@@ -63,6 +63,29 @@ MEASURED_TRAFFIC = {
 }
 
 
+# Warp instructions per value of the column (Hadamard + SR) cast kernels, from
+# ncu's smsp__inst_executed.sum on one launch divided by the launch's values;
+# the same source-hash rule as MEASURED_TRAFFIC.  They give the instruction-
+# issue roofline of those casts: at most 4 warp instructions per clock per SM.
+MEASURED_INSTR = {
+    "cast_cols_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"), None, {}),
+    "cast_dual_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"), None, {}),
+}
+
+
+def measured_instr(kernel: str, workload: str):
+    names, sha, table = MEASURED_INSTR[kernel]
+    if sha is None or workload not in table or sources_sha256(names) != sha:
+        return None
+    return table[workload]
+
+
+def issue_bound_us(instr_per_value: float, values: int, sms: int, sm_mhz: float) -> float:
+    """Time at the instruction-issue roofline: every SM issues at most one warp
+    instruction per clock on each of its four schedulers."""
+    return instr_per_value * values / (sms * 4 * sm_mhz * 1e6) * 1e6
+
+
 def sources_sha256(names) -> str:
     h = hashlib.sha256()
     for n in names:
@@ -595,7 +618,10 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
             fn()
     torch.cuda.synchronize()
     ms = timed(lambda: [fn() for fn in ops.values()], steps)      # the whole step
-    us = {k: 1e3 * timed(fn, steps) / steps for k, fn in ops.items()}
+    with ClockSampler(dev.index or 0) as clk:
+        us = {k: 1e3 * timed(fn, steps) / steps for k, fn in ops.items()}
+    sm_mhz = clk.summary()["sm_mhz"] or 1965.0
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     cast_bytes = {"cast_dY": T * Do * 2 + T * Do // 2 + T * Do // 32,
                   "cast_X": T * Di * 2 + T * Di // 2 + T * Di // 32}
     flops = 2.0 * Do * Di * T
@@ -603,9 +629,20 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
     hbm = float(peaks["hbm_gbs"])
     out = {"workload": "wgrad_mxfp4 dY 16384x4096, X 16384x14336 (Student-t), Hadamard+SR along tokens, "
                        "dW fp32", "steps": steps, "ms_per_step": round(ms / steps, 4)}
+    values = {"cast_dY": T * Do, "cast_X": T * Di}
+    shape = {"cast_dY": f"{T}x{Do}", "cast_X": f"{T}x{Di}"}
     for k in ("cast_dY", "cast_X"):
         gbs = cast_bytes[k] / (us[k] * 1e-6) / 1e9
+        hbm_us = cast_bytes[k] / (hbm * 1e9) * 1e6
         out[k] = {"us": round(us[k], 1), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+        ipv = measured_instr("cast_cols_had_sr", f"e2m1_bf16_{shape[k]}")
+        if ipv is not None:
+            alu_us = issue_bound_us(ipv, values[k], sms, sm_mhz)
+            out[k]["alu"] = {"warp_instr_per_value": ipv, "bound_us": round(alu_us, 1), "sm_mhz": sm_mhz,
+                             "frac": round(alu_us / us[k], 4)}
+            # the roofline is the slower of the two bounds
+            out[k]["roofline"] = {"bound": "alu" if alu_us > hbm_us else "hbm",
+                                  "frac": round(max(alu_us, hbm_us) / us[k], 4)}
     tf = flops / (us["gemm_dW"] * 1e-6) / 1e12
     out["gemm_dW"] = {"us": round(us["gemm_dW"], 1), "tflops": round(tf, 1), "frac": round(tf / fp4_peak, 4),
                       "peak": round(fp4_peak, 1)}

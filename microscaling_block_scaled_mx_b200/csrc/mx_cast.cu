@@ -275,17 +275,30 @@ __device__ __forceinline__ void stage_tile(const CastParams &p, uint8_t *buf, in
 // (sr_base 0 and sr_stride = rows for a whole tensor).
 // KEYED: the caller passes the packed 16-bit maxima of |bf16| of the two
 // columns (bf16_pair_max over the raw words), valid without the Hadamard.
-template <int FMT, bool SR, bool HAD, bool KEYED = false>
+// Sign flip of the fixed-sign Hadamard with the default mask, applied while
+// loading: row j of a block is negated (both columns of the pair, an exact
+// sign-bit flip, the same as multiplying by -1) unless bit j of the mask is
+// set.  With the mask a compile-time constant this is one XOR on half of the
+// rows and nothing on the others.
+__device__ __forceinline__ constexpr bool default_mask_negates(int j) {
+    return ((MX_DEFAULT_SIGN_MASK >> j) & 1u) == 0u;
+}
+
+// SIGNED: the caller has already applied the Hadamard's sign flips to x
+// (the default mask, folded into the loads).
+template <int FMT, bool SR, bool HAD, bool KEYED = false, bool SIGNED = false>
 __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&x)[32], int64_t gc, int64_t gr0,
                                                 uint32_t pair_max16 = 0) {
     static_assert(!(KEYED && HAD), "the bf16 maxima describe the values before the Hadamard");
     constexpr int BITS = Fmt<FMT>::bits;
     const int64_t R = p.rows, C = p.cols;
     if (HAD) {
+        if (!SIGNED) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const float sg = ((p.sign_mask >> j) & 1u) ? 1.0f : -1.0f;
-            x[j] = f2_mul(x[j], f2_pack(sg, sg));
+            for (int j = 0; j < 32; ++j) {
+                const float sg = ((p.sign_mask >> j) & 1u) ? 1.0f : -1.0f;
+                x[j] = f2_mul(x[j], f2_pack(sg, sg));
+            }
         }
 #pragma unroll
         for (int h = 1; h < 32; h <<= 1) {
@@ -380,7 +393,8 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
     }
 }
 
-template <int FMT, bool SR, bool BF16_IN, bool HAD>
+// DEFM: the Hadamard uses the default sign mask, folded into the loads.
+template <int FMT, bool SR, bool BF16_IN, bool HAD, bool DEFM = false>
 __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p) {
     using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
     constexpr int TILE_BYTES = COL_TILE_R * COL_TILE_C * sizeof(TIn);
@@ -419,15 +433,17 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
             for (int j = 0; j < 32; ++j) {
                 const int off = (blk * 32 + j) * COL_TILE_C + 2 * pair;
                 if (BF16_IN) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t *>(tile + off);
+                    uint32_t w = *reinterpret_cast<const uint32_t *>(tile + off);
                     words[j] = w;
+                    if (HAD && DEFM && default_mask_negates(j)) w ^= 0x80008000u;
                     x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
                 } else {
                     x[j] = *reinterpret_cast<const uint64_t *>(tile + off);
+                    if (HAD && DEFM && default_mask_negates(j)) x[j] ^= 0x8000000080000000ull;
                 }
             }
             if (BF16_IN && !HAD) encode_col_pair<FMT, SR, false, true>(p, x, gc, gr0, bf16_pair_max<32>(words));
-            else encode_col_pair<FMT, SR, HAD>(p, x, gc, gr0);
+            else encode_col_pair<FMT, SR, HAD, false, DEFM>(p, x, gc, gr0);
         }
         __syncthreads();             // everyone is done with `buf` before it is refilled
     }
@@ -445,7 +461,7 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
 // thread encodes one column pair of one 32-row block (as cast_cols) and two
 // 32-element row blocks (as cast_rows, RNE or SR with its own seed).  The
 // result equals mx_quantize along rows plus mx_quantize along columns.
-template <int FMT, bool BF16_IN, bool HAD>
+template <int FMT, bool BF16_IN, bool HAD, bool DEFM = false>
 __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr, CastParams pc, int sr_rows,
                                                                    int sr_cols) {
     using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
@@ -494,11 +510,13 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
             for (int j = 0; j < 32; ++j) {
                 const uint8_t *src = tile + (blk * 32 + j) * ROW_BYTES + col_off[j & 1];
                 if (BF16_IN) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t *>(src);
+                    uint32_t w = *reinterpret_cast<const uint32_t *>(src);
                     words[j] = w;
+                    if (HAD && DEFM && default_mask_negates(j)) w ^= 0x80008000u;
                     x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
                 } else {
                     x[j] = *reinterpret_cast<const uint64_t *>(src);
+                    if (HAD && DEFM && default_mask_negates(j)) x[j] ^= 0x8000000080000000ull;
                 }
             }
             if (BF16_IN && !HAD) {
@@ -506,8 +524,8 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
                 if (sr_cols) encode_col_pair<FMT, true, false, true>(pc, x, gc, gr0, m16);
                 else encode_col_pair<FMT, false, false, true>(pc, x, gc, gr0, m16);
             } else {
-                if (sr_cols) encode_col_pair<FMT, true, HAD>(pc, x, gc, gr0);
-                else encode_col_pair<FMT, false, HAD>(pc, x, gc, gr0);
+                if (sr_cols) encode_col_pair<FMT, true, HAD, false, DEFM>(pc, x, gc, gr0);
+                else encode_col_pair<FMT, false, HAD, false, DEFM>(pc, x, gc, gr0);
             }
         }
         // ---- row blocks ----
@@ -738,6 +756,10 @@ static cudaError_t launch_cast_fmt(const CastParams &p, int xdt, int block_axis,
         }
     } else {
         const int64_t tiles = ((p.rows + COL_TILE_R - 1) / COL_TILE_R) * ((p.cols + COL_TILE_C - 1) / COL_TILE_C);
+        if (had && p.sign_mask == MX_DEFAULT_SIGN_MASK) {
+            if (bf) return launch_cols<cast_cols_kernel<FMT, SR, true, true, true>>(2, p, tiles, sms, st);
+            return launch_cols<cast_cols_kernel<FMT, SR, false, true, true>>(4, p, tiles, sms, st);
+        }
         if (had) {
             if (bf) return launch_cols<cast_cols_kernel<FMT, SR, true, true>>(2, p, tiles, sms, st);
             return launch_cols<cast_cols_kernel<FMT, SR, false, true>>(4, p, tiles, sms, st);
@@ -771,6 +793,10 @@ static cudaError_t launch_dual_fmt(const CastParams &pr, const CastParams &pc, i
                                    int sr_cols, int sms, cudaStream_t st) {
     const int64_t tiles = ((pc.rows + COL_TILE_R - 1) / COL_TILE_R) * ((pc.cols + COL_TILE_C - 1) / COL_TILE_C);
     const bool bf = xdt == MX_BF16;
+    if (had && pc.sign_mask == MX_DEFAULT_SIGN_MASK) {
+        if (bf) return launch_dual<cast_dual_kernel<FMT, true, true, true>>(2, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+        return launch_dual<cast_dual_kernel<FMT, false, true, true>>(4, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+    }
     if (had) {
         if (bf) return launch_dual<cast_dual_kernel<FMT, true, true>>(2, pr, pc, sr_rows, sr_cols, tiles, sms, st);
         return launch_dual<cast_dual_kernel<FMT, false, true>>(4, pr, pc, sr_rows, sr_cols, tiles, sms, st);

@@ -594,30 +594,35 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
 // (the pair-wide tcgen05.cp copies each CTA's shared memory into its own
 // tensor memory).  All loads of both CTAs complete on CTA 0's stage barrier
 // (the two-SM form of the TMA load); CTA 0's commit frees the stage in both
-// CTAs.  A 256-column fp32 accumulator leaves no room for a second one next to
-// the scale factors, so the epilogue first drains the accumulator into
-// registers, releases it to the MMA issuer, and only then stores to C.
+// CTAs.  Two tile widths: 256 columns, whose fp32 accumulator leaves no room
+// for a second one next to the scale factors (the epilogue first drains the
+// accumulator into registers, releases it to the MMA issuer, and only then
+// stores to C), and 192 columns with two accumulators, so the next tile's
+// MMAs run while the epilogue drains the previous one.  A 192-column tile at
+// an odd position starts 64 rows into a 128-row B scale atom: its B scale
+// factors are addressed two tensor-memory columns later.
 // ------------------------------------------------------------------------
 constexpr int PAIR_BM = 256;
-constexpr int PAIR_BN = 256;
-constexpr int PAIR_B_ROWS = PAIR_BN / 2;                 // B rows per CTA
 constexpr int PAIR_A_BYTES = 128 * BK_BYTES;             // 16 KiB per CTA per stage
-constexpr int PAIR_B_BYTES = PAIR_B_ROWS * BK_BYTES;     // 16 KiB per CTA per stage
-constexpr uint32_t PAIR_SF_COL = PAIR_BN;                // scale factors after the accumulator
 
-template <bool FP4> struct PairCfg {
+template <bool FP4, int PBN> struct PairCfg {
+    static constexpr int BN = PBN;                       // tile columns (B rows)
+    static constexpr int B_ROWS = PBN / 2;               // B rows per CTA
+    static constexpr int B_BYTES = B_ROWS * BK_BYTES;    // per CTA per stage
+    static constexpr int ACC_BUFS = PBN == 256 ? 1 : 2;  // accumulators in tensor memory
+    static constexpr uint32_t SF_COL = ACC_BUFS * PBN;   // scale factors after the accumulators
     static constexpr int G = FP4 ? 2 : 1;                // scale atoms along K per stage
-    static constexpr int STAGES = 5;
+    static constexpr int STAGES = (PBN == 192 && !FP4) ? 6 : 5;
     static constexpr int SFA_BYTES = ATOM * G;
     static constexpr int SFB_BYTES = 2 * ATOM * G;       // both 128-row scale blocks the tile touches
     static constexpr int SFA_COLS = 4 * G;
     static constexpr int SFB_COLS = 8 * G;
     static constexpr int SF_STAGE_COLS = SFA_COLS + SFB_COLS;
-    static constexpr int STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES;
+    static constexpr int STAGE_BYTES = PAIR_A_BYTES + B_BYTES;
     // shared-memory layout
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * PAIR_A_BYTES;
-    static constexpr int OFF_SFA = OFF_B + STAGES * PAIR_B_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_EPI = (OFF_SFB + STAGES * SFB_BYTES + 1023) / 1024 * 1024;
     static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_WARP_BYTES;
@@ -625,8 +630,9 @@ template <bool FP4> struct PairCfg {
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
     static constexpr int SMEM = OFF_ABORT + 4 + 1024;    // + alignment slack
-    static_assert(PAIR_BN + STAGES * SF_STAGE_COLS <= 512, "tensor memory columns");
+    static_assert(SF_COL + STAGES * SF_STAGE_COLS <= 512, "tensor memory columns");
     static_assert(SMEM <= 232448, "shared memory per block");
+    static_assert(PBN == 256 || PBN == 192, "pair tile widths");
 };
 
 struct PairParams {
@@ -635,7 +641,7 @@ struct PairParams {
     int M, N, K;
     int k_tiles;
     int k_groups;
-    int tiles_m, tiles_n;      // 256 x 256 pair tiles
+    int tiles_m, tiles_n;      // 256-row pair tiles
     float alpha;
     uint32_t idesc;
     uint32_t ab_tx;            // bytes one CTA's A and B loads of a stage deliver
@@ -695,12 +701,12 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
     }
 }
 
-template <bool FP4, int OUT>
+template <bool FP4, int OUT, int PBN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                     const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
                     const __grid_constant__ CUtensorMap tma_c, PairParams p) {
-    using C = PairCfg<FP4>;
+    using C = PairCfg<FP4, PBN>;
     constexpr int STAGES_P = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -760,8 +766,8 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                 // only feeds discarded outputs, so its loads are clamped to rows
                 // that exist and no TMA box is ever entirely outside its tensor
                 const int m0 = min(tm * PAIR_BM + 128 * static_cast<int>(rank), p.M - 1);
-                const int nb0 = min(tn * PAIR_BN + PAIR_B_ROWS * static_cast<int>(rank), p.N - 1);
-                const int rb_a = m0 / 128, rb_b = (tn * PAIR_BN) / 128;
+                const int nb0 = min(tn * PBN + C::B_ROWS * static_cast<int>(rank), p.N - 1);
+                const int rb_a = m0 / 128, rb_b = (tn * PBN) / 128;
                 const int rb_b1 = min(rb_b + 1, (p.N - 1) / 128);
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
@@ -772,7 +778,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                     const uint32_t fb = map_to_rank(full_bar(s), 0);
                     if (rank == 0) mbar_expect_tx(full_bar(s), stage_bytes);
                     tma_load_2d_pair(sbase + C::OFF_A + s * PAIR_A_BYTES, &tma_a, kt * BK_BYTES, m0, fb);
-                    tma_load_2d_pair(sbase + C::OFF_B + s * PAIR_B_BYTES, &tma_b, kt * BK_BYTES, nb0, fb);
+                    tma_load_2d_pair(sbase + C::OFF_B + s * C::B_BYTES, &tma_b, kt * BK_BYTES, nb0, fb);
                     // scale atoms: a scale buffer is viewed as rows of 256 bytes, two per atom
                     const int kg = kt * C::G;
                     tma_load_2d_pair(sbase + C::OFF_SFA + s * C::SFA_BYTES, &tma_sfa, 0,
@@ -802,16 +808,18 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             bool issued = false;
             int local = 0;
             for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters, ++local) {
-                const int b = 0;
-                const uint32_t acc_ph = local & 1;
+                const int b = local % C::ACC_BUFS;
+                const uint32_t acc_ph = (local / C::ACC_BUFS) & 1;
                 if (!wait_bounded(acc_empty(b), acc_ph ^ 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem;
-                const uint32_t sfb_shift = 0u;
+                int tm, tn;
+                tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
+                const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * PBN);
+                const uint32_t sfb_shift = ((tn * PBN) & 127) ? 2u : 0u;   // tile starts 64 rows into an atom
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!wait_bounded(full_bar(s), ph, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t sfa_t = tmem + PAIR_SF_COL + s * C::SF_STAGE_COLS;
+                    const uint32_t sfa_t = tmem + C::SF_COL + s * C::SF_STAGE_COLS;
                     const uint32_t sfb_t = sfa_t + C::SFA_COLS;
                     const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
@@ -824,7 +832,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                                                   scale_atom_desc(sfb_s + h * (C::SFB_BYTES / 2) + g * ATOM));
                     }
                     const uint32_t a_s = sbase + C::OFF_A + s * PAIR_A_BYTES;
-                    const uint32_t b_s = sbase + C::OFF_B + s * PAIR_B_BYTES;
+                    const uint32_t b_s = sbase + C::OFF_B + s * C::B_BYTES;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t g = FP4 ? (k >> 1) : 0u;
@@ -852,10 +860,10 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
         const int half = (warp - 2) >> 2;
         EpiWriter ew{&tma_c, sbase + C::OFF_EPI + static_cast<uint32_t>(warp - 2) * EPI_WARP_BYTES, 0, lane};
         int local = 0;
-        constexpr int NCH = PAIR_BN / 2 / 32;    // 32-column chunks per warp
+        constexpr int NCH = PBN / 2 / 32;        // 32-column chunks per warp
         for (int tile = cluster_id; tile < num_tiles; tile += n_clusters, ++local) {
-            const int b = 0;
-            const uint32_t acc_ph = local & 1;
+            const int b = local % C::ACC_BUFS;
+            const uint32_t acc_ph = (local / C::ACC_BUFS) & 1;
             int ok = 1;
             if (lane == 0) ok = wait_bounded(acc_full(b), acc_ph, abort_flag) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -864,8 +872,8 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             int tm, tn;
             tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
             const int m = tm * PAIR_BM + 128 * static_cast<int>(rank) + q * 32 + lane;
-            const int c0 = half * (PAIR_BN / 2);
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + c0;
+            const int c0 = half * (PBN / 2);
+            const uint32_t taddr = tmem + static_cast<uint32_t>(b * PBN) + (static_cast<uint32_t>(q * 32) << 16) + c0;
             uint32_t r[32 * NCH];
 #pragma unroll
             for (int j = 0; j < NCH; ++j) tmem_ld_x32_nowait(taddr + 32 * j, r + 32 * j);
@@ -874,7 +882,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(map_to_rank(acc_empty(b), 0));
-            const int n_base = tn * PAIR_BN + c0;
+            const int n_base = tn * PBN + c0;
             if constexpr (OUT == OUT_MX) {
                 Params pp;
                 pp.c = p.c; pp.ldc = p.ldc; pp.M = p.M; pp.N = p.N; pp.alpha = p.alpha; pp.q = p.q;
@@ -885,7 +893,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                 constexpr int PC = OUT == OUT_BF16 ? 32 : 16;   // columns per piece
                 if (m_warp < p.M) {
 #pragma unroll
-                    for (int j = 0; j < (PAIR_BN / 2) / PC; ++j)
+                    for (int j = 0; j < (PBN / 2) / PC; ++j)
                         if (n_base + PC * j < p.N) epi_piece<OUT>(ew, r + PC * j, p.alpha, n_base + PC * j, m_warp);
                 }
             }
@@ -1063,14 +1071,15 @@ cudaError_t launch_overlapped(Kern kern, int grid, int smem, cudaStream_t st, co
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <bool FP4, int OUT>
+template <bool FP4, int OUT, int PBN>
 cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
                         const CUtensorMap &tsb, const CUtensorMap &tc, const PairParams &p, int grid,
                         cudaStream_t st) {
-    auto kern = mx_gemm_pair_kernel<FP4, OUT>;
+    auto kern = mx_gemm_pair_kernel<FP4, OUT, PBN>;
+    constexpr int smem = PairCfg<FP4, PBN>::SMEM;
     static std::atomic<uint64_t> configured{0};   // per instantiation, one bit per device
-    if (cudaError_t e = ensure_smem_limit(kern, PairCfg<FP4>::SMEM, configured); e != cudaSuccess) return e;
-    return launch_overlapped(kern, grid, PairCfg<FP4>::SMEM, st, ta, tb, tsa, tsb, tc, p);
+    if (cudaError_t e = ensure_smem_limit(kern, smem, configured); e != cudaSuccess) return e;
+    return launch_overlapped(kern, grid, smem, st, ta, tb, tsa, tsb, tc, p);
 }
 
 template <bool FP4, int OUT>
@@ -1082,13 +1091,13 @@ cudaError_t launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorM
     return launch_overlapped(kern, grid, SMEM_BYTES, st, ta, tb, tc, p);
 }
 
-template <bool FP4>
+template <bool FP4, int PBN>
 cudaError_t launch_pair_out(int out, const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
                             const CUtensorMap &tsb, const CUtensorMap &tc, const PairParams &p, int grid,
                             cudaStream_t st) {
-    if (out == OUT_MX) return launch_pair<FP4, OUT_MX>(ta, tb, tsa, tsb, tc, p, grid, st);
-    if (out == OUT_BF16) return launch_pair<FP4, OUT_BF16>(ta, tb, tsa, tsb, tc, p, grid, st);
-    return launch_pair<FP4, OUT_F32>(ta, tb, tsa, tsb, tc, p, grid, st);
+    if (out == OUT_MX) return launch_pair<FP4, OUT_MX, PBN>(ta, tb, tsa, tsb, tc, p, grid, st);
+    if (out == OUT_BF16) return launch_pair<FP4, OUT_BF16, PBN>(ta, tb, tsa, tsb, tc, p, grid, st);
+    return launch_pair<FP4, OUT_F32, PBN>(ta, tb, tsa, tsb, tc, p, grid, st);
 }
 
 template <bool FP4>
@@ -1119,6 +1128,14 @@ MxOut mx_out(const MxGemmArgs &a) {
 namespace {
 // armed by mx_debug_gemm_skip_stage; consumed by the next GEMM call of the same host thread
 thread_local int g_skip_k_tile = -1;
+// set by mx_debug_gemm_force_kernel for this host thread's GEMM calls (-1: automatic)
+thread_local int g_force_kernel = -1;
+}
+
+extern "C" int mx_debug_gemm_force_kernel(int tile_n) {
+    if (tile_n != -1 && tile_n != 0 && tile_n != 192 && tile_n != 256) return MX_ERR_ARG;
+    g_force_kernel = tile_n;
+    return MX_OK;
 }
 
 extern "C" int mx_debug_gemm_skip_stage(int k_tile) {
@@ -1146,8 +1163,8 @@ bool use_mxf4(const MxGemmArgs &a) {
     return a.fa == MX_E2M1 && a.fb == MX_E2M1 && a.K % 256 == 0;
 }
 
-// M > 128: the two-SM kernel (256 x 256 tiles over CTA pairs).
-int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
+// The two-SM kernel: 256 x pbn tiles over CTA pairs (pbn 256 or 192).
+int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
     using namespace mxg;
     const bool fp4 = use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;     // K bytes of a uint8 stage view
@@ -1156,7 +1173,7 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     CUtensorMap ta, tb, tsa, tsb, tc;
     if (!make_c_map(&tc, a)) return MX_ERR_CUDA;
     if (!make_operand_map(&ta, a.a_codes, a.M, a.K, a.fa, fp4, 128)) return MX_ERR_CUDA;
-    if (!make_operand_map(&tb, a.b_codes, a.N, a.K, a.fb, fp4, PAIR_B_ROWS)) return MX_ERR_CUDA;
+    if (!make_operand_map(&tb, a.b_codes, a.N, a.K, a.fb, fp4, pbn / 2)) return MX_ERR_CUDA;
     const int64_t sa_bytes = (a.M + 127) / 128 * 128 * k_groups * 4;
     const int64_t sb_bytes = (a.N + 127) / 128 * 128 * k_groups * 4;
     if (!make_scale_map(&tsa, a.a_scales, sa_bytes, G)) return MX_ERR_CUDA;
@@ -1170,10 +1187,10 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     p.k_tiles = static_cast<int>(k_bytes / BK_BYTES);
     p.k_groups = static_cast<int>(k_groups);
     p.tiles_m = static_cast<int>((a.M + PAIR_BM - 1) / PAIR_BM);
-    p.tiles_n = static_cast<int>((a.N + PAIR_BN - 1) / PAIR_BN);
+    p.tiles_n = static_cast<int>((a.N + pbn - 1) / pbn);
     p.alpha = a.alpha;
-    p.idesc = make_idesc(a.fa, a.fb, fp4, PAIR_BM, PAIR_BN);
-    p.ab_tx = stage_tx_bytes(a.fa, fp4, 128) + stage_tx_bytes(a.fb, fp4, PAIR_B_ROWS);
+    p.idesc = make_idesc(a.fa, a.fb, fp4, PAIR_BM, pbn);
+    p.ab_tx = stage_tx_bytes(a.fa, fp4, 128) + stage_tx_bytes(a.fb, fp4, pbn / 2);
     raster_for(a, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major);
     p.skip_k_tile = g_skip_k_tile;
     g_skip_k_tile = -1;
@@ -1183,27 +1200,31 @@ int launch_gemm_pair(const MxGemmArgs &a, cudaStream_t st) {
     cudaError_t e;
     p.q = mx_out(a);
     const int out = out_mode(a);
-    if (fp4) e = launch_pair_out<true>(out, ta, tb, tsa, tsb, tc, p, grid, st);
-    else e = launch_pair_out<false>(out, ta, tb, tsa, tsb, tc, p, grid, st);
+    if (pbn == 256) e = fp4 ? launch_pair_out<true, 256>(out, ta, tb, tsa, tsb, tc, p, grid, st)
+                            : launch_pair_out<false, 256>(out, ta, tb, tsa, tsb, tc, p, grid, st);
+    else e = fp4 ? launch_pair_out<true, 192>(out, ta, tb, tsa, tsb, tc, p, grid, st)
+                 : launch_pair_out<false, 192>(out, ta, tb, tsa, tsb, tc, p, grid, st);
     return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
 }  // namespace
 
-// Kernel choice.  CTA pairs on 256 x 256 tiles have the higher steady-state
+// Kernel choice.  CTA pairs on 256-row tiles have the higher steady-state
 // rate (each MMA and scale copy covers two SMs, each SM loads half of B), but
 // a shape with few such tiles or few K steps per tile is dominated by wave
 // quantisation and per-tile start-up, where the one-SM kernel's smaller tiles
 // and overlapped epilogue win (measured on the GPT-2-shaped GEMMs).
-bool use_pair_kernel(const MxGemmArgs &a) {
-    if (a.M <= 128 || a.K < 2048) return false;
+// Returns the pair tile width to use, or 0 for the one-SM kernel.
+int pair_tile_n(const MxGemmArgs &a) {
+    if (g_force_kernel >= 0) return g_force_kernel;
+    if (a.M <= 128 || a.K < 2048) return 0;
     const int64_t pair_tiles = ((a.M + 255) / 256) * ((a.N + 255) / 256);
-    return pair_tiles >= a.num_sms;
+    return pair_tiles >= a.num_sms ? 256 : 0;
 }
 
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     using namespace mxg;
-    if (use_pair_kernel(a)) return launch_gemm_pair(a, st);
+    if (const int pbn = pair_tile_n(a); pbn != 0) return launch_gemm_pair(a, pbn, st);
     const bool fp4 = use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;
     CUtensorMap ta, tb, tc;

@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
             L.mx_abi_version.argtypes = []
             L.mx_debug_gemm_skip_stage.restype = i32
             L.mx_debug_gemm_skip_stage.argtypes = [i32]
+            L.mx_debug_gemm_force_kernel.restype = i32
+            L.mx_debug_gemm_force_kernel.argtypes = [i32]
             _lib = L
     return _lib
 

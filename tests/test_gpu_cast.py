@@ -310,3 +310,23 @@ def test_wgrad_casts_full_size(oracle, wgrad_oracle_operands):
     for name, t, seed, want in (("dY", d["dy"], 42, d["dy_q"]), ("X", d["xx"], 43, d["xx_q"])):
         got = gpu_cast(t, 0, "e2m1", "sr", seed=seed, hadamard=True)
         assert_same(got, want, name)
+
+
+@pytest.mark.parametrize("mask", [0x00000000, 0xFFFFFFFF, 0x12345678, MASK ^ 1])
+@pytest.mark.parametrize("bf16", [True, False])
+def test_hadamard_any_sign_mask(oracle, mask, bf16):
+    """The default mask is compiled into the loads; any other mask takes the
+    general path.  Both match the oracle byte for byte (column cast and the
+    dual cast's column output), SR and RNE."""
+    x = mixed_input(256, 96, 77, bf16)
+    xd = to_device(x)
+    for rnd in ("rne", "sr"):
+        codes, scales = mx.quantize(xd, 0, "e2m1", rnd=rnd, seed=3, hadamard=True, sign_mask=mask)
+        torch.cuda.synchronize()
+        oc, os_ = oracle.quantize(x, 0, oracle.E2M1, rnd=1 if rnd == "sr" else 0, seed=3, hadamard=True,
+                                  sign_mask=mask, scale_layout=oracle.MMA)
+        assert np.array_equal(host(codes), oc), (hex(mask), rnd, first_mismatch(host(codes), oc))
+        assert np.array_equal(host(scales)[:os_.size], os_), (hex(mask), rnd)
+        _, _, cc, sc = mx.quantize_dual(xd, "e2m1", rnd_cols=rnd, seed_cols=3, hadamard=True, sign_mask=mask)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(cc), oc) and np.array_equal(host(sc)[:os_.size], os_), (hex(mask), rnd)

@@ -353,3 +353,79 @@ def test_gemm_writes_only_inside_c(oracle, M, N, K, out_dtype):
     obc, obs = oracle.quantize(b, 1, oracle.E4M3, scale_layout=oracle.MMA)
     ref, bound = oracle.gemm_decoded(oac, oas, oracle.E4M3, obc, obs, oracle.E4M3, M, N, K)
     check(h[:M, :N], ref, bound, out_dtype, (M, N, K))
+
+
+# Every kernel on every shape: the automatic choice picks one kernel per
+# shape; mx_debug_gemm_force_kernel (include/mx_debug.h) lets these tests run
+# the one-SM kernel (0) and both CTA-pair tile widths (256, 192) on the same
+# operands.
+KERNELS = [0, 256, 192]
+
+
+class forced_kernel:
+    def __init__(self, tile_n):
+        self.tile_n = tile_n
+
+    def __enter__(self):
+        assert mx.lib().mx_debug_gemm_force_kernel(self.tile_n) == 0
+        return self
+
+    def __exit__(self, *exc):
+        mx.lib().mx_debug_gemm_force_kernel(-1)
+        return False
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("fa,fb,K", [("e4m3", "e4m3", 512), ("e2m1", "e2m1", 1024), ("e3m2", "e2m1", 384),
+                                     ("e5m2", "e2m3", 256)])
+def test_gemm_each_kernel_bit_exact(oracle, kernel, fa, fb, K):
+    """Exact partial sums, so every kernel must return the oracle's C bit for
+    bit; shapes with several tiles along both axes, odd 192-column tiles and
+    ragged edges on both axes."""
+    for (M, N) in [(512, 576), (300, 200), (640, 1000)]:
+        rng = np.random.default_rng(M + N + K + kernel)
+        a = np.clip(small_int_operand(rng, M, K), -3, 3)
+        b = np.clip(small_int_operand(rng, N, K), -3, 3)
+        with forced_kernel(kernel):
+            got, ref, bound = run_gemm(oracle, a, b, fa, M, N, K, fb=fb)
+        exact = oracle.round_f32(ref).astype(np.float64)
+        assert np.array_equal(got, exact), (kernel, fa, fb, M, N, np.argwhere(got != exact)[:5])
+    assert mx.last_device_status() == 0
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_each_kernel_tolerance_and_window(oracle, kernel, out_dtype):
+    """General data on every kernel, pitched C with sentinels around the
+    M x N window (nothing outside it is written)."""
+    rng = np.random.default_rng(23 + kernel)
+    for (M, N, K, fmt) in [(700, 900, 2048, "e2m1"), (264, 392, 768, "e4m3")]:
+        a = (rng.standard_normal((M, K)) * np.exp2(rng.uniform(-3, 3, (M, 1)))).astype(np.float32)
+        b = rng.standard_t(3, size=(N, K)).astype(np.float32)
+        ac, as_ = mx.quantize(to_device(a), 1, fmt)
+        bc, bs = mx.quantize(to_device(b), 1, fmt)
+        ldc = (N + 7) // 8 * 8 + 24
+        buf = torch.full((M + 2, ldc), -5.0, dtype=out_dtype, device=dev())
+        with forced_kernel(kernel):
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, alpha=0.5, out=buf[:M, :N])
+        torch.cuda.synchronize()
+        h = to_f64(buf)
+        assert np.all(h[:M, N:] == -5.0) and np.all(h[M:, :] == -5.0), (kernel, M, N)
+        f = oracle.FORMATS[fmt]
+        oac, oas = oracle.quantize(a, 1, f, scale_layout=oracle.MMA)
+        obc, obs = oracle.quantize(b, 1, f, scale_layout=oracle.MMA)
+        ref, bound = oracle.gemm_decoded(oac, oas, f, obc, obs, f, M, N, K, alpha=0.5)
+        check(h[:M, :N], ref, bound, out_dtype, (kernel, M, N, K))
+    assert mx.last_device_status() == 0
+
+
+@pytest.mark.parametrize("kernel", [256, 192])
+def test_gemm_pair_kernels_on_llama_shape(oracle, kernel):
+    """The first Llama-3 MXFP4 shape (8192 x 6144 x 4096) on both pair tile
+    widths: 512 sampled rows against the oracle."""
+    M, N, K = I.LLAMA3_GEMMS[0]
+    x, w = I.linear_operands(M, K, N, 3, stream=0)
+    rows = np.sort(np.random.default_rng(kernel).choice(M, 512, replace=False))
+    with forced_kernel(kernel):
+        got, ref, bound = run_gemm(oracle, x, w, "e2m1", M, N, K, out_dtype=torch.bfloat16, rows=rows)
+    check(got, ref, bound, torch.bfloat16, (kernel, M, N, K))

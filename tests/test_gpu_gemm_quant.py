@@ -175,3 +175,24 @@ def test_gemm_quantize_k_zero_empty_and_shape():
     mx.gemm_quantize(z, z, z, z, 0, 64, 128, out_fmt="e4m3", out=(z, z))
     with pytest.raises(mx.MxError, match="MX_ERR_SHAPE"):
         mx.gemm_quantize(z, z, z, z, 4, 48, 128, out_fmt="e4m3", out=(codes, scales))
+
+
+@pytest.mark.parametrize("kernel", [0, 256, 192])
+@pytest.mark.parametrize("out_fmt", ["e4m3", "e2m1", "e3m2", "int8"])
+def test_gemm_quantize_each_kernel_bit_exact(oracle, kernel, out_fmt):
+    """The quantizing epilogue on every kernel (forced with
+    mx_debug_gemm_force_kernel), exact partial sums: codes and scales equal
+    the oracle's cast of the exact C, ragged M and several N tiles."""
+    M, N, K = 520, 640, 512
+    rng = np.random.default_rng(kernel + len(out_fmt))
+    a = np.clip(small_int_operand(rng, M, K), -3, 3)
+    b = np.clip(small_int_operand(rng, N, K), -3, 3)
+    ga, gb, oa, ob = operands(oracle, a, b, "e4m3", "e4m3")
+    c, _ = oracle_c(oracle, oa, ob, "e4m3", "e4m3", M, N, K, 0.25)
+    c32 = oracle.round_f32(c)
+    assert mx.lib().mx_debug_gemm_force_kernel(kernel) == 0
+    try:
+        got = gpu_gemm_quant(ga, gb, M, N, K, "e4m3", "e4m3", 0.25, out_fmt, "sr", 11, "mma")
+    finally:
+        mx.lib().mx_debug_gemm_force_kernel(-1)
+    assert_same(got, oracle_quant(oracle, c32, out_fmt, "sr", 11, "mma"), (kernel, out_fmt))
