@@ -17,14 +17,14 @@ pytestmark = pytest.mark.gpu
 MASK = mx.DEFAULT_SIGN_MASK
 
 
-def gpu_cast(x_np, axis, fmt, rnd="rne", seed=0, hadamard=False, sl="mma", ldx=None, cols=None):
+def gpu_cast(x_np, axis, fmt, rnd="rne", seed=0, hadamard=False, sl="mma", ldx=None, cols=None, sign_mask=MASK):
     x = to_device(x_np)
     if cols is not None:
         x = x[:, :cols]
     outer, inner = (x.shape[0], x.shape[1]) if axis == 1 else (x.shape[1], x.shape[0])
     codes = torch.full((outer, mx.codes_row_bytes(fmt, inner)), 0xAB, dtype=torch.uint8, device=dev())
     scales = torch.full((max(mx.scales_bytes(sl, outer, inner), 1),), 0xAB, dtype=torch.uint8, device=dev())
-    mx.quantize(x, axis, fmt, rnd=rnd, seed=seed, hadamard=hadamard, sign_mask=MASK,
+    mx.quantize(x, axis, fmt, rnd=rnd, seed=seed, hadamard=hadamard, sign_mask=sign_mask,
                 scale_layout=sl, codes=codes, scales=scales)
     torch.cuda.synchronize()
     return host(codes), host(scales)
@@ -321,12 +321,11 @@ def test_hadamard_any_sign_mask(oracle, mask, bf16):
     x = mixed_input(256, 96, 77, bf16)
     xd = to_device(x)
     for rnd in ("rne", "sr"):
-        codes, scales = mx.quantize(xd, 0, "e2m1", rnd=rnd, seed=3, hadamard=True, sign_mask=mask)
-        torch.cuda.synchronize()
+        got = gpu_cast(x, 0, "e2m1", rnd, seed=3, hadamard=True, sign_mask=mask, sl="plain")
         oc, os_ = oracle.quantize(x, 0, oracle.E2M1, rnd=1 if rnd == "sr" else 0, seed=3, hadamard=True,
-                                  sign_mask=mask, scale_layout=oracle.MMA)
-        assert np.array_equal(host(codes), oc), (hex(mask), rnd, first_mismatch(host(codes), oc))
-        assert np.array_equal(host(scales)[:os_.size], os_), (hex(mask), rnd)
-        _, _, cc, sc = mx.quantize_dual(xd, "e2m1", rnd_cols=rnd, seed_cols=3, hadamard=True, sign_mask=mask)
+                                  sign_mask=mask, scale_layout=oracle.PLAIN)
+        assert_same(got, (oc, os_), (hex(mask), rnd))
+        _, _, cc, sc = mx.quantize_dual(xd, "e2m1", rnd_cols=rnd, seed_cols=3, hadamard=True, sign_mask=mask,
+                                        scale_layout="plain")
         torch.cuda.synchronize()
-        assert np.array_equal(host(cc), oc) and np.array_equal(host(sc)[:os_.size], os_), (hex(mask), rnd)
+        assert np.array_equal(host(cc), oc) and np.array_equal(host(sc), os_), (hex(mask), rnd)

@@ -47,12 +47,15 @@ def test_shard_cast_parity(oracle, fmt, axis, hadamard):
     outer, inner = (R, C) if axis == 1 else (C, R)
     wc = ind.unpack_codes(fmt, host(whole_c), inner)
     ws = plain_scales(host(whole_s), outer, inner)
+    # cuts along the block axis fall on block boundaries; across it, rows are cut
+    # anywhere and columns on 8-column (16-byte) boundaries, the row-pitch rule
     row_cuts = [96, 224] if axis == 0 else [45, 200]
-    col_cuts = [64, 160] if axis == 1 else [33, 170]
+    col_cuts = [64, 160] if axis == 1 else [40, 168]
     for r0, r1 in pieces(R, row_cuts):
         for c0, c1 in pieces(C, col_cuts):
             piece = np.ascontiguousarray(x[r0:r1, c0:c1])
-            gc, gs = mx.quantize(xd[r0:r1, c0:c1], axis, fmt, rnd="sr", seed=99, hadamard=hadamard,
+            # each piece in its own (aligned) buffer, as a rank would hold it
+            gc, gs = mx.quantize(to_device(piece), axis, fmt, rnd="sr", seed=99, hadamard=hadamard,
                                  sign_mask=MASK, scale_layout="plain", shard=(r0, c0, R, C))
             torch.cuda.synchronize()
             oc, os_ = oracle.quantize(piece, axis, f, rnd=oracle.SR, seed=99, hadamard=hadamard, sign_mask=MASK,
@@ -69,20 +72,21 @@ def test_dual_shard_parity(oracle, fmt):
     rng = np.random.default_rng(3)
     R, C = 256, 320
     x = ind.f32_to_bf16_bits_rne(rng.standard_normal((R, C)).astype(np.float32))
-    xd = to_device(x)
     f = oracle.FORMATS[fmt]
     for r0, r1 in pieces(R, [64, 192]):
         for c0, c1 in pieces(C, [96]):
             piece = np.ascontiguousarray(x[r0:r1, c0:c1])
-            cr, sr_, cc, sc = mx.quantize_dual(xd[r0:r1, c0:c1], fmt, rnd_rows="sr", seed_rows=5, rnd_cols="sr",
-                                               seed_cols=6, hadamard=True, sign_mask=MASK, shard=(r0, c0, R, C))
+            # plain scale layout: the tensor-core layout pads these piece shapes, and
+            # padding bytes are never written
+            cr, sr_, cc, sc = mx.quantize_dual(to_device(piece), fmt, rnd_rows="sr", seed_rows=5, rnd_cols="sr",
+                                               seed_cols=6, hadamard=True, sign_mask=MASK, scale_layout="plain",
+                                               shard=(r0, c0, R, C))
             torch.cuda.synchronize()
-            ocr, osr = oracle.quantize(piece, 1, f, rnd=oracle.SR, seed=5, scale_layout=oracle.MMA,
-                                       shard=(r0, c0, R, C))
+            ocr, osr = oracle.quantize(piece, 1, f, rnd=oracle.SR, seed=5, shard=(r0, c0, R, C))
             occ, osc = oracle.quantize(piece, 0, f, rnd=oracle.SR, seed=6, hadamard=True, sign_mask=MASK,
-                                       scale_layout=oracle.MMA, shard=(r0, c0, R, C))
+                                       shard=(r0, c0, R, C))
             assert np.array_equal(host(cr), ocr) and np.array_equal(host(cc), occ), (r0, c0)
-            assert np.array_equal(host(sr_)[:osr.size], osr) and np.array_equal(host(sc)[:osc.size], osc)
+            assert np.array_equal(host(sr_), osr) and np.array_equal(host(sc), osc), (r0, c0)
 
 
 def test_wgrad_token_shards_reproduce_whole_cast():
