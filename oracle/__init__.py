@@ -92,6 +92,13 @@ def lib() -> ctypes.CDLL:
                                                ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
                                                ctypes.c_int, ctypes.c_uint32, _i64, _i64, _i64, _i64,
                                                _vp, _vp, ctypes.c_int]
+            L.mxref_nvfp4_scales_bytes.restype = _i64
+            L.mxref_nvfp4_scales_bytes.argtypes = [ctypes.c_int, _i64, _i64]
+            L.mxref_nvfp4_quantize.restype = ctypes.c_int
+            L.mxref_nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i64, _i64, _vp, _vp,
+                                               ctypes.c_int, _vp]
+            L.mxref_nvfp4_dequantize.restype = ctypes.c_int
+            L.mxref_nvfp4_dequantize.argtypes = [_vp, _vp, ctypes.c_int, _i64, _i64, _vp, _i64, _vp]
             L.mxref_dequantize.restype = ctypes.c_int
             L.mxref_dequantize.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _i64, _i64, _vp]
             L.mxref_round_f32.restype = None
@@ -292,3 +299,59 @@ def gemm_decoded(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha=1.
     c = alpha * (A @ B.T)
     bound = abs(alpha) * (np.abs(A) @ np.abs(B).T)
     return c, bound
+
+
+# --------------------------------------------------------------------------
+# NVFP4 scale domains (reading; see mx_oracle.c): 16-element E2M1 blocks with
+# an E4M3 block scale and one fp32 encode scale per domain.
+# --------------------------------------------------------------------------
+
+NV_SCALE_NAN = 0x7F
+
+
+def nvfp4_scales_bytes(sl: int, rows: int, cols: int) -> int:
+    return lib().mxref_nvfp4_scales_bytes(sl, rows, cols)
+
+
+def nvfp4_quantize(x: np.ndarray, domain_lines: int = 0, scale_layout: int = PLAIN, fill: int = 0):
+    """Cast a rows x cols float32 array (or bf16 bits as uint16) along its rows
+    to NVFP4.  domain_lines 0: one global domain; else one domain per that many
+    rows.  Returns (codes, scales, enc_scales)."""
+    if x.dtype == np.float32:
+        xdt = F32
+    elif x.dtype == np.uint16:
+        xdt = BF16
+    else:
+        raise TypeError("x must be float32 or bf16 bits (uint16)")
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    n_dom = 1 if domain_lines == 0 else (rows + domain_lines - 1) // domain_lines
+    codes = np.full((rows, cols // 2), fill, dtype=np.uint8)
+    scales = np.full(max(nvfp4_scales_bytes(scale_layout, rows, cols), 0), fill, dtype=np.uint8)
+    enc = np.zeros(max(n_dom, 1), dtype=np.float32)
+    rc = lib().mxref_nvfp4_quantize(_ptr(x), xdt, rows, cols, cols, domain_lines, _ptr(codes), _ptr(scales),
+                                    scale_layout, _ptr(enc))
+    _check(rc, "mxref_nvfp4_quantize")
+    return codes, scales, enc
+
+
+def nvfp4_dequantize(codes, scales, enc_scales, rows: int, cols: int, domain_lines: int = 0,
+                     scale_layout: int = PLAIN) -> np.ndarray:
+    y = np.empty((rows, cols), dtype=np.float64)
+    rc = lib().mxref_nvfp4_dequantize(_ptr(np.ascontiguousarray(codes)), _ptr(np.ascontiguousarray(scales)),
+                                      scale_layout, rows, cols,
+                                      _ptr(np.ascontiguousarray(enc_scales, dtype=np.float32)),
+                                      domain_lines, _ptr(y))
+    _check(rc, "mxref_nvfp4_dequantize")
+    return y
+
+
+def nvfp4_gemm_decoded(a, b, M, N, K, alpha=1.0, a_lines=0, b_lines=0, scale_layout: int = MMA, rows=None):
+    """C = alpha * A * B^T on NVFP4 operands a = (codes, scales, enc) (M x K)
+    and b (N x K), both cast along K: exact decode, numpy fp64 matrix product.
+    Returns (C, bound) with bound = |alpha| * sum_k |a b|."""
+    A = nvfp4_dequantize(a[0], a[1], a[2], M, K, a_lines, scale_layout)
+    B = nvfp4_dequantize(b[0], b[1], b[2], N, K, b_lines, scale_layout)
+    if rows is not None:
+        A = A[np.asarray(rows)]
+    return alpha * (A @ B.T), abs(alpha) * (np.abs(A) @ np.abs(B).T)

@@ -589,3 +589,125 @@ int mxref_gemm_entries(const uint8_t *a_codes, const uint8_t *a_scales, int fa,
                    &c[i], &bound[i]);
     return MXO_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 scale domains (reading of "global NVFP4" and "cooperative-thread-  */
+/* array-local NVFP4", FP4 pretraining abstract; the pages name these       */
+/* domains but do not define them, so this follows the public NVFP4         */
+/* format):                                                                 */
+/*  - blocks of 16 consecutive elements along the block axis (rows, here);   */
+/*    elements E2M1; one E4M3 block scale (positive; 0x7F, the E4M3 NaN     */
+/*    code, marks a block holding a NaN or Inf, whose codes are then 0);     */
+/*  - one fp32 encode scale E per domain: the whole tensor ("global"), or    */
+/*    each group of domain_lines consecutive rows ("CTA-local": the rows one */
+/*    CTA of the cast owns, all of the block axis);                          */
+/*  - every step in fp32 IEEE arithmetic (round to nearest even, no fused    */
+/*    multiply-add, no flush): a_D = largest finite |x| of the domain,       */
+/*    E = 2688 / a_D (6 * 448: the largest E2M1 and E4M3 values; 1 when      */
+/*    a_D = 0, the largest finite fp32 when the quotient overflows); per     */
+/*    block a_b = largest |x|, block scale s = E4M3(RNE, saturating) of      */
+/*    (a_b / 6) * E, d its value, r = E / d (0 when d = 0), and each code    */
+/*    E2M1(RNE, saturating) of x * r;                                        */
+/*  - the value of a code P in a block with scale value d is P * d / E.      */
+/* ------------------------------------------------------------------------ */
+#define NV_BLOCK 16
+#define NV_SCALE_NAN 0x7Fu
+
+static float nv_encode_scale(float amax)
+{
+    if (!(amax > 0.0f)) return 1.0f;
+    float e = 2688.0f / amax;
+    if (isinf(e)) e = 3.40282346638528859812e+38f;      /* largest finite fp32 */
+    return e;
+}
+
+int64_t mxref_nvfp4_scales_bytes(int sl, int64_t rows, int64_t cols)
+{
+    /* one byte per 16-block; the MMA layout is the MX atom layout over 16-blocks */
+    return mxref_scales_bytes(sl, rows, cols * 2);
+}
+
+/* Cast along rows (block axis 1).  domain_lines 0: one global domain, else
+ * rows are grouped domain_lines at a time.  codes: rows x cols/2 bytes (E2M1,
+ * even element in the low nibble); scales: plain rows x cols/16 or the MMA
+ * atom layout; enc_scales: one fp32 per domain. */
+int mxref_nvfp4_quantize(const void *x, int xdt, int64_t rows, int64_t cols, int64_t ldx,
+                         int64_t domain_lines, uint8_t *codes, uint8_t *scales, int sl, float *enc_scales)
+{
+    build_tables();
+    if (!x || !codes || !scales || !enc_scales) return MXO_ERR_ARG;
+    if ((xdt != DT_F32 && xdt != DT_BF16) || rows < 0 || cols < 0 || ldx < cols || domain_lines < 0)
+        return MXO_ERR_ARG;
+    if (cols % NV_BLOCK != 0) return MXO_ERR_SHAPE;
+    const int64_t lines = domain_lines == 0 ? (rows > 0 ? rows : 1) : domain_lines;
+    const int64_t n_dom = (rows + lines - 1) / lines;
+    const int64_t kb_total = cols / NV_BLOCK;
+    const int64_t row_bytes = cols / 2;
+
+    for (int64_t d = 0; d < n_dom; ++d) {
+        float amax = 0.0f;
+        for (int64_t r = d * lines; r < rows && r < (d + 1) * lines; ++r)
+            for (int64_t c = 0; c < cols; ++c) {
+                float v = load_elem(x, xdt, r * ldx + c);
+                if (isfinite(v) && fabsf(v) > amax) amax = fabsf(v);
+            }
+        enc_scales[d] = nv_encode_scale(amax);
+    }
+
+    #pragma omp parallel for schedule(static)
+    for (int64_t o = 0; o < rows; ++o) {
+        const float E = enc_scales[o / lines];
+        uint8_t *crow = codes + o * row_bytes;
+        for (int64_t kb = 0; kb < kb_total; ++kb) {
+            float v[NV_BLOCK];
+            int finite = 1;
+            float amax = 0.0f;
+            for (int j = 0; j < NV_BLOCK; ++j) {
+                v[j] = load_elem(x, xdt, o * ldx + kb * NV_BLOCK + j);
+                if (!isfinite(v[j])) finite = 0;
+                else if (fabsf(v[j]) > amax) amax = fabsf(v[j]);
+            }
+            unsigned s;
+            if (!finite) {
+                s = NV_SCALE_NAN;
+                for (int j = 0; j < NV_BLOCK; ++j) put_code(FMT_E2M1, crow, kb * NV_BLOCK + j, 0);
+            } else {
+                float t = (amax / 6.0f) * E;
+                s = mxref_encode_rne(FMT_E4M3, (double)t);      /* t >= 0: a positive code */
+                float dval = (float)mxref_decode_elem(FMT_E4M3, s);
+                float r = dval > 0.0f ? E / dval : 0.0f;
+                for (int j = 0; j < NV_BLOCK; ++j) {
+                    float u = v[j] * r;
+                    put_code(FMT_E2M1, crow, kb * NV_BLOCK + j, mxref_encode_rne(FMT_E2M1, (double)u));
+                }
+            }
+            scales[scale_offset(sl, o, kb, kb_total)] = (uint8_t)s;
+        }
+    }
+    return MXO_OK;
+}
+
+/* Decode: P * d / E in double (P * d is exact; the one division rounds); a
+ * 0x7F block scale gives NaN for its block. */
+int mxref_nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, int sl, int64_t rows, int64_t cols,
+                           const float *enc_scales, int64_t domain_lines, double *y)
+{
+    build_tables();
+    if (!codes || !scales || !enc_scales || !y || domain_lines < 0) return MXO_ERR_ARG;
+    if (cols % NV_BLOCK != 0) return MXO_ERR_SHAPE;
+    const int64_t lines = domain_lines == 0 ? (rows > 0 ? rows : 1) : domain_lines;
+    const int64_t kb_total = cols / NV_BLOCK;
+    for (int64_t o = 0; o < rows; ++o) {
+        const double E = (double)enc_scales[o / lines];
+        const uint8_t *crow = codes + o * (cols / 2);
+        for (int64_t kb = 0; kb < kb_total; ++kb) {
+            unsigned s = scales[scale_offset(sl, o, kb, kb_total)];
+            double dval = s == NV_SCALE_NAN ? NAN : mxref_decode_elem(FMT_E4M3, s);
+            for (int j = 0; j < NV_BLOCK; ++j) {
+                double p = mxref_decode_elem(FMT_E2M1, mxref_get_code(FMT_E2M1, crow, kb * NV_BLOCK + j));
+                y[o * cols + kb * NV_BLOCK + j] = (p * dval) / E;
+            }
+        }
+    }
+    return MXO_OK;
+}
