@@ -228,6 +228,48 @@ MX_API int mx_quantize_dual_shard(const void *x, mx_dtype xdt, int64_t rows, int
                                   mx_scale_layout sl, void *stream);
 
 /*
+ * mx_quantize_nvfp4 -- the NVFP4 cast with a global or a CTA-local scale
+ * domain, the two NVFP4 variants the abstract of "Format-Aware Fusion for
+ * Fast FP4 Pretraining" names next to native MXFP4.  The pages do not define
+ * them; the reading taken here is the public NVFP4 format:
+ *  - blocks of 16 consecutive elements along the rows (block axis 1), E2M1
+ *    elements (the MXFP4 codes), one E4M3 block scale per block;
+ *  - one fp32 encode scale E per domain: the whole tensor (domain_rows = 0,
+ *    "global"), or each group of domain_rows consecutive rows, all columns
+ *    ("CTA-local": the rows one CTA of this cast owns; 32 matches the rows
+ *    one epilogue thread of the GEMM covers);
+ *  - with a_D the largest finite |x| of a domain, E = 2688 / a_D (6 * 448, the
+ *    largest E2M1 and E4M3 values; 1 when a_D = 0, the largest finite fp32
+ *    when the quotient overflows); per block, with a_b its largest |x|, the
+ *    block scale is the E4M3 code of (a_b / 6) * E (round to nearest even,
+ *    saturating at 448), d its value, and each code the E2M1 code of
+ *    x * (E / d) (nearest even, saturating at 6; 0 when d = 0); every step one
+ *    IEEE fp32 operation, no flush.  A block holding a NaN or Inf gets the
+ *    E4M3 NaN code 0x7F and zero codes;
+ *  - a code P in a block of scale value d stands for P * d / E.
+ *
+ *  x          device, rows x cols (ldx elements per row), fp32 or bf16,
+ *             16-byte aligned, ldx * sizeof(elem) a multiple of 16.
+ *  cols       a multiple of 16 (MX_ERR_SHAPE).
+ *  codes      device, rows x cols / 2 bytes (two codes per byte, even element
+ *             in the low nibble), 16-byte aligned.
+ *  scales     device, mx_nvfp4_scales_bytes(sl, rows, cols) bytes: plain
+ *             (rows x cols / 16) or the tensor-core atom layout of
+ *             MX_SCALES_MMA over 16-element blocks.
+ *  enc_scales device, mx_nvfp4_domains(rows, domain_rows) fp32 values: E of
+ *             each domain (written; the global form also uses it while it
+ *             runs, starting from zero).
+ * Errors: MX_ERR_ARG, MX_ERR_ALIGN, MX_ERR_SHAPE, MX_ERR_UNSUPPORTED,
+ * MX_ERR_CUDA.
+ */
+MX_API int mx_quantize_nvfp4(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                             int64_t domain_rows, void *codes, void *scales, mx_scale_layout sl,
+                             float *enc_scales, void *stream);
+/* Byte size of mx_quantize_nvfp4's scales, and its number of domains. */
+MX_API size_t mx_nvfp4_scales_bytes(mx_scale_layout sl, int64_t rows, int64_t cols);
+MX_API int64_t mx_nvfp4_domains(int64_t rows, int64_t domain_rows);
+
+/*
  * mx_dequantize -- v = X * P (section 2), exact, rounded once to ydt.
  *
  *  codes, scales  device, as written by mx_quantize for (outer, inner).

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmx.so")
-SOURCES = ["mx_api.cu", "mx_cast.cu", "mx_gemm.cu"]
+SOURCES = ["mx_api.cu", "mx_cast.cu", "mx_gemm.cu", "mx_nvfp4.cu"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

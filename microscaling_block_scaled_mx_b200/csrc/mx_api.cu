@@ -226,6 +226,37 @@ int mx_quantize_dual_shard(const void *x, mx_dtype xdt, int64_t rows, int64_t co
                               shard, codes_rows, scales_rows, codes_cols, scales_cols, sl, stream);
 }
 
+size_t mx_nvfp4_scales_bytes(mx_scale_layout sl, int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return 0;
+    return mx_scales_bytes(sl, rows, 2 * cols);       // one byte per 16-block, the same atoms
+}
+
+int64_t mx_nvfp4_domains(int64_t rows, int64_t domain_rows) {
+    if (rows < 0 || domain_rows < 0) return 0;
+    if (domain_rows == 0) return 1;
+    return (rows + domain_rows - 1) / domain_rows;
+}
+
+int mx_quantize_nvfp4(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, int64_t domain_rows,
+                      void *codes, void *scales, mx_scale_layout sl, float *enc_scales, void *stream) {
+    if (xdt != MX_F32 && xdt != MX_BF16) return MX_ERR_ARG;
+    if (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA) return MX_ERR_ARG;
+    if (rows < 0 || cols < 0 || domain_rows < 0) return MX_ERR_ARG;
+    if (cols % 16 != 0) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;             // empty: pointers may be NULL
+    if (!x || !codes || !scales || !enc_scales || ldx < cols) return MX_ERR_ARG;
+    if (!aligned16(x) || (ldx * dtype_bytes(xdt)) % 16 != 0 || !aligned16(codes) ||
+        (reinterpret_cast<uintptr_t>(enc_scales) & 3u) != 0)
+        return MX_ERR_ALIGN;
+    if (mx_nvfp4_scales_bytes(sl, rows, cols) >= (1ull << 32)) return MX_ERR_UNSUPPORTED;
+    MxNvfp4Args a;
+    a.x = x; a.xdt = xdt; a.rows = rows; a.cols = cols; a.ldx = ldx; a.domain_rows = domain_rows;
+    a.codes = codes; a.scales = scales; a.sl = sl; a.enc_scales = enc_scales;
+    a.num_sms = sm_count(nullptr);
+    if (a.num_sms <= 0) return MX_ERR_CUDA;
+    return mx_launch_quantize_nvfp4(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
 int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_scale_layout sl,
                   int64_t outer, int64_t inner, void *y, mx_dtype ydt, int64_t ldy, void *stream) {
     if (elem_bits(fmt) == 0 || (ydt != MX_F32 && ydt != MX_BF16)) return MX_ERR_ARG;

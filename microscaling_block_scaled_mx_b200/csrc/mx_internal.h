@@ -42,6 +42,18 @@ struct MxQuantizeDualArgs {
     uint64_t sr_base_rows, sr_stride_rows, sr_base_cols, sr_stride_cols;
 };
 
+struct MxNvfp4Args {
+    const void *x;
+    int xdt;
+    int64_t rows, cols, ldx;
+    int64_t domain_rows;       // 0: one global domain
+    void *codes;
+    void *scales;
+    int sl;
+    float *enc_scales;
+    int num_sms;
+};
+
 struct MxDequantArgs {
     const void *codes;
     const void *scales;
@@ -83,6 +95,7 @@ inline uint32_t fmix32_host(uint32_t h) {
 cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st);
 cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st);
 cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st);
+cudaError_t mx_launch_quantize_nvfp4(const MxNvfp4Args &a, cudaStream_t st);
 // returns an mx_status (MX_OK, MX_ERR_CUDA, MX_ERR_UNSUPPORTED)
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st);
 // reads and clears the device status word of the current device (after a sync)

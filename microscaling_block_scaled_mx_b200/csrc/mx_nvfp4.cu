@@ -1,0 +1,255 @@
+// mx_nvfp4.cu -- the NVFP4 cast: 16-element E2M1 blocks with an E4M3 block
+// scale and one fp32 encode scale per scale domain, the "global NVFP4" and
+// "cooperative-thread-array-local NVFP4" domains named by the abstract of
+// "Format-Aware Fusion for Fast FP4 Pretraining".  The pages do not define
+// them; the reading taken (the public NVFP4 format) is stated in include/mx.h
+// at mx_quantize_nvfp4.
+//
+// Kernels (blocks along rows, the K axis of a GEMM operand):
+//   global domain      nv_amax_kernel   largest finite |x| of the tensor, an
+//                                       atomic max into enc_scales[0] (as bits)
+//                      nv_quant_kernel  every block, E from that maximum
+//                      nv_final_kernel  enc_scales[0] <- E
+//   CTA-local domains  nv_local_kernel  one CTA per domain of domain_rows rows:
+//                                       its maximum (CTA reduction), E, then
+//                                       its blocks (the second read is served
+//                                       by L2)
+// Every step is one IEEE fp32 operation (no fused multiply-add, no flush), in
+// the order the reading states, so results equal the CPU reference bit for
+// bit.
+#include <algorithm>
+#include <cfloat>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "mx.h"
+#include "mx_device.cuh"
+#include "mx_internal.h"
+
+namespace mxnv {
+
+constexpr int NV_BLOCK = 16;
+constexpr uint32_t NV_SCALE_NAN = 0x7Fu;
+constexpr int THREADS = 256;
+
+struct NvParams {
+    const void *x;
+    int64_t rows, cols, ldx;
+    uint8_t *codes;
+    uint8_t *scales;
+    int mma;               // MMA scale layout (else plain)
+    uint32_t k_blocks;     // cols / 16
+    uint32_t k_groups;     // ceil(k_blocks / 4)
+    float *enc;            // one fp32 per domain
+    int64_t lines;         // rows per domain
+};
+
+__device__ __forceinline__ float encode_scale(float amax) {
+    if (!(amax > 0.0f)) return 1.0f;
+    float e = __fdiv_rn(2688.0f, amax);
+    if (isinf(e)) e = FLT_MAX;
+    return e;
+}
+
+// value of a positive E4M3 code (sign bit clear, not 0x7F)
+__device__ __forceinline__ float e4m3_value(uint32_t s) {
+    const uint32_t e = (s >> 3) & 15u, m = s & 7u;
+    return e == 0 ? static_cast<float>(m) * 0.001953125f                                   // m * 2^-9
+                  : __uint_as_float(((e + 120u) << 23) | (m << 20));                       // (1 + m/8) 2^(e-7)
+}
+
+// the 16 values of block kb of row `row`, widened to fp32
+template <bool BF16_IN>
+__device__ __forceinline__ void load_block(const NvParams &p, int64_t row, int64_t kb, float (&v)[NV_BLOCK]) {
+    if (BF16_IN) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.x) + row * p.ldx + kb * 16);
+        const uint4 a = __ldcs(src), b = __ldcs(src + 1);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    } else {
+        const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(p.x) + row * p.ldx + kb * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 f = __ldcs(src + i);
+            v[4 * i] = f.x;
+            v[4 * i + 1] = f.y;
+            v[4 * i + 2] = f.z;
+            v[4 * i + 3] = f.w;
+        }
+    }
+}
+
+// largest finite magnitude; `finite` false when a NaN or Inf is present
+__device__ __forceinline__ float block_max(const float (&v)[NV_BLOCK], bool &finite) {
+    float m = 0.0f;
+    finite = true;
+#pragma unroll
+    for (int i = 0; i < NV_BLOCK; ++i) {
+        const float a = fabsf(v[i]);
+        if (!(a <= FLT_MAX)) finite = false;
+        else m = fmaxf(m, a);
+    }
+    return m;
+}
+
+template <bool BF16_IN>
+__device__ __forceinline__ void quant_block(const NvParams &p, int64_t row, int64_t kb, float E) {
+    float v[NV_BLOCK];
+    load_block<BF16_IN>(p, row, kb, v);
+    bool finite;
+    const float amax = block_max(v, finite);
+    uint32_t s = NV_SCALE_NAN;
+    uint2 c = make_uint2(0u, 0u);
+    if (finite) {
+        const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), E);
+        s = mxk::cvt_pair<MX_E4M3>(t, 0.0f) & 0xffu;          // t >= 0: a positive code
+        const float d = e4m3_value(s);
+        const float r = d > 0.0f ? __fdiv_rn(E, d) : 0.0f;
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < NV_BLOCK; i += 2) {
+            const uint32_t byte = mxk::cvt_pair<MX_E2M1>(__fmul_rn(v[i], r), __fmul_rn(v[i + 1], r));
+            w[i >> 3] |= byte << (4 * (i & 7));
+        }
+        c = make_uint2(w[0], w[1]);
+    }
+    *reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + kb * 8) = c;
+    const uint32_t off = p.mma ? mxk::mma_scale_offset32(static_cast<uint32_t>(row), static_cast<uint32_t>(kb),
+                                                         p.k_groups)
+                               : static_cast<uint32_t>(row) * p.k_blocks + static_cast<uint32_t>(kb);
+    p.scales[off] = static_cast<uint8_t>(s);
+}
+
+// largest value over the CTA (every thread gets it)
+__device__ __forceinline__ float cta_max(float m, float *red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (warp == 0) {
+        m = lane < THREADS / 32 ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) red[0] = m;
+    }
+    __syncthreads();
+    m = red[0];
+    __syncthreads();
+    return m;
+}
+
+template <bool BF16_IN>
+__global__ void __launch_bounds__(THREADS) nv_amax_kernel(NvParams p) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float red[THREADS / 32];
+    const int64_t n = p.rows * static_cast<int64_t>(p.k_blocks);
+    float m = 0.0f;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(THREADS) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * THREADS) {
+        float v[NV_BLOCK];
+        load_block<BF16_IN>(p, i / p.k_blocks, i % p.k_blocks, v);
+        bool finite;
+        m = fmaxf(m, block_max(v, finite));
+    }
+    m = cta_max(m, red);
+    // non-negative floats order as their bit patterns
+    if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int *>(p.enc), __float_as_uint(m));
+}
+
+template <bool BF16_IN>
+__global__ void __launch_bounds__(THREADS) nv_quant_kernel(NvParams p) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const float E = encode_scale(p.enc[0]);              // enc[0] holds the tensor's maximum here
+    const int64_t n = p.rows * static_cast<int64_t>(p.k_blocks);
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(THREADS) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * THREADS)
+        quant_block<BF16_IN>(p, i / p.k_blocks, i % p.k_blocks, E);
+}
+
+__global__ void nv_final_kernel(float *enc) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (blockIdx.x == 0 && threadIdx.x == 0) enc[0] = encode_scale(enc[0]);
+}
+
+template <bool BF16_IN>
+__global__ void __launch_bounds__(THREADS) nv_local_kernel(NvParams p, int64_t n_dom) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float red[THREADS / 32];
+    for (int64_t d = blockIdx.x; d < n_dom; d += gridDim.x) {
+        const int64_t r0 = d * p.lines;
+        const int64_t nr = min(p.lines, p.rows - r0);
+        const int64_t n = nr * static_cast<int64_t>(p.k_blocks);
+        float m = 0.0f;
+        for (int64_t i = threadIdx.x; i < n; i += THREADS) {
+            float v[NV_BLOCK];
+            load_block<BF16_IN>(p, r0 + i / p.k_blocks, i % p.k_blocks, v);
+            bool finite;
+            m = fmaxf(m, block_max(v, finite));
+        }
+        const float E = encode_scale(cta_max(m, red));
+        if (threadIdx.x == 0) p.enc[d] = E;
+        for (int64_t i = threadIdx.x; i < n; i += THREADS)
+            quant_block<BF16_IN>(p, r0 + i / p.k_blocks, i % p.k_blocks, E);
+    }
+}
+
+template <auto Kernel, typename... Args>
+cudaError_t launch(int grid, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, Kernel, args...);
+}
+
+template <bool BF16_IN>
+cudaError_t run(const NvParams &p, int64_t domain_rows, int sms, cudaStream_t st) {
+    const int64_t blocks = p.rows * static_cast<int64_t>(p.k_blocks);
+    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    if (domain_rows == 0) {
+        // the maximum accumulates in enc_scales[0], which starts at zero
+        cudaError_t e = cudaMemsetAsync(p.enc, 0, sizeof(float), st);
+        if (e != cudaSuccess) return e;
+        int grid = static_cast<int>(std::min<int64_t>((blocks + THREADS - 1) / THREADS, cap));
+        if (grid < 1) grid = 1;
+        if ((e = launch<nv_amax_kernel<BF16_IN>>(grid, st, p)) != cudaSuccess) return e;
+        if ((e = launch<nv_quant_kernel<BF16_IN>>(grid, st, p)) != cudaSuccess) return e;
+        return launch<nv_final_kernel>(1, st, p.enc);
+    }
+    const int64_t n_dom = (p.rows + domain_rows - 1) / domain_rows;
+    const int grid = static_cast<int>(std::min<int64_t>(n_dom, cap));
+    return launch<nv_local_kernel<BF16_IN>>(grid < 1 ? 1 : grid, st, p, n_dom);
+}
+
+}  // namespace mxnv
+
+cudaError_t mx_launch_quantize_nvfp4(const MxNvfp4Args &a, cudaStream_t st) {
+    using namespace mxnv;
+    NvParams p;
+    p.x = a.x;
+    p.rows = a.rows;
+    p.cols = a.cols;
+    p.ldx = a.ldx;
+    p.codes = static_cast<uint8_t *>(a.codes);
+    p.scales = static_cast<uint8_t *>(a.scales);
+    p.mma = a.sl == MX_SCALES_MMA;
+    p.k_blocks = static_cast<uint32_t>(a.cols / NV_BLOCK);
+    p.k_groups = (p.k_blocks + 3) / 4;
+    p.enc = a.enc_scales;
+    p.lines = a.domain_rows == 0 ? a.rows : a.domain_rows;
+    return a.xdt == MX_BF16 ? run<true>(p, a.domain_rows, a.num_sms, st) : run<false>(p, a.domain_rows, a.num_sms, st);
+}

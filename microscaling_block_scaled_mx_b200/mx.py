@@ -76,6 +76,12 @@ def lib() -> ctypes.CDLL:
             L.mx_quantize_dual.restype = i32
             L.mx_quantize_dual.argtypes = [vp, i32, i64, i64, i64, i32, i32, u64, i32, u64,
                                            ctypes.POINTER(_Precond), vp, vp, vp, vp, i32, vp]
+            L.mx_quantize_nvfp4.restype = i32
+            L.mx_quantize_nvfp4.argtypes = [vp, i32, i64, i64, i64, i64, vp, vp, i32, vp, vp]
+            L.mx_nvfp4_scales_bytes.restype = ctypes.c_size_t
+            L.mx_nvfp4_scales_bytes.argtypes = [i32, i64, i64]
+            L.mx_nvfp4_domains.restype = i64
+            L.mx_nvfp4_domains.argtypes = [i64, i64]
             L.mx_dequantize.restype = i32
             L.mx_dequantize.argtypes = [vp, vp, i32, i32, i64, i64, vp, i32, i64, vp]
             L.mx_gemm.restype = i32
@@ -219,6 +225,29 @@ def quantize_dual(x: torch.Tensor, fmt="e4m3", rnd_rows="rne", seed_rows: int = 
                                           sl, _stream(stream))
         _check(rc, "mx_quantize_dual_shard")
     return cr, sr_, cc, sc
+
+
+def quantize_nvfp4(x: torch.Tensor, domain_rows: int = 0, scale_layout="mma", out=None, stream=None):
+    """NVFP4 cast of a 2-D CUDA tensor along its rows (mx_quantize_nvfp4):
+    domain_rows 0 for one global scale domain, else rows per CTA-local domain.
+    Returns (codes, scales, enc_scales)."""
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    if x.dtype not in DTYPE:
+        raise TypeError("x must be float32 or bfloat16")
+    rows, cols = x.shape
+    sl = _layout(scale_layout)
+    if out is None:
+        u8 = dict(dtype=torch.uint8, device=x.device)
+        out = (torch.empty((rows, cols // 2), **u8),
+               torch.empty(max(lib().mx_nvfp4_scales_bytes(sl, rows, cols), 1), **u8),
+               torch.empty(max(lib().mx_nvfp4_domains(rows, domain_rows), 1), dtype=torch.float32,
+                           device=x.device))
+    codes, scales, enc = out
+    rc = lib().mx_quantize_nvfp4(x.data_ptr(), DTYPE[x.dtype], rows, cols, x.stride(0), domain_rows,
+                                 codes.data_ptr(), scales.data_ptr(), sl, enc.data_ptr(), _stream(stream))
+    _check(rc, "mx_quantize_nvfp4")
+    return codes, scales, enc
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, fmt, outer: int, inner: int,

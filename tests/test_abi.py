@@ -217,3 +217,17 @@ def test_shard_validation(mx):
     assert d((16, 0, 128, 64)) == -3                    # both axes are block axes in the dual cast
     assert d((0, 16, 64, 128)) == -3
     assert d((96, 0, 128, 64)) == -1
+
+
+def test_nvfp4_validation(mx):
+    """Host-side checks of mx_quantize_nvfp4 (nothing is launched)."""
+    L = mx.lib()
+    assert L.mx_quantize_nvfp4(16, 1, 64, 40, 64, 0, 16, 16, 1, 16, None) == -3     # cols % 16
+    assert L.mx_quantize_nvfp4(16, 1, 64, 64, 64, -1, 16, 16, 1, 16, None) == -1    # domain_rows
+    assert L.mx_quantize_nvfp4(16, 3, 64, 64, 64, 0, 16, 16, 1, 16, None) == -1     # dtype
+    assert L.mx_quantize_nvfp4(24, 1, 64, 64, 64, 0, 16, 16, 1, 16, None) == -2     # x alignment
+    assert L.mx_quantize_nvfp4(16, 1, 64, 64, 64, 0, 16, 16, 1, 18, None) == -2     # enc alignment
+    assert L.mx_quantize_nvfp4(16, 1, 0, 64, 64, 0, None, None, 1, None, None) == 0  # empty
+    assert L.mx_nvfp4_domains(100, 32) == 4 and L.mx_nvfp4_domains(100, 0) == 1
+    assert L.mx_nvfp4_scales_bytes(0, 100, 64) == 400
+    assert L.mx_nvfp4_scales_bytes(1, 100, 64) == 128 * 4
