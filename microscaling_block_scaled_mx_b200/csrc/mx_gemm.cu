@@ -19,6 +19,12 @@
 //               to fp32 / bf16, written to a per-warp shared-memory piece of
 //               32 rows x 64 bytes and stored to C by one TMA store per piece
 //               (the copy engine clips the ragged edges of C).
+// A tcgen05.cp costs tensor-pipe time per instruction, nearly whatever its
+// size: the scale copies take about a fifth of the MXFP4 pair kernel's time.
+// Fewer, wider copies (128x256b from atoms replicated four times in shared
+// memory) measured slower end to end, as did writing the scale factors with
+// tcgen05.st from the epilogue warps: both need a per-stage handshake that
+// costs more than the copies.
 // A 192-column tile starts 64 rows into a 128-row scale atom on odd tiles;
 // the B scale-factor TMEM address then starts two columns later.
 // Every mbarrier wait is bounded; on expiry the kernel records MX_ERR_TIMEOUT
@@ -326,16 +332,40 @@ __device__ __forceinline__ void quantize_chunk(const Params &p, int m, int n0, c
 // C with one TMA store.  The buffers use the copy engine's 64-byte swizzle
 // (16-byte granule g of row r sits at granule g ^ ((r >> 1) & 3)), so the
 // lanes' 16-byte writes spread over all banks.  The tensor map clips rows
-// >= M and columns >= N.
+// >= M exactly, but along a row the copy engine writes whole 16-byte units,
+// so the one piece of a row of tiles that reaches past column N is written
+// with bounds-checked plain stores instead.
 struct EpiWriter {
     const CUtensorMap *map;
     uint32_t buf;      // this warp's two pieces (1024-byte aligned)
     int count;         // pieces issued so far (selects the buffer)
     int lane;
+    void *c;           // C and its shape, for the piece at the right edge
+    int64_t ldc;
+    int M, N;
 };
 // vals: 32 accumulator words (bf16 output) or 16 (fp32 output) of this lane's row
 template <int OUT>
 __device__ __forceinline__ void epi_piece(EpiWriter &w, const uint32_t *vals, float alpha, int x, int y) {
+    constexpr int PC = OUT == OUT_BF16 ? 32 : 16;   // columns per piece
+    if (x + PC > w.N) {
+        // right edge of C: plain stores of the columns that exist, rows < M
+        const int m = y + w.lane;
+        if (m < w.M) {
+            if constexpr (OUT == OUT_BF16) {
+                __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(w.c) + static_cast<int64_t>(m) * w.ldc + x;
+#pragma unroll
+                for (int i = 0; i < PC; ++i)
+                    if (x + i < w.N) row[i] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(vals[i]), alpha));
+            } else {
+                float *row = static_cast<float *>(w.c) + static_cast<int64_t>(m) * w.ldc + x;
+#pragma unroll
+                for (int i = 0; i < PC; ++i)
+                    if (x + i < w.N) row[i] = __fmul_rn(__uint_as_float(vals[i]), alpha);
+            }
+        }
+        return;
+    }
     const uint32_t b = w.buf + static_cast<uint32_t>(w.count & 1) * EPI_PIECE;
     if (w.lane == 0) bulk_wait_read<1>();       // this buffer's previous store has read it
     __syncwarp();
@@ -532,7 +562,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         // ------------------------------ epilogue ------------------------------
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
         const int half = (warp - 2) >> 2;        // which 96 columns of the tile
-        EpiWriter ew{&tma_c, sbase + Smem::EPI + static_cast<uint32_t>(warp - 2) * EPI_WARP_BYTES, 0, lane};
+        EpiWriter ew{&tma_c, sbase + Smem::EPI + static_cast<uint32_t>(warp - 2) * EPI_WARP_BYTES, 0, lane,
+                     p.c, p.ldc, p.M, p.N};
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int b = local & 1;
@@ -858,7 +889,8 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
         // ------------------------------ epilogue (both CTAs) -------------------
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
-        EpiWriter ew{&tma_c, sbase + C::OFF_EPI + static_cast<uint32_t>(warp - 2) * EPI_WARP_BYTES, 0, lane};
+        EpiWriter ew{&tma_c, sbase + C::OFF_EPI + static_cast<uint32_t>(warp - 2) * EPI_WARP_BYTES, 0, lane,
+                     p.c, p.ldc, p.M, p.N};
         int local = 0;
         constexpr int NCH = PBN / 2 / 32;        // 32-column chunks per warp
         for (int tile = cluster_id; tile < num_tiles; tile += n_clusters, ++local) {

@@ -24,8 +24,8 @@ def special_input(rows, cols, seed, bf16):
     sub = rng.choice(flat.size, flat.size // 200, replace=False)
     flat[sub] = (rng.integers(1, 1 << 23, sub.size).astype(np.uint32)
                  | (rng.integers(0, 2, sub.size).astype(np.uint32) << 31)).view(np.float32)
-    x[3, 17] = np.nan
-    x[5, 40] = np.inf
+    x[3, 17 % cols] = np.nan
+    x[5, 40 % cols] = np.inf
     x[7, :] = 0.0
     return ind.f32_to_bf16_bits_rne(x) if bf16 else x
 
