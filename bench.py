@@ -44,7 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
 # the roofline kernels, from one ncu capture of this benchmark's own launches
-# (summaries in profiles/dram_traffic_bench.md).  Each entry holds the kernel
+# (summaries under profiles/).  Each entry holds the kernel
 # sources, the sha256 of their contents at capture time and bytes per launch
 # by workload.  A figure is reported only while the sources still hash to that
 # value; after any change to them it reads null until captured again.
@@ -418,6 +418,10 @@ def run_mx(args):
     dual = None if args.no_dual else run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world)
     if dual is not None:
         launches_gemm += dual.pop("_launches")
+    nvfp4 = None if args.no_nvfp4 else run_nvfp4_phase(args, dev, stream, peaks, peak_kind, barrier,
+                                                        max_over_ranks, world)
+    if nvfp4 is not None:
+        launches_gemm += nvfp4.pop("_launches")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -451,6 +455,8 @@ def run_mx(args):
             line["wgrad"] = wgrad
         if dual is not None:
             line["dual_cast"] = dual
+        if nvfp4 is not None:
+            line["nvfp4"] = nvfp4
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -709,6 +715,90 @@ def run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world):
     return out
 
 
+def run_nvfp4_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world):
+    """NVFP4 (16-element E2M1 blocks, E4M3 block scales, one fp32 encode scale
+    per domain): the cast of a Llama-3-8B activation 8192 x 4096 bf16 with a
+    global domain and with CTA-local domains of 128 rows, and the three
+    Llama-3-8B GEMM shapes on NVFP4 operands (activations CTA-local, weights
+    global), bf16 out."""
+    import torch
+    from microscaling_block_scaled_mx_b200 import inputs as I
+    from microscaling_block_scaled_mx_b200 import mx
+    local_rows = 128
+    steps = max(3, min(args.steps, 50))
+    hbm = float(peaks["hbm_gbs"])
+    fp4_peak = 4.0 * float(peaks["bf16_tflops"])
+    launches = 0
+
+    def timed(fn, n):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(1e3 * e0.elapsed_time(e1) / n)
+
+    out = {"workload": "nvfp4: cast of a Llama-3-8B activation 8192x4096 bf16 (global, and CTA-local "
+                       f"domains of {local_rows} rows); Llama-3-8B GEMMs M=8192 on NVFP4 operands "
+                       "(activations CTA-local, weights global), bf16 out", "steps": steps}
+    # cast: inputs rotate over three device copies (> L2)
+    xb, _ = I.linear_operands(8192, 4096, 128, 3, stream=0)
+    xs = [torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev) for _ in range(N_ROTATE)]
+    rows, cols = xs[0].shape
+    cast = {}
+    for label, dom in (("global", 0), ("cta_local", local_rows)):
+        bufs = [mx.quantize_nvfp4(x, dom) for x in xs]
+        it = [0]
+
+        def one(dom=dom, bufs=bufs, it=it):
+            r = it[0] % N_ROTATE
+            it[0] += 1
+            mx.quantize_nvfp4(xs[r], dom, out=bufs[r])
+        for _ in range(args.warmup):
+            one()
+        us = timed(one, steps)
+        launches += steps * (3 if dom == 0 else 1)
+        n = rows * cols
+        alg = n * 2 + n // 2 + n // 16 + 4 * mx.lib().mx_nvfp4_domains(rows, dom)
+        cast[label] = {"us": round(us, 1), "gbs": round(alg / (us * 1e-6) / 1e9, 1),
+                       "frac_hbm": round(alg / (us * 1e-6) / 1e9 / hbm, 4),
+                       "kernels": "nv_amax + nv_quant + nv_final" if dom == 0 else "nv_local"}
+    out["cast"] = cast
+    del xs
+    gemm = {}
+    total_flops = total_us = 0.0
+    for idx, (M, N, K) in enumerate(I.LLAMA3_GEMMS):
+        xb, wb = I.linear_operands(M, K, N, 3, stream=idx)
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
+        a = mx.quantize_nvfp4(x, local_rows)
+        b = mx.quantize_nvfp4(w, 0)
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        del x, w
+
+        def g(a=a, b=b, c=c, M=M, N=N, K=K):
+            mx.gemm_nvfp4(a, b, M, N, K, local_rows, 0, out=c)
+        for _ in range(args.warmup):
+            g()
+        us = timed(g, steps)
+        launches += steps
+        fl = 2.0 * M * N * K
+        total_flops += fl
+        total_us += us
+        tf = fl / (us * 1e-6) / 1e12
+        gemm[f"{M}x{N}x{K}"] = {"us": round(us, 1), "tflops": round(tf, 1), "frac": round(tf / fp4_peak, 4)}
+    out["gemm"] = {"kernel": "mx_gemm_pair_kernel (cta_group::2, kind::mxf4nvf4, scale_vec::4X)",
+                   "per_shape": gemm, "tflops": round(total_flops / (total_us * 1e-6) / 1e12, 1),
+                   "peak": round(fp4_peak, 1),
+                   "peak_kind": f"{peak_kind} bf16 burst x 4 (nominal ratio for FP4 operands)"}
+    out["_launches"] = launches
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -721,6 +811,7 @@ def main():
     ap.add_argument("--no-cast", action="store_true", help="GEMM phases only (profiling)")
     ap.add_argument("--no-wgrad", action="store_true", help="skip the weight-gradient phase")
     ap.add_argument("--no-dual", action="store_true", help="skip the dual-cast phase")
+    ap.add_argument("--no-nvfp4", action="store_true", help="skip the NVFP4 phase")
     ap.add_argument("--no-fused", action="store_true", help="skip the quantizing-epilogue comparison")
     ap.add_argument("--fmts", default=",".join(FMTS), help="comma-separated cast formats (profiling)")
     ap.add_argument("--gemm-shapes", default="0,1,2", help="indices of the Llama-3 GEMM shapes to time")

@@ -347,6 +347,37 @@ MX_API int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa
                             mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
                             void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream);
 
+/*
+ * mx_gemm_nvfp4 -- C = alpha * A * B^T on NVFP4 operands written by
+ * mx_quantize_nvfp4 (MX_SCALES_MMA), each element taken as P * d / E (the
+ * reading of the global / CTA-local NVFP4 variants given at
+ * mx_quantize_nvfp4).  The tensor cores accumulate sum_k (P_a d_a)(P_b d_b)
+ * in fp32 (kind::mxf4nvf4, E4M3 block scales); the epilogue multiplies each
+ * element by fl32(fl32(alpha / E_A[m]) / E_B[n]), E_A[m] being the encode
+ * scale of the domain that holds row m of A and E_B[n] that of row n of B,
+ * and rounds once to cdt.
+ *
+ *  a_codes, b_codes  device, M x K / 2 and N x K / 2 bytes (mx_quantize_nvfp4
+ *             codes of A and B, K contiguous), 16-byte aligned.
+ *  a_scales, b_scales  device, mx_nvfp4_scales_bytes(MX_SCALES_MMA, M, K) and
+ *             (.., N, K) bytes, 16-byte aligned.
+ *  a_enc, b_enc  device, mx_nvfp4_domains(M, a_domain_rows) and
+ *             mx_nvfp4_domains(N, b_domain_rows) fp32 encode scales, 4-byte
+ *             aligned; read only.
+ *  a_domain_rows  rows of A per domain (0: one domain).
+ *  b_domain_rows  rows of B per domain: 0 or a multiple of 32
+ *             (MX_ERR_UNSUPPORTED otherwise; the epilogue applies one E_B per
+ *             32 columns of C).
+ *  K          a multiple of 16 (MX_ERR_SHAPE) and of 256 (MX_ERR_UNSUPPORTED).
+ *  c, cdt, ldc  as for mx_gemm (MX_F32 or MX_BF16).
+ * Errors: MX_ERR_ARG, MX_ERR_ALIGN, MX_ERR_SHAPE, MX_ERR_UNSUPPORTED,
+ * MX_ERR_CUDA; MX_ERR_TIMEOUT later through mx_last_device_status.
+ */
+MX_API int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float *a_enc, int64_t a_domain_rows,
+                         const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
+                         int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
+                         void *stream);
+
 /* Byte sizes of the buffers above (0 for invalid arguments). */
 MX_API size_t mx_codes_bytes(mx_fmt fmt, int64_t outer, int64_t inner);
 MX_API size_t mx_scales_bytes(mx_scale_layout sl, int64_t outer, int64_t inner);

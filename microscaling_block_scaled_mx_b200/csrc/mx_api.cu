@@ -308,6 +308,7 @@ MxGemmArgs gemm_args(const void *a_codes, const void *a_scales, mx_fmt fa, const
     a.fa = fa; a.fb = fb; a.M = M; a.N = N; a.K = K; a.alpha = alpha;
     a.c = nullptr; a.cdt = MX_F32; a.ldc = 0;
     a.q_codes = nullptr; a.q_scales = nullptr; a.q_fmt = 0; a.q_rnd = MX_RNE; a.q_sl = MX_SCALES_MMA; a.q_seed = 0;
+    a.nv = false; a.enc_a = nullptr; a.enc_b = nullptr; a.a_lines = 0; a.b_lines = 0;
     a.num_sms = 0; a.device = 0;
     return a;
 }
@@ -372,6 +373,37 @@ int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa,
     MxGemmArgs a = gemm_args(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha);
     a.q_codes = out_codes; a.q_scales = out_scales; a.q_fmt = out_fmt; a.q_rnd = out_rnd; a.q_sl = out_sl;
     a.q_seed = out_seed;
+    a.num_sms = sm_count(&a.device);
+    if (a.num_sms <= 0) return MX_ERR_CUDA;
+    return mx_launch_gemm(a, st);
+}
+
+int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float *a_enc, int64_t a_domain_rows,
+                  const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
+                  int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
+                  void *stream) {
+    if (cdt != MX_F32 && cdt != MX_BF16) return MX_ERR_ARG;
+    if (M < 0 || N < 0 || K < 0 || a_domain_rows < 0 || b_domain_rows < 0) return MX_ERR_ARG;
+    if (!gemm_dims_fit(M, N, K)) return MX_ERR_UNSUPPORTED;
+    if (K % 16 != 0) return MX_ERR_SHAPE;
+    if (K % 256 != 0 || b_domain_rows % 32 != 0) return MX_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return MX_OK;                  // empty: pointers may be NULL
+    if (!c || ldc < N) return MX_ERR_ARG;
+    if (!aligned16(c) || (ldc * dtype_bytes(cdt)) % 16 != 0) return MX_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) {
+        const size_t esz = static_cast<size_t>(dtype_bytes(cdt));
+        return cudaMemset2DAsync(c, ldc * esz, 0, N * esz, M, st) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+    }
+    if (!a_codes || !a_scales || !a_enc || !b_codes || !b_scales || !b_enc) return MX_ERR_ARG;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
+        (reinterpret_cast<uintptr_t>(a_enc) & 3u) != 0 || (reinterpret_cast<uintptr_t>(b_enc) & 3u) != 0)
+        return MX_ERR_ALIGN;
+    MxGemmArgs a = gemm_args(a_codes, a_scales, MX_E2M1, b_codes, b_scales, MX_E2M1, M, N, K, alpha);
+    a.c = c; a.cdt = cdt; a.ldc = ldc;
+    a.nv = true; a.enc_a = a_enc; a.enc_b = b_enc;
+    a.a_lines = a_domain_rows >= M ? 0 : a_domain_rows;   // a domain covering every row: one domain
+    a.b_lines = b_domain_rows >= N ? 0 : b_domain_rows;
     a.num_sms = sm_count(&a.device);
     if (a.num_sms <= 0) return MX_ERR_CUDA;
     return mx_launch_gemm(a, st);

@@ -636,13 +636,15 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
 constexpr int PAIR_BM = 256;
 constexpr int PAIR_A_BYTES = 128 * BK_BYTES;             // 16 KiB per CTA per stage
 
-template <bool FP4, int PBN> struct PairCfg {
+// NV: NVFP4 operands (kind::mxf4nvf4, 16-element blocks with E4M3 scales, so
+// four scale atoms per 256-element stage instead of two).
+template <bool FP4, int PBN, bool NV = false> struct PairCfg {
     static constexpr int BN = PBN;                       // tile columns (B rows)
     static constexpr int B_ROWS = PBN / 2;               // B rows per CTA
     static constexpr int B_BYTES = B_ROWS * BK_BYTES;    // per CTA per stage
     static constexpr int ACC_BUFS = PBN == 256 ? 1 : 2;  // accumulators in tensor memory
     static constexpr uint32_t SF_COL = ACC_BUFS * PBN;   // scale factors after the accumulators
-    static constexpr int G = FP4 ? 2 : 1;                // scale atoms along K per stage
+    static constexpr int G = NV ? 4 : (FP4 ? 2 : 1);     // scale atoms along K per stage
     static constexpr int STAGES = (PBN == 192 && !FP4) ? 6 : 5;
     static constexpr int SFA_BYTES = ATOM * G;
     static constexpr int SFB_BYTES = 2 * ATOM * G;       // both 128-row scale blocks the tile touches
@@ -679,6 +681,10 @@ struct PairParams {
     int skip_k_tile;
     int raster_group, raster_n_major;   // tile order (tile_coords)
     MxOut q;                   // OUT_MX only
+    // NVFP4 only: the operands' per-domain encode scales and rows per domain
+    // (0: one domain); C = alpha * acc / (E_A[m / a_lines] * E_B[n / b_lines])
+    const float *enc_a, *enc_b;
+    int a_lines, b_lines;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -714,10 +720,16 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
 __device__ __forceinline__ void tc_cp_scale_atom_pair(uint32_t taddr, uint64_t desc) {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
-template <bool FP4>
+template <bool FP4, bool NV = false>
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-    if (FP4) {
+    if (NV) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+            : "memory");
+    } else if (FP4) {
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
             "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
@@ -732,12 +744,12 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
     }
 }
 
-template <bool FP4, int OUT, int PBN>
+template <bool FP4, int OUT, int PBN, bool NV = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                     const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
                     const __grid_constant__ CUtensorMap tma_c, PairParams p) {
-    using C = PairCfg<FP4, PBN>;
+    using C = PairCfg<FP4, PBN, NV>;
     constexpr int STAGES_P = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -866,10 +878,12 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                     const uint32_t b_s = sbase + C::OFF_B + s * C::B_BYTES;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint32_t g = FP4 ? (k >> 1) : 0u;
-                        const uint32_t sf_id = FP4 ? ((2u * k) & 3u) : static_cast<uint32_t>(k);
+                        // MXFP8: k-block k of the atom; MXFP4: k-blocks 2k, 2k + 1 of atom k / 2;
+                        // NVFP4: all four 16-element blocks of atom k
+                        const uint32_t g = NV ? static_cast<uint32_t>(k) : (FP4 ? (k >> 1) : 0u);
+                        const uint32_t sf_id = NV ? 0u : (FP4 ? ((2u * k) & 3u) : static_cast<uint32_t>(k));
                         const uint32_t idesc = p.idesc | (sf_id << 4) | (sf_id << 29);
-                        tc_mma_pair<FP4>(d_tmem, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k), idesc,
+                        tc_mma_pair<FP4, NV>(d_tmem, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k), idesc,
                                          sfa_t + 4 * g, sfb_t + 8 * g + sfb_shift, (kt > 0 || k > 0) ? 1u : 0u);
                     }
                     issued = true;
@@ -923,10 +937,17 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             } else {
                 const int m_warp = tm * PAIR_BM + 128 * static_cast<int>(rank) + q * 32;
                 constexpr int PC = OUT == OUT_BF16 ? 32 : 16;   // columns per piece
+                // NVFP4: alpha / E_A of this row, then / E_B of the piece's columns
+                float fa = p.alpha;
+                if (NV) fa = __fdiv_rn(p.alpha, p.enc_a[p.a_lines ? min(m, p.M - 1) / p.a_lines : 0]);
                 if (m_warp < p.M) {
 #pragma unroll
-                    for (int j = 0; j < (PBN / 2) / PC; ++j)
-                        if (n_base + PC * j < p.N) epi_piece<OUT>(ew, r + PC * j, p.alpha, n_base + PC * j, m_warp);
+                    for (int j = 0; j < (PBN / 2) / PC; ++j) {
+                        const int n0 = n_base + PC * j;
+                        if (n0 >= p.N) continue;
+                        const float f = NV ? __fdiv_rn(fa, p.enc_b[p.b_lines ? n0 / p.b_lines : 0]) : fa;
+                        epi_piece<OUT>(ew, r + PC * j, f, n0, m_warp);
+                    }
                 }
             }
         }
@@ -1066,7 +1087,7 @@ bool make_c_map(CUtensorMap *map, const MxGemmArgs &a) {
                      bf16 ? 32u : 16u, 32u, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN) {
+uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN, bool nv = false) {
     auto code = [&](int f) -> uint32_t {
         if (fp4) return 1u;               // kind::mxf4: E2M1
         switch (f) {                      // kind::mxf8f6f4 operand type codes
@@ -1081,7 +1102,7 @@ uint32_t make_idesc(int fa, int fb, bool fp4, int m = BM, int n = BN) {
     d |= code(fa) << 7;
     d |= code(fb) << 10;
     d |= static_cast<uint32_t>(n >> 3) << 17;
-    d |= 1u << 23;                         // scale factors are UE8M0
+    if (!nv) d |= 1u << 23;                // scale factors are UE8M0 (NVFP4: UE4M3, bit clear)
     d |= static_cast<uint32_t>(m >> 4) << 24;
     return d;
 }
@@ -1103,12 +1124,12 @@ cudaError_t launch_overlapped(Kern kern, int grid, int smem, cudaStream_t st, co
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <bool FP4, int OUT, int PBN>
+template <bool FP4, int OUT, int PBN, bool NV = false>
 cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
                         const CUtensorMap &tsb, const CUtensorMap &tc, const PairParams &p, int grid,
                         cudaStream_t st) {
-    auto kern = mx_gemm_pair_kernel<FP4, OUT, PBN>;
-    constexpr int smem = PairCfg<FP4, PBN>::SMEM;
+    auto kern = mx_gemm_pair_kernel<FP4, OUT, PBN, NV>;
+    constexpr int smem = PairCfg<FP4, PBN, NV>::SMEM;
     static std::atomic<uint64_t> configured{0};   // per instantiation, one bit per device
     if (cudaError_t e = ensure_smem_limit(kern, smem, configured); e != cudaSuccess) return e;
     return launch_overlapped(kern, grid, smem, st, ta, tb, tsa, tsb, tc, p);
@@ -1195,13 +1216,15 @@ bool use_mxf4(const MxGemmArgs &a) {
     return a.fa == MX_E2M1 && a.fb == MX_E2M1 && a.K % 256 == 0;
 }
 
-// The two-SM kernel: 256 x pbn tiles over CTA pairs (pbn 256 or 192).
+// The two-SM kernel: 256 x pbn tiles over CTA pairs (pbn 256 or 192; NVFP4
+// operands 256 only).
 int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
     using namespace mxg;
-    const bool fp4 = use_mxf4(a);
+    const bool fp4 = a.nv || use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;     // K bytes of a uint8 stage view
-    const int G = fp4 ? 2 : 1;
-    const int64_t k_groups = a.K / 128;
+    const int G = a.nv ? 4 : (fp4 ? 2 : 1);
+    // scale atoms along K: four blocks each, of 32 elements (MX) or 16 (NVFP4)
+    const int64_t k_groups = a.nv ? a.K / 64 : a.K / 128;
     CUtensorMap ta, tb, tsa, tsb, tc;
     if (!make_c_map(&tc, a)) return MX_ERR_CUDA;
     if (!make_operand_map(&ta, a.a_codes, a.M, a.K, a.fa, fp4, 128)) return MX_ERR_CUDA;
@@ -1221,8 +1244,12 @@ int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
     p.tiles_m = static_cast<int>((a.M + PAIR_BM - 1) / PAIR_BM);
     p.tiles_n = static_cast<int>((a.N + pbn - 1) / pbn);
     p.alpha = a.alpha;
-    p.idesc = make_idesc(a.fa, a.fb, fp4, PAIR_BM, pbn);
+    p.idesc = make_idesc(a.fa, a.fb, fp4, PAIR_BM, pbn, a.nv);
     p.ab_tx = stage_tx_bytes(a.fa, fp4, 128) + stage_tx_bytes(a.fb, fp4, pbn / 2);
+    p.enc_a = a.enc_a;
+    p.enc_b = a.enc_b;
+    p.a_lines = static_cast<int>(a.a_lines);
+    p.b_lines = static_cast<int>(a.b_lines);
     raster_for(a, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major);
     p.skip_k_tile = g_skip_k_tile;
     g_skip_k_tile = -1;
@@ -1232,7 +1259,11 @@ int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
     cudaError_t e;
     p.q = mx_out(a);
     const int out = out_mode(a);
-    if (pbn == 256) e = fp4 ? launch_pair_out<true, 256>(out, ta, tb, tsa, tsb, tc, p, grid, st)
+    if (a.nv) {
+        if (pbn != 256 || out == OUT_MX) return MX_ERR_UNSUPPORTED;
+        e = out == OUT_BF16 ? launch_pair<true, OUT_BF16, 256, true>(ta, tb, tsa, tsb, tc, p, grid, st)
+                            : launch_pair<true, OUT_F32, 256, true>(ta, tb, tsa, tsb, tc, p, grid, st);
+    } else if (pbn == 256) e = fp4 ? launch_pair_out<true, 256>(out, ta, tb, tsa, tsb, tc, p, grid, st)
                             : launch_pair_out<false, 256>(out, ta, tb, tsa, tsb, tc, p, grid, st);
     else e = fp4 ? launch_pair_out<true, 192>(out, ta, tb, tsa, tsb, tc, p, grid, st)
                  : launch_pair_out<false, 192>(out, ta, tb, tsa, tsb, tc, p, grid, st);
@@ -1256,6 +1287,7 @@ int pair_tile_n(const MxGemmArgs &a) {
 
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     using namespace mxg;
+    if (a.nv) return launch_gemm_pair(a, 256, st);   // NVFP4 runs on the CTA-pair kernel only
     if (const int pbn = pair_tile_n(a); pbn != 0) return launch_gemm_pair(a, pbn, st);
     const bool fp4 = use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;

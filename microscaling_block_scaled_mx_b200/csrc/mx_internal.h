@@ -78,6 +78,11 @@ struct MxGemmArgs {
     void *q_codes, *q_scales;
     int q_fmt, q_rnd, q_sl;
     uint64_t q_seed;
+    // NVFP4 operands (mx_gemm_nvfp4): E2M1 codes with 16-element E4M3 blocks
+    // and per-domain fp32 encode scales; a_lines / b_lines rows per domain (0: one)
+    bool nv;
+    const float *enc_a, *enc_b;
+    int64_t a_lines, b_lines;
     int num_sms;
     int device;
 };

@@ -231,3 +231,22 @@ def test_nvfp4_validation(mx):
     assert L.mx_nvfp4_domains(100, 32) == 4 and L.mx_nvfp4_domains(100, 0) == 1
     assert L.mx_nvfp4_scales_bytes(0, 100, 64) == 400
     assert L.mx_nvfp4_scales_bytes(1, 100, 64) == 128 * 4
+
+
+def test_nvfp4_gemm_validation(mx):
+    """Host-side checks of mx_gemm_nvfp4 (nothing is launched)."""
+    L = mx.lib()
+
+    def call(M=256, N=256, K=512, a_dom=0, b_dom=0, cdt=1, ldc=256, c=16, a_codes=16, a_enc=16, b_enc=16):
+        return L.mx_gemm_nvfp4(a_codes, 16, a_enc, a_dom, 16, 16, b_enc, b_dom, M, N, K, 1.0, c, cdt, ldc, None)
+
+    assert call(K=520) == -3                    # K % 16
+    assert call(K=384) == -4                    # K % 256
+    assert call(b_dom=48) == -4                 # E_B per 32 columns
+    assert call(a_dom=-1) == -1 and call(M=-1) == -1
+    assert call(cdt=2) == -1                    # output dtype
+    assert call(ldc=100) == -1                  # ldc < N
+    assert call(c=24) == -2 and call(a_codes=8) == -2 and call(a_enc=18) == -2 and call(b_enc=2) == -2
+    assert call(M=1 << 31) == -4                # past 32-bit indexing
+    assert L.mx_gemm_nvfp4(None, None, None, 0, None, None, None, 0, 0, 256, 512, 1.0, None, 1, 256,
+                           None) == 0          # empty
