@@ -124,3 +124,18 @@ def test_gemm_reference_is_matmul(oracle):
     A, B = dec(a, M, 32), dec(b, N, 0)
     assert np.allclose(c, 0.5 * (A @ B.T), rtol=0, atol=1e-12 * np.abs(c).max())
     assert np.all(bound >= np.abs(c) - 1e-12)
+
+
+def test_local_domains_are_global_casts_of_their_rows(oracle):
+    """A CTA-local cast is, domain by domain, the global cast of that
+    domain's rows alone (a ragged last domain included)."""
+    rng = np.random.default_rng(6)
+    x = (rng.standard_normal((100, 64)) * np.exp2(rng.uniform(-5, 5, (100, 1)))).astype(np.float32)
+    c, s, e = oracle.nvfp4_quantize(x, 32)
+    s = s.reshape(100, 4)
+    for d, r0 in enumerate(range(0, 100, 32)):
+        r1 = min(r0 + 32, 100)
+        cg, sg, eg = oracle.nvfp4_quantize(np.ascontiguousarray(x[r0:r1]), 0)
+        assert e[d] == eg[0]
+        assert np.array_equal(c[r0:r1], cg)
+        assert np.array_equal(s[r0:r1].reshape(-1), sg)
