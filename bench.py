@@ -50,16 +50,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # value; after any change to them it reads null until captured again.
 _CSRC = os.path.join(ROOT, "microscaling_block_scaled_mx_b200", "csrc")
 MEASURED_TRAFFIC = {
+    # the third of three consecutive casts of one format captured with
+    # --cache-control none, so each launch also carries the write-back of its
+    # predecessor's output still in L2 (steady state: reads + writes of one cast)
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "21c13cd4e7a3657226ce260915a58d45276e77cba8f53b8744192be6197a113e",
-                  {"e4m3_bf16_8192x8192": 169430272, "e5m2_bf16_8192x8192": 166759168,
-                   "e2m3_bf16_8192x8192": 158376192, "e3m2_bf16_8192x8192": 157790976,
-                   "e2m1_bf16_8192x8192": 148557312, "int8_bf16_8192x8192": 169712384}),
+                  "05265ce9ff1cd80a87eeb3540ef2af52f9b9c025ae52f0c590bcb67a3bd81420",
+                  {"e4m3_bf16_8192x8192": 202876928, "e5m2_bf16_8192x8192": 201791744,
+                   "e2m3_bf16_8192x8192": 186473728, "e3m2_bf16_8192x8192": 186313984,
+                   "e2m1_bf16_8192x8192": 170129920, "int8_bf16_8192x8192": 203687680}),
+    # the GEMMs: default cache control (L2 flushed before the launch), so reads
+    # show re-reads and writes count only what left L2 during the launch
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "c0792af6b749f96e1b6170749458bf04f9760c61c60696dc34860212860cebd0",
-             {"e2m1_8192x6144x4096": 78123264, "e2m1_8192x14336x4096": 227853056,
-              "e2m1_8192x4096x14336": 138795520, "e4m3_8192x3072x768": 9282304,
-              "e4m3_8192x768x3072": 28421120}),
+             "47937c20e39ed097a06bafbb8a85a90bf2b036ff2ef83db3ebc74c540197e9e9",
+             {"e2m1_8192x6144x4096": 85044224, "e2m1_8192x14336x4096": 235565824,
+              "e2m1_8192x4096x14336": 150462464, "e4m3_8192x3072x768": 10886912,
+              "e4m3_8192x768x3072": 28439296}),
 }
 
 
@@ -68,8 +73,14 @@ MEASURED_TRAFFIC = {
 # the same source-hash rule as MEASURED_TRAFFIC.  They give the instruction-
 # issue roofline of those casts: at most 4 warp instructions per clock per SM.
 MEASURED_INSTR = {
-    "cast_cols_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"), None, {}),
-    "cast_dual_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"), None, {}),
+    "cast_cols_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
+                         "05265ce9ff1cd80a87eeb3540ef2af52f9b9c025ae52f0c590bcb67a3bd81420",
+                         {"e2m1_bf16_16384x4096": 38797248 / (16384 * 4096),
+                          "e2m1_bf16_16384x14336": 135299008 / (16384 * 14336)}),
+    "cast_dual_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
+                         "05265ce9ff1cd80a87eeb3540ef2af52f9b9c025ae52f0c590bcb67a3bd81420",
+                         {"e2m1_bf16_16384x4096": 52169344 / (16384 * 4096),
+                          "e2m1_bf16_16384x14336": 182012544 / (16384 * 14336)}),
 }
 
 
@@ -261,14 +272,29 @@ def run_mx(args):
 
     peaks, peak_kind = load_peaks()
     stream = torch.cuda.current_stream()
-    if args.no_cast:
-        gemm = run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world)
-        gemm8 = run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks, world, fmt="e4m3")
-        if rank == 0:
-            print(json.dumps({"gemm_only": True, "gemm": gemm, "gemm_fp8": gemm8}), flush=True)
-        if world > 1:
-            dist.destroy_process_group()
-        return 0
+    if args.only:
+        # profiling: the named phases alone, on their own workloads (not a bench line)
+        phases = {"gemm": lambda: run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
+                                                 world),
+                  "gemm_fp8": lambda: run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier,
+                                                     max_over_ranks, world, fmt="e4m3"),
+                  "wgrad": lambda: run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
+                                                   world),
+                  "dual": lambda: run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world),
+                  "nvfp4": lambda: run_nvfp4_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
+                                                   world)}
+        names = args.only.split(",")
+        if "cast" in names and len(names) > 1:
+            raise SystemExit("--only cast runs alone")
+        res = {name: phases[name]() for name in names if name != "cast"}
+        if "cast" not in names:
+            if rank == 0:
+                print(json.dumps({"profiling_only": args.only, **res}), flush=True)
+            if world > 1:
+                dist.destroy_process_group()
+            return 0
+        args.no_gemm = args.no_wgrad = args.no_dual = args.no_nvfp4 = True
+        args.no_e2e = args.no_cpu_baseline = True
 
     # ---- inputs (host generation, then resident in HBM) ----
     bits = I.cast_sweep_input(ROWS, COLS, seed_stream=rank)
@@ -644,7 +670,7 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
         ipv = measured_instr("cast_cols_had_sr", f"e2m1_bf16_{shape[k]}")
         if ipv is not None:
             alu_us = issue_bound_us(ipv, values[k], sms, sm_mhz)
-            out[k]["alu"] = {"warp_instr_per_value": ipv, "bound_us": round(alu_us, 1), "sm_mhz": sm_mhz,
+            out[k]["alu"] = {"warp_instr_per_value": round(ipv, 4), "bound_us": round(alu_us, 1), "sm_mhz": sm_mhz,
                              "frac": round(alu_us / us[k], 4)}
             # the roofline is the slower of the two bounds
             out[k]["roofline"] = {"bound": "alu" if alu_us > hbm_us else "hbm",
@@ -691,6 +717,7 @@ def run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world):
 
     steps = max(3, min(args.steps, 20))
     hbm = float(peaks["hbm_gbs"])
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     out = {"workload": "dual cast: dY 16384x4096 and X 16384x14336 bf16 to E2M1 (rows RNE, tokens Hadamard+SR); "
                        "Llama-3 activation 8192x4096 bf16 to E4M3 (RNE both axes)", "steps": steps}
     for name, t, f, rc, had, o in ops:
@@ -703,7 +730,9 @@ def run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world):
         for _ in range(args.warmup):
             dual()
             two()
-        d, s2 = timed(dual, steps), timed(two, steps)
+        with ClockSampler(dev.index or 0) as clk:
+            d, s2 = timed(dual, steps), timed(two, steps)
+        sm_mhz = clk.summary()["sm_mhz"] or 1965.0
         launches += 3 * steps
         n = t.numel()
         bits = mx.FMT_BITS[mx.FMT[f]]
@@ -711,6 +740,14 @@ def run_dual_phase(args, dev, stream, peaks, barrier, max_over_ranks, world):
         out[name] = {"dual_us": round(d, 1), "two_casts_us": round(s2, 1), "speedup": round(s2 / d, 3),
                      "dual_gbs": round(alg / (d * 1e-6) / 1e9, 1),
                      "frac_hbm": round(alg / (d * 1e-6) / 1e9 / hbm, 4)}
+        ipv = measured_instr("cast_dual_had_sr", f"{f}_bf16_{t.shape[0]}x{t.shape[1]}") if had else None
+        if ipv is not None:
+            alu_us = issue_bound_us(ipv, n, sms, sm_mhz)
+            hbm_us = alg / (hbm * 1e9) * 1e6
+            out[name]["alu"] = {"warp_instr_per_value": round(ipv, 4), "bound_us": round(alu_us, 1),
+                                "sm_mhz": sm_mhz, "frac": round(alu_us / d, 4)}
+            out[name]["roofline"] = {"bound": "alu" if alu_us > hbm_us else "hbm",
+                                     "frac": round(max(alu_us, hbm_us) / d, 4)}
     out["_launches"] = launches
     return out
 
@@ -761,12 +798,12 @@ def run_nvfp4_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
         for _ in range(args.warmup):
             one()
         us = timed(one, steps)
-        launches += steps * (3 if dom == 0 else 1)
+        launches += steps * 3
         n = rows * cols
         alg = n * 2 + n // 2 + n // 16 + 4 * mx.lib().mx_nvfp4_domains(rows, dom)
         cast[label] = {"us": round(us, 1), "gbs": round(alg / (us * 1e-6) / 1e9, 1),
                        "frac_hbm": round(alg / (us * 1e-6) / 1e9 / hbm, 4),
-                       "kernels": "nv_amax + nv_quant + nv_final" if dom == 0 else "nv_local"}
+                       "kernels": "nv_amax + nv_quant + nv_final"}
     out["cast"] = cast
     del xs
     gemm = {}
@@ -808,7 +845,8 @@ def main():
     ap.add_argument("--no-gemm", action="store_true", help="skip the GEMM phase")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phase")
-    ap.add_argument("--no-cast", action="store_true", help="GEMM phases only (profiling)")
+    ap.add_argument("--only", default="", help="profiling: comma-separated phases to run alone "
+                    "(cast, gemm, gemm_fp8, wgrad, dual, nvfp4)")
     ap.add_argument("--no-wgrad", action="store_true", help="skip the weight-gradient phase")
     ap.add_argument("--no-dual", action="store_true", help="skip the dual-cast phase")
     ap.add_argument("--no-nvfp4", action="store_true", help="skip the NVFP4 phase")

@@ -236,8 +236,9 @@ MX_API int mx_quantize_dual_shard(const void *x, mx_dtype xdt, int64_t rows, int
  *    elements (the MXFP4 codes), one E4M3 block scale per block;
  *  - one fp32 encode scale E per domain: the whole tensor (domain_rows = 0,
  *    "global"), or each group of domain_rows consecutive rows, all columns
- *    ("CTA-local": the rows one CTA of this cast owns; 32 matches the rows
- *    one epilogue thread of the GEMM covers);
+ *    ("CTA-local": rows that one CTA of a fused producer can own, so that in
+ *    such a producer the scale needs no grid-wide reduction; this cast runs
+ *    both kinds as the same two passes over the input);
  *  - with a_D the largest finite |x| of a domain, E = 2688 / a_D (6 * 448, the
  *    largest E2M1 and E4M3 values; 1 when a_D = 0, the largest finite fp32
  *    when the quotient overflows); per block, with a_b its largest |x|, the

@@ -5,15 +5,19 @@
 // them; the reading taken (the public NVFP4 format) is stated in include/mx.h
 // at mx_quantize_nvfp4.
 //
-// Kernels (blocks along rows, the K axis of a GEMM operand):
-//   global domain      nv_amax_kernel   largest finite |x| of the tensor, an
-//                                       atomic max into enc_scales[0] (as bits)
-//                      nv_quant_kernel  every block, E from that maximum
-//                      nv_final_kernel  enc_scales[0] <- E
-//   CTA-local domains  nv_local_kernel  one CTA per domain of domain_rows rows:
-//                                       its maximum (CTA reduction), E, then
-//                                       its blocks (the second read is served
-//                                       by L2)
+// Kernels (blocks along rows, the K axis of a GEMM operand), the same three
+// for both kinds of domain (the global domain is one domain of all rows):
+//   nv_amax_kernel   largest finite |x| of each domain: every CTA reduces a
+//                    contiguous piece of one domain and adds it to
+//                    enc_scales[d] with one atomic max (as bits; non-negative
+//                    floats order as their bit patterns)
+//   nv_quant_kernel  every block, E from its domain's maximum (the same
+//                    pieces, so E is computed once per CTA; the second read of
+//                    a tensor that fits in L2 is served from there)
+//   nv_final_kernel  enc_scales[d] <- E of domain d
+// A domain's blocks are contiguous in row-major order and are split evenly
+// over `parts` CTAs, so there are enough CTAs to fill the GPU whether there is
+// one domain or thousands.
 // Every step is one IEEE fp32 operation (no fused multiply-add, no flush), in
 // the order the reading states, so results equal the CPU reference bit for
 // bit.
@@ -42,6 +46,9 @@ struct NvParams {
     uint32_t k_groups;     // ceil(k_blocks / 4)
     float *enc;            // one fp32 per domain
     int64_t lines;         // rows per domain
+    int64_t n_dom;         // domains
+    int parts;             // CTAs per domain
+    uint32_t row_step, kb_step;   // THREADS blocks = row_step rows + kb_step blocks
 };
 
 __device__ __forceinline__ float encode_scale(float amax) {
@@ -58,12 +65,13 @@ __device__ __forceinline__ float e4m3_value(uint32_t s) {
                   : __uint_as_float(((e + 120u) << 23) | (m << 20));                       // (1 + m/8) 2^(e-7)
 }
 
-// the 16 values of block kb of row `row`, widened to fp32
-template <bool BF16_IN>
+// the 16 values of block kb of row `row`, widened to fp32; LAST: the last read
+// of these bytes (streaming), else keep them in L2 for the second pass
+template <bool BF16_IN, bool LAST>
 __device__ __forceinline__ void load_block(const NvParams &p, int64_t row, int64_t kb, float (&v)[NV_BLOCK]) {
     if (BF16_IN) {
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.x) + row * p.ldx + kb * 16);
-        const uint4 a = __ldcs(src), b = __ldcs(src + 1);
+        const uint4 a = LAST ? __ldcs(src) : __ldg(src), b = LAST ? __ldcs(src + 1) : __ldg(src + 1);
         const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -74,7 +82,7 @@ __device__ __forceinline__ void load_block(const NvParams &p, int64_t row, int64
         const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(p.x) + row * p.ldx + kb * 16);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float4 f = __ldcs(src + i);
+            const float4 f = LAST ? __ldcs(src + i) : __ldg(src + i);
             v[4 * i] = f.x;
             v[4 * i + 1] = f.y;
             v[4 * i + 2] = f.z;
@@ -99,7 +107,7 @@ __device__ __forceinline__ float block_max(const float (&v)[NV_BLOCK], bool &fin
 template <bool BF16_IN>
 __device__ __forceinline__ void quant_block(const NvParams &p, int64_t row, int64_t kb, float E) {
     float v[NV_BLOCK];
-    load_block<BF16_IN>(p, row, kb, v);
+    load_block<BF16_IN, true>(p, row, kb, v);
     bool finite;
     const float amax = block_max(v, finite);
     uint32_t s = NV_SCALE_NAN;
@@ -143,63 +151,70 @@ __device__ __forceinline__ float cta_max(float m, float *red) {
     return m;
 }
 
+// The piece of domain d that this CTA covers: blocks [b0, b1) of the domain,
+// counted row-major from its first row r0.
+struct Piece {
+    int64_t d, r0, b0, b1;
+};
+__device__ __forceinline__ Piece piece_of(const NvParams &p) {
+    Piece q;
+    q.d = blockIdx.x / p.parts;
+    const int64_t part = blockIdx.x % p.parts;
+    q.r0 = q.d * p.lines;
+    const int64_t nb = min(p.lines, p.rows - q.r0) * static_cast<int64_t>(p.k_blocks);
+    const int64_t chunk = (nb + p.parts - 1) / p.parts;
+    q.b0 = min(nb, part * chunk);
+    q.b1 = min(nb, q.b0 + chunk);
+    return q;
+}
+
+// Calls f(row, kb) for this thread's blocks of the piece: block b0 + tid, then
+// every THREADS blocks, stepping (row, kb) without a division per block.
+template <typename F>
+__device__ __forceinline__ void for_each_block(const NvParams &p, const Piece &q, F f) {
+    int64_t i = q.b0 + threadIdx.x;
+    if (i >= q.b1) return;
+    int64_t row = q.r0 + i / p.k_blocks;
+    uint32_t kb = static_cast<uint32_t>(i % p.k_blocks);
+    for (; i < q.b1; i += THREADS) {
+        f(row, kb);
+        row += p.row_step;
+        kb += p.kb_step;
+        if (kb >= p.k_blocks) { kb -= p.k_blocks; ++row; }
+    }
+}
+
 template <bool BF16_IN>
 __global__ void __launch_bounds__(THREADS) nv_amax_kernel(NvParams p) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ float red[THREADS / 32];
-    const int64_t n = p.rows * static_cast<int64_t>(p.k_blocks);
+    const Piece q = piece_of(p);
     float m = 0.0f;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(THREADS) + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * THREADS) {
+    for_each_block(p, q, [&](int64_t row, uint32_t kb) {
         float v[NV_BLOCK];
-        load_block<BF16_IN>(p, i / p.k_blocks, i % p.k_blocks, v);
+        load_block<BF16_IN, false>(p, row, kb, v);
         bool finite;
         m = fmaxf(m, block_max(v, finite));
-    }
+    });
     m = cta_max(m, red);
-    // non-negative floats order as their bit patterns
-    if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int *>(p.enc), __float_as_uint(m));
+    if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int *>(p.enc + q.d), __float_as_uint(m));
 }
 
 template <bool BF16_IN>
 __global__ void __launch_bounds__(THREADS) nv_quant_kernel(NvParams p) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const float E = encode_scale(p.enc[0]);              // enc[0] holds the tensor's maximum here
-    const int64_t n = p.rows * static_cast<int64_t>(p.k_blocks);
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(THREADS) + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * THREADS)
-        quant_block<BF16_IN>(p, i / p.k_blocks, i % p.k_blocks, E);
+    const Piece q = piece_of(p);
+    const float E = encode_scale(p.enc[q.d]);             // enc[d] holds the domain's maximum here
+    for_each_block(p, q, [&](int64_t row, uint32_t kb) { quant_block<BF16_IN>(p, row, kb, E); });
 }
 
-__global__ void nv_final_kernel(float *enc) {
+__global__ void __launch_bounds__(THREADS) nv_final_kernel(float *enc, int64_t n_dom) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (blockIdx.x == 0 && threadIdx.x == 0) enc[0] = encode_scale(enc[0]);
-}
-
-template <bool BF16_IN>
-__global__ void __launch_bounds__(THREADS) nv_local_kernel(NvParams p, int64_t n_dom) {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    __shared__ float red[THREADS / 32];
-    for (int64_t d = blockIdx.x; d < n_dom; d += gridDim.x) {
-        const int64_t r0 = d * p.lines;
-        const int64_t nr = min(p.lines, p.rows - r0);
-        const int64_t n = nr * static_cast<int64_t>(p.k_blocks);
-        float m = 0.0f;
-        for (int64_t i = threadIdx.x; i < n; i += THREADS) {
-            float v[NV_BLOCK];
-            load_block<BF16_IN>(p, r0 + i / p.k_blocks, i % p.k_blocks, v);
-            bool finite;
-            m = fmaxf(m, block_max(v, finite));
-        }
-        const float E = encode_scale(cta_max(m, red));
-        if (threadIdx.x == 0) p.enc[d] = E;
-        for (int64_t i = threadIdx.x; i < n; i += THREADS)
-            quant_block<BF16_IN>(p, r0 + i / p.k_blocks, i % p.k_blocks, E);
-    }
+    const int64_t d = blockIdx.x * static_cast<int64_t>(THREADS) + threadIdx.x;
+    if (d < n_dom) enc[d] = encode_scale(enc[d]);
 }
 
 template <auto Kernel, typename... Args>
@@ -217,22 +232,14 @@ cudaError_t launch(int grid, cudaStream_t st, Args... args) {
 }
 
 template <bool BF16_IN>
-cudaError_t run(const NvParams &p, int64_t domain_rows, int sms, cudaStream_t st) {
-    const int64_t blocks = p.rows * static_cast<int64_t>(p.k_blocks);
-    const int64_t cap = static_cast<int64_t>(sms) * 8;
-    if (domain_rows == 0) {
-        // the maximum accumulates in enc_scales[0], which starts at zero
-        cudaError_t e = cudaMemsetAsync(p.enc, 0, sizeof(float), st);
-        if (e != cudaSuccess) return e;
-        int grid = static_cast<int>(std::min<int64_t>((blocks + THREADS - 1) / THREADS, cap));
-        if (grid < 1) grid = 1;
-        if ((e = launch<nv_amax_kernel<BF16_IN>>(grid, st, p)) != cudaSuccess) return e;
-        if ((e = launch<nv_quant_kernel<BF16_IN>>(grid, st, p)) != cudaSuccess) return e;
-        return launch<nv_final_kernel>(1, st, p.enc);
-    }
-    const int64_t n_dom = (p.rows + domain_rows - 1) / domain_rows;
-    const int grid = static_cast<int>(std::min<int64_t>(n_dom, cap));
-    return launch<nv_local_kernel<BF16_IN>>(grid < 1 ? 1 : grid, st, p, n_dom);
+cudaError_t run(const NvParams &p, cudaStream_t st) {
+    // the maxima accumulate in enc_scales, which start at zero
+    cudaError_t e = cudaMemsetAsync(p.enc, 0, static_cast<size_t>(p.n_dom) * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    const int grid = static_cast<int>(p.n_dom * p.parts);
+    if ((e = launch<nv_amax_kernel<BF16_IN>>(grid, st, p)) != cudaSuccess) return e;
+    if ((e = launch<nv_quant_kernel<BF16_IN>>(grid, st, p)) != cudaSuccess) return e;
+    return launch<nv_final_kernel>(static_cast<int>((p.n_dom + THREADS - 1) / THREADS), st, p.enc, p.n_dom);
 }
 
 }  // namespace mxnv
@@ -250,6 +257,16 @@ cudaError_t mx_launch_quantize_nvfp4(const MxNvfp4Args &a, cudaStream_t st) {
     p.k_blocks = static_cast<uint32_t>(a.cols / NV_BLOCK);
     p.k_groups = (p.k_blocks + 3) / 4;
     p.enc = a.enc_scales;
-    p.lines = a.domain_rows == 0 ? a.rows : a.domain_rows;
-    return a.xdt == MX_BF16 ? run<true>(p, a.domain_rows, a.num_sms, st) : run<false>(p, a.domain_rows, a.num_sms, st);
+    p.lines = (a.domain_rows == 0 || a.domain_rows > a.rows) ? a.rows : a.domain_rows;
+    p.n_dom = (a.rows + p.lines - 1) / p.lines;
+    // about eight CTAs of THREADS per SM over all domains, at least one per domain
+    const int64_t target = static_cast<int64_t>(a.num_sms) * 8;
+    const int64_t per_dom = p.lines * static_cast<int64_t>(p.k_blocks);
+    int64_t parts = (target + p.n_dom - 1) / p.n_dom;
+    parts = std::min<int64_t>(parts, (per_dom + THREADS - 1) / THREADS);   // no CTA without a block
+    p.parts = static_cast<int>(std::max<int64_t>(parts, 1));
+    if (p.n_dom * p.parts > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+    p.row_step = static_cast<uint32_t>(THREADS / p.k_blocks);
+    p.kb_step = static_cast<uint32_t>(THREADS % p.k_blocks);
+    return a.xdt == MX_BF16 ? run<true>(p, st) : run<false>(p, st);
 }
