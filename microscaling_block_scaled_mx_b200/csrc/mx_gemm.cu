@@ -344,8 +344,10 @@ struct EpiWriter {
     int64_t ldc;
     int M, N;
 };
-// vals: 32 accumulator words (bf16 output) or 16 (fp32 output) of this lane's row
-template <int OUT>
+// vals: 32 accumulator words (bf16 output) or 16 (fp32 output) of this lane's row;
+// NBUF staging buffers per warp (2: a store may still read one while the
+// other is written; 1: each piece waits for the previous store's read)
+template <int OUT, int NBUF = 2>
 __device__ __forceinline__ void epi_piece(EpiWriter &w, const uint32_t *vals, float alpha, int x, int y) {
     constexpr int PC = OUT == OUT_BF16 ? 32 : 16;   // columns per piece
     if (x + PC > w.N) {
@@ -366,8 +368,8 @@ __device__ __forceinline__ void epi_piece(EpiWriter &w, const uint32_t *vals, fl
         }
         return;
     }
-    const uint32_t b = w.buf + static_cast<uint32_t>(w.count & 1) * EPI_PIECE;
-    if (w.lane == 0) bulk_wait_read<1>();       // this buffer's previous store has read it
+    const uint32_t b = w.buf + static_cast<uint32_t>(w.count % NBUF) * EPI_PIECE;
+    if (w.lane == 0) bulk_wait_read<NBUF - 1>();   // this buffer's previous store has read it
     __syncwarp();
     uint32_t q[16];
     if constexpr (OUT == OUT_BF16) {
@@ -637,32 +639,50 @@ constexpr int PAIR_BM = 256;
 constexpr int PAIR_A_BYTES = 128 * BK_BYTES;             // 16 KiB per CTA per stage
 
 // NV: NVFP4 operands (kind::mxf4nvf4, 16-element blocks with E4M3 scales, so
-// four scale atoms per 256-element stage instead of two).
+// four scale atoms per 256-element K slice instead of two).
+// KS: 128-byte K slices per pipeline stage.  Two slices per stage halve the
+// barrier handshakes per K step between the producers and the MMA thread,
+// which set the stage rate more than the bytes do (a loads-only probe of this
+// operand stream: 18.4 TB/s with one slice per stage for any stage count from
+// 3 to 6, 22.3 TB/s with two slices in 3 stages); the 256-column tiles of MX
+// operands take them, the tensor memory of the other configurations has no
+// room for the doubled scale columns.
 template <bool FP4, int PBN, bool NV = false> struct PairCfg {
     static constexpr int BN = PBN;                       // tile columns (B rows)
     static constexpr int B_ROWS = PBN / 2;               // B rows per CTA
-    static constexpr int B_BYTES = B_ROWS * BK_BYTES;    // per CTA per stage
+    static constexpr int B_SLICE = B_ROWS * BK_BYTES;    // B bytes per CTA per K slice
     static constexpr int ACC_BUFS = PBN == 256 ? 1 : 2;  // accumulators in tensor memory
     static constexpr uint32_t SF_COL = ACC_BUFS * PBN;   // scale factors after the accumulators
-    static constexpr int G = NV ? 4 : (FP4 ? 2 : 1);     // scale atoms along K per stage
-    static constexpr int STAGES = (PBN == 192 && !FP4) ? 6 : 5;
+    static constexpr int KS = (PBN == 256 && !NV) ? 2 : 1;
+    static constexpr int G1 = NV ? 4 : (FP4 ? 2 : 1);    // scale atoms along K per slice
+    static constexpr int G = KS * G1;                    // scale atoms along K per stage
+    static constexpr int STAGES = KS == 2 ? 3 : ((PBN == 192 && !FP4) ? 6 : 5);
+    static constexpr int A_BYTES = KS * PAIR_A_BYTES;    // per CTA per stage
+    static constexpr int B_BYTES = KS * B_SLICE;
     static constexpr int SFA_BYTES = ATOM * G;
     static constexpr int SFB_BYTES = 2 * ATOM * G;       // both 128-row scale blocks the tile touches
     static constexpr int SFA_COLS = 4 * G;
     static constexpr int SFB_COLS = 8 * G;
     static constexpr int SF_STAGE_COLS = SFA_COLS + SFB_COLS;
-    static constexpr int STAGE_BYTES = PAIR_A_BYTES + B_BYTES;
+    static constexpr int EPI_BUFS = KS == 2 ? 1 : 2;     // staged pieces of C per epilogue warp
     // shared-memory layout
     static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + STAGES * PAIR_A_BYTES;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_EPI = (OFF_SFB + STAGES * SFB_BYTES + 1023) / 1024 * 1024;
-    static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_WARP_BYTES;
+    static constexpr int EPI_WARP = EPI_BUFS * EPI_PIECE;
+    static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_WARP;
     static constexpr int NUM_BARS = 2 * STAGES + 5;      // full, empty, acc_full, acc_empty, drain (+2 spare)
     static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
-    static constexpr int SMEM = OFF_ABORT + 4 + 1024;    // + alignment slack
+    static constexpr int USED = OFF_ABORT + 4;
+    // Slack for aligning the dynamic shared memory to 1024 bytes (128-byte
+    // swizzled operand tiles).  Where the layout leaves no room for it, the
+    // kernel requires the base to be aligned already and reports
+    // MX_ERR_ALIGN through the device status word otherwise.
+    static constexpr bool SLACK = USED + 1024 <= 232448;
+    static constexpr int SMEM = USED + (SLACK ? 1024 : 0);
     static_assert(SF_COL + STAGES * SF_STAGE_COLS <= 512, "tensor memory columns");
     static_assert(SMEM <= 232448, "shared memory per block");
     static_assert(PBN == 256 || PBN == 192, "pair tile widths");
@@ -752,6 +772,11 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
     using C = PairCfg<FP4, PBN, NV>;
     constexpr int STAGES_P = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if (!C::SLACK && (smem_u32(smem_raw) & 1023u) != 0) {
+        // no room to realign (both CTAs of the pair see the same base and leave here)
+        if (threadIdx.x == 0) atomicExch(&g_mx_status, MX_ERR_ALIGN);
+        return;
+    }
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -801,7 +826,6 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            const uint32_t stage_bytes = 2 * (p.ab_tx + C::SFA_BYTES + C::SFB_BYTES);
             for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
                 int tm, tn;
                 tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
@@ -812,18 +836,29 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                 const int nb0 = min(tn * PBN + C::B_ROWS * static_cast<int>(rank), p.N - 1);
                 const int rb_a = m0 / 128, rb_b = (tn * PBN) / 128;
                 const int rb_b1 = min(rb_b + 1, (p.N - 1) / 128);
-                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                for (int kt = 0; kt < p.k_tiles; kt += C::KS) {
                     if (!wait_bounded(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
-                    if (rank == 0 && kt == p.skip_k_tile && tile == cluster_id && cluster_id == 0) {
+                    if (rank == 0 && p.skip_k_tile >= kt && p.skip_k_tile < kt + C::KS && tile == cluster_id &&
+                        cluster_id == 0) {
                         ok = false;          // injected stall: CTA 0 never arms this stage
                         break;
                     }
+                    // K slices in this stage (the last stage may hold fewer); the
+                    // scale boxes always cover the stage's G atoms, the atoms past
+                    // the slices present being read but unused (zero past the end)
+                    const int ns = min(C::KS, p.k_tiles - kt);
                     const uint32_t fb = map_to_rank(full_bar(s), 0);
-                    if (rank == 0) mbar_expect_tx(full_bar(s), stage_bytes);
-                    tma_load_2d_pair(sbase + C::OFF_A + s * PAIR_A_BYTES, &tma_a, kt * BK_BYTES, m0, fb);
-                    tma_load_2d_pair(sbase + C::OFF_B + s * C::B_BYTES, &tma_b, kt * BK_BYTES, nb0, fb);
+                    if (rank == 0)
+                        mbar_expect_tx(full_bar(s), 2 * (static_cast<uint32_t>(ns) * p.ab_tx + C::SFA_BYTES +
+                                                         C::SFB_BYTES));
+                    for (int q = 0; q < ns; ++q) {
+                        tma_load_2d_pair(sbase + C::OFF_A + s * C::A_BYTES + q * PAIR_A_BYTES, &tma_a,
+                                         (kt + q) * BK_BYTES, m0, fb);
+                        tma_load_2d_pair(sbase + C::OFF_B + s * C::B_BYTES + q * C::B_SLICE, &tma_b,
+                                         (kt + q) * BK_BYTES, nb0, fb);
+                    }
                     // scale atoms: a scale buffer is viewed as rows of 256 bytes, two per atom
-                    const int kg = kt * C::G;
+                    const int kg = kt * C::G1;
                     tma_load_2d_pair(sbase + C::OFF_SFA + s * C::SFA_BYTES, &tma_sfa, 0,
                                      2 * (rb_a * p.k_groups + kg), fb);
                     tma_load_2d_pair(sbase + C::OFF_SFB + s * C::SFB_BYTES, &tma_sfb, 0,
@@ -859,32 +894,41 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                 tile_coords(tile, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major, tm, tn);
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * PBN);
                 const uint32_t sfb_shift = ((tn * PBN) & 127) ? 2u : 0u;   // tile starts 64 rows into an atom
-                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                for (int kt = 0; kt < p.k_tiles; kt += C::KS) {
                     if (!wait_bounded(full_bar(s), ph, abort_flag)) { ok = false; break; }
                     tc_fence_after();
+                    const int ns = min(C::KS, p.k_tiles - kt);
                     const uint32_t sfa_t = tmem + C::SF_COL + s * C::SF_STAGE_COLS;
                     const uint32_t sfb_t = sfa_t + C::SFA_COLS;
                     const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
 #pragma unroll
                     for (int g = 0; g < C::G; ++g) {
-                        tc_cp_scale_atom_pair(sfa_t + 4 * g, scale_atom_desc(sfa_s + g * ATOM));
+                        if (g < ns * C::G1) {
+                            tc_cp_scale_atom_pair(sfa_t + 4 * g, scale_atom_desc(sfa_s + g * ATOM));
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            tc_cp_scale_atom_pair(sfb_t + 8 * g + 4 * h,
-                                                  scale_atom_desc(sfb_s + h * (C::SFB_BYTES / 2) + g * ATOM));
+                            for (int h = 0; h < 2; ++h)
+                                tc_cp_scale_atom_pair(sfb_t + 8 * g + 4 * h,
+                                                      scale_atom_desc(sfb_s + h * (C::SFB_BYTES / 2) + g * ATOM));
+                        }
                     }
-                    const uint32_t a_s = sbase + C::OFF_A + s * PAIR_A_BYTES;
-                    const uint32_t b_s = sbase + C::OFF_B + s * C::B_BYTES;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        // MXFP8: k-block k of the atom; MXFP4: k-blocks 2k, 2k + 1 of atom k / 2;
-                        // NVFP4: all four 16-element blocks of atom k
-                        const uint32_t g = NV ? static_cast<uint32_t>(k) : (FP4 ? (k >> 1) : 0u);
-                        const uint32_t sf_id = NV ? 0u : (FP4 ? ((2u * k) & 3u) : static_cast<uint32_t>(k));
-                        const uint32_t idesc = p.idesc | (sf_id << 4) | (sf_id << 29);
-                        tc_mma_pair<FP4, NV>(d_tmem, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k), idesc,
-                                         sfa_t + 4 * g, sfb_t + 8 * g + sfb_shift, (kt > 0 || k > 0) ? 1u : 0u);
+                    for (int q = 0; q < C::KS; ++q) {
+                        if (q < ns) {
+                            const uint32_t a_s = sbase + C::OFF_A + s * C::A_BYTES + q * PAIR_A_BYTES;
+                            const uint32_t b_s = sbase + C::OFF_B + s * C::B_BYTES + q * C::B_SLICE;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                // MXFP8: k-block k of the slice's atom; MXFP4: k-blocks 2k, 2k + 1
+                                // of atom k / 2; NVFP4: all four 16-element blocks of atom k
+                                const uint32_t g = q * C::G1 + (NV ? static_cast<uint32_t>(k) : (FP4 ? (k >> 1) : 0u));
+                                const uint32_t sf_id = NV ? 0u : (FP4 ? ((2u * k) & 3u) : static_cast<uint32_t>(k));
+                                const uint32_t idesc = p.idesc | (sf_id << 4) | (sf_id << 29);
+                                tc_mma_pair<FP4, NV>(d_tmem, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k),
+                                                     idesc, sfa_t + 4 * g, sfb_t + 8 * g + sfb_shift,
+                                                     (kt > 0 || q > 0 || k > 0) ? 1u : 0u);
+                            }
+                        }
                     }
                     issued = true;
                     tc_commit_pair(empty_bar(s));
@@ -903,7 +947,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
         // ------------------------------ epilogue (both CTAs) -------------------
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
-        EpiWriter ew{&tma_c, sbase + C::OFF_EPI + static_cast<uint32_t>(warp - 2) * EPI_WARP_BYTES, 0, lane,
+        EpiWriter ew{&tma_c, sbase + C::OFF_EPI + static_cast<uint32_t>(warp - 2) * C::EPI_WARP, 0, lane,
                      p.c, p.ldc, p.M, p.N};
         int local = 0;
         constexpr int NCH = PBN / 2 / 32;        // 32-column chunks per warp
@@ -946,7 +990,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                         const int n0 = n_base + PC * j;
                         if (n0 >= p.N) continue;
                         const float f = NV ? __fdiv_rn(fa, p.enc_b[p.b_lines ? n0 / p.b_lines : 0]) : fa;
-                        epi_piece<OUT>(ew, r + PC * j, f, n0, m_warp);
+                        epi_piece<OUT, C::EPI_BUFS>(ew, r + PC * j, f, n0, m_warp);
                     }
                 }
             }
@@ -1222,7 +1266,9 @@ int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
     using namespace mxg;
     const bool fp4 = a.nv || use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;     // K bytes of a uint8 stage view
-    const int G = a.nv ? 4 : (fp4 ? 2 : 1);
+    // scale atoms one stage's boxes cover: per 128-byte K slice, times the
+    // slices per stage (PairCfg::KS: two on 256-column tiles of MX operands)
+    const int G = (a.nv ? 4 : (fp4 ? 2 : 1)) * ((pbn == 256 && !a.nv) ? 2 : 1);
     // scale atoms along K: four blocks each, of 32 elements (MX) or 16 (NVFP4)
     const int64_t k_groups = a.nv ? a.K / 64 : a.K / 128;
     CUtensorMap ta, tb, tsa, tsb, tc;
