@@ -61,10 +61,10 @@ MEASURED_TRAFFIC = {
     # the GEMMs: default cache control (L2 flushed before the launch), so reads
     # show re-reads and writes count only what left L2 during the launch
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "47937c20e39ed097a06bafbb8a85a90bf2b036ff2ef83db3ebc74c540197e9e9",
-             {"e2m1_8192x6144x4096": 85044224, "e2m1_8192x14336x4096": 235565824,
-              "e2m1_8192x4096x14336": 150462464, "e4m3_8192x3072x768": 10886912,
-              "e4m3_8192x768x3072": 28439296}),
+             "5f42b5547c2bdbf3d3e990563c14d3a8491634cca05f78bb356c715b535ca8e6",
+             {"e2m1_8192x6144x4096": 85373440, "e2m1_8192x14336x4096": 236292864,
+              "e2m1_8192x4096x14336": 150680576, "e4m3_8192x3072x768": 10714880,
+              "e4m3_8192x768x3072": 28427008, "e2m1_4096x14336x16384": 493558272}),
 }
 
 
@@ -677,7 +677,7 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
                                   "frac": round(max(alu_us, hbm_us) / us[k], 4)}
     tf = flops / (us["gemm_dW"] * 1e-6) / 1e12
     out["gemm_dW"] = {"us": round(us["gemm_dW"], 1), "tflops": round(tf, 1), "frac": round(tf / fp4_peak, 4),
-                      "peak": round(fp4_peak, 1)}
+                      "peak": round(fp4_peak, 1), "traffic": measured_traffic("gemm", f"e2m1_{Do}x{Di}x{T}")}
     return out
 
 
