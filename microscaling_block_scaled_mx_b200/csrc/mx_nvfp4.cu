@@ -132,6 +132,75 @@ __device__ __forceinline__ void quant_block(const NvParams &p, int64_t row, int6
     p.scales[off] = static_cast<uint8_t>(s);
 }
 
+// bf16 input, a block as the 8 words of its 16 values (element 2i in the low
+// half of word i).  |x| of a bf16 is its bits with the sign cleared, and
+// magnitudes order as those 16-bit integers (Inf and NaN at 0x7F80 and above),
+// so the block maximum is a packed 16-bit integer max.
+constexpr uint32_t ABS16 = 0x7fff7fffu;
+constexpr uint32_t NONFINITE16 = 0x7f80u;
+
+__device__ __forceinline__ uint32_t max_half(uint32_t m) { return max(m & 0xffffu, m >> 16); }
+
+// largest |x| bits of the block (>= 0x7F80 when it holds a NaN or Inf)
+__device__ __forceinline__ uint32_t block_max_bits(const uint4 &a, const uint4 &b) {
+    uint32_t m = __vimax3_u16x2(a.x & ABS16, a.y & ABS16, a.z & ABS16);
+    m = __vimax3_u16x2(m, a.w & ABS16, b.x & ABS16);
+    m = __vimax3_u16x2(m, b.y & ABS16, b.z & ABS16);
+    return max_half(__vmaxu2(m, b.w & ABS16));
+}
+
+// largest finite |x| bits of the block (non-finite values count as zero)
+__device__ __forceinline__ uint32_t block_finite_max_bits(const uint4 &a, const uint4 &b) {
+    auto fin = [](uint32_t w) {
+        const uint32_t h = w & ABS16;
+        return h & ~__vcmpgeu2(h, (NONFINITE16 << 16) | NONFINITE16);
+    };
+    uint32_t m = __vimax3_u16x2(fin(a.x), fin(a.y), fin(a.z));
+    m = __vimax3_u16x2(m, fin(a.w), fin(b.x));
+    m = __vimax3_u16x2(m, fin(b.y), fin(b.z));
+    return max_half(__vmaxu2(m, fin(b.w)));
+}
+
+__device__ __forceinline__ uint64_t f2_mul_rn(uint64_t a, uint64_t b) {   // two IEEE fp32 products
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ const uint4 *bf16_block_ptr(const NvParams &p, int64_t row, uint32_t kb) {
+    return reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.x) + row * p.ldx + kb * 16);
+}
+
+// quant_block for bf16 input whose 32 bytes are already loaded
+__device__ __forceinline__ void quant_block_bf16(const NvParams &p, int64_t row, uint32_t kb, float E,
+                                                 const uint4 &a, const uint4 &b) {
+    const uint32_t mb = block_max_bits(a, b);
+    uint32_t s = NV_SCALE_NAN;
+    uint2 c = make_uint2(0u, 0u);
+    if (mb < NONFINITE16) {
+        const float amax = __uint_as_float(mb << 16);
+        const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), E);
+        s = mxk::cvt_pair<MX_E4M3>(t, 0.0f) & 0xffu;          // t >= 0: a positive code
+        const float d = e4m3_value(s);
+        const float r = d > 0.0f ? __fdiv_rn(E, d) : 0.0f;
+        const uint64_t rr = (static_cast<uint64_t>(__float_as_uint(r)) << 32) | __float_as_uint(r);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t q[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint64_t pr = f2_mul_rn((static_cast<uint64_t>(w[i] & 0xffff0000u) << 32) | (w[i] << 16), rr);
+            const uint32_t byte = mxk::cvt_pair<MX_E2M1>(__uint_as_float(static_cast<uint32_t>(pr)),
+                                                         __uint_as_float(static_cast<uint32_t>(pr >> 32)));
+            q[i >> 2] |= byte << (8 * (i & 3));
+        }
+        c = make_uint2(q[0], q[1]);
+    }
+    *reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + kb * 8) = c;
+    const uint32_t off = p.mma ? mxk::mma_scale_offset32(static_cast<uint32_t>(row), kb, p.k_groups)
+                               : static_cast<uint32_t>(row) * p.k_blocks + kb;
+    p.scales[off] = static_cast<uint8_t>(s);
+}
+
 // largest value over the CTA (every thread gets it)
 __device__ __forceinline__ float cta_max(float m, float *red) {
 #pragma unroll
@@ -184,6 +253,34 @@ __device__ __forceinline__ void for_each_block(const NvParams &p, const Piece &q
     }
 }
 
+// bf16: this thread's blocks of the piece with the next block's two loads
+// issued before the current block is processed; f(row, kb, a, b)
+template <bool LAST, typename F>
+__device__ __forceinline__ void for_each_bf16_block(const NvParams &p, const Piece &q, F f) {
+    int64_t i = q.b0 + threadIdx.x;
+    if (i >= q.b1) return;
+    int64_t row = q.r0 + i / p.k_blocks;
+    uint32_t kb = static_cast<uint32_t>(i % p.k_blocks);
+    const uint4 *src = bf16_block_ptr(p, row, kb);
+    uint4 a = LAST ? __ldcs(src) : __ldg(src), b = LAST ? __ldcs(src + 1) : __ldg(src + 1);
+    for (; i < q.b1; i += THREADS) {
+        int64_t row_n = row + p.row_step;
+        uint32_t kb_n = kb + p.kb_step;
+        if (kb_n >= p.k_blocks) { kb_n -= p.k_blocks; ++row_n; }
+        uint4 an = a, bn = b;
+        if (i + THREADS < q.b1) {
+            const uint4 *nx = bf16_block_ptr(p, row_n, kb_n);
+            an = LAST ? __ldcs(nx) : __ldg(nx);
+            bn = LAST ? __ldcs(nx + 1) : __ldg(nx + 1);
+        }
+        f(row, kb, a, b);
+        row = row_n;
+        kb = kb_n;
+        a = an;
+        b = bn;
+    }
+}
+
 template <bool BF16_IN>
 __global__ void __launch_bounds__(THREADS) nv_amax_kernel(NvParams p) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -191,12 +288,20 @@ __global__ void __launch_bounds__(THREADS) nv_amax_kernel(NvParams p) {
     __shared__ float red[THREADS / 32];
     const Piece q = piece_of(p);
     float m = 0.0f;
-    for_each_block(p, q, [&](int64_t row, uint32_t kb) {
-        float v[NV_BLOCK];
-        load_block<BF16_IN, false>(p, row, kb, v);
-        bool finite;
-        m = fmaxf(m, block_max(v, finite));
-    });
+    if constexpr (BF16_IN) {
+        uint32_t mb = 0;
+        for_each_bf16_block<false>(p, q, [&](int64_t, uint32_t, const uint4 &a, const uint4 &b) {
+            mb = max(mb, block_finite_max_bits(a, b));
+        });
+        m = __uint_as_float(mb << 16);
+    } else {
+        for_each_block(p, q, [&](int64_t row, uint32_t kb) {
+            float v[NV_BLOCK];
+            load_block<BF16_IN, false>(p, row, kb, v);
+            bool finite;
+            m = fmaxf(m, block_max(v, finite));
+        });
+    }
     m = cta_max(m, red);
     if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int *>(p.enc + q.d), __float_as_uint(m));
 }
@@ -207,7 +312,12 @@ __global__ void __launch_bounds__(THREADS) nv_quant_kernel(NvParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const Piece q = piece_of(p);
     const float E = encode_scale(p.enc[q.d]);             // enc[d] holds the domain's maximum here
-    for_each_block(p, q, [&](int64_t row, uint32_t kb) { quant_block<BF16_IN>(p, row, kb, E); });
+    if constexpr (BF16_IN)
+        for_each_bf16_block<true>(p, q, [&](int64_t row, uint32_t kb, const uint4 &a, const uint4 &b) {
+            quant_block_bf16(p, row, kb, E, a, b);
+        });
+    else
+        for_each_block(p, q, [&](int64_t row, uint32_t kb) { quant_block<BF16_IN>(p, row, kb, E); });
 }
 
 __global__ void __launch_bounds__(THREADS) nv_final_kernel(float *enc, int64_t n_dom) {
