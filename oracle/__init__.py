@@ -34,7 +34,7 @@ FORMATS = {"e4m3": E4M3, "e5m2": E5M2, "e2m3": E2M3, "e3m2": E3M2, "e2m1": E2M1,
 BITS = {E4M3: 8, E5M2: 8, E2M3: 6, E3M2: 6, E2M1: 4, INT8: 8}
 F32, BF16 = 0, 1
 RNE, SR = 0, 1
-PLAIN, MMA = 0, 1
+PLAIN, MMA, MMA_X4 = 0, 1, 2
 
 _lock = threading.Lock()
 _lib = None

@@ -52,7 +52,7 @@ enum { FMT_E4M3 = 0, FMT_E5M2 = 1, FMT_E2M3 = 2, FMT_E3M2 = 3, FMT_E2M1 = 4,
        FMT_INT8 = 5, FMT_COUNT = 6 };
 enum { DT_F32 = 0, DT_BF16 = 1 };
 enum { RND_RNE = 0, RND_SR = 1 };
-enum { SL_PLAIN = 0, SL_MMA = 1 };
+enum { SL_PLAIN = 0, SL_MMA = 1, SL_MMA_X4 = 2 };
 
 #define BLOCK 32
 
@@ -273,7 +273,9 @@ void mxref_hadamard32(float *x, uint32_t sign_mask)
 /*         byte, even element in the low nibble.                            */
 /*  scales: plain = outer x (inner/32) row-major; MMA = rows padded to 128, */
 /*         k-blocks padded to 4, 512-byte atoms of 128 rows x 4 k-blocks,   */
-/*         atoms k-fastest, inside an atom (r%32)*16 + ((r/32)%4)*4 + kb%4. */
+/*         atoms k-fastest, inside an atom (r%32)*16 + ((r/32)%4)*4 + kb%4; */
+/*         MMA x4 = the MMA layout with every atom stored four times in a   */
+/*         row (2048 bytes per atom; reads use the first copy).             */
 /* ------------------------------------------------------------------------ */
 
 int64_t mxref_codes_bytes(int fmt, int64_t outer, int64_t inner)
@@ -288,7 +290,17 @@ int64_t mxref_scales_bytes(int sl, int64_t outer, int64_t inner)
     if (sl == SL_PLAIN) return outer * kb;
     int64_t rows = (outer + 127) / 128 * 128;
     int64_t kbp = (kb + 3) / 4 * 4;
-    return rows * kbp;
+    return rows * kbp * (sl == SL_MMA_X4 ? 4 : 1);
+}
+
+static int64_t scale_offset(int sl, int64_t outer_idx, int64_t kb, int64_t kb_total);
+
+/* writes the scale byte of (outer_idx, kb): once, or in all four copies of
+ * its atom in the x4 layout */
+static void put_scale(uint8_t *scales, int sl, int64_t outer_idx, int64_t kb, int64_t kb_total, unsigned s)
+{
+    int64_t off = scale_offset(sl, outer_idx, kb, kb_total);
+    for (int j = 0; j < (sl == SL_MMA_X4 ? 4 : 1); ++j) scales[off + 512 * j] = (uint8_t)s;
 }
 
 static int64_t scale_offset(int sl, int64_t outer_idx, int64_t kb, int64_t kb_total)
@@ -297,7 +309,7 @@ static int64_t scale_offset(int sl, int64_t outer_idx, int64_t kb, int64_t kb_to
     int64_t katoms = (kb_total + 3) / 4;
     int64_t atom = (outer_idx / 128) * katoms + kb / 4;
     int64_t r = outer_idx % 128;
-    return atom * 512 + (r % 32) * 16 + (r / 32) * 4 + (kb % 4);
+    return atom * (sl == SL_MMA_X4 ? 2048 : 512) + (r % 32) * 16 + (r / 32) * 4 + (kb % 4);
 }
 
 static void put_code(int fmt, uint8_t *row, int64_t i, unsigned code)
@@ -449,7 +461,7 @@ int mxref_quantize_shard(const void *x, int xdt, int64_t rows, int64_t cols, int
             uint64_t idx0 = (uint64_t)((outer_off + o) * inner_total + inner_off + kb * BLOCK);
             unsigned s = quantize_block(fmt, rnd, seed, v, idx0, c);
             for (int j = 0; j < BLOCK; ++j) put_code(fmt, crow, kb * BLOCK + j, c[j]);
-            scales[scale_offset(sl, o, kb, kb_total)] = (uint8_t)s;
+            put_scale(scales, sl, o, kb, kb_total, s);
         }
     }
     return MXO_OK;
@@ -681,7 +693,7 @@ int mxref_nvfp4_quantize(const void *x, int xdt, int64_t rows, int64_t cols, int
                     put_code(FMT_E2M1, crow, kb * NV_BLOCK + j, mxref_encode_rne(FMT_E2M1, (double)u));
                 }
             }
-            scales[scale_offset(sl, o, kb, kb_total)] = (uint8_t)s;
+            put_scale(scales, sl, o, kb, kb_total, s);
         }
     }
     return MXO_OK;

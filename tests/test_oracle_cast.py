@@ -301,3 +301,34 @@ def test_round_f32_is_nearest(oracle):
     got = oracle.round_f32(y)
     np.testing.assert_array_equal(got, np.array([1.0, 1.0 + 2.0 ** -22, -(1.0 + 2.0 ** -23)],
                                                 dtype=np.float32))
+
+
+def test_mma_x4_scale_layout(oracle):
+    """The x4 layout: the MMA layout's 512-byte atoms, each stored four times
+    in a row (built here by repeating the plain scales through the MMA index
+    map), for both block axes, every format, SR and the Hadamard; decodes
+    agree with the plain layout's."""
+    rng = np.random.default_rng(44)
+    for outer, inner in [(128, 128), (200, 96), (300, 32 * 9)]:
+        for axis in (0, 1):
+            rows, cols = (outer, inner) if axis == 1 else (inner, outer)
+            x = rng.standard_normal((rows, cols)).astype(np.float32)
+            for name in ("e4m3", "e2m1", "e3m2", "int8"):
+                kw = dict(rnd=oracle.SR, seed=5, hadamard=axis == 0)
+                c_plain, plain = oracle.quantize(x, axis, fid(name), scale_layout=oracle.PLAIN, **kw)
+                c_x4, x4 = oracle.quantize(x, axis, fid(name), scale_layout=oracle.MMA_X4, fill=0xAB, **kw)
+                kb = inner // 32
+                assert x4.size == 4 * ((outer + 127) // 128 * 128) * ((kb + 3) // 4 * 4)
+                perm = ind.mma_scale_permutation(outer, kb)            # MMA layout positions
+                atom, within = perm // 512, perm % 512
+                for j in range(4):
+                    np.testing.assert_array_equal(x4[atom * 2048 + 512 * j + within], plain.reshape(outer, kb))
+                written = np.zeros(x4.size, bool)
+                for j in range(4):
+                    written[(atom * 2048 + 512 * j + within).reshape(-1)] = True
+                assert np.all(x4[~written] == 0xAB)
+                assert np.array_equal(c_x4, c_plain)
+                y_plain = oracle.dequantize(c_plain, plain, fid(name), outer, inner, oracle.PLAIN)
+                y_x4 = oracle.dequantize(c_x4, x4, fid(name), outer, inner, oracle.MMA_X4)
+                np.testing.assert_array_equal(y_x4, y_plain)
+    assert oracle.scales_bytes(oracle.MMA_X4, 129, 32 * 5) == 4 * 256 * 8

@@ -68,11 +68,12 @@ def test_gemm_plain_and_mma_layouts_agree(oracle):
     a = rng.standard_normal((M, K)).astype(np.float32)
     b = rng.standard_normal((N, K)).astype(np.float32)
     res = []
-    for sl in (0, 1):
+    for sl in (0, 1, 2):                      # plain, MMA, MMA x4
         ac, as_ = oracle.quantize(a, 1, 0, scale_layout=sl)
         bc, bs = oracle.quantize(b, 1, 0, scale_layout=sl)
         res.append(oracle.gemm(ac, as_, 0, bc, bs, 0, M, N, K, scale_layout=sl)[0])
     np.testing.assert_array_equal(res[0], res[1])
+    np.testing.assert_array_equal(res[0], res[2])
 
 
 def test_gemm_random_close_to_fp64_of_inputs(oracle):
