@@ -53,6 +53,12 @@
  *    fastest; inside an atom the byte for row r, k-block kb is at
  *    (r % 32) * 16 + ((r / 32) % 4) * 4 + (kb % 4).  Padding bytes are never
  *    written by mx_quantize.
+ *    MX_SCALES_MMA_X4: the MMA layout with every atom stored four times in a
+ *    row, 2048 bytes per atom (the byte above at atom * 2048 + j * 512 + its
+ *    offset in the atom, j = 0..3; four times the MMA bytes).  The tensor
+ *    cores read each atom into all four 32-lane quarters of tensor memory;
+ *    with the copies already in memory the GEMM moves them with plain
+ *    128-lane copies instead of the replicating copy (mx_gemm_x4).
  */
 #ifndef MX_H
 #define MX_H
@@ -86,7 +92,7 @@ typedef enum {
     MX_SR = 1     /* stochastic rounding, see mx_quantize */
 } mx_round;
 
-typedef enum { MX_SCALES_PLAIN = 0, MX_SCALES_MMA = 1 } mx_scale_layout;
+typedef enum { MX_SCALES_PLAIN = 0, MX_SCALES_MMA = 1, MX_SCALES_MMA_X4 = 2 } mx_scale_layout;
 
 /* Optional preconditioning of each 32-block before the cast.
  * hadamard != 0: x_j <- s_j * x_j with s_j = +1 where bit j of sign_mask is
@@ -378,6 +384,28 @@ MX_API int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float 
                          const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
                          int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
                          void *stream);
+
+/*
+ * mx_gemm_x4, mx_gemm_quantize_x4 -- mx_gemm and mx_gemm_quantize with both
+ * operands' scales in MX_SCALES_MMA_X4 (mx_scales_bytes(MX_SCALES_MMA_X4, ..)
+ * bytes each) instead of MX_SCALES_MMA: the same arguments (mx_gemm_x4 has no
+ * workspace), the same results bit for bit.  They run the 256 x 256 CTA-pair
+ * kernel for every shape, whose tensor-memory scale copies are then the
+ * 128-lane shapes instead of the replicating ones: fewer copy instructions
+ * per K step (measured 9-11 % faster on the MXFP4 GEMMs of the benchmark).
+ * The quantizing form writes C's scales in out_sl, any layout (MX_SCALES_MMA_X4
+ * for a chain of such GEMMs).  The kernel-forcing debug hook accepts only the
+ * pair kernel here (MX_ERR_UNSUPPORTED otherwise).
+ */
+MX_API int mx_gemm_x4(const void *a_codes, const void *a_scales, mx_fmt fa,
+                      const void *b_codes, const void *b_scales, mx_fmt fb,
+                      int64_t M, int64_t N, int64_t K, float alpha,
+                      void *c, mx_dtype cdt, int64_t ldc, void *stream);
+MX_API int mx_gemm_quantize_x4(const void *a_codes, const void *a_scales, mx_fmt fa,
+                               const void *b_codes, const void *b_scales, mx_fmt fb,
+                               int64_t M, int64_t N, int64_t K, float alpha,
+                               mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
+                               void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream);
 
 /* Byte sizes of the buffers above (0 for invalid arguments). */
 MX_API size_t mx_codes_bytes(mx_fmt fmt, int64_t outer, int64_t inner);

@@ -27,6 +27,10 @@ int sm_count(int *device_out) {
     return g_sm_count[dev];
 }
 
+bool valid_layout(mx_scale_layout sl) {
+    return sl == MX_SCALES_PLAIN || sl == MX_SCALES_MMA || sl == MX_SCALES_MMA_X4;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
@@ -71,8 +75,9 @@ size_t mx_scales_bytes(mx_scale_layout sl, int64_t outer, int64_t inner) {
     if (outer < 0 || inner < 0 || inner % 32 != 0) return 0;
     const int64_t kb = inner / 32;
     if (sl == MX_SCALES_PLAIN) return static_cast<size_t>(outer * kb);
-    if (sl != MX_SCALES_MMA) return 0;
-    return static_cast<size_t>((outer + 127) / 128 * 128) * static_cast<size_t>((kb + 3) / 4 * 4);
+    if (sl != MX_SCALES_MMA && sl != MX_SCALES_MMA_X4) return 0;
+    return static_cast<size_t>((outer + 127) / 128 * 128) * static_cast<size_t>((kb + 3) / 4 * 4) *
+           (sl == MX_SCALES_MMA_X4 ? 4u : 1u);
 }
 
 size_t mx_gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
@@ -118,7 +123,7 @@ int quantize_impl(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64
                   mx_fmt fmt, mx_round rnd, uint64_t seed, const mx_precond *pre, const mx_shard *shard,
                   void *codes, void *scales, mx_scale_layout sl, void *stream) {
     if ((xdt != MX_F32 && xdt != MX_BF16) || elem_bits(fmt) == 0) return MX_ERR_ARG;
-    if ((rnd != MX_RNE && rnd != MX_SR) || (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA)) return MX_ERR_ARG;
+    if ((rnd != MX_RNE && rnd != MX_SR) || !valid_layout(sl)) return MX_ERR_ARG;
     if (block_axis != 0 && block_axis != 1) return MX_ERR_ARG;
     if (rows < 0 || cols < 0) return MX_ERR_ARG;
     Placement pl;
@@ -156,7 +161,7 @@ int quantize_dual_impl(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, 
                        void *codes_cols, void *scales_cols, mx_scale_layout sl, void *stream) {
     if ((xdt != MX_F32 && xdt != MX_BF16) || elem_bits(fmt) == 0) return MX_ERR_ARG;
     if ((rnd_rows != MX_RNE && rnd_rows != MX_SR) || (rnd_cols != MX_RNE && rnd_cols != MX_SR)) return MX_ERR_ARG;
-    if (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA) return MX_ERR_ARG;
+    if (!valid_layout(sl)) return MX_ERR_ARG;
     if (rows < 0 || cols < 0) return MX_ERR_ARG;
     Placement pl;
     if (int rc = place(shard, rows, cols, pl); rc != MX_OK) return rc;
@@ -260,7 +265,7 @@ int mx_quantize_nvfp4(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, i
 int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_scale_layout sl,
                   int64_t outer, int64_t inner, void *y, mx_dtype ydt, int64_t ldy, void *stream) {
     if (elem_bits(fmt) == 0 || (ydt != MX_F32 && ydt != MX_BF16)) return MX_ERR_ARG;
-    if (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA) return MX_ERR_ARG;
+    if (!valid_layout(sl)) return MX_ERR_ARG;
     if (outer < 0 || inner < 0) return MX_ERR_ARG;
     if (inner % 32 != 0) return MX_ERR_SHAPE;
     if (outer == 0 || inner == 0) return MX_OK;          // empty: pointers may be NULL
@@ -308,21 +313,14 @@ MxGemmArgs gemm_args(const void *a_codes, const void *a_scales, mx_fmt fa, const
     a.fa = fa; a.fb = fb; a.M = M; a.N = N; a.K = K; a.alpha = alpha;
     a.c = nullptr; a.cdt = MX_F32; a.ldc = 0;
     a.q_codes = nullptr; a.q_scales = nullptr; a.q_fmt = 0; a.q_rnd = MX_RNE; a.q_sl = MX_SCALES_MMA; a.q_seed = 0;
-    a.nv = false; a.enc_a = nullptr; a.enc_b = nullptr; a.a_lines = 0; a.b_lines = 0;
+    a.nv = false; a.x4 = false; a.enc_a = nullptr; a.enc_b = nullptr; a.a_lines = 0; a.b_lines = 0;
     a.num_sms = 0; a.device = 0;
     return a;
 }
 
-}  // namespace
-
-extern "C" {
-
-int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
-            const void *b_codes, const void *b_scales, mx_fmt fb,
-            int64_t M, int64_t N, int64_t K, float alpha,
-            void *c, mx_dtype cdt, int64_t ldc, void *workspace, size_t ws_bytes, void *stream) {
-    (void)workspace;
-    (void)ws_bytes;
+int gemm_impl(const void *a_codes, const void *a_scales, mx_fmt fa, const void *b_codes, const void *b_scales,
+              mx_fmt fb, int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
+              bool x4, void *stream) {
     if (elem_bits(fa) == 0 || elem_bits(fb) == 0 || (cdt != MX_F32 && cdt != MX_BF16)) return MX_ERR_ARG;
     if (M < 0 || N < 0 || K < 0) return MX_ERR_ARG;
     if (!gemm_dims_fit(M, N, K)) return MX_ERR_UNSUPPORTED;
@@ -338,19 +336,18 @@ int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
         return cudaMemset2DAsync(c, ldc * esz, 0, N * esz, M, st) == cudaSuccess ? MX_OK : MX_ERR_CUDA;
     }
     MxGemmArgs a = gemm_args(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha);
-    a.c = c; a.cdt = cdt; a.ldc = ldc;
+    a.c = c; a.cdt = cdt; a.ldc = ldc; a.x4 = x4;
     a.num_sms = sm_count(&a.device);
     if (a.num_sms <= 0) return MX_ERR_CUDA;
     return mx_launch_gemm(a, st);
 }
 
-int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa,
-                     const void *b_codes, const void *b_scales, mx_fmt fb,
-                     int64_t M, int64_t N, int64_t K, float alpha,
-                     mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
-                     void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream) {
+int gemm_quantize_impl(const void *a_codes, const void *a_scales, mx_fmt fa, const void *b_codes,
+                       const void *b_scales, mx_fmt fb, int64_t M, int64_t N, int64_t K, float alpha,
+                       mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed, void *out_codes, void *out_scales,
+                       mx_scale_layout out_sl, bool x4, void *stream) {
     if (elem_bits(fa) == 0 || elem_bits(fb) == 0 || elem_bits(out_fmt) == 0) return MX_ERR_ARG;
-    if ((out_rnd != MX_RNE && out_rnd != MX_SR) || (out_sl != MX_SCALES_PLAIN && out_sl != MX_SCALES_MMA))
+    if ((out_rnd != MX_RNE && out_rnd != MX_SR) || !valid_layout(out_sl))
         return MX_ERR_ARG;
     if (M < 0 || N < 0 || K < 0) return MX_ERR_ARG;
     if (!gemm_dims_fit(M, N, K)) return MX_ERR_UNSUPPORTED;
@@ -372,10 +369,48 @@ int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa,
     }
     MxGemmArgs a = gemm_args(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha);
     a.q_codes = out_codes; a.q_scales = out_scales; a.q_fmt = out_fmt; a.q_rnd = out_rnd; a.q_sl = out_sl;
-    a.q_seed = out_seed;
+    a.q_seed = out_seed; a.x4 = x4;
     a.num_sms = sm_count(&a.device);
     if (a.num_sms <= 0) return MX_ERR_CUDA;
     return mx_launch_gemm(a, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
+            const void *b_codes, const void *b_scales, mx_fmt fb,
+            int64_t M, int64_t N, int64_t K, float alpha,
+            void *c, mx_dtype cdt, int64_t ldc, void *workspace, size_t ws_bytes, void *stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    return gemm_impl(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha, c, cdt, ldc, false, stream);
+}
+
+int mx_gemm_x4(const void *a_codes, const void *a_scales, mx_fmt fa,
+               const void *b_codes, const void *b_scales, mx_fmt fb,
+               int64_t M, int64_t N, int64_t K, float alpha,
+               void *c, mx_dtype cdt, int64_t ldc, void *stream) {
+    return gemm_impl(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha, c, cdt, ldc, true, stream);
+}
+
+int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa,
+                     const void *b_codes, const void *b_scales, mx_fmt fb,
+                     int64_t M, int64_t N, int64_t K, float alpha,
+                     mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
+                     void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream) {
+    return gemm_quantize_impl(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha, out_fmt, out_rnd,
+                              out_seed, out_codes, out_scales, out_sl, false, stream);
+}
+
+int mx_gemm_quantize_x4(const void *a_codes, const void *a_scales, mx_fmt fa,
+                        const void *b_codes, const void *b_scales, mx_fmt fb,
+                        int64_t M, int64_t N, int64_t K, float alpha,
+                        mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
+                        void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream) {
+    return gemm_quantize_impl(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha, out_fmt, out_rnd,
+                              out_seed, out_codes, out_scales, out_sl, true, stream);
 }
 
 int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float *a_enc, int64_t a_domain_rows,

@@ -30,7 +30,7 @@ struct CastParams {
     int64_t rows, cols, ldx;
     uint8_t *codes;
     uint8_t *scales;
-    int mma_scales;      // 0 plain, 1 MMA layout
+    int mma_scales;      // scale layout: 0 plain, 1 MMA, 2 MMA x4
     int64_t k_blocks;    // blocks per output row (inner / 32)
     int64_t k_groups;    // ceil(k_blocks / 4), MMA layout
     uint32_t key;        // stochastic-rounding seed key
@@ -41,10 +41,8 @@ struct CastParams {
 
 __device__ __forceinline__ void store_scale(const CastParams &p, int64_t o, int64_t kb, uint32_t s) {
     // scale buffers are far below 4 GiB: offsets in 32-bit arithmetic
-    const uint32_t oo = static_cast<uint32_t>(o), k = static_cast<uint32_t>(kb);
-    const uint32_t off = p.mma_scales ? mma_scale_offset32(oo, k, static_cast<uint32_t>(p.k_groups))
-                                      : oo * static_cast<uint32_t>(p.k_blocks) + k;
-    p.scales[off] = static_cast<uint8_t>(s);
+    put_scale(p.scales, p.mma_scales, static_cast<uint32_t>(o), static_cast<uint32_t>(kb),
+              static_cast<uint32_t>(p.k_blocks), static_cast<uint32_t>(p.k_groups), s);
 }
 
 // ---------------------------------------------------------------------------
@@ -635,7 +633,10 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t o = i / octs_per_row, oc = i - o * octs_per_row;
         const int64_t kb = oc >> 2;
-        const uint32_t s = p.scales[p.mma_scales ? mma_scale_offset(o, kb, p.k_groups) : o * p.k_blocks + kb];
+        const int64_t so = p.mma_scales == SL_MMA_X4 ? static_cast<int64_t>(x4_scale_offset32(
+                               static_cast<uint32_t>(o), static_cast<uint32_t>(kb), static_cast<uint32_t>(p.k_groups)))
+                           : p.mma_scales == SL_MMA ? mma_scale_offset(o, kb, p.k_groups) : o * p.k_blocks + kb;
+        const uint32_t s = p.scales[so];
         uint32_t pairs[4];
         if (BITS == 8) {
             uint2 w = *reinterpret_cast<const uint2 *>(p.codes + o * p.inner + oc * 8);
@@ -816,7 +817,7 @@ cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st) {
     p.ldx = a.ldx;
     p.codes = static_cast<uint8_t *>(a.codes);
     p.scales = static_cast<uint8_t *>(a.scales);
-    p.mma_scales = a.sl == MX_SCALES_MMA;
+    p.mma_scales = a.sl;
     const int64_t inner = a.block_axis == 1 ? a.cols : a.rows;
     p.k_blocks = inner / 32;
     p.k_groups = (p.k_blocks + 3) / 4;
@@ -841,7 +842,7 @@ cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st) {
     DequantParams p;
     p.codes = static_cast<const uint8_t *>(a.codes);
     p.scales = static_cast<const uint8_t *>(a.scales);
-    p.mma_scales = a.sl == MX_SCALES_MMA;
+    p.mma_scales = a.sl;
     p.outer = a.outer;
     p.inner = a.inner;
     p.k_blocks = a.inner / 32;
@@ -876,7 +877,7 @@ cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st
     pr.rows = pc.rows = a.rows;
     pr.cols = pc.cols = a.cols;
     pr.ldx = pc.ldx = a.ldx;
-    pr.mma_scales = pc.mma_scales = a.sl == MX_SCALES_MMA;
+    pr.mma_scales = pc.mma_scales = a.sl;
     pr.codes = static_cast<uint8_t *>(a.codes_rows);
     pr.scales = static_cast<uint8_t *>(a.scales_rows);
     pr.k_blocks = a.cols / 32;

@@ -224,4 +224,27 @@ __device__ __forceinline__ uint32_t mma_scale_offset32(uint32_t o, uint32_t kb, 
     return (atom << 9) + ((o & 31u) << 4) + (((o >> 5) & 3u) << 2) + (kb & 3u);
 }
 
+// Scale layout codes of the kernels (the mx_scale_layout values).
+constexpr int SL_PLAIN = 0, SL_MMA = 1, SL_MMA_X4 = 2;
+
+// Byte offset of the first copy of (o, kb)'s scale in the x4 layout: atoms of
+// 2048 bytes, each holding the MMA atom four times.
+__device__ __forceinline__ uint32_t x4_scale_offset32(uint32_t o, uint32_t kb, uint32_t k_groups) {
+    const uint32_t atom = (o >> 7) * k_groups + (kb >> 2);
+    return (atom << 11) + ((o & 31u) << 4) + (((o >> 5) & 3u) << 2) + (kb & 3u);
+}
+
+// Writes scale byte s of (o, kb) in layout sl (plain rows of k_blocks bytes,
+// MMA atoms, or the four copies of the x4 layout).
+__device__ __forceinline__ void put_scale(uint8_t *scales, int sl, uint32_t o, uint32_t kb, uint32_t k_blocks,
+                                          uint32_t k_groups, uint32_t s) {
+    if (sl == SL_MMA_X4) {
+        const uint32_t off = x4_scale_offset32(o, kb, k_groups);
+#pragma unroll
+        for (uint32_t j = 0; j < 4; ++j) scales[off + 512u * j] = static_cast<uint8_t>(s);
+    } else {
+        scales[sl == SL_MMA ? mma_scale_offset32(o, kb, k_groups) : o * k_blocks + kb] = static_cast<uint8_t>(s);
+    }
+}
+
 }  // namespace mxk

@@ -17,7 +17,7 @@ struct BlockSink {
     int64_t inner;
     uint32_t k_blocks;   // inner / 32
     uint32_t k_groups;   // ceil(k_blocks / 4), MMA layout
-    int mma_scales;
+    int mma_scales;      // scale layout: 0 plain, 1 MMA, 2 MMA x4
     uint32_t key;        // stochastic-rounding seed key
     // stochastic-rounding position of element (row, i): sr_base + row * sr_stride + i
     // (a whole tensor: 0 and inner; a shard: its place in the whole tensor's output)
@@ -26,9 +26,8 @@ struct BlockSink {
 
 __device__ __forceinline__ void sink_scale(const BlockSink &o, int64_t row, int64_t kb, uint32_t s) {
     // scale buffers are far below 4 GiB: offsets in 32-bit arithmetic
-    const uint32_t r = static_cast<uint32_t>(row), k = static_cast<uint32_t>(kb);
-    const uint32_t off = o.mma_scales ? mma_scale_offset32(r, k, o.k_groups) : r * o.k_blocks + k;
-    o.scales[off] = static_cast<uint8_t>(s);
+    put_scale(o.scales, o.mma_scales, static_cast<uint32_t>(row), static_cast<uint32_t>(kb), o.k_blocks,
+              o.k_groups, s);
 }
 
 __device__ __forceinline__ uint64_t f2_mul_ftz(uint64_t a, uint64_t b) {

@@ -103,7 +103,7 @@ struct MxOut {
     uint8_t *scales;     // plain or MMA layout for (M, N)
     int fmt;             // element format
     int sr;              // stochastic rounding (else RNE)
-    int mma;             // MMA scale layout (else plain)
+    int mma;             // scale layout: 0 plain, 1 MMA, 2 MMA x4
     uint32_t key;        // stochastic-rounding seed key
 };
 
@@ -647,20 +647,27 @@ constexpr int PAIR_A_BYTES = 128 * BK_BYTES;             // 16 KiB per CTA per s
 // 3 to 6, 22.3 TB/s with two slices in 3 stages); the 256-column tiles of MX
 // operands take them, the tensor memory of the other configurations has no
 // room for the doubled scale columns.
-template <bool FP4, int PBN, bool NV = false> struct PairCfg {
+// X4: operand scales in the x4 layout (each 512-byte atom stored four times,
+// 2048 bytes): TMA lands the copies in the source layout of the 128-lane
+// tcgen05.cp shapes, so a stage needs three copies (MXFP4: one 128x256b for
+// A's two atoms, one 128x256b per k-group for B's two row blocks) instead of
+// six replicating 32x128b.warpx4 copies.  One slice per stage (the scale
+// bytes per stage are four times larger).
+template <bool FP4, int PBN, bool NV = false, bool X4 = false> struct PairCfg {
     static constexpr int BN = PBN;                       // tile columns (B rows)
     static constexpr int B_ROWS = PBN / 2;               // B rows per CTA
     static constexpr int B_SLICE = B_ROWS * BK_BYTES;    // B bytes per CTA per K slice
     static constexpr int ACC_BUFS = PBN == 256 ? 1 : 2;  // accumulators in tensor memory
     static constexpr uint32_t SF_COL = ACC_BUFS * PBN;   // scale factors after the accumulators
-    static constexpr int KS = (PBN == 256 && !NV) ? 2 : 1;
+    static constexpr int KS = (PBN == 256 && !NV && !X4) ? 2 : 1;
     static constexpr int G1 = NV ? 4 : (FP4 ? 2 : 1);    // scale atoms along K per slice
     static constexpr int G = KS * G1;                    // scale atoms along K per stage
-    static constexpr int STAGES = KS == 2 ? 3 : ((PBN == 192 && !FP4) ? 6 : 5);
+    static constexpr int STAGES = X4 ? (FP4 ? 4 : 5) : (KS == 2 ? 3 : ((PBN == 192 && !FP4) ? 6 : 5));
     static constexpr int A_BYTES = KS * PAIR_A_BYTES;    // per CTA per stage
     static constexpr int B_BYTES = KS * B_SLICE;
-    static constexpr int SFA_BYTES = ATOM * G;
-    static constexpr int SFB_BYTES = 2 * ATOM * G;       // both 128-row scale blocks the tile touches
+    static constexpr int ATOM_BYTES = X4 ? 4 * ATOM : ATOM;   // one atom's bytes in memory
+    static constexpr int SFA_BYTES = ATOM_BYTES * G;
+    static constexpr int SFB_BYTES = 2 * ATOM_BYTES * G; // both 128-row scale blocks the tile touches
     static constexpr int SFA_COLS = 4 * G;
     static constexpr int SFB_COLS = 8 * G;
     static constexpr int SF_STAGE_COLS = SFA_COLS + SFB_COLS;
@@ -686,6 +693,7 @@ template <bool FP4, int PBN, bool NV = false> struct PairCfg {
     static_assert(SF_COL + STAGES * SF_STAGE_COLS <= 512, "tensor memory columns");
     static_assert(SMEM <= 232448, "shared memory per block");
     static_assert(PBN == 256 || PBN == 192, "pair tile widths");
+    static_assert(!X4 || (PBN == 256 && !NV), "x4 scales: 256-column tiles of MX operands");
 };
 
 struct PairParams {
@@ -737,6 +745,16 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
         ::"r"(bar), "h"(static_cast<uint16_t>(3)) : "memory");
 }
+// x4 scales: 128 lanes x 256 bits (two 2048-byte atom copies, `lbo` bytes
+// apart, into 8 columns) or 128 lanes x 128 bits (one, into 4 columns)
+__device__ __forceinline__ void tc_cp_x4_pair_256b(uint32_t taddr, uint32_t src, uint32_t lbo) {
+    asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;"
+                 ::"r"(taddr), "l"(smem_desc(src, lbo, 128, LAYOUT_NONE)) : "memory");
+}
+__device__ __forceinline__ void tc_cp_x4_pair_128b(uint32_t taddr, uint32_t src) {
+    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;"
+                 ::"r"(taddr), "l"(smem_desc(src, 16, 128, LAYOUT_NONE)) : "memory");
+}
 __device__ __forceinline__ void tc_cp_scale_atom_pair(uint32_t taddr, uint64_t desc) {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
@@ -764,12 +782,12 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
     }
 }
 
-template <bool FP4, int OUT, int PBN, bool NV = false>
+template <bool FP4, int OUT, int PBN, bool NV = false, bool X4 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                     const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
                     const __grid_constant__ CUtensorMap tma_c, PairParams p) {
-    using C = PairCfg<FP4, PBN, NV>;
+    using C = PairCfg<FP4, PBN, NV, X4>;
     constexpr int STAGES_P = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     if (!C::SLACK && (smem_u32(smem_raw) & 1023u) != 0) {
@@ -857,14 +875,15 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                         tma_load_2d_pair(sbase + C::OFF_B + s * C::B_BYTES + q * C::B_SLICE, &tma_b,
                                          (kt + q) * BK_BYTES, nb0, fb);
                     }
-                    // scale atoms: a scale buffer is viewed as rows of 256 bytes, two per atom
+                    // scale atoms: a scale buffer is viewed as rows of 256 bytes (two per
+                    // atom; eight per x4 atom)
                     const int kg = kt * C::G1;
                     tma_load_2d_pair(sbase + C::OFF_SFA + s * C::SFA_BYTES, &tma_sfa, 0,
-                                     2 * (rb_a * p.k_groups + kg), fb);
+                                     C::ATOM_BYTES / 256 * (rb_a * p.k_groups + kg), fb);
                     tma_load_2d_pair(sbase + C::OFF_SFB + s * C::SFB_BYTES, &tma_sfb, 0,
-                                     2 * (rb_b * p.k_groups + kg), fb);
+                                     C::ATOM_BYTES / 256 * (rb_b * p.k_groups + kg), fb);
                     tma_load_2d_pair(sbase + C::OFF_SFB + s * C::SFB_BYTES + C::SFB_BYTES / 2, &tma_sfb, 0,
-                                     2 * (rb_b1 * p.k_groups + kg), fb);
+                                     C::ATOM_BYTES / 256 * (rb_b1 * p.k_groups + kg), fb);
                     if (++s == STAGES_P) { s = 0; ph ^= 1u; }
                 }
             }
@@ -902,9 +921,18 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                     const uint32_t sfb_t = sfa_t + C::SFA_COLS;
                     const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
+                    if constexpr (X4) {
+                        // A: both atoms of the slice (MXFP4) or its one atom; B: per
+                        // k-group, its two row blocks' atoms side by side
+                        if (FP4) tc_cp_x4_pair_256b(sfa_t, sfa_s, C::ATOM_BYTES);
+                        else tc_cp_x4_pair_128b(sfa_t, sfa_s);
+#pragma unroll
+                        for (int g = 0; g < C::G; ++g)
+                            tc_cp_x4_pair_256b(sfb_t + 8 * g, sfb_s + g * C::ATOM_BYTES, C::SFB_BYTES / 2);
+                    }
 #pragma unroll
                     for (int g = 0; g < C::G; ++g) {
-                        if (g < ns * C::G1) {
+                        if (!X4 && g < ns * C::G1) {
                             tc_cp_scale_atom_pair(sfa_t + 4 * g, scale_atom_desc(sfa_s + g * ATOM));
 #pragma unroll
                             for (int h = 0; h < 2; ++h)
@@ -1168,12 +1196,12 @@ cudaError_t launch_overlapped(Kern kern, int grid, int smem, cudaStream_t st, co
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <bool FP4, int OUT, int PBN, bool NV = false>
+template <bool FP4, int OUT, int PBN, bool NV = false, bool X4 = false>
 cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
                         const CUtensorMap &tsb, const CUtensorMap &tc, const PairParams &p, int grid,
                         cudaStream_t st) {
-    auto kern = mx_gemm_pair_kernel<FP4, OUT, PBN, NV>;
-    constexpr int smem = PairCfg<FP4, PBN, NV>::SMEM;
+    auto kern = mx_gemm_pair_kernel<FP4, OUT, PBN, NV, X4>;
+    constexpr int smem = PairCfg<FP4, PBN, NV, X4>::SMEM;
     static std::atomic<uint64_t> configured{0};   // per instantiation, one bit per device
     if (cudaError_t e = ensure_smem_limit(kern, smem, configured); e != cudaSuccess) return e;
     return launch_overlapped(kern, grid, smem, st, ta, tb, tsa, tsb, tc, p);
@@ -1215,7 +1243,7 @@ MxOut mx_out(const MxGemmArgs &a) {
     q.scales = static_cast<uint8_t *>(a.q_scales);
     q.fmt = a.q_fmt;
     q.sr = a.q_rnd == MX_SR;
-    q.mma = a.q_sl == MX_SCALES_MMA;
+    q.mma = a.q_sl;
     q.key = fmix32_host(static_cast<uint32_t>(a.q_seed)) ^ static_cast<uint32_t>(a.q_seed >> 32);
     return q;
 }
@@ -1267,18 +1295,21 @@ int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
     const bool fp4 = a.nv || use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;     // K bytes of a uint8 stage view
     // scale atoms one stage's boxes cover: per 128-byte K slice, times the
-    // slices per stage (PairCfg::KS: two on 256-column tiles of MX operands)
-    const int G = (a.nv ? 4 : (fp4 ? 2 : 1)) * ((pbn == 256 && !a.nv) ? 2 : 1);
+    // slices per stage (PairCfg::KS: two on 256-column tiles of MX operands
+    // with MMA-layout scales); a box row is 256 bytes, two per atom, eight
+    // per x4 atom
+    const int G = (a.nv ? 4 : (fp4 ? 2 : 1)) * ((pbn == 256 && !a.nv && !a.x4) ? 2 : 1);
+    const int box_atoms = a.x4 ? 4 * G : G;
     // scale atoms along K: four blocks each, of 32 elements (MX) or 16 (NVFP4)
     const int64_t k_groups = a.nv ? a.K / 64 : a.K / 128;
     CUtensorMap ta, tb, tsa, tsb, tc;
     if (!make_c_map(&tc, a)) return MX_ERR_CUDA;
     if (!make_operand_map(&ta, a.a_codes, a.M, a.K, a.fa, fp4, 128)) return MX_ERR_CUDA;
     if (!make_operand_map(&tb, a.b_codes, a.N, a.K, a.fb, fp4, pbn / 2)) return MX_ERR_CUDA;
-    const int64_t sa_bytes = (a.M + 127) / 128 * 128 * k_groups * 4;
-    const int64_t sb_bytes = (a.N + 127) / 128 * 128 * k_groups * 4;
-    if (!make_scale_map(&tsa, a.a_scales, sa_bytes, G)) return MX_ERR_CUDA;
-    if (!make_scale_map(&tsb, a.b_scales, sb_bytes, G)) return MX_ERR_CUDA;
+    const int64_t sa_bytes = (a.M + 127) / 128 * 128 * k_groups * 4 * (a.x4 ? 4 : 1);
+    const int64_t sb_bytes = (a.N + 127) / 128 * 128 * k_groups * 4 * (a.x4 ? 4 : 1);
+    if (!make_scale_map(&tsa, a.a_scales, sa_bytes, box_atoms)) return MX_ERR_CUDA;
+    if (!make_scale_map(&tsb, a.b_scales, sb_bytes, box_atoms)) return MX_ERR_CUDA;
     PairParams p;
     p.c = a.c;
     p.ldc = a.ldc;
@@ -1305,7 +1336,16 @@ int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
     cudaError_t e;
     p.q = mx_out(a);
     const int out = out_mode(a);
-    if (a.nv) {
+    if (a.x4) {
+        if (pbn != 256 || a.nv) return MX_ERR_UNSUPPORTED;
+        if (out == OUT_MX) e = fp4 ? launch_pair<true, OUT_MX, 256, false, true>(ta, tb, tsa, tsb, tc, p, grid, st)
+                                   : launch_pair<false, OUT_MX, 256, false, true>(ta, tb, tsa, tsb, tc, p, grid, st);
+        else if (out == OUT_BF16)
+            e = fp4 ? launch_pair<true, OUT_BF16, 256, false, true>(ta, tb, tsa, tsb, tc, p, grid, st)
+                    : launch_pair<false, OUT_BF16, 256, false, true>(ta, tb, tsa, tsb, tc, p, grid, st);
+        else e = fp4 ? launch_pair<true, OUT_F32, 256, false, true>(ta, tb, tsa, tsb, tc, p, grid, st)
+                     : launch_pair<false, OUT_F32, 256, false, true>(ta, tb, tsa, tsb, tc, p, grid, st);
+    } else if (a.nv) {
         if (pbn != 256 || out == OUT_MX) return MX_ERR_UNSUPPORTED;
         e = out == OUT_BF16 ? launch_pair<true, OUT_BF16, 256, true>(ta, tb, tsa, tsb, tc, p, grid, st)
                             : launch_pair<true, OUT_F32, 256, true>(ta, tb, tsa, tsb, tc, p, grid, st);
@@ -1334,6 +1374,11 @@ int pair_tile_n(const MxGemmArgs &a) {
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     using namespace mxg;
     if (a.nv) return launch_gemm_pair(a, 256, st);   // NVFP4 runs on the CTA-pair kernel only
+    if (a.x4) {
+        // x4 scales: the 256-column pair kernel only (any shape)
+        if (g_force_kernel >= 0 && g_force_kernel != 256) return MX_ERR_UNSUPPORTED;
+        return launch_gemm_pair(a, 256, st);
+    }
     if (const int pbn = pair_tile_n(a); pbn != 0) return launch_gemm_pair(a, pbn, st);
     const bool fp4 = use_mxf4(a);
     const int64_t k_bytes = fp4 ? a.K / 2 : a.K;

@@ -81,6 +81,7 @@ struct MxGemmArgs {
     // NVFP4 operands (mx_gemm_nvfp4): E2M1 codes with 16-element E4M3 blocks
     // and per-domain fp32 encode scales; a_lines / b_lines rows per domain (0: one)
     bool nv;
+    bool x4;                   // operand scales in MX_SCALES_MMA_X4
     const float *enc_a, *enc_b;
     int64_t a_lines, b_lines;
     int num_sms;

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libmx.so")
 FMT = {"e4m3": 0, "e5m2": 1, "e2m3": 2, "e3m2": 3, "e2m1": 4, "int8": 5}
 FMT_BITS = {0: 8, 1: 8, 2: 6, 3: 6, 4: 4, 5: 8}
 ROUND = {"rne": 0, "sr": 1}
-LAYOUT = {"plain": 0, "mma": 1}
+LAYOUT = {"plain": 0, "mma": 1, "mma_x4": 2}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 DEFAULT_SIGN_MASK = 0x6A09E667
 
@@ -90,6 +90,11 @@ def lib() -> ctypes.CDLL:
             L.mx_gemm_nvfp4.restype = i32
             L.mx_gemm_nvfp4.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float,
                                         vp, i32, i64, vp]
+            L.mx_gemm_x4.restype = i32
+            L.mx_gemm_x4.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, ctypes.c_float, vp, i32, i64, vp]
+            L.mx_gemm_quantize_x4.restype = i32
+            L.mx_gemm_quantize_x4.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, ctypes.c_float,
+                                              i32, i32, u64, vp, vp, i32, vp]
             L.mx_gemm_quantize.restype = i32
             L.mx_gemm_quantize.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, ctypes.c_float,
                                            i32, i32, u64, vp, vp, i32, vp]
@@ -268,15 +273,23 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, fmt, outer: int, inner
 
 def gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
          b_scales: torch.Tensor, M: int, N: int, K: int, fa="e4m3", fb=None, alpha: float = 1.0,
-         out_dtype=torch.bfloat16, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """C = alpha * A * B^T on MX operands quantized along K (MMA scale layout)."""
+         out_dtype=torch.bfloat16, out: torch.Tensor | None = None, stream=None,
+         scale_layout="mma") -> torch.Tensor:
+    """C = alpha * A * B^T on MX operands quantized along K; scale_layout is the
+    operands' scale layout, "mma" (mx_gemm) or "mma_x4" (mx_gemm_x4)."""
     fb = fa if fb is None else fb
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=a_codes.device)
-    rc = lib().mx_gemm(a_codes.data_ptr(), a_scales.data_ptr(), _fmt(fa),
-                       b_codes.data_ptr(), b_scales.data_ptr(), _fmt(fb), M, N, K, float(alpha),
-                       out.data_ptr(), DTYPE[out.dtype], out.stride(0), None, 0, _stream(stream))
-    _check(rc, "mx_gemm")
+    args = (a_codes.data_ptr(), a_scales.data_ptr(), _fmt(fa), b_codes.data_ptr(), b_scales.data_ptr(), _fmt(fb),
+            M, N, K, float(alpha), out.data_ptr(), DTYPE[out.dtype], out.stride(0))
+    if _layout(scale_layout) == LAYOUT["mma_x4"]:
+        rc = lib().mx_gemm_x4(*args, _stream(stream))
+        _check(rc, "mx_gemm_x4")
+    elif _layout(scale_layout) == LAYOUT["mma"]:
+        rc = lib().mx_gemm(*args, None, 0, _stream(stream))
+        _check(rc, "mx_gemm")
+    else:
+        raise ValueError("GEMM operand scales are in the mma or mma_x4 layout")
     return out
 
 
@@ -297,7 +310,8 @@ def gemm_nvfp4(a, b, M: int, N: int, K: int, a_domain_rows: int = 0, b_domain_ro
 
 def gemm_quantize(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
                   b_scales: torch.Tensor, M: int, N: int, K: int, fa="e4m3", fb=None, alpha: float = 1.0,
-                  out_fmt="e4m3", rnd="rne", seed: int = 0, scale_layout="mma", out=None, stream=None):
+                  out_fmt="e4m3", rnd="rne", seed: int = 0, scale_layout="mma", out=None, stream=None,
+                  operand_layout="mma"):
     """alpha * A * B^T quantized along its rows in the GEMM epilogue.
 
     Returns (codes, scales): M x (N * bits / 8) codes and the scales of an
@@ -310,11 +324,14 @@ def gemm_quantize(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.
         out = (torch.empty((M, codes_row_bytes(of, N)), dtype=torch.uint8, device=dev),
                torch.empty(max(scales_bytes(sl, M, N), 1), dtype=torch.uint8, device=dev))
     codes, scales = out
-    rc = lib().mx_gemm_quantize(a_codes.data_ptr(), a_scales.data_ptr(), _fmt(fa), b_codes.data_ptr(),
-                                b_scales.data_ptr(), _fmt(fb), M, N, K, float(alpha), of,
-                                ROUND[rnd] if isinstance(rnd, str) else int(rnd), seed & (2**64 - 1),
-                                codes.data_ptr(), scales.data_ptr(), sl, _stream(stream))
-    _check(rc, "mx_gemm_quantize")
+    fn = {LAYOUT["mma"]: "mx_gemm_quantize", LAYOUT["mma_x4"]: "mx_gemm_quantize_x4"}.get(_layout(operand_layout))
+    if fn is None:
+        raise ValueError("GEMM operand scales are in the mma or mma_x4 layout")
+    rc = getattr(lib(), fn)(a_codes.data_ptr(), a_scales.data_ptr(), _fmt(fa), b_codes.data_ptr(),
+                            b_scales.data_ptr(), _fmt(fb), M, N, K, float(alpha), of,
+                            ROUND[rnd] if isinstance(rnd, str) else int(rnd), seed & (2**64 - 1),
+                            codes.data_ptr(), scales.data_ptr(), sl, _stream(stream))
+    _check(rc, fn)
     return codes, scales
 
 

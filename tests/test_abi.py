@@ -58,7 +58,7 @@ def test_sizes_agree_with_oracle(mx, oracle, fmt, outer, inner):
 def test_sizes_reject_bad_shapes(mx):
     assert mx.codes_bytes(0, 4, 33) == 0
     assert mx.codes_bytes(9, 4, 32) == 0
-    assert mx.scales_bytes(2, 4, 32) == 0
+    assert mx.scales_bytes(3, 4, 32) == 0
 
 
 def _q(mx, x=16, dt=1, rows=64, cols=64, ldx=64, axis=1, fmt=0, rnd=0, codes=16, scales=16,
@@ -167,7 +167,7 @@ def _gq(mx, M=128, N=128, K=256, fa=0, fb=0, of=0, rnd=0, codes=16, scales=16, s
 def test_gemm_quantize_validation(mx):
     assert _gq(mx, of=6) == -1
     assert _gq(mx, rnd=5) == -1
-    assert _gq(mx, sl=2) == -1
+    assert _gq(mx, sl=3) == -1
     assert _gq(mx, M=-1) == -1
     assert _gq(mx, N=48) == -3                    # C's blocks run along N
     assert _gq(mx, K=48) == -3
@@ -250,3 +250,20 @@ def test_nvfp4_gemm_validation(mx):
     assert call(M=1 << 31) == -4                # past 32-bit indexing
     assert L.mx_gemm_nvfp4(None, None, None, 0, None, None, None, 0, 0, 256, 512, 1.0, None, 1, 256,
                            None) == 0          # empty
+
+
+def test_x4_layout_sizes_and_entries(mx):
+    """The x4 scale layout's sizes, its acceptance by the casts' checks and its
+    refusal by the NVFP4 cast; the x4 GEMM entries validate like mx_gemm."""
+    L = mx.lib()
+    assert L.mx_scales_bytes(2, 129, 32 * 5) == 4 * L.mx_scales_bytes(1, 129, 32 * 5)
+    assert L.mx_scales_bytes(3, 128, 128) == 0
+    assert L.mx_quantize_nvfp4(16, 1, 64, 64, 64, 0, 16, 16, 2, 16, None) == -1
+    # empty casts and GEMMs are no-ops for the x4 layout as for the others
+    assert L.mx_quantize(None, 1, 0, 64, 64, 1, 0, 0, 0, None, None, None, 2, None) == 0
+    assert L.mx_gemm_x4(None, None, 0, None, None, 0, 0, 64, 128, 1.0, None, 0, 64, None) == 0
+    # argument checks before any launch
+    assert L.mx_gemm_x4(16, 16, 0, 16, 16, 0, 128, 128, 100, 1.0, 16, 0, 128, None) == -3     # K % 32
+    assert L.mx_gemm_x4(16, 16, 5, 16, 16, 0, 128, 128, 128, 1.0, 16, 0, 128, None) == -4     # INT8
+    assert L.mx_gemm_x4(16, 16, 0, 16, 16, 0, 128, 128, 128, 1.0, 24, 0, 128, None) == -2     # C alignment
+    assert L.mx_gemm_quantize_x4(16, 16, 0, 16, 16, 0, 128, 100, 128, 1.0, 0, 0, 0, 16, 16, 2, None) == -3
