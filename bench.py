@@ -500,6 +500,9 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         return None
     shapes = I.LLAMA3_GEMMS if fmt == "e2m1" else I.GPT2_GEMMS
     cfg_index = 3 if fmt == "e2m1" else 2
+    # MXFP4 operands carry x4 scales (the pair kernel's cheaper scale copies);
+    # the short-K MXFP8 shapes keep the MMA layout and the one-SM kernel
+    sl = "mma_x4" if fmt == "e2m1" else "mma"
     ops = []
     for idx, (M, N, K) in enumerate(shapes):
         if fmt == "e2m1" and str(idx) not in args.gemm_shapes.split(","):
@@ -507,14 +510,14 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         xb, wb = I.linear_operands(M, K, N, cfg_index, stream=idx)
         x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
         w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
-        ac, as_ = mx.quantize(x, 1, fmt)
-        bc, bs = mx.quantize(w, 1, fmt)
+        ac, as_ = mx.quantize(x, 1, fmt, scale_layout=sl)
+        bc, bs = mx.quantize(w, 1, fmt, scale_layout=sl)
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ops.append((M, N, K, ac, as_, bc, bs, c))
         del x, w
     try:
         M, N, K, ac, as_, bc, bs, c = ops[0]
-        mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
+        mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c, scale_layout=sl)
     except mx.MxError as e:
         if e.status == -4:
             return None
@@ -522,7 +525,7 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
     flops_step = sum(2.0 * M * N * K for (M, N, K, *_r) in ops)
     for _ in range(args.warmup):
         for (M, N, K, ac, as_, bc, bs, c) in ops:
-            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c, scale_layout=sl)
     torch.cuda.synchronize()
 
     def timed_region(body, n):
@@ -539,7 +542,7 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
 
     def step(i):
         for (M, N, K, ac, as_, bc, bs, c) in ops:
-            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c, scale_layout=sl)
 
     ms = timed_region(step, args.steps)
     launches = len(ops) * args.steps
@@ -548,12 +551,12 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
     n_shape = max(3, min(args.steps, 200))
     for (M, N, K, ac, as_, bc, bs, c) in ops:
         def one(i, M=M, N=N, K=K, ac=ac, as_=as_, bc=bc, bs=bs, c=c):
-            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
+            mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c, scale_layout=sl)
         us = 1e3 * timed_region(one, n_shape) / n_shape
         launches += n_shape
         per_shape[f"{M}x{N}x{K}"] = {"us": round(us, 1), "tflops": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 1)}
     traffic = None
-    t_shape = {k: measured_traffic("gemm", f"{fmt}_{k}") for k in per_shape}
+    t_shape = {k: measured_traffic("gemm", f"{fmt}_{'x4_' if sl == 'mma_x4' else ''}{k}") for k in per_shape}
     if all(v is not None for v in t_shape.values()):
         traffic = round(statistics.mean(t_shape.values()))
         for k in per_shape:
@@ -571,9 +574,10 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         for label in ("gemm_then_cast", "fused"):
             def once(label=label, M=M, N=N, K=K, ac=ac, as_=as_, bc=bc, bs=bs, c=c, qc=qc, qs=qs):
                 if label == "fused":
-                    mx.gemm_quantize(ac, as_, bc, bs, M, N, K, fa=fmt, out_fmt=fmt, out=(qc, qs))
+                    mx.gemm_quantize(ac, as_, bc, bs, M, N, K, fa=fmt, out_fmt=fmt, out=(qc, qs),
+                                     operand_layout=sl)
                 else:
-                    mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c)
+                    mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c, scale_layout=sl)
                     mx.quantize(c, 1, fmt, codes=qc, scales=qs)
             for _ in range(args.warmup):
                 once()
@@ -594,8 +598,9 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
     ratio = 4.0 if fmt == "e2m1" else 2.0             # nominal fp4 : fp8 : bf16 = 9 : 4.5 : 2.25
     peak = ratio * float(peaks["bf16_tflops"])
     if fmt == "e2m1":
-        workload = "llama3_8b_mxfp4_gemms_m8192 (4096->6144, 4096->14336, 14336->4096), bf16 out"
-        kernel = "mx_gemm_pair_kernel (cta_group::2, kind::mxf4)"
+        workload = ("llama3_8b_mxfp4_gemms_m8192 (4096->6144, 4096->14336, 14336->4096), bf16 out, "
+                    "x4 operand scales")
+        kernel = "mx_gemm_pair_kernel (cta_group::2, kind::mxf4, x4 scales)"
     else:
         workload = "gpt2_small_mxfp8_gemms_m8192 (768->3072, 3072->768), bf16 out"
         kernel = "mx_gemm_kernel (cta_group::1, kind::mxf8f6f4; short K / few tiles)"
@@ -624,13 +629,17 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
     x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
     del dyb, xb
     ac = torch.empty((Do, T // 2), dtype=torch.uint8, device=dev)
-    as_ = torch.empty(mx.scales_bytes("mma", Do, T), dtype=torch.uint8, device=dev)
+    as_ = torch.empty(mx.scales_bytes("mma_x4", Do, T), dtype=torch.uint8, device=dev)
     bc = torch.empty((Di, T // 2), dtype=torch.uint8, device=dev)
-    bs = torch.empty(mx.scales_bytes("mma", Di, T), dtype=torch.uint8, device=dev)
+    bs = torch.empty(mx.scales_bytes("mma_x4", Di, T), dtype=torch.uint8, device=dev)
     dw = torch.empty((Do, Di), dtype=torch.float32, device=dev)
-    ops = {"cast_dY": lambda: mx.quantize(dy, 0, "e2m1", rnd="sr", seed=42, hadamard=True, codes=ac, scales=as_),
-           "cast_X": lambda: mx.quantize(x, 0, "e2m1", rnd="sr", seed=43, hadamard=True, codes=bc, scales=bs),
-           "gemm_dW": lambda: mx.gemm(ac, as_, bc, bs, Do, Di, T, fa="e2m1", alpha=1.0 / 32, out=dw)}
+    # x4 scales for the dW GEMM (the pair kernel's cheaper scale copies)
+    ops = {"cast_dY": lambda: mx.quantize(dy, 0, "e2m1", rnd="sr", seed=42, hadamard=True, codes=ac, scales=as_,
+                                          scale_layout="mma_x4"),
+           "cast_X": lambda: mx.quantize(x, 0, "e2m1", rnd="sr", seed=43, hadamard=True, codes=bc, scales=bs,
+                                         scale_layout="mma_x4"),
+           "gemm_dW": lambda: mx.gemm(ac, as_, bc, bs, Do, Di, T, fa="e2m1", alpha=1.0 / 32, out=dw,
+                                      scale_layout="mma_x4")}
 
     def timed(fn, n):
         barrier()
@@ -660,14 +669,14 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
     fp4_peak = 4.0 * float(peaks["bf16_tflops"])
     hbm = float(peaks["hbm_gbs"])
     out = {"workload": "wgrad_mxfp4 dY 16384x4096, X 16384x14336 (Student-t), Hadamard+SR along tokens, "
-                       "dW fp32", "steps": steps, "ms_per_step": round(ms / steps, 4)}
+                       "x4 scales, dW fp32", "steps": steps, "ms_per_step": round(ms / steps, 4)}
     values = {"cast_dY": T * Do, "cast_X": T * Di}
     shape = {"cast_dY": f"{T}x{Do}", "cast_X": f"{T}x{Di}"}
     for k in ("cast_dY", "cast_X"):
         gbs = cast_bytes[k] / (us[k] * 1e-6) / 1e9
         hbm_us = cast_bytes[k] / (hbm * 1e9) * 1e6
         out[k] = {"us": round(us[k], 1), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
-        ipv = measured_instr("cast_cols_had_sr", f"e2m1_bf16_{shape[k]}")
+        ipv = measured_instr("cast_cols_had_sr", f"e2m1_bf16_x4_{shape[k]}")
         if ipv is not None:
             alu_us = issue_bound_us(ipv, values[k], sms, sm_mhz)
             out[k]["alu"] = {"warp_instr_per_value": round(ipv, 4), "bound_us": round(alu_us, 1), "sm_mhz": sm_mhz,
@@ -677,7 +686,7 @@ def run_wgrad_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
                                   "frac": round(max(alu_us, hbm_us) / us[k], 4)}
     tf = flops / (us["gemm_dW"] * 1e-6) / 1e12
     out["gemm_dW"] = {"us": round(us["gemm_dW"], 1), "tflops": round(tf, 1), "frac": round(tf / fp4_peak, 4),
-                      "peak": round(fp4_peak, 1), "traffic": measured_traffic("gemm", f"e2m1_{Do}x{Di}x{T}")}
+                      "peak": round(fp4_peak, 1), "traffic": measured_traffic("gemm", f"e2m1_x4_{Do}x{Di}x{T}")}
     return out
 
 
