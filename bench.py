@@ -789,8 +789,8 @@ def run_nvfp4_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
         return max_over_ranks(1e3 * e0.elapsed_time(e1) / n)
 
     out = {"workload": "nvfp4: cast of a Llama-3-8B activation 8192x4096 bf16 (global, and CTA-local "
-                       f"domains of {local_rows} rows); Llama-3-8B GEMMs M=8192 on NVFP4 operands "
-                       "(activations CTA-local, weights global), bf16 out", "steps": steps}
+                       f"domains of {local_rows} rows), MMA scale layout; Llama-3-8B GEMMs M=8192 on NVFP4 "
+                       "operands (activations CTA-local, weights global, x4 scales), bf16 out", "steps": steps}
     # cast: inputs rotate over three device copies (> L2)
     xb, _ = I.linear_operands(8192, 4096, 128, 3, stream=0)
     xs = [torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev) for _ in range(N_ROTATE)]
@@ -821,13 +821,13 @@ def run_nvfp4_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
         xb, wb = I.linear_operands(M, K, N, 3, stream=idx)
         x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
         w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
-        a = mx.quantize_nvfp4(x, local_rows)
-        b = mx.quantize_nvfp4(w, 0)
+        a = mx.quantize_nvfp4(x, local_rows, scale_layout="mma_x4")
+        b = mx.quantize_nvfp4(w, 0, scale_layout="mma_x4")
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         del x, w
 
         def g(a=a, b=b, c=c, M=M, N=N, K=K):
-            mx.gemm_nvfp4(a, b, M, N, K, local_rows, 0, out=c)
+            mx.gemm_nvfp4(a, b, M, N, K, local_rows, 0, out=c, scale_layout="mma_x4")
         for _ in range(args.warmup):
             g()
         us = timed(g, steps)
@@ -837,7 +837,7 @@ def run_nvfp4_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks
         total_us += us
         tf = fl / (us * 1e-6) / 1e12
         gemm[f"{M}x{N}x{K}"] = {"us": round(us, 1), "tflops": round(tf, 1), "frac": round(tf / fp4_peak, 4)}
-    out["gemm"] = {"kernel": "mx_gemm_pair_kernel (cta_group::2, kind::mxf4nvf4, scale_vec::4X)",
+    out["gemm"] = {"kernel": "mx_gemm_pair_kernel (cta_group::2, kind::mxf4nvf4, scale_vec::4X, x4 scales)",
                    "per_shape": gemm, "tflops": round(total_flops / (total_us * 1e-6) / 1e12, 1),
                    "peak": round(fp4_peak, 1),
                    "peak_kind": f"{peak_kind} bf16 burst x 4 (nominal ratio for FP4 operands)"}

@@ -261,8 +261,8 @@ MX_API int mx_quantize_dual_shard(const void *x, mx_dtype xdt, int64_t rows, int
  *  codes      device, rows x cols / 2 bytes (two codes per byte, even element
  *             in the low nibble), 16-byte aligned.
  *  scales     device, mx_nvfp4_scales_bytes(sl, rows, cols) bytes: plain
- *             (rows x cols / 16) or the tensor-core atom layout of
- *             MX_SCALES_MMA over 16-element blocks.
+ *             (rows x cols / 16), or the tensor-core atom layout of
+ *             MX_SCALES_MMA (or MX_SCALES_MMA_X4) over 16-element blocks.
  *  enc_scales device, mx_nvfp4_domains(rows, domain_rows) fp32 values: E of
  *             each domain (written; the global form also uses it while it
  *             runs, starting from zero).
@@ -384,6 +384,15 @@ MX_API int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float 
                          const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
                          int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
                          void *stream);
+
+/* mx_gemm_nvfp4 with both operands' block scales in MX_SCALES_MMA_X4
+ * (mx_nvfp4_scales_bytes(MX_SCALES_MMA_X4, ..) bytes, written by
+ * mx_quantize_nvfp4 with that layout): the same results bit for bit, with
+ * the 128-lane scale copies (six per 256-element slice instead of twelve). */
+MX_API int mx_gemm_nvfp4_x4(const void *a_codes, const void *a_scales, const float *a_enc, int64_t a_domain_rows,
+                            const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
+                            int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
+                            void *stream);
 
 /*
  * mx_gemm_x4, mx_gemm_quantize_x4 -- mx_gemm and mx_gemm_quantize with both

@@ -245,7 +245,7 @@ int64_t mx_nvfp4_domains(int64_t rows, int64_t domain_rows) {
 int mx_quantize_nvfp4(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, int64_t domain_rows,
                       void *codes, void *scales, mx_scale_layout sl, float *enc_scales, void *stream) {
     if (xdt != MX_F32 && xdt != MX_BF16) return MX_ERR_ARG;
-    if (sl != MX_SCALES_PLAIN && sl != MX_SCALES_MMA) return MX_ERR_ARG;
+    if (!valid_layout(sl)) return MX_ERR_ARG;
     if (rows < 0 || cols < 0 || domain_rows < 0) return MX_ERR_ARG;
     if (cols % 16 != 0) return MX_ERR_SHAPE;
     if (rows == 0 || cols == 0) return MX_OK;             // empty: pointers may be NULL
@@ -413,10 +413,14 @@ int mx_gemm_quantize_x4(const void *a_codes, const void *a_scales, mx_fmt fa,
                               out_seed, out_codes, out_scales, out_sl, true, stream);
 }
 
-int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float *a_enc, int64_t a_domain_rows,
-                  const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
-                  int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
-                  void *stream) {
+}  // extern "C"
+
+namespace {
+
+int gemm_nvfp4_impl(const void *a_codes, const void *a_scales, const float *a_enc, int64_t a_domain_rows,
+                    const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
+                    int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc, bool x4,
+                    void *stream) {
     if (cdt != MX_F32 && cdt != MX_BF16) return MX_ERR_ARG;
     if (M < 0 || N < 0 || K < 0 || a_domain_rows < 0 || b_domain_rows < 0) return MX_ERR_ARG;
     if (!gemm_dims_fit(M, N, K)) return MX_ERR_UNSUPPORTED;
@@ -436,12 +440,32 @@ int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float *a_enc,
         return MX_ERR_ALIGN;
     MxGemmArgs a = gemm_args(a_codes, a_scales, MX_E2M1, b_codes, b_scales, MX_E2M1, M, N, K, alpha);
     a.c = c; a.cdt = cdt; a.ldc = ldc;
-    a.nv = true; a.enc_a = a_enc; a.enc_b = b_enc;
+    a.nv = true; a.x4 = x4; a.enc_a = a_enc; a.enc_b = b_enc;
     a.a_lines = a_domain_rows >= M ? 0 : a_domain_rows;   // a domain covering every row: one domain
     a.b_lines = b_domain_rows >= N ? 0 : b_domain_rows;
     a.num_sms = sm_count(&a.device);
     if (a.num_sms <= 0) return MX_ERR_CUDA;
     return mx_launch_gemm(a, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float *a_enc, int64_t a_domain_rows,
+                  const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
+                  int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
+                  void *stream) {
+    return gemm_nvfp4_impl(a_codes, a_scales, a_enc, a_domain_rows, b_codes, b_scales, b_enc, b_domain_rows, M, N,
+                           K, alpha, c, cdt, ldc, false, stream);
+}
+
+int mx_gemm_nvfp4_x4(const void *a_codes, const void *a_scales, const float *a_enc, int64_t a_domain_rows,
+                     const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
+                     int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
+                     void *stream) {
+    return gemm_nvfp4_impl(a_codes, a_scales, a_enc, a_domain_rows, b_codes, b_scales, b_enc, b_domain_rows, M, N,
+                           K, alpha, c, cdt, ldc, true, stream);
 }
 
 int mx_last_device_status(void *stream) {

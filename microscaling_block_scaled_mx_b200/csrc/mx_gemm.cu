@@ -662,7 +662,7 @@ template <bool FP4, int PBN, bool NV = false, bool X4 = false> struct PairCfg {
     static constexpr int KS = (PBN == 256 && !NV && !X4) ? 2 : 1;
     static constexpr int G1 = NV ? 4 : (FP4 ? 2 : 1);    // scale atoms along K per slice
     static constexpr int G = KS * G1;                    // scale atoms along K per stage
-    static constexpr int STAGES = X4 ? (FP4 ? 4 : 5) : (KS == 2 ? 3 : ((PBN == 192 && !FP4) ? 6 : 5));
+    static constexpr int STAGES = X4 ? (NV ? 3 : (FP4 ? 4 : 5)) : (KS == 2 ? 3 : ((PBN == 192 && !FP4) ? 6 : 5));
     static constexpr int A_BYTES = KS * PAIR_A_BYTES;    // per CTA per stage
     static constexpr int B_BYTES = KS * B_SLICE;
     static constexpr int ATOM_BYTES = X4 ? 4 * ATOM : ATOM;   // one atom's bytes in memory
@@ -693,7 +693,7 @@ template <bool FP4, int PBN, bool NV = false, bool X4 = false> struct PairCfg {
     static_assert(SF_COL + STAGES * SF_STAGE_COLS <= 512, "tensor memory columns");
     static_assert(SMEM <= 232448, "shared memory per block");
     static_assert(PBN == 256 || PBN == 192, "pair tile widths");
-    static_assert(!X4 || (PBN == 256 && !NV), "x4 scales: 256-column tiles of MX operands");
+    static_assert(!X4 || PBN == 256, "x4 scales: 256-column tiles");
 };
 
 struct PairParams {
@@ -922,10 +922,15 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_cons
                     const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
                     if constexpr (X4) {
-                        // A: both atoms of the slice (MXFP4) or its one atom; B: per
+                        // A: the slice's atoms two per copy (one for MXFP8); B: per
                         // k-group, its two row blocks' atoms side by side
-                        if (FP4) tc_cp_x4_pair_256b(sfa_t, sfa_s, C::ATOM_BYTES);
-                        else tc_cp_x4_pair_128b(sfa_t, sfa_s);
+                        if (FP4) {
+#pragma unroll
+                            for (int i = 0; i < C::G / 2; ++i)
+                                tc_cp_x4_pair_256b(sfa_t + 8 * i, sfa_s + 2 * i * C::ATOM_BYTES, C::ATOM_BYTES);
+                        } else {
+                            tc_cp_x4_pair_128b(sfa_t, sfa_s);
+                        }
 #pragma unroll
                         for (int g = 0; g < C::G; ++g)
                             tc_cp_x4_pair_256b(sfb_t + 8 * g, sfb_s + g * C::ATOM_BYTES, C::SFB_BYTES / 2);
@@ -1336,8 +1341,12 @@ int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
     cudaError_t e;
     p.q = mx_out(a);
     const int out = out_mode(a);
-    if (a.x4) {
-        if (pbn != 256 || a.nv) return MX_ERR_UNSUPPORTED;
+    if (a.x4 && a.nv) {
+        if (pbn != 256 || out == OUT_MX) return MX_ERR_UNSUPPORTED;
+        e = out == OUT_BF16 ? launch_pair<true, OUT_BF16, 256, true, true>(ta, tb, tsa, tsb, tc, p, grid, st)
+                            : launch_pair<true, OUT_F32, 256, true, true>(ta, tb, tsa, tsb, tc, p, grid, st);
+    } else if (a.x4) {
+        if (pbn != 256) return MX_ERR_UNSUPPORTED;
         if (out == OUT_MX) e = fp4 ? launch_pair<true, OUT_MX, 256, false, true>(ta, tb, tsa, tsb, tc, p, grid, st)
                                    : launch_pair<false, OUT_MX, 256, false, true>(ta, tb, tsa, tsb, tc, p, grid, st);
         else if (out == OUT_BF16)

@@ -41,7 +41,7 @@ struct NvParams {
     int64_t rows, cols, ldx;
     uint8_t *codes;
     uint8_t *scales;
-    int mma;               // MMA scale layout (else plain)
+    int mma;               // scale layout: 0 plain, 1 MMA, 2 MMA x4
     uint32_t k_blocks;     // cols / 16
     uint32_t k_groups;     // ceil(k_blocks / 4)
     float *enc;            // one fp32 per domain
@@ -126,10 +126,8 @@ __device__ __forceinline__ void quant_block(const NvParams &p, int64_t row, int6
         c = make_uint2(w[0], w[1]);
     }
     *reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + kb * 8) = c;
-    const uint32_t off = p.mma ? mxk::mma_scale_offset32(static_cast<uint32_t>(row), static_cast<uint32_t>(kb),
-                                                         p.k_groups)
-                               : static_cast<uint32_t>(row) * p.k_blocks + static_cast<uint32_t>(kb);
-    p.scales[off] = static_cast<uint8_t>(s);
+    mxk::put_scale(p.scales, p.mma, static_cast<uint32_t>(row), static_cast<uint32_t>(kb), p.k_blocks, p.k_groups,
+                   s);
 }
 
 // bf16 input, a block as the 8 words of its 16 values (element 2i in the low
@@ -196,9 +194,7 @@ __device__ __forceinline__ void quant_block_bf16(const NvParams &p, int64_t row,
         c = make_uint2(q[0], q[1]);
     }
     *reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + kb * 8) = c;
-    const uint32_t off = p.mma ? mxk::mma_scale_offset32(static_cast<uint32_t>(row), kb, p.k_groups)
-                               : static_cast<uint32_t>(row) * p.k_blocks + kb;
-    p.scales[off] = static_cast<uint8_t>(s);
+    mxk::put_scale(p.scales, p.mma, static_cast<uint32_t>(row), kb, p.k_blocks, p.k_groups, s);
 }
 
 // largest value over the CTA (every thread gets it)
@@ -363,7 +359,7 @@ cudaError_t mx_launch_quantize_nvfp4(const MxNvfp4Args &a, cudaStream_t st) {
     p.ldx = a.ldx;
     p.codes = static_cast<uint8_t *>(a.codes);
     p.scales = static_cast<uint8_t *>(a.scales);
-    p.mma = a.sl == MX_SCALES_MMA;
+    p.mma = a.sl;
     p.k_blocks = static_cast<uint32_t>(a.cols / NV_BLOCK);
     p.k_groups = (p.k_blocks + 3) / 4;
     p.enc = a.enc_scales;

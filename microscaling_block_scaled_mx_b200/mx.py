@@ -87,6 +87,9 @@ def lib() -> ctypes.CDLL:
             L.mx_gemm.restype = i32
             L.mx_gemm.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, i64, ctypes.c_float,
                                   vp, i32, i64, vp, ctypes.c_size_t, vp]
+            L.mx_gemm_nvfp4_x4.restype = i32
+            L.mx_gemm_nvfp4_x4.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float,
+                                           vp, i32, i64, vp]
             L.mx_gemm_nvfp4.restype = i32
             L.mx_gemm_nvfp4.argtypes = [vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float,
                                         vp, i32, i64, vp]
@@ -295,16 +298,20 @@ def gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
 
 def gemm_nvfp4(a, b, M: int, N: int, K: int, a_domain_rows: int = 0, b_domain_rows: int = 0,
                alpha: float = 1.0, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
-    """C = alpha * A * B^T on NVFP4 operands (mx_gemm_nvfp4): a and b are the
-    (codes, scales, enc_scales) triples quantize_nvfp4 returns (MMA layout)."""
+               stream=None, scale_layout="mma") -> torch.Tensor:
+    """C = alpha * A * B^T on NVFP4 operands (mx_gemm_nvfp4, or mx_gemm_nvfp4_x4
+    for scale_layout "mma_x4"): a and b are the (codes, scales, enc_scales)
+    triples quantize_nvfp4 returns in that layout."""
     (ac, asc, ae), (bc, bsc, be) = a, b
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=ac.device)
-    rc = lib().mx_gemm_nvfp4(ac.data_ptr(), asc.data_ptr(), ae.data_ptr(), a_domain_rows,
-                             bc.data_ptr(), bsc.data_ptr(), be.data_ptr(), b_domain_rows, M, N, K,
-                             float(alpha), out.data_ptr(), DTYPE[out.dtype], out.stride(0), _stream(stream))
-    _check(rc, "mx_gemm_nvfp4")
+    fn = {LAYOUT["mma"]: "mx_gemm_nvfp4", LAYOUT["mma_x4"]: "mx_gemm_nvfp4_x4"}.get(_layout(scale_layout))
+    if fn is None:
+        raise ValueError("NVFP4 GEMM operand scales are in the mma or mma_x4 layout")
+    rc = getattr(lib(), fn)(ac.data_ptr(), asc.data_ptr(), ae.data_ptr(), a_domain_rows,
+                            bc.data_ptr(), bsc.data_ptr(), be.data_ptr(), b_domain_rows, M, N, K,
+                            float(alpha), out.data_ptr(), DTYPE[out.dtype], out.stride(0), _stream(stream))
+    _check(rc, fn)
     return out
 
 

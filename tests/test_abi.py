@@ -253,12 +253,12 @@ def test_nvfp4_gemm_validation(mx):
 
 
 def test_x4_layout_sizes_and_entries(mx):
-    """The x4 scale layout's sizes, its acceptance by the casts' checks and its
-    refusal by the NVFP4 cast; the x4 GEMM entries validate like mx_gemm."""
+    """The x4 scale layout's sizes and an unknown layout code's refusal; the
+    x4 GEMM entries validate like mx_gemm."""
     L = mx.lib()
     assert L.mx_scales_bytes(2, 129, 32 * 5) == 4 * L.mx_scales_bytes(1, 129, 32 * 5)
     assert L.mx_scales_bytes(3, 128, 128) == 0
-    assert L.mx_quantize_nvfp4(16, 1, 64, 64, 64, 0, 16, 16, 2, 16, None) == -1
+    assert L.mx_quantize_nvfp4(16, 1, 64, 64, 64, 0, 16, 16, 3, 16, None) == -1     # layout code
     # empty casts and GEMMs are no-ops for the x4 layout as for the others
     assert L.mx_quantize(None, 1, 0, 64, 64, 1, 0, 0, 0, None, None, None, 2, None) == 0
     assert L.mx_gemm_x4(None, None, 0, None, None, 0, 0, 64, 128, 1.0, None, 0, 64, None) == 0
@@ -267,3 +267,5 @@ def test_x4_layout_sizes_and_entries(mx):
     assert L.mx_gemm_x4(16, 16, 5, 16, 16, 0, 128, 128, 128, 1.0, 16, 0, 128, None) == -4     # INT8
     assert L.mx_gemm_x4(16, 16, 0, 16, 16, 0, 128, 128, 128, 1.0, 24, 0, 128, None) == -2     # C alignment
     assert L.mx_gemm_quantize_x4(16, 16, 0, 16, 16, 0, 128, 100, 128, 1.0, 0, 0, 0, 16, 16, 2, None) == -3
+    assert L.mx_gemm_nvfp4_x4(16, 16, 16, 0, 16, 16, 16, 0, 256, 256, 384, 1.0, 16, 1, 256, None) == -4   # K % 256
+    assert L.mx_nvfp4_scales_bytes(2, 100, 64) == 4 * L.mx_nvfp4_scales_bytes(1, 100, 64)

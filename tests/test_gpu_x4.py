@@ -183,3 +183,29 @@ def test_gemm_x4_force_hook():
             assert rc == want, (kern, rc)
     finally:
         L.mx_debug_gemm_force_kernel(-1)
+
+
+@pytest.mark.parametrize("domain_rows", [0, 32])
+def test_nvfp4_x4_cast_and_gemm(oracle, domain_rows):
+    """NVFP4 with x4 block scales: the cast writes the oracle's bytes and the
+    x4 GEMM equals the MMA-layout NVFP4 GEMM bit for bit."""
+    rng = np.random.default_rng(940 + domain_rows)
+    M, N, K = 300, 264, 768
+    a = (rng.standard_normal((M, K)) * np.exp2(rng.uniform(-6, 6, (M, 1)))).astype(np.float32)
+    b = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    a4 = mx.quantize_nvfp4(to_device(a), domain_rows, scale_layout="mma_x4")
+    b4 = mx.quantize_nvfp4(to_device(b), 0, scale_layout="mma_x4")
+    a1 = mx.quantize_nvfp4(to_device(a), domain_rows)
+    b1 = mx.quantize_nvfp4(to_device(b), 0)
+    torch.cuda.synchronize()
+    oc, os_, oe = oracle.nvfp4_quantize(a, domain_rows, scale_layout=X4, fill=0xAB)
+    written = os_ != 0xAB
+    assert np.array_equal(host(a4[0]), oc)
+    assert np.array_equal(host(a4[1])[written], os_[written])
+    for out_dtype in (torch.float32, torch.bfloat16):
+        c4 = mx.gemm_nvfp4(a4, b4, M, N, K, domain_rows, 0, alpha=0.5, out_dtype=out_dtype, scale_layout="mma_x4")
+        c1 = mx.gemm_nvfp4(a1, b1, M, N, K, domain_rows, 0, alpha=0.5, out_dtype=out_dtype)
+        torch.cuda.synchronize()
+        assert mx.last_device_status() == 0
+        iv = torch.int16 if out_dtype == torch.bfloat16 else torch.int32
+        assert torch.equal(c4.view(iv), c1.view(iv)), (domain_rows, out_dtype)
