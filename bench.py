@@ -54,17 +54,18 @@ MEASURED_TRAFFIC = {
     # --cache-control none, so each launch also carries the write-back of its
     # predecessor's output still in L2 (steady state: reads + writes of one cast)
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "05265ce9ff1cd80a87eeb3540ef2af52f9b9c025ae52f0c590bcb67a3bd81420",
-                  {"e4m3_bf16_8192x8192": 202876928, "e5m2_bf16_8192x8192": 201791744,
-                   "e2m3_bf16_8192x8192": 186473728, "e3m2_bf16_8192x8192": 186313984,
-                   "e2m1_bf16_8192x8192": 170129920, "int8_bf16_8192x8192": 203687680}),
+                  "dc0cae36612ead6afd7a6cc8d22f277164ab2de0155b11959810e1bb1b51b96d",
+                  {"e4m3_bf16_8192x8192": 201026048, "e5m2_bf16_8192x8192": 201932800,
+                   "e2m3_bf16_8192x8192": 186476544, "e3m2_bf16_8192x8192": 186476288,
+                   "e2m1_bf16_8192x8192": 170484480, "int8_bf16_8192x8192": 203712256}),
     # the GEMMs: default cache control (L2 flushed before the launch), so reads
-    # show re-reads and writes count only what left L2 during the launch
+    # show re-reads and writes count only what left L2 during the launch; "x4":
+    # operands with x4 scales
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "5f42b5547c2bdbf3d3e990563c14d3a8491634cca05f78bb356c715b535ca8e6",
-             {"e2m1_8192x6144x4096": 85373440, "e2m1_8192x14336x4096": 236292864,
-              "e2m1_8192x4096x14336": 150680576, "e4m3_8192x3072x768": 10714880,
-              "e4m3_8192x768x3072": 28427008, "e2m1_4096x14336x16384": 493558272}),
+             "0b94d08768d8eddd2b0b1e5d8cab398da5ef1bf8cf06b62cbad88ce42aea3855",
+             {"e2m1_x4_8192x6144x4096": 94986752, "e2m1_x4_8192x14336x4096": 248997120,
+              "e2m1_x4_8192x4096x14336": 195028480, "e4m3_8192x3072x768": 10663168,
+              "e4m3_8192x768x3072": 28427264, "e2m1_x4_4096x14336x16384": 639930112}),
 }
 
 
@@ -74,13 +75,13 @@ MEASURED_TRAFFIC = {
 # issue roofline of those casts: at most 4 warp instructions per clock per SM.
 MEASURED_INSTR = {
     "cast_cols_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                         "05265ce9ff1cd80a87eeb3540ef2af52f9b9c025ae52f0c590bcb67a3bd81420",
-                         {"e2m1_bf16_16384x4096": 38797248 / (16384 * 4096),
-                          "e2m1_bf16_16384x14336": 135299008 / (16384 * 14336)}),
+                         "dc0cae36612ead6afd7a6cc8d22f277164ab2de0155b11959810e1bb1b51b96d",
+                         {"e2m1_bf16_x4_16384x4096": 39026624 / (16384 * 4096),
+                          "e2m1_bf16_x4_16384x14336": 136101824 / (16384 * 14336)}),
     "cast_dual_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                         "05265ce9ff1cd80a87eeb3540ef2af52f9b9c025ae52f0c590bcb67a3bd81420",
-                         {"e2m1_bf16_16384x4096": 52169344 / (16384 * 4096),
-                          "e2m1_bf16_16384x14336": 182012544 / (16384 * 14336)}),
+                         "dc0cae36612ead6afd7a6cc8d22f277164ab2de0155b11959810e1bb1b51b96d",
+                         {"e2m1_bf16_16384x4096": 52669952 / (16384 * 4096),
+                          "e2m1_bf16_16384x14336": 183823872 / (16384 * 14336)}),
 }
 
 
