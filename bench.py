@@ -605,6 +605,36 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
     else:
         workload = "gpt2_small_mxfp8_gemms_m8192 (768->3072, 3072->768), bf16 out"
         kernel = "mx_gemm_kernel (cta_group::1, kind::mxf8f6f4; short K / few tiles)"
+    # Llama-3 "quantized along K, and again along M": the first shape's
+    # activation X (8192 x 4096) and output C (8192 x 6144, bf16) cast with
+    # blocks along M (tokens, transposed out), and the weight-gradient-shaped
+    # product C^T X contracting over the 8192 tokens
+    along_m = None
+    if fmt == "e2m1" and ops and not args.no_fused:
+        M, N, K, ac, as_, bc, bs, c = ops[0]
+        xb, _ = I.linear_operands(M, K, N, cfg_index, stream=0)
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c, scale_layout=sl)
+        xc, xs = mx.quantize(x, 0, fmt, scale_layout=sl)         # K x M codes: x^T along tokens
+        cc, cs = mx.quantize(c, 0, fmt, scale_layout=sl)         # N x M codes: C^T along tokens
+        ct = torch.empty((N, K), dtype=torch.float32, device=dev)
+        steps_m = max(3, min(args.steps, 20))
+        timings = {}
+        for label, fn in (("cast_x_along_m", lambda: mx.quantize(x, 0, fmt, codes=xc, scales=xs, scale_layout=sl)),
+                          ("cast_c_along_m", lambda: mx.quantize(c, 0, fmt, codes=cc, scales=cs, scale_layout=sl)),
+                          ("gemm_ct_x", lambda: mx.gemm(cc, cs, xc, xs, N, K, M, fa=fmt, out=ct, scale_layout=sl))):
+            for _ in range(args.warmup):
+                fn()
+            timings[label] = 1e3 * timed_region(lambda i, fn=fn: fn(), steps_m) / steps_m
+            launches += steps_m
+        along_m = {"workload": f"X {M}x{K} and C {M}x{N} bf16 cast along M to E2M1 (RNE, x4 scales); "
+                               f"C^T X = {N}x{K}x{M}, fp32 out"}
+        for label, n in (("cast_x_along_m", M * K), ("cast_c_along_m", M * N)):
+            alg = n * 2 + n // 2 + n // 32
+            along_m[label] = {"us": round(timings[label], 1), "gbs": round(alg / (timings[label] * 1e-6) / 1e9, 1)}
+        along_m["gemm_ct_x"] = {"us": round(timings["gemm_ct_x"], 1),
+                                "tflops": round(2.0 * N * K * M / (timings["gemm_ct_x"] * 1e-6) / 1e12, 1)}
+        del x, xc, xs, cc, cs, ct
     return {"metric": "MX GEMM TFLOP/s", "value": round(value, 1), "unit": "TFLOP/s",
             "workload": workload, "ms_per_step": round(ms / args.steps, 4),
             "roofline": {"bound": "tensor", "kernel": kernel,
@@ -613,6 +643,7 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
                          "peak_kind": f"{peak_kind} bf16 burst x {ratio:g} (nominal ratio for the operand type)",
                          "traffic": traffic, "per_shape": per_shape},
             "quantizing_epilogue": fused,
+            "along_m": along_m,
             "_launches": launches}
 
 
