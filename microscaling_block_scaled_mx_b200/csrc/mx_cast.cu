@@ -2,7 +2,8 @@
 // Learning", summary page, section 3) and exact decode (section 2) on sm_100a.
 //
 // The casts are streaming kernels: every input byte is read once, every code
-// and scale byte written once.
+// and scale byte written once (a scale byte four times in the x4 layout, one
+// per copy of its atom).
 //  * cast_rows: blocks run along the contiguous axis.  One lane owns one
 //    32-block (two 32-byte loads for bf16); a warp covers 32 consecutive
 //    blocks of a row, with the next two chunks' loads in flight in a ring of

@@ -19,12 +19,15 @@
 //               to fp32 / bf16, written to a per-warp shared-memory piece of
 //               32 rows x 64 bytes and stored to C by one TMA store per piece
 //               (the copy engine clips the ragged edges of C).
-// A tcgen05.cp costs tensor-pipe time per instruction, nearly whatever its
-// size: the scale copies take about a fifth of the MXFP4 pair kernel's time.
-// Fewer, wider copies (128x256b from atoms replicated four times in shared
-// memory) measured slower end to end, as did writing the scale factors with
-// tcgen05.st from the epilogue warps: both need a per-stage handshake that
-// costs more than the copies.
+// The scale copies are the largest cost after the MMAs: with the replicating
+// 32x128b.warpx4 form (one per 512-byte atom) they take a fifth to a third of
+// the MXFP4 pair kernel's time.  With operand scales in the x4 layout (each
+// atom stored four times, written so by the cast) the pair kernel uses the
+// 128-lane 128x256b / 128x128b forms instead, two atoms per copy: half the
+// copy instructions and 9-11 % less time on MXFP4.  Building those replicas
+// inside the SM (an expander warp, or the epilogue warps writing the scale
+// factors with tcgen05.st) measured slower: both need a per-stage cross-CTA
+// handshake that costs more than the copies.
 // A 192-column tile starts 64 rows into a 128-row scale atom on odd tiles;
 // the B scale-factor TMEM address then starts two columns later.
 // Every mbarrier wait is bounded; on expiry the kernel records MX_ERR_TIMEOUT
