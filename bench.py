@@ -54,7 +54,7 @@ MEASURED_TRAFFIC = {
     # --cache-control none, so each launch also carries the write-back of its
     # predecessor's output still in L2 (steady state: reads + writes of one cast)
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "dc0cae36612ead6afd7a6cc8d22f277164ab2de0155b11959810e1bb1b51b96d",
+                  "fd12806ddd982f7d8ade8fbaff3a2fb32e12af6eef26beb9256acfbf6d8c5916",
                   {"e4m3_bf16_8192x8192": 201026048, "e5m2_bf16_8192x8192": 201932800,
                    "e2m3_bf16_8192x8192": 186476544, "e3m2_bf16_8192x8192": 186476288,
                    "e2m1_bf16_8192x8192": 170484480, "int8_bf16_8192x8192": 203712256}),
@@ -62,7 +62,7 @@ MEASURED_TRAFFIC = {
     # show re-reads and writes count only what left L2 during the launch; "x4":
     # operands with x4 scales
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "0b94d08768d8eddd2b0b1e5d8cab398da5ef1bf8cf06b62cbad88ce42aea3855",
+             "c89c1e54c65172af272a90f7d63214df974483241caf85d202f5132976ecac2e",
              {"e2m1_x4_8192x6144x4096": 94986752, "e2m1_x4_8192x14336x4096": 248997120,
               "e2m1_x4_8192x4096x14336": 195028480, "e4m3_8192x3072x768": 10663168,
               "e4m3_8192x768x3072": 28427264, "e2m1_x4_4096x14336x16384": 639930112}),
@@ -75,11 +75,11 @@ MEASURED_TRAFFIC = {
 # issue roofline of those casts: at most 4 warp instructions per clock per SM.
 MEASURED_INSTR = {
     "cast_cols_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                         "dc0cae36612ead6afd7a6cc8d22f277164ab2de0155b11959810e1bb1b51b96d",
+                         "fd12806ddd982f7d8ade8fbaff3a2fb32e12af6eef26beb9256acfbf6d8c5916",
                          {"e2m1_bf16_x4_16384x4096": 39026624 / (16384 * 4096),
                           "e2m1_bf16_x4_16384x14336": 136101824 / (16384 * 14336)}),
     "cast_dual_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                         "dc0cae36612ead6afd7a6cc8d22f277164ab2de0155b11959810e1bb1b51b96d",
+                         "fd12806ddd982f7d8ade8fbaff3a2fb32e12af6eef26beb9256acfbf6d8c5916",
                          {"e2m1_bf16_16384x4096": 52669952 / (16384 * 4096),
                           "e2m1_bf16_16384x14336": 183823872 / (16384 * 14336)}),
 }
