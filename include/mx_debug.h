@@ -29,7 +29,9 @@ MX_API int mx_debug_gemm_skip_stage(int k_tile);
  * mx_debug_gemm_force_kernel -- choose the GEMM kernel of the calling host
  * thread's later mx_gemm / mx_gemm_quantize calls instead of the automatic
  * choice, so that tests reach every kernel on any shape: 0 the one-SM kernel
- * (128 x 192 tiles), 256 or 192 the CTA-pair kernel with 256 x 256 or
+ * (128 x 192 tiles), 1 the one-SM kernel with a resident B panel (128 x 192
+ * tiles, at most six 128-byte K slices: a GEMM with a longer K then returns
+ * MX_ERR_UNSUPPORTED), 256 or 192 the CTA-pair kernel with 256 x 256 or
  * 256 x 192 tiles, -1 back to automatic.  Results are the same up to the
  * order of the fp32 sums.  Returns MX_OK, or MX_ERR_ARG for another value.
  */

@@ -122,6 +122,7 @@ struct Params {
     float alpha;
     uint32_t idesc;  // instruction descriptor without the scale-factor ids
     uint32_t ab_tx;  // bytes the A and B loads of one stage deliver (packed size in global)
+    uint32_t a_tx;   // the A load's share of ab_tx
     int skip_k_tile; // testing hook: CTA 0 withholds this k-tile of its first tile (-1: off)
     int raster_group, raster_n_major;   // tile order (tile_coords)
     MxOut q;         // OUT_MX only
@@ -605,6 +606,278 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
 #pragma unroll
                     for (int j = 0; j < (BN / 2) / PC; ++j)
                         if (n_base + PC * j < p.N) epi_piece<OUT>(ew, r + PC * j, p.alpha, n_base + PC * j, m_warp);
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_all();          // stores done reading shared memory and written
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------------
+// Resident-B kernel for short K (one SM per CTA, 128 x 192 tiles): when the
+// whole K of a 192-row B panel fits in shared memory (at most six 128-byte K
+// slices: K <= 768 for MXFP8, 1536 for MXFP4), each CTA takes a contiguous
+// range of tiles in panel-major order (all M tiles of one N panel, then the
+// next), loads its B panel and the panel's scale atoms once, and streams only
+// A per tile.  The one-SM kernel reloads a 24 KiB B slice with every 16 KiB
+// A slice; on such shapes the operand stream from L2 is what bounds it.  The
+// panel's B scale factors stay in tensor memory for the whole panel, so a K
+// slice needs one scale copy (A's) instead of three.
+// ------------------------------------------------------------------------
+constexpr int PANEL_MAX_SLICES = 6;
+constexpr int PANEL_A_STAGES = 3;
+
+template <bool FP4> struct PanelCfg {
+    static constexpr int G = FP4 ? 2 : 1;                        // scale atoms along K per slice
+    static constexpr int MAX_ATOMS = PANEL_MAX_SLICES * G;       // per 128-row scale block
+    static constexpr int OFF_B = 0;                              // the panel: slice k at k * B_STAGE_BYTES
+    static constexpr int OFF_SFB = OFF_B + PANEL_MAX_SLICES * B_STAGE_BYTES;   // two row blocks of atoms
+    static constexpr int OFF_A = OFF_SFB + 2 * MAX_ATOMS * ATOM;
+    static constexpr int OFF_SFA = OFF_A + PANEL_A_STAGES * A_STAGE_BYTES;
+    static constexpr int OFF_EPI = (OFF_SFA + PANEL_A_STAGES * G * ATOM + 1023) / 1024 * 1024;
+    static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_PIECE;          // one staged piece per warp
+    // a_full[S], a_empty[S], acc_full[2], acc_empty[2], panel_full, panel_empty, drain
+    static constexpr int NUM_BARS = 2 * PANEL_A_STAGES + 7;
+    static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM + 4;
+    static constexpr int SMEM = OFF_ABORT + 4 + 1024;                        // + alignment slack
+    // tensor memory: two 192-column accumulators, the panel's B scale factors
+    // (8 columns per k-group: both row blocks), then A's per stage
+    static constexpr uint32_t SFB_COL = 2 * ACC_COLS;
+    static constexpr uint32_t SFA_COL = SFB_COL + 8 * MAX_ATOMS;
+    static_assert(OFF_A % 1024 == 0, "operand tiles 1024-byte aligned");
+    static_assert(SFA_COL + PANEL_A_STAGES * 4 * G <= TMEM_COLS, "tensor memory columns");
+    static_assert(SMEM <= 232448, "shared memory per block");
+};
+
+template <bool FP4, int OUT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+mx_gemm_panel_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                     const __grid_constant__ CUtensorMap tma_c, Params p) {
+    using C = Cfg<FP4>;
+    using PC = PanelCfg<FP4>;
+    constexpr int S = PANEL_A_STAGES;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + PC::OFF_ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + PC::OFF_TMEM);
+
+    auto a_full = [&](int s) { return sbase + PC::OFF_BAR + 8u * s; };
+    auto a_empty = [&](int s) { return sbase + PC::OFF_BAR + 8u * (S + s); };
+    auto acc_full = [&](int b) { return sbase + PC::OFF_BAR + 8u * (2 * S + b); };
+    auto acc_empty = [&](int b) { return sbase + PC::OFF_BAR + 8u * (2 * S + 2 + b); };
+    const uint32_t panel_full = sbase + PC::OFF_BAR + 8u * (2 * S + 4);
+    const uint32_t panel_empty = sbase + PC::OFF_BAR + 8u * (2 * S + 5);
+    const uint32_t drain_bar = sbase + PC::OFF_BAR + 8u * (2 * S + 6);
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < S; ++s) {
+            mbar_init(a_full(s), 1);
+            mbar_init(a_empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full(b), 1);
+            mbar_init(acc_empty(b), EPI_WARPS);
+        }
+        mbar_init(panel_full, 1);
+        mbar_init(panel_empty, 1);
+        mbar_init(drain_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // this CTA's tiles: a contiguous range in panel-major order (tile t: N panel
+    // t / tiles_m, M tile t % tiles_m)
+    const int64_t num_tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+    const int t_begin = static_cast<int>(num_tiles * blockIdx.x / gridDim.x);
+    const int t_end = static_cast<int>(num_tiles * (blockIdx.x + 1) / gridDim.x);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t outstanding = 0;   // bit s: stage s has loads in flight not yet observed
+            int panel = -1, panels = 0;
+            bool panel_out = false;     // the latest panel load may still be in flight
+            bool ok = true;
+            for (int t = t_begin; t < t_end && ok; ++t) {
+                const int tn = t / p.tiles_m, tm = t % p.tiles_m;
+                if (tn != panel) {
+                    // the MMAs are done with the previous panel; load this one
+                    if (panels > 0 && !wait_bounded(panel_empty, (panels - 1) & 1, abort_flag)) { ok = false; break; }
+                    const int n0 = tn * BN, rb_b = n0 / 128;
+                    const bool b_second = (rb_b + 1) * 128 < p.N;
+                    const uint32_t at_bytes = static_cast<uint32_t>(p.k_groups) * ATOM;
+                    mbar_expect_tx(panel_full, static_cast<uint32_t>(p.k_tiles) * (p.ab_tx - p.a_tx) +
+                                                   (b_second ? 2u : 1u) * at_bytes);
+                    for (int kt = 0; kt < p.k_tiles; ++kt)
+                        tma_load_2d(sbase + PC::OFF_B + kt * B_STAGE_BYTES, &tma_b, kt * BK_BYTES, n0, panel_full);
+                    bulk_load(sbase + PC::OFF_SFB, p.b_scales + static_cast<int64_t>(rb_b) * p.k_groups * ATOM,
+                              at_bytes, panel_full);
+                    if (b_second)
+                        bulk_load(sbase + PC::OFF_SFB + PC::MAX_ATOMS * ATOM,
+                                  p.b_scales + static_cast<int64_t>(rb_b + 1) * p.k_groups * ATOM, at_bytes,
+                                  panel_full);
+                    panel = tn;
+                    ++panels;
+                    panel_out = true;
+                }
+                const int m0 = tm * BM, rb_a = m0 / 128;
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!wait_bounded(a_empty(s), ph ^ 1u, abort_flag)) { ok = false; break; }
+                    if (kt == p.skip_k_tile && t == t_begin && blockIdx.x == 0) {
+                        ok = false;          // injected stall: this stage is never filled
+                        break;
+                    }
+                    const uint32_t fb = a_full(s);
+                    mbar_expect_tx(fb, p.a_tx + C::G * ATOM);
+                    tma_load_2d(sbase + PC::OFF_A + s * A_STAGE_BYTES, &tma_a, kt * BK_BYTES, m0, fb);
+                    bulk_load(sbase + PC::OFF_SFA + s * C::G * ATOM,
+                              p.a_scales + (static_cast<int64_t>(rb_a) * p.k_groups + kt * C::G) * ATOM,
+                              C::G * ATOM, fb);
+                    outstanding |= 1u << s;
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                    outstanding &= ~(1u << s);   // its previous use was released by the MMA
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for every stage and the panel whose loads may still land
+                volatile int no_abort = 0;
+                int ds = s;
+                uint32_t dph = ph;
+                for (int i = 0; i < S; ++i) {
+                    ds = ds == 0 ? S - 1 : ds - 1;
+                    if (ds == S - 1) dph ^= 1u;
+                    if (outstanding & (1u << ds)) (void)wait_bounded(a_full(ds), dph, &no_abort, DRAIN_LIMIT_NS);
+                }
+                if (panel_out) (void)wait_bounded(panel_full, (panels - 1) & 1, &no_abort, DRAIN_LIMIT_NS);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ----------------------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            bool issued = false;
+            int panel = -1, panels = 0;
+            int local = 0;
+            for (int t = t_begin; t < t_end && ok; ++t, ++local) {
+                const int tn = t / p.tiles_m;
+                if (tn != panel) {
+                    // the previous panel is free once its MMAs complete
+                    if (panels > 0) tc_commit(panel_empty);
+                    if (!wait_bounded(panel_full, panels & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    // the panel's B scale atoms -> tensor memory, 8 columns per k-group
+                    const uint32_t sfb_s = sbase + PC::OFF_SFB;
+                    for (int g = 0; g < p.k_groups; ++g)
+                        for (int h = 0; h < 2; ++h)
+                            tc_cp_scale_atom(tmem + PC::SFB_COL + 8 * g + 4 * h,
+                                             scale_atom_desc(sfb_s + h * PC::MAX_ATOMS * ATOM + g * ATOM));
+                    issued = true;
+                    panel = tn;
+                    ++panels;
+                }
+                const int b = local & 1;
+                const uint32_t acc_ph = (local >> 1) & 1;
+                if (!wait_bounded(acc_empty(b), acc_ph ^ 1u, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + b * ACC_COLS;
+                const uint32_t sfb_shift = (tn & 1) ? 2u : 0u;   // odd 192-column tiles
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!wait_bounded(a_full(s), ph, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sfa_t = tmem + PC::SFA_COL + s * 4 * C::G;
+                    const uint32_t sfa_s = sbase + PC::OFF_SFA + s * C::G * ATOM;
+#pragma unroll
+                    for (int g = 0; g < C::G; ++g) tc_cp_scale_atom(sfa_t + 4 * g, scale_atom_desc(sfa_s + g * ATOM));
+                    const uint32_t a_s = sbase + PC::OFF_A + s * A_STAGE_BYTES;
+                    const uint32_t b_s = sbase + PC::OFF_B + kt * B_STAGE_BYTES;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        // FP8: k-block k of the atom; FP4: k-blocks 2k, 2k+1 (atom k/2, bytes 2k%4..)
+                        const uint32_t g = FP4 ? (k >> 1) : 0u;
+                        const uint32_t sf_id = FP4 ? ((2u * k) & 3u) : static_cast<uint32_t>(k);
+                        const uint32_t idesc = p.idesc | (sf_id << 4) | (sf_id << 29);
+                        tc_mma<FP4>(d_tmem, operand_desc(a_s, 32u * k), operand_desc(b_s, 32u * k), idesc,
+                                    sfa_t + 4 * g,
+                                    tmem + PC::SFB_COL + 8 * (kt * C::G + g) + sfb_shift, (kt > 0 || k > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit(a_empty(s));
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(acc_full(b));
+            }
+            if (issued) {
+                // all issued MMAs and copies must finish before TMEM is released
+                tc_commit(drain_bar);
+                volatile int no_abort = 0;
+                (void)wait_bounded(drain_bar, 0, &no_abort, ok ? WAIT_LIMIT_NS : DRAIN_LIMIT_NS);
+            }
+        }
+    } else {
+        // ------------------------------ epilogue ------------------------------
+        const int q = warp & 3;                  // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;        // which 96 columns of the tile
+        EpiWriter ew{&tma_c, sbase + PC::OFF_EPI + static_cast<uint32_t>(warp - 2) * EPI_PIECE, 0, lane,
+                     p.c, p.ldc, p.M, p.N};
+        int local = 0;
+        for (int t = t_begin; t < t_end; ++t, ++local) {
+            const int b = local & 1;
+            const uint32_t acc_ph = (local >> 1) & 1;
+            int ok = 1;
+            if (lane == 0) ok = wait_bounded(acc_full(b), acc_ph, abort_flag) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const int tn = t / p.tiles_m, tm = t % p.tiles_m;
+            const int m = tm * BM + q * 32 + lane;
+            const int c0 = half * (BN / 2);
+            const uint32_t taddr = tmem + b * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16) + c0;
+            uint32_t r[96];
+            tmem_ld_x32_nowait(taddr, r);
+            tmem_ld_x32_nowait(taddr + 32, r + 32);
+            tmem_ld_x32_nowait(taddr + 64, r + 64);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty(b));
+            const int n_base = tn * BN + c0;
+            if constexpr (OUT == OUT_MX) {
+#pragma unroll
+                for (int j = 0; j < 3; ++j) store_chunk_mx(p, m, n_base + 32 * j, r + 32 * j);
+            } else {
+                const int m_warp = tm * BM + q * 32;
+                constexpr int PCOL = OUT == OUT_BF16 ? 32 : 16;  // columns per piece
+                if (m_warp < p.M) {
+#pragma unroll
+                    for (int j = 0; j < (BN / 2) / PCOL; ++j)
+                        if (n_base + PCOL * j < p.N)
+                            epi_piece<OUT, 1>(ew, r + PCOL * j, p.alpha, n_base + PCOL * j, m_warp);
                 }
             }
         }
@@ -1233,6 +1506,24 @@ cudaError_t launch_pair_out(int out, const CUtensorMap &ta, const CUtensorMap &t
     return launch_pair<FP4, OUT_F32, PBN>(ta, tb, tsa, tsb, tc, p, grid, st);
 }
 
+template <bool FP4, int OUT>
+cudaError_t launch_panel(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc, const Params &p,
+                         int grid, cudaStream_t st) {
+    auto kern = mx_gemm_panel_kernel<FP4, OUT>;
+    constexpr int smem = PanelCfg<FP4>::SMEM;
+    static std::atomic<uint64_t> configured{0};   // per instantiation, one bit per device
+    if (cudaError_t e = ensure_smem_limit(kern, smem, configured); e != cudaSuccess) return e;
+    return launch_overlapped(kern, grid, smem, st, ta, tb, tc, p);
+}
+
+template <bool FP4>
+cudaError_t launch_panel_out(int out, const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
+                             const Params &p, int grid, cudaStream_t st) {
+    if (out == OUT_MX) return launch_panel<FP4, OUT_MX>(ta, tb, tc, p, grid, st);
+    if (out == OUT_BF16) return launch_panel<FP4, OUT_BF16>(ta, tb, tc, p, grid, st);
+    return launch_panel<FP4, OUT_F32>(ta, tb, tc, p, grid, st);
+}
+
 template <bool FP4>
 cudaError_t launch_out(int out, const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
                        const Params &p, int grid, cudaStream_t st) {
@@ -1266,7 +1557,7 @@ thread_local int g_force_kernel = -1;
 }
 
 extern "C" int mx_debug_gemm_force_kernel(int tile_n) {
-    if (tile_n != -1 && tile_n != 0 && tile_n != 192 && tile_n != 256) return MX_ERR_ARG;
+    if (tile_n != -1 && tile_n != 0 && tile_n != 1 && tile_n != 192 && tile_n != 256) return MX_ERR_ARG;
     g_force_kernel = tile_n;
     return MX_OK;
 }
@@ -1377,7 +1668,7 @@ int launch_gemm_pair(const MxGemmArgs &a, int pbn, cudaStream_t st) {
 // and overlapped epilogue win (measured on the GPT-2-shaped GEMMs).
 // Returns the pair tile width to use, or 0 for the one-SM kernel.
 int pair_tile_n(const MxGemmArgs &a) {
-    if (g_force_kernel >= 0) return g_force_kernel;
+    if (g_force_kernel >= 0) return g_force_kernel == 1 ? 0 : g_force_kernel;   // 1: the panel kernel
     if (a.M <= 128 || a.K < 2048) return 0;
     const int64_t pair_tiles = ((a.M + 255) / 256) * ((a.N + 255) / 256);
     return pair_tiles >= a.num_sms ? 256 : 0;
@@ -1413,6 +1704,7 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     p.alpha = a.alpha;
     p.idesc = make_idesc(a.fa, a.fb, fp4);
     p.ab_tx = stage_tx_bytes(a.fa, fp4, BM) + stage_tx_bytes(a.fb, fp4, BN);
+    p.a_tx = stage_tx_bytes(a.fa, fp4, BM);
     raster_for(a, p.tiles_m, p.tiles_n, p.raster_group, p.raster_n_major);
     p.skip_k_tile = g_skip_k_tile;
     g_skip_k_tile = -1;
@@ -1421,8 +1713,17 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
     cudaError_t e;
     p.q = mx_out(a);
     const int out = out_mode(a);
-    if (fp4) e = launch_out<true>(out, ta, tb, tc, p, grid, st);
-    else e = launch_out<false>(out, ta, tb, tc, p, grid, st);
+    // the resident-B kernel where a B panel's whole K fits in shared memory and
+    // each panel serves several M tiles (or when forced)
+    const bool panel = g_force_kernel == 1 ||
+                       (g_force_kernel < 0 && p.k_tiles <= PANEL_MAX_SLICES && p.tiles_m >= 4);
+    if (panel) {
+        if (p.k_tiles > PANEL_MAX_SLICES) return MX_ERR_UNSUPPORTED;
+        e = fp4 ? launch_panel_out<true>(out, ta, tb, tc, p, grid, st)
+                : launch_panel_out<false>(out, ta, tb, tc, p, grid, st);
+    } else {
+        e = fp4 ? launch_out<true>(out, ta, tb, tc, p, grid, st) : launch_out<false>(out, ta, tb, tc, p, grid, st);
+    }
     return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 

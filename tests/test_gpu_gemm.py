@@ -310,11 +310,11 @@ def test_gemm_wgrad_config(oracle, wgrad_oracle_operands):
               ("wgrad tile", m0, n0))
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 256, 1024), (4096, 2560, 2048)])
+@pytest.mark.parametrize("M,N,K", [(256, 256, 1024), (1024, 384, 512), (4096, 2560, 2048)])
 def test_gemm_bounded_wait_reports_timeout(M, N, K):
     """A stage that is never filled: the MMA issuer's bounded wait runs out, the
     kernel records MX_ERR_TIMEOUT and returns; the context stays usable.  The
-    first shape runs on the one-SM kernel, the second on CTA pairs."""
+    shapes run on the one-SM kernel, the resident-B kernel and CTA pairs."""
     rng = np.random.default_rng(1)
     a = to_device(rng.standard_normal((M, K)).astype(np.float32))
     b = to_device(rng.standard_normal((N, K)).astype(np.float32))
@@ -359,7 +359,7 @@ def test_gemm_writes_only_inside_c(oracle, M, N, K, out_dtype):
 # shape; mx_debug_gemm_force_kernel (include/mx_debug.h) lets these tests run
 # the one-SM kernel (0) and both CTA-pair tile widths (256, 192) on the same
 # operands.
-KERNELS = [0, 256, 192]
+KERNELS = [0, 1, 256, 192]   # one-SM, one-SM with a resident B panel, CTA pairs
 
 
 class forced_kernel:
@@ -399,7 +399,8 @@ def test_gemm_each_kernel_tolerance_and_window(oracle, kernel, out_dtype):
     """General data on every kernel, pitched C with sentinels around the
     M x N window (nothing outside it is written)."""
     rng = np.random.default_rng(23 + kernel)
-    for (M, N, K, fmt) in [(700, 900, 2048, "e2m1"), (264, 392, 768, "e4m3")]:
+    # the resident-B kernel holds at most six K slices (MXFP4 K <= 1536)
+    for (M, N, K, fmt) in [(700, 900, 1536 if kernel == 1 else 2048, "e2m1"), (264, 392, 768, "e4m3")]:
         a = (rng.standard_normal((M, K)) * np.exp2(rng.uniform(-3, 3, (M, 1)))).astype(np.float32)
         b = rng.standard_t(3, size=(N, K)).astype(np.float32)
         ac, as_ = mx.quantize(to_device(a), 1, fmt)
@@ -429,3 +430,34 @@ def test_gemm_pair_kernels_on_llama_shape(oracle, kernel):
     with forced_kernel(kernel):
         got, ref, bound = run_gemm(oracle, x, w, "e2m1", M, N, K, out_dtype=torch.bfloat16, rows=rows)
     check(got, ref, bound, torch.bfloat16, (kernel, M, N, K))
+
+
+def test_gemm_panel_kernel_refuses_long_k():
+    """Forced onto the resident-B kernel, a K of more than six slices is refused."""
+    z = torch.zeros(1 << 20, dtype=torch.uint8, device=dev())
+    c = torch.empty((256, 256), dtype=torch.float32, device=dev())
+    with forced_kernel(1):
+        rc = mx.lib().mx_gemm(z.data_ptr(), z.data_ptr(), 0, z.data_ptr(), z.data_ptr(), 0, 256, 256, 1024, 1.0,
+                              c.data_ptr(), 0, 256, None, 0, None)
+    assert rc == -4
+
+
+def test_gemm_panel_kernel_gpt2_up_projection(oracle):
+    """The GPT-2 MLP up-projection shape (8192 x 3072 x 768, MXFP8), which the
+    automatic choice gives to the resident-B kernel: all of C within the
+    tolerance, and equal to the one-SM kernel's C bit for bit (same sums in
+    the same order)."""
+    M, N, K = 8192, 3072, 768
+    x, w = I.linear_operands(M, K, N, 2, stream=0)
+    ac, as_ = mx.quantize(to_device(x), 1, "e4m3")
+    bc, bs = mx.quantize(to_device(w), 1, "e4m3")
+    c_auto = mx.gemm(ac, as_, bc, bs, M, N, K, fa="e4m3", out_dtype=torch.float32)
+    with forced_kernel(0):
+        c_one = mx.gemm(ac, as_, bc, bs, M, N, K, fa="e4m3", out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert mx.last_device_status() == 0
+    assert torch.equal(c_auto.view(torch.int32), c_one.view(torch.int32))
+    oac, oas = oracle.quantize(x, 1, oracle.E4M3, scale_layout=oracle.MMA)
+    obc, obs = oracle.quantize(w, 1, oracle.E4M3, scale_layout=oracle.MMA)
+    ref, bound = oracle.gemm_decoded(oac, oas, oracle.E4M3, obc, obs, oracle.E4M3, M, N, K)
+    check(to_f64(c_auto), ref, bound, torch.float32, "gpt2 up-projection")

@@ -177,7 +177,7 @@ def test_gemm_quantize_k_zero_empty_and_shape():
         mx.gemm_quantize(z, z, z, z, 4, 48, 128, out_fmt="e4m3", out=(codes, scales))
 
 
-@pytest.mark.parametrize("kernel", [0, 256, 192])
+@pytest.mark.parametrize("kernel", [0, 1, 256, 192])
 @pytest.mark.parametrize("out_fmt", ["e4m3", "e2m1", "e3m2", "int8"])
 def test_gemm_quantize_each_kernel_bit_exact(oracle, kernel, out_fmt):
     """The quantizing epilogue on every kernel (forced with
