@@ -604,7 +604,8 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         kernel = "mx_gemm_pair_kernel (cta_group::2, kind::mxf4, x4 scales)"
     else:
         workload = "gpt2_small_mxfp8_gemms_m8192 (768->3072, 3072->768), bf16 out"
-        kernel = "mx_gemm_kernel (cta_group::1, kind::mxf8f6f4; short K / few tiles)"
+        kernel = ("mx_gemm_panel_kernel (768->3072: resident B panel) and mx_gemm_kernel (3072->768); "
+                  "cta_group::1, kind::mxf8f6f4")
     # Llama-3 "quantized along K, and again along M": the first shape's
     # activation X (8192 x 4096) and output C (8192 x 6144, bf16) cast with
     # blocks along M (tokens, transposed out), and the weight-gradient-shaped
