@@ -62,10 +62,10 @@ MEASURED_TRAFFIC = {
     # show re-reads and writes count only what left L2 during the launch; "x4":
     # operands with x4 scales
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "c89c1e54c65172af272a90f7d63214df974483241caf85d202f5132976ecac2e",
-             {"e2m1_x4_8192x6144x4096": 94986752, "e2m1_x4_8192x14336x4096": 248997120,
-              "e2m1_x4_8192x4096x14336": 195028480, "e4m3_8192x3072x768": 10663168,
-              "e4m3_8192x768x3072": 28427264, "e2m1_x4_4096x14336x16384": 639930112}),
+             "81602d7c28146bb2866e48d7318af51587248677cb59052448cece18862c8f55",
+             {"e2m1_x4_8192x6144x4096": 37114880 + 57409280, "e2m1_x4_8192x14336x4096": 58781184 + 190069760,
+              "e2m1_x4_8192x4096x14336": 139339520 + 52288512, "e4m3_8192x3072x768": 8977664 + 3238144,
+              "e4m3_8192x768x3072": 28427520 + 0, "e2m1_x4_4096x14336x16384": 402007040 + 213721600}),
 }
 
 
