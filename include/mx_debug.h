@@ -37,6 +37,30 @@ MX_API int mx_debug_gemm_skip_stage(int k_tile);
  */
 MX_API int mx_debug_gemm_force_kernel(int tile_n);
 
+/*
+ * mx_debug_cast_force_cpasync -- on != 0: the calling host thread's later
+ * column and dual casts (mx_quantize with block_axis 0, mx_quantize_dual and
+ * their shard forms) stage their input tiles with 16-byte cp.async copies
+ * instead of TMA tensor copies, the path taken otherwise only for inputs a
+ * tensor map cannot describe (a row or column count beyond int32 range).  The
+ * results are identical.  on == 0 restores the automatic choice.  Returns
+ * MX_OK.
+ */
+MX_API int mx_debug_cast_force_cpasync(int on);
+
+/*
+ * mx_debug_cast_skip_tile -- arm (on != 0) or disarm a one-shot injected
+ * stall for the next column or dual cast of the calling host thread: the
+ * first CTA does not issue the TMA copy of its first tile, so its bounded
+ * wait on that tile runs out (after about 2 s).  The CTA records
+ * MX_ERR_TIMEOUT in the cast status word (read with mx_last_device_status),
+ * waits, again bounded, for the copies it did issue, and returns; the CUDA
+ * context stays usable and the outputs are left partly unwritten.  A call
+ * that stages with cp.async (mx_debug_cast_force_cpasync) consumes the hook
+ * without effect.  Returns MX_OK.
+ */
+MX_API int mx_debug_cast_skip_tile(int on);
+
 #ifdef __cplusplus
 }
 #endif

@@ -469,7 +469,10 @@ int mx_gemm_nvfp4_x4(const void *a_codes, const void *a_scales, const float *a_e
 }
 
 int mx_last_device_status(void *stream) {
-    return mx_read_device_status(static_cast<cudaStream_t>(stream));
+    // the GEMMs' and the casts' status words, both read and cleared
+    const int g = mx_read_device_status(static_cast<cudaStream_t>(stream));
+    const int c = mx_read_cast_status();
+    return g != MX_OK ? g : c;
 }
 
 }  // extern "C"

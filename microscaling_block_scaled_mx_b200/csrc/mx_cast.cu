@@ -9,19 +9,22 @@
 //    blocks of a row, with the next two chunks' loads in flight in a ring of
 //    register slots.
 //  * cast_cols: blocks run down columns.  A CTA stages 128 x 128 tiles in
-//    shared memory (double-buffered cp.async); each thread owns one column
+//    shared memory (double-buffered; one TMA tensor copy per tile, or 16-byte
+//    cp.async copies when the input is not 16-byte aligned); each thread owns one column
 //    pair of a 32-row block, where the optional fixed-sign 32-point Hadamard
 //    ("Format-Aware Fusion for Fast FP4 Pretraining", abstract) runs as five
 //    packed fp32 butterfly stages, and writes its codes as rows of the
 //    transposed (block-axis-major) output.
 //  * cast_dual: both of the above from one staged tile.
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "mx.h"
 #include "mx_device.cuh"
 #include "mx_encode.cuh"
+#include "mx_debug.h"
 #include "mx_internal.h"
 
 namespace mxk {
@@ -38,6 +41,7 @@ struct CastParams {
     uint32_t sign_mask;  // Hadamard signs
     // stochastic-rounding position of output element (o, i): sr_base + o * sr_stride + i
     uint64_t sr_base, sr_stride;
+    int skip_first;      // testing hook: CTA 0 withholds the copy of its first staged tile
 };
 
 __device__ __forceinline__ void store_scale(const CastParams &p, int64_t o, int64_t kb, uint32_t s) {
@@ -234,6 +238,73 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// Tile staging by the tensor-memory-access (TMA) engine: one thread issues a
+// tensor copy per tile (per 128-byte-wide box for the swizzled dual-cast
+// layout) that completes on the buffer's mbarrier; every thread waits on that
+// barrier.  Compared with 16-byte cp.async copies this takes the per-chunk
+// address, bounds and zero-fill arithmetic off every thread (the copy engine
+// fills the part of a box outside the tensor with zeros).
+__device__ int g_cast_status;   // MX_ERR_TIMEOUT once a staging wait gave up
+
+constexpr unsigned long long STAGE_WAIT_NS = 2000000000ull;    // 2 s per tile wait
+constexpr unsigned long long STAGE_DRAIN_NS = 200000000ull;    // 0.2 s for copies in flight after that
+
+__device__ __forceinline__ void stage_bar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void stage_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_tile_load(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ bool stage_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait for phase `parity` of a staging barrier: false after `limit`
+// ns, with the timeout recorded in the status word (read by
+// mx_last_device_status).
+__device__ __noinline__ bool stage_wait_slow(uint32_t bar, uint32_t parity, unsigned long long limit) {
+    unsigned long long t0;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (uint32_t it = 0;; ++it) {
+        if (stage_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 63u) {
+            unsigned long long t;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+            if (t - t0 > limit) {
+                atomicExch(&g_cast_status, MX_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ bool stage_wait(uint32_t bar, uint32_t parity, unsigned long long limit = STAGE_WAIT_NS) {
+    return stage_try_wait(bar, parity) || stage_wait_slow(bar, parity, limit);
+}
+
+// Shared-memory layout of a TMA-staged tile: the buffers start at the first
+// ALIGN boundary of the dynamic buffer (1024 bytes for the 128-byte swizzle,
+// whose pattern repeats every 1024 bytes), followed by one mbarrier per buffer.
+template <int ALIGN>
+struct StagedTiles {
+    uint8_t *tiles;     // generic pointer to buffer 0
+    uint32_t base;      // its shared-memory address
+    uint32_t bars;      // barrier of buffer b at bars + 8 b
+    __device__ StagedTiles(uint8_t *raw, int tile_bytes) {
+        const uint32_t r = static_cast<uint32_t>(__cvta_generic_to_shared(raw));
+        base = (r + ALIGN - 1) & ~static_cast<uint32_t>(ALIGN - 1);
+        tiles = raw + (base - r);
+        bars = base + 2 * tile_bytes;
+    }
+};
+
 // Shared-memory position of 16-byte chunk q of tile row rr.  Unswizzled for
 // the column cast.  The dual cast, which also reads 32-element row segments,
 // XORs the chunk's index inside its 128-byte span with the span index and the
@@ -392,12 +463,24 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
     }
 }
 
+// After a staging wait gave up at tile use `use` (buffer `buf`): wait, again
+// bounded, for the copies that may still be landing in shared memory (that
+// tile's, and the next one's if it was issued) before the CTA exits.
+__device__ __noinline__ void drain_staged(uint32_t bars, int buf, uint32_t use, bool next_issued) {
+    (void)stage_wait(bars + 8 * buf, (use >> 1) & 1u, STAGE_DRAIN_NS);
+    if (next_issued) (void)stage_wait(bars + 8 * (buf ^ 1), ((use + 1) >> 1) & 1u, STAGE_DRAIN_NS);
+}
+
 // DEFM: the Hadamard uses the default sign mask, folded into the loads.
-template <int FMT, bool SR, bool BF16_IN, bool HAD, bool DEFM = false>
-__global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p) {
+// TMA: tiles staged by tensor copies of `tmap` (the input as a rows x cols
+// tensor, boxes of 128 x 128), else by cp.async.
+template <int FMT, bool SR, bool BF16_IN, bool HAD, bool DEFM, bool TMA>
+__global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p, const __grid_constant__ CUtensorMap tmap) {
     using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
     constexpr int TILE_BYTES = COL_TILE_R * COL_TILE_C * sizeof(TIn);
     extern __shared__ __align__(16) uint8_t col_smem[];
+    const StagedTiles<128> st(col_smem, TILE_BYTES);
+    uint8_t *const tiles = TMA ? st.tiles : col_smem;
 
     const int64_t R = p.rows, C = p.cols;
     const int64_t tiles_r = (R + COL_TILE_R - 1) / COL_TILE_R;
@@ -406,25 +489,50 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int blk = warp & 3;                       // 32-row block inside the tile
     const int pair = (warp >> 2) * 32 + lane;       // column pair inside the tile
+    // thread 0: the copy of tile `tile` into buffer b (TMA staging)
+    auto issue = [&](int64_t tile, int b) {
+        stage_expect(st.bars + 8 * b, TILE_BYTES);
+        tma_tile_load(st.base + b * TILE_BYTES, &tmap, static_cast<int>((tile % tiles_c) * COL_TILE_C),
+                      static_cast<int>((tile / tiles_c) * COL_TILE_R), st.bars + 8 * b);
+    };
+    if (TMA) {
+        if (threadIdx.x == 0) {
+            stage_bar_init(st.bars);
+            stage_bar_init(st.bars + 8);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        __syncthreads();
+    }
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");     // inputs of the previous kernel are visible
     int64_t t = blockIdx.x;
-    if (t < n_tiles) stage_tile<BF16_IN>(p, col_smem, (t / tiles_c) * COL_TILE_R, (t % tiles_c) * COL_TILE_C);
-    cp_async_commit();
-    for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1) {
-        const int64_t tn = t + gridDim.x;
-        if (tn < n_tiles)
-            stage_tile<BF16_IN>(p, col_smem + (buf ^ 1) * TILE_BYTES, (tn / tiles_c) * COL_TILE_R,
-                                (tn % tiles_c) * COL_TILE_C);
+    if (TMA) {
+        if (t < n_tiles && threadIdx.x == 0 && !(p.skip_first && blockIdx.x == 0)) issue(t, 0);
+    } else {
+        if (t < n_tiles) stage_tile<BF16_IN>(p, col_smem, (t / tiles_c) * COL_TILE_R, (t % tiles_c) * COL_TILE_C);
         cp_async_commit();
-        cp_async_wait_prev();        // this tile's copies (the older group) have landed
-        __syncthreads();
+    }
+    uint32_t use = 0;                // tiles this CTA has taken: buffer use % 2, phase (use / 2) % 2
+    bool ok = true;
+    for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1, ++use) {
+        const int64_t tn = t + gridDim.x;
+        if (TMA) {
+            if (tn < n_tiles && threadIdx.x == 0) issue(tn, buf ^ 1);
+            ok = stage_wait(st.bars + 8 * buf, (use >> 1) & 1u);
+        } else {
+            if (tn < n_tiles)
+                stage_tile<BF16_IN>(p, col_smem + (buf ^ 1) * TILE_BYTES, (tn / tiles_c) * COL_TILE_R,
+                                    (tn % tiles_c) * COL_TILE_C);
+            cp_async_commit();
+            cp_async_wait_prev();        // this tile's copies (the older group) have landed
+            __syncthreads();
+        }
 
         const int64_t r0 = (t / tiles_c) * COL_TILE_R, c0 = (t % tiles_c) * COL_TILE_C;
         const int64_t gc = c0 + 2 * pair, gr0 = r0 + blk * 32;
-        if (gc < C && gr0 < R) {
-            const TIn *tile = reinterpret_cast<const TIn *>(col_smem + buf * TILE_BYTES);
+        if (ok && gc < C && gr0 < R) {
+            const TIn *tile = reinterpret_cast<const TIn *>(tiles + buf * TILE_BYTES);
             // x[j] = (column gc, column gc + 1) at row gr0 + j, as packed f32x2
             uint64_t x[32];
             uint32_t words[32];
@@ -444,9 +552,18 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
             if (BF16_IN && !HAD) encode_col_pair<FMT, SR, false, true>(p, x, gc, gr0, bf16_pair_max<32>(words));
             else encode_col_pair<FMT, SR, HAD, false, DEFM>(p, x, gc, gr0);
         }
-        __syncthreads();             // everyone is done with `buf` before it is refilled
+        // everyone is done with `buf` before it is refilled; with TMA staging
+        // a wait that gave up (in any thread) ends the CTA's loop
+        if (TMA) {
+            if (!__syncthreads_and(ok)) {
+                if (threadIdx.x == 0) drain_staged(st.bars, buf, use, tn < n_tiles);
+                break;
+            }
+        } else {
+            __syncthreads();
+        }
     }
-    cp_async_wait_all();
+    if (!TMA) cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -460,14 +577,27 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p)
 // thread encodes one column pair of one 32-row block (as cast_cols) and two
 // 32-element row blocks (as cast_rows, RNE or SR with its own seed).  The
 // result equals mx_quantize along rows plus mx_quantize along columns.
-template <int FMT, bool BF16_IN, bool HAD, bool DEFM = false>
+// TMA: the tile is staged by tensor copies of `tmap` in boxes 128 bytes wide
+// (64 bf16 or 32 fp32 columns) with the copy engine's 128-byte swizzle: box h
+// of the tile occupies 16 KiB at h * 16 KiB, tile row r at r * 128 bytes, and
+// its 16-byte chunk c at position c XOR (r % 8).  The column reads (a warp
+// reads one 128-byte box row) and the row reads (eight lanes read the same
+// chunk of eight consecutive rows) then touch distinct banks.  Without TMA,
+// cp.async copies with the tile_chunk swizzle.
+template <int FMT, bool BF16_IN, bool HAD, bool DEFM, bool TMA>
 __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr, CastParams pc, int sr_rows,
-                                                                   int sr_cols) {
+                                                                   int sr_cols,
+                                                                   const __grid_constant__ CUtensorMap tmap) {
     using TIn = typename std::conditional<BF16_IN, uint16_t, float>::type;
     constexpr int TILE_BYTES = COL_TILE_R * COL_TILE_C * sizeof(TIn);
     constexpr int ROW_BYTES = COL_TILE_C * sizeof(TIn);
     constexpr int CPB = 32 * sizeof(TIn) / 16;              // 16-byte chunks per 32-element row block
+    constexpr int BOX_C = 128 / sizeof(TIn);                // columns per 128-byte box (TMA)
+    constexpr int BOXES = COL_TILE_C / BOX_C;
+    constexpr int BOX_BYTES = COL_TILE_R * 128;
     extern __shared__ __align__(16) uint8_t col_smem[];
+    const StagedTiles<1024> st(col_smem, TILE_BYTES);
+    uint8_t *const tiles = TMA ? st.tiles : col_smem;
 
     const int64_t R = pc.rows, C = pc.cols;
     const int64_t tiles_r = (R + COL_TILE_R - 1) / COL_TILE_R;
@@ -476,38 +606,71 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int blk = warp & 3;                       // column part: 32-row block inside the tile
     const int pair = (warp >> 2) * 32 + lane;       // column part: column pair inside the tile
-    const int rb = threadIdx.x & 3;                 // row part: 32-column block inside the tile
-    const int rrow = threadIdx.x >> 2;              // row part: tile rows rrow and rrow + 64
+    // row part: 32-column block rb of tile rows rrow and rrow + 64 (with TMA,
+    // eight consecutive lanes take the same block of eight consecutive rows)
+    const int rb = TMA ? (lane >> 3) : (threadIdx.x & 3);
+    const int rrow = TMA ? (warp * 8 + (lane & 7)) : (threadIdx.x >> 2);
 
-    // the column pair's byte offset inside even and odd tile rows
+    // the column pair's byte offset inside even and odd tile rows (cp.async
+    // layout), or inside tile row blk * 32 before the row's swizzle (TMA)
     const int cbyte = 2 * pair * static_cast<int>(sizeof(TIn));
     const int col_off[2] = {tile_chunk<BF16_IN, true>(0, cbyte >> 4) * 16 + (cbyte & 15),
                             tile_chunk<BF16_IN, true>(1, cbyte >> 4) * 16 + (cbyte & 15)};
+    const int col_box = (cbyte >> 7) * BOX_BYTES + blk * 32 * 128 + (cbyte & 127);
+
+    auto issue = [&](int64_t tile, int b) {     // thread 0, TMA staging
+        stage_expect(st.bars + 8 * b, TILE_BYTES);
+        const int x0 = static_cast<int>((tile % tiles_c) * COL_TILE_C), y0 = static_cast<int>((tile / tiles_c) * COL_TILE_R);
+#pragma unroll
+        for (int h = 0; h < BOXES; ++h)
+            tma_tile_load(st.base + b * TILE_BYTES + h * BOX_BYTES, &tmap, x0 + h * BOX_C, y0, st.bars + 8 * b);
+    };
+    if (TMA) {
+        if (threadIdx.x == 0) {
+            stage_bar_init(st.bars);
+            stage_bar_init(st.bars + 8);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        __syncthreads();
+    }
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");     // inputs of the previous kernel are visible
     int64_t t = blockIdx.x;
-    if (t < n_tiles) stage_tile<BF16_IN, true>(pc, col_smem, (t / tiles_c) * COL_TILE_R, (t % tiles_c) * COL_TILE_C);
-    cp_async_commit();
-    for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1) {
-        const int64_t tn = t + gridDim.x;
-        if (tn < n_tiles)
-            stage_tile<BF16_IN, true>(pc, col_smem + (buf ^ 1) * TILE_BYTES, (tn / tiles_c) * COL_TILE_R,
-                                      (tn % tiles_c) * COL_TILE_C);
+    if (TMA) {
+        if (t < n_tiles && threadIdx.x == 0 && !(pc.skip_first && blockIdx.x == 0)) issue(t, 0);
+    } else {
+        if (t < n_tiles) stage_tile<BF16_IN, true>(pc, col_smem, (t / tiles_c) * COL_TILE_R, (t % tiles_c) * COL_TILE_C);
         cp_async_commit();
-        cp_async_wait_prev();        // this tile's copies (the older group) have landed
-        __syncthreads();
+    }
+    uint32_t use = 0;                // tiles this CTA has taken: buffer use % 2, phase (use / 2) % 2
+    bool ok = true;
+    for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1, ++use) {
+        const int64_t tn = t + gridDim.x;
+        if (TMA) {
+            if (tn < n_tiles && threadIdx.x == 0) issue(tn, buf ^ 1);
+            ok = stage_wait(st.bars + 8 * buf, (use >> 1) & 1u);
+        } else {
+            if (tn < n_tiles)
+                stage_tile<BF16_IN, true>(pc, col_smem + (buf ^ 1) * TILE_BYTES, (tn / tiles_c) * COL_TILE_R,
+                                          (tn % tiles_c) * COL_TILE_C);
+            cp_async_commit();
+            cp_async_wait_prev();        // this tile's copies (the older group) have landed
+            __syncthreads();
+        }
 
-        const uint8_t *tile = col_smem + buf * TILE_BYTES;
+        const uint8_t *tile = tiles + buf * TILE_BYTES;
         const int64_t r0 = (t / tiles_c) * COL_TILE_R, c0 = (t % tiles_c) * COL_TILE_C;
         // ---- column blocks ----
         const int64_t gc = c0 + 2 * pair, gr0 = r0 + blk * 32;
-        if (gc < C && gr0 < R) {
+        if (ok && gc < C && gr0 < R) {
             uint64_t x[32];
             uint32_t words[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const uint8_t *src = tile + (blk * 32 + j) * ROW_BYTES + col_off[j & 1];
+                // TMA: row blk * 32 + j, whose chunks are permuted by j % 8
+                const uint8_t *src = TMA ? tile + ((col_box ^ ((j & 7) << 4)) + j * 128)
+                                         : tile + (blk * 32 + j) * ROW_BYTES + col_off[j & 1];
                 if (BF16_IN) {
                     uint32_t w = *reinterpret_cast<const uint32_t *>(src);
                     words[j] = w;
@@ -532,13 +695,16 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
         for (int h = 0; h < 2; ++h) {
             const int rr = rrow + 64 * h;
             const int64_t row = r0 + rr, kb = (c0 >> 5) + rb;
-            if (row >= R || 32 * kb >= C) continue;
+            if (!ok || row >= R || 32 * kb >= C) continue;
             uint32_t b[32];
             uint32_t words[16];
 #pragma unroll
             for (int i = 0; i < CPB; ++i) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(
-                    tile + rr * ROW_BYTES + tile_chunk<BF16_IN, true>(rr, rb * CPB + i) * 16);
+                // chunk q of the row: box q / 8, chunk q % 8 permuted by rr % 8 (TMA)
+                const int q = rb * CPB + i;
+                const int off = TMA ? (q >> 3) * BOX_BYTES + rr * 128 + (((q & 7) ^ (rr & 7)) << 4)
+                                    : rr * ROW_BYTES + tile_chunk<BF16_IN, true>(rr, q) * 16;
+                const uint4 w = *reinterpret_cast<const uint4 *>(tile + off);
                 if (BF16_IN) {
                     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -560,9 +726,18 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
                 else encode_row_block<FMT, false, false>(pr, row, kb, b);
             }
         }
-        __syncthreads();             // everyone is done with `buf` before it is refilled
+        // everyone is done with `buf` before it is refilled; with TMA staging
+        // a wait that gave up (in any thread) ends the CTA's loop
+        if (TMA) {
+            if (!__syncthreads_and(ok)) {
+                if (threadIdx.x == 0) drain_staged(st.bars, buf, use, tn < n_tiles);
+                break;
+            }
+        } else {
+            __syncthreads();
+        }
     }
-    cp_async_wait_all();
+    if (!TMA) cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -719,14 +894,50 @@ static cudaError_t launch_overlapped(int grid, int block, int smem, cudaStream_t
     return cudaLaunchKernelEx(&cfg, Kernel, args...);
 }
 
+// Testing hooks (include/mx_debug.h), per host thread.
+thread_local bool t_force_cpasync = false;
+thread_local bool t_skip_first = false;
+
+// Tensor map of a cast's input for TMA staging: the rows x cols tensor in
+// boxes of 128 rows x 128 columns, unswizzled (column cast), or x 128 bytes
+// with the 128-byte swizzle (dual cast).  False when the input cannot be
+// staged that way (base address or row pitch not a multiple of 16 bytes, a
+// coordinate beyond int32, an encoding the driver refuses): the kernels then
+// stage with cp.async.
+static bool make_input_map(CUtensorMap *map, const CastParams &p, bool bf16, bool swizzled) {
+    if (t_force_cpasync) return false;
+    const int64_t esz = bf16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(p.x) & 15u) != 0 || ((p.ldx * esz) & 15) != 0) return false;
+    if (p.rows > INT32_MAX - COL_TILE_R || p.cols > INT32_MAX - COL_TILE_C) return false;
+    return mxg::encode_2d(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.x,
+                          static_cast<uint64_t>(p.cols), static_cast<uint64_t>(p.rows),
+                          static_cast<uint64_t>(p.ldx * esz), swizzled ? static_cast<uint32_t>(128 / esz) : COL_TILE_C,
+                          COL_TILE_R, swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Dynamic shared memory of the column and dual casts: two tile buffers, their
+// two staging barriers, and slack to align the buffers for TMA.
+static int staged_smem_bytes(int in_bytes, int align) {
+    return 2 * COL_TILE_R * COL_TILE_C * in_bytes + 16 + align;
+}
+
 // Column cast: two tile buffers of dynamic shared memory, a resident grid.
 template <auto Kernel>
-static cudaError_t launch_cols(int in_bytes, const CastParams &p, int64_t tiles, int sms, cudaStream_t st) {
-    const int smem = 2 * COL_TILE_R * COL_TILE_C * in_bytes;
+static cudaError_t launch_cols(int in_bytes, const CastParams &p, int64_t tiles, int sms, cudaStream_t st,
+                               const CUtensorMap &map) {
+    const int smem = staged_smem_bytes(in_bytes, 128);
     static std::atomic<uint64_t> configured{0};    // per kernel, one bit per device
     if (cudaError_t e = ensure_smem_limit(Kernel, smem, configured); e != cudaSuccess) return e;
     return launch_overlapped<Kernel>(grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)),
-                                     COL_THREADS, smem, st, p);
+                                     COL_THREADS, smem, st, p, map);
+}
+
+// The TMA-staged instance when `map` is set, else the cp.async one.
+template <int FMT, bool SR, bool BF, bool HAD, bool DEFM>
+static cudaError_t launch_cols_staged(const CastParams &p, int64_t tiles, int sms, cudaStream_t st,
+                                      const CUtensorMap *map) {
+    if (map) return launch_cols<cast_cols_kernel<FMT, SR, BF, HAD, DEFM, true>>(BF ? 2 : 4, p, tiles, sms, st, *map);
+    return launch_cols<cast_cols_kernel<FMT, SR, BF, HAD, DEFM, false>>(BF ? 2 : 4, p, tiles, sms, st, CUtensorMap{});
 }
 
 template <int FMT, bool SR>
@@ -758,16 +969,18 @@ static cudaError_t launch_cast_fmt(const CastParams &p, int xdt, int block_axis,
         }
     } else {
         const int64_t tiles = ((p.rows + COL_TILE_R - 1) / COL_TILE_R) * ((p.cols + COL_TILE_C - 1) / COL_TILE_C);
+        CUtensorMap m;
+        const CUtensorMap *map = make_input_map(&m, p, bf, false) ? &m : nullptr;
         if (had && p.sign_mask == MX_DEFAULT_SIGN_MASK) {
-            if (bf) return launch_cols<cast_cols_kernel<FMT, SR, true, true, true>>(2, p, tiles, sms, st);
-            return launch_cols<cast_cols_kernel<FMT, SR, false, true, true>>(4, p, tiles, sms, st);
+            if (bf) return launch_cols_staged<FMT, SR, true, true, true>(p, tiles, sms, st, map);
+            return launch_cols_staged<FMT, SR, false, true, true>(p, tiles, sms, st, map);
         }
         if (had) {
-            if (bf) return launch_cols<cast_cols_kernel<FMT, SR, true, true>>(2, p, tiles, sms, st);
-            return launch_cols<cast_cols_kernel<FMT, SR, false, true>>(4, p, tiles, sms, st);
+            if (bf) return launch_cols_staged<FMT, SR, true, true, false>(p, tiles, sms, st, map);
+            return launch_cols_staged<FMT, SR, false, true, false>(p, tiles, sms, st, map);
         }
-        if (bf) return launch_cols<cast_cols_kernel<FMT, SR, true, false>>(2, p, tiles, sms, st);
-        return launch_cols<cast_cols_kernel<FMT, SR, false, false>>(4, p, tiles, sms, st);
+        if (bf) return launch_cols_staged<FMT, SR, true, false, false>(p, tiles, sms, st, map);
+        return launch_cols_staged<FMT, SR, false, false, false>(p, tiles, sms, st, map);
     }
     return cudaGetLastError();
 }
@@ -782,12 +995,22 @@ static cudaError_t launch_cast_rnd(const CastParams &p, int xdt, int block_axis,
 // Dual cast: the column cast's tile buffers and resident grid.
 template <auto Kernel>
 static cudaError_t launch_dual(int in_bytes, const CastParams &pr, const CastParams &pc, int sr_rows, int sr_cols,
-                               int64_t tiles, int sms, cudaStream_t st) {
-    const int smem = 2 * COL_TILE_R * COL_TILE_C * in_bytes;
+                               int64_t tiles, int sms, cudaStream_t st, const CUtensorMap &map) {
+    const int smem = staged_smem_bytes(in_bytes, 1024);
     static std::atomic<uint64_t> configured{0};    // per kernel, one bit per device
     if (cudaError_t e = ensure_smem_limit(Kernel, smem, configured); e != cudaSuccess) return e;
     return launch_overlapped<Kernel>(grid_for(tiles, 1, sms * resident_blocks_per_sm<Kernel>(COL_THREADS, smem)),
-                                     COL_THREADS, smem, st, pr, pc, sr_rows, sr_cols);
+                                     COL_THREADS, smem, st, pr, pc, sr_rows, sr_cols, map);
+}
+
+template <int FMT, bool BF, bool HAD, bool DEFM>
+static cudaError_t launch_dual_staged(const CastParams &pr, const CastParams &pc, int sr_rows, int sr_cols,
+                                      int64_t tiles, int sms, cudaStream_t st, const CUtensorMap *map) {
+    if (map)
+        return launch_dual<cast_dual_kernel<FMT, BF, HAD, DEFM, true>>(BF ? 2 : 4, pr, pc, sr_rows, sr_cols, tiles,
+                                                                       sms, st, *map);
+    return launch_dual<cast_dual_kernel<FMT, BF, HAD, DEFM, false>>(BF ? 2 : 4, pr, pc, sr_rows, sr_cols, tiles, sms,
+                                                                    st, CUtensorMap{});
 }
 
 template <int FMT>
@@ -795,16 +1018,18 @@ static cudaError_t launch_dual_fmt(const CastParams &pr, const CastParams &pc, i
                                    int sr_cols, int sms, cudaStream_t st) {
     const int64_t tiles = ((pc.rows + COL_TILE_R - 1) / COL_TILE_R) * ((pc.cols + COL_TILE_C - 1) / COL_TILE_C);
     const bool bf = xdt == MX_BF16;
+    CUtensorMap m;
+    const CUtensorMap *map = make_input_map(&m, pc, bf, true) ? &m : nullptr;
     if (had && pc.sign_mask == MX_DEFAULT_SIGN_MASK) {
-        if (bf) return launch_dual<cast_dual_kernel<FMT, true, true, true>>(2, pr, pc, sr_rows, sr_cols, tiles, sms, st);
-        return launch_dual<cast_dual_kernel<FMT, false, true, true>>(4, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+        if (bf) return launch_dual_staged<FMT, true, true, true>(pr, pc, sr_rows, sr_cols, tiles, sms, st, map);
+        return launch_dual_staged<FMT, false, true, true>(pr, pc, sr_rows, sr_cols, tiles, sms, st, map);
     }
     if (had) {
-        if (bf) return launch_dual<cast_dual_kernel<FMT, true, true>>(2, pr, pc, sr_rows, sr_cols, tiles, sms, st);
-        return launch_dual<cast_dual_kernel<FMT, false, true>>(4, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+        if (bf) return launch_dual_staged<FMT, true, true, false>(pr, pc, sr_rows, sr_cols, tiles, sms, st, map);
+        return launch_dual_staged<FMT, false, true, false>(pr, pc, sr_rows, sr_cols, tiles, sms, st, map);
     }
-    if (bf) return launch_dual<cast_dual_kernel<FMT, true, false>>(2, pr, pc, sr_rows, sr_cols, tiles, sms, st);
-    return launch_dual<cast_dual_kernel<FMT, false, false>>(4, pr, pc, sr_rows, sr_cols, tiles, sms, st);
+    if (bf) return launch_dual_staged<FMT, true, false, false>(pr, pc, sr_rows, sr_cols, tiles, sms, st, map);
+    return launch_dual_staged<FMT, false, false, false>(pr, pc, sr_rows, sr_cols, tiles, sms, st, map);
 }
 
 }  // namespace mxk
@@ -826,6 +1051,11 @@ cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st) {
     p.sign_mask = a.sign_mask;
     p.sr_base = a.sr_base;
     p.sr_stride = a.sr_stride;
+    p.skip_first = 0;
+    if (a.block_axis == 0) {         // the one-shot hook applies to staged (column) casts
+        p.skip_first = t_skip_first ? 1 : 0;
+        t_skip_first = false;
+    }
     const bool sr = a.rnd == MX_SR;
     switch (a.fmt) {
         case MX_E4M3: return launch_cast_rnd<MX_E4M3>(p, a.xdt, a.block_axis, sr, a.hadamard, a.num_sms, st);
@@ -895,6 +1125,9 @@ cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st
     pc.sign_mask = a.sign_mask;
     pc.sr_base = a.sr_base_cols;
     pc.sr_stride = a.sr_stride_cols;
+    pr.skip_first = 0;
+    pc.skip_first = t_skip_first ? 1 : 0;
+    t_skip_first = false;
     const int sr_r = a.rnd_rows == MX_SR, sr_c = a.rnd_cols == MX_SR;
     switch (a.fmt) {
         case MX_E4M3: return launch_dual_fmt<MX_E4M3>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);
@@ -905,4 +1138,23 @@ cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st
         case MX_INT8: return launch_dual_fmt<MX_INT8>(pr, pc, a.xdt, a.hadamard, sr_r, sr_c, a.num_sms, st);
     }
     return cudaErrorInvalidValue;
+}
+
+// Reads and clears the casts' status word (after the caller synchronised).
+int mx_read_cast_status() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, mxk::g_cast_status, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(mxk::g_cast_status, &zero, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
+    return v;
+}
+
+extern "C" int mx_debug_cast_force_cpasync(int on) {
+    mxk::t_force_cpasync = on != 0;
+    return MX_OK;
+}
+
+extern "C" int mx_debug_cast_skip_tile(int on) {
+    mxk::t_skip_first = on != 0;
+    return MX_OK;
 }

@@ -5,6 +5,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "mx.h"
@@ -106,6 +107,16 @@ cudaError_t mx_launch_quantize_nvfp4(const MxNvfp4Args &a, cudaStream_t st);
 int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st);
 // reads and clears the device status word of the current device (after a sync)
 int mx_read_device_status(cudaStream_t st);
+// reads and clears the cast kernels' status word (the caller has synchronised)
+int mx_read_cast_status();
+
+namespace mxg {
+// Encodes (or takes from a per-process cache) a 2-D tiled tensor map: d0 x d1
+// elements of type dt at base, row stride `stride` bytes, boxes of b0 x b1,
+// no interleave, zero fill outside the tensor.  False if the driver refuses.
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t d0, uint64_t d1,
+               uint64_t stride, uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz);
+}
 
 // Raises a kernel's dynamic shared-memory limit on the current device the
 // first time that device launches it.  The attribute belongs to the device's

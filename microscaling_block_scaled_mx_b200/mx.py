@@ -117,6 +117,10 @@ def lib() -> ctypes.CDLL:
             L.mx_debug_gemm_skip_stage.argtypes = [i32]
             L.mx_debug_gemm_force_kernel.restype = i32
             L.mx_debug_gemm_force_kernel.argtypes = [i32]
+            L.mx_debug_cast_force_cpasync.restype = i32
+            L.mx_debug_cast_force_cpasync.argtypes = [i32]
+            L.mx_debug_cast_skip_tile.restype = i32
+            L.mx_debug_cast_skip_tile.argtypes = [i32]
             _lib = L
     return _lib
 
