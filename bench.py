@@ -545,7 +545,9 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
         for (M, N, K, ac, as_, bc, bs, c) in ops:
             mx.gemm(ac, as_, bc, bs, M, N, K, fa=fmt, out=c, scale_layout=sl)
 
-    ms = timed_region(step, args.steps)
+    with ClockSampler(dev.index or 0) as clk:
+        ms = timed_region(step, args.steps)
+    clocks = clk.summary()
     launches = len(ops) * args.steps
     value = world * flops_step * args.steps / (ms * 1e-3) / 1e12
     per_shape = {}
@@ -597,7 +599,11 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
                                  "fused_us": round(res["fused"], 1),
                                  "speedup": round(res["gemm_then_cast"] / res["fused"], 3)}
     ratio = 4.0 if fmt == "e2m1" else 2.0             # nominal fp4 : fp8 : bf16 = 9 : 4.5 : 2.25
-    peak = ratio * float(peaks["bf16_tflops"])
+    # A GEMM loop of a quarter second or more runs into the board's power cap
+    # and settles at the sustained clock: the sustained cuBLAS figure is its
+    # denominator then, the burst one for a shorter loop.
+    sustained = ms >= 250.0
+    peak = ratio * float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
     if fmt == "e2m1":
         workload = ("llama3_8b_mxfp4_gemms_m8192 (4096->6144, 4096->14336, 14336->4096), bf16 out, "
                     "x4 operand scales")
@@ -641,8 +647,9 @@ def run_gemm_phase(args, dev, stream, peaks, peak_kind, barrier, max_over_ranks,
             "roofline": {"bound": "tensor", "kernel": kernel,
                          "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4),
-                         "peak_kind": f"{peak_kind} bf16 burst x {ratio:g} (nominal ratio for the operand type)",
-                         "traffic": traffic, "per_shape": per_shape},
+                         "peak_kind": f"{peak_kind} bf16 {'sustained' if sustained else 'burst'} x {ratio:g} "
+                                      f"(nominal ratio for the operand type; timed loop {ms:.0f} ms)",
+                         "clocks": clocks, "traffic": traffic, "per_shape": per_shape},
             "quantizing_epilogue": fused,
             "along_m": along_m,
             "_launches": launches}
