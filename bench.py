@@ -54,10 +54,10 @@ MEASURED_TRAFFIC = {
     # --cache-control none, so each launch also carries the write-back of its
     # predecessor's output still in L2 (steady state: reads + writes of one cast)
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "fd12806ddd982f7d8ade8fbaff3a2fb32e12af6eef26beb9256acfbf6d8c5916",
-                  {"e4m3_bf16_8192x8192": 201026048, "e5m2_bf16_8192x8192": 201932800,
-                   "e2m3_bf16_8192x8192": 186476544, "e3m2_bf16_8192x8192": 186476288,
-                   "e2m1_bf16_8192x8192": 170484480, "int8_bf16_8192x8192": 203712256}),
+                  "ee3a7c00ba6555c8e6c466c1c7004995e131e3aeb5d5ebeba7e82b3dbd2e2aa1",
+                  {"e4m3_bf16_8192x8192": 134246912 + 68575744, "e5m2_bf16_8192x8192": 134269184 + 68492544,
+                   "e2m3_bf16_8192x8192": 134221312 + 52434688, "e3m2_bf16_8192x8192": 134225920 + 52307200,
+                   "e2m1_bf16_8192x8192": 134224128 + 36084224, "int8_bf16_8192x8192": 134248704 + 68609536}),
     # the GEMMs: default cache control (L2 flushed before the launch), so reads
     # show re-reads and writes count only what left L2 during the launch; "x4":
     # operands with x4 scales
@@ -75,13 +75,13 @@ MEASURED_TRAFFIC = {
 # issue roofline of those casts: at most 4 warp instructions per clock per SM.
 MEASURED_INSTR = {
     "cast_cols_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                         "fd12806ddd982f7d8ade8fbaff3a2fb32e12af6eef26beb9256acfbf6d8c5916",
-                         {"e2m1_bf16_x4_16384x4096": 39026624 / (16384 * 4096),
-                          "e2m1_bf16_x4_16384x14336": 136101824 / (16384 * 14336)}),
+                         "ee3a7c00ba6555c8e6c466c1c7004995e131e3aeb5d5ebeba7e82b3dbd2e2aa1",
+                         {"e2m1_bf16_x4_16384x4096": 27703560 / (16384 * 4096),
+                          "e2m1_bf16_x4_16384x14336": 96526600 / (16384 * 14336)}),
     "cast_dual_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                         "fd12806ddd982f7d8ade8fbaff3a2fb32e12af6eef26beb9256acfbf6d8c5916",
-                         {"e2m1_bf16_16384x4096": 52669952 / (16384 * 4096),
-                          "e2m1_bf16_16384x14336": 183823872 / (16384 * 14336)}),
+                         "ee3a7c00ba6555c8e6c466c1c7004995e131e3aeb5d5ebeba7e82b3dbd2e2aa1",
+                         {"e2m1_bf16_16384x4096": 41922952 / (16384 * 4096),
+                          "e2m1_bf16_16384x14336": 146329992 / (16384 * 14336)}),
 }
 
 
