@@ -424,11 +424,11 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
         constexpr int SLOT = BITS == 4 ? 4 : 8;
         uint32_t pw[8];
         if (SR) {
-            const uint32_t g = static_cast<uint32_t>(
-                (p.sr_base + static_cast<uint64_t>(oc) * p.sr_stride + static_cast<uint64_t>(gr0)) >> 2);
+            uint32_t rw[8];
+            sr_block_words(p.sr_base + static_cast<uint64_t>(oc) * p.sr_stride + static_cast<uint64_t>(gr0), p.key, rw);
 #pragma unroll
             for (int w = 0; w < 8; ++w)
-                pw[w] = sr_quad<FMT>(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3], fmix32((g + w) ^ p.key));
+                pw[w] = sr_quad<FMT>(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3], rw[w]);
         } else {
 #pragma unroll
             for (int w = 0; w < 8; ++w)

@@ -201,14 +201,34 @@ __device__ __forceinline__ float max_abs3(float m, float a, float b) {
     return r;
 }
 
-// MurmurHash3 32-bit finaliser (public domain, A. Appleby).
-__device__ __forceinline__ uint32_t fmix32(uint32_t h) {
-    h ^= h >> 16;
+// MurmurHash3 32-bit finaliser (public domain, A. Appleby), and its steps
+// after the first (h ^= h >> 16).
+__device__ __forceinline__ uint32_t fmix32_rest(uint32_t h) {
     h *= 0x85ebca6bu;
     h ^= h >> 13;
     h *= 0xc2b2ae35u;
     h ^= h >> 16;
     return h;
+}
+__device__ __forceinline__ uint32_t fmix32(uint32_t h) { return fmix32_rest(h ^ (h >> 16)); }
+
+// The eight random words of a 32-value block whose first value has
+// stochastic-rounding index i0: word w = fmix32((floor(i0 / 4) + w) ^ key),
+// whose bytes round values 4w .. 4w + 3.  When i0 is a multiple of 32 the
+// words are g .. g + 7 with g a multiple of 8, so (g + w) ^ key = G ^ w for
+// G = g ^ key, and the finaliser's first step maps G ^ w to H ^ w for
+// H = G ^ (G >> 16) (w < 8 leaves the high half alone): one XOR per word
+// replaces the add, the key XOR and that step.
+__device__ __forceinline__ void sr_block_words(uint64_t i0, uint32_t key, uint32_t (&rw)[8]) {
+    const uint32_t g = static_cast<uint32_t>(i0 >> 2);
+    if ((i0 & 31u) == 0) {
+        const uint32_t G = g ^ key, H = G ^ (G >> 16);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) rw[w] = fmix32_rest(H ^ static_cast<uint32_t>(w));
+    } else {
+#pragma unroll
+        for (int w = 0; w < 8; ++w) rw[w] = fmix32((g + static_cast<uint32_t>(w)) ^ key);
+    }
 }
 
 // Byte offset of the scale of (outer row o, k-block kb) in the MMA layout:

@@ -110,11 +110,11 @@ __device__ __forceinline__ void encode_block32_amax(const BlockSink &o, int64_t 
     constexpr int SLOT = BITS == 4 ? 4 : 8;
     uint32_t pw[8];
     if (SR) {
-        const uint32_t g = static_cast<uint32_t>(
-            (o.sr_base + static_cast<uint64_t>(row) * o.sr_stride + static_cast<uint64_t>(kb * 32)) >> 2);
+        uint32_t rw[8];
+        sr_block_words(o.sr_base + static_cast<uint64_t>(row) * o.sr_stride + static_cast<uint64_t>(kb * 32), o.key, rw);
 #pragma unroll
         for (int w = 0; w < 8; ++w)
-            pw[w] = sr_quad<FMT>(u[4 * w], u[4 * w + 1], u[4 * w + 2], u[4 * w + 3], fmix32((g + w) ^ o.key));
+            pw[w] = sr_quad<FMT>(u[4 * w], u[4 * w + 1], u[4 * w + 2], u[4 * w + 3], rw[w]);
     } else {
 #pragma unroll
         for (int w = 0; w < 8; ++w)
