@@ -42,6 +42,7 @@ struct CastParams {
     // stochastic-rounding position of output element (o, i): sr_base + o * sr_stride + i
     uint64_t sr_base, sr_stride;
     int skip_first;      // testing hook: CTA 0 withholds the copy of its first staged tile
+    int stage_scales;    // column casts: a full tile's scale atom goes out through shared memory
 };
 
 __device__ __forceinline__ void store_scale(const CastParams &p, int64_t o, int64_t kb, uint32_t s) {
@@ -289,19 +290,23 @@ __device__ __forceinline__ bool stage_wait(uint32_t bar, uint32_t parity, unsign
     return stage_try_wait(bar, parity) || stage_wait_slow(bar, parity, limit);
 }
 
-// Shared-memory layout of a TMA-staged tile: the buffers start at the first
+// Shared-memory layout of a staged tile: the buffers start at the first
 // ALIGN boundary of the dynamic buffer (1024 bytes for the 128-byte swizzle,
-// whose pattern repeats every 1024 bytes), followed by one mbarrier per buffer.
+// whose pattern repeats every 1024 bytes), followed by one mbarrier per buffer
+// and two 512-byte scale atoms (one per buffer).  The cp.async path uses the
+// same layout with ALIGN's slack left unused.
 template <int ALIGN>
 struct StagedTiles {
     uint8_t *tiles;     // generic pointer to buffer 0
     uint32_t base;      // its shared-memory address
     uint32_t bars;      // barrier of buffer b at bars + 8 b
+    uint8_t *atoms;     // scale atom of buffer b at atoms + 512 b
     __device__ StagedTiles(uint8_t *raw, int tile_bytes) {
         const uint32_t r = static_cast<uint32_t>(__cvta_generic_to_shared(raw));
         base = (r + ALIGN - 1) & ~static_cast<uint32_t>(ALIGN - 1);
         tiles = raw + (base - r);
         bars = base + 2 * tile_bytes;
+        atoms = tiles + 2 * tile_bytes + 16;
     }
 };
 
@@ -356,9 +361,11 @@ __device__ __forceinline__ constexpr bool default_mask_negates(int j) {
 
 // SIGNED: the caller has already applied the Hadamard's sign flips to x
 // (the default mask, folded into the loads).
+// satom: when set, the scale bytes go to this 512-byte shared-memory copy of
+// the tile's scale atom (the caller writes the atom out), else to global memory.
 template <int FMT, bool SR, bool HAD, bool KEYED = false, bool SIGNED = false>
 __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&x)[32], int64_t gc, int64_t gr0,
-                                                uint32_t pair_max16 = 0) {
+                                                uint32_t pair_max16 = 0, uint8_t *satom = nullptr) {
     static_assert(!(KEYED && HAD), "the bf16 maxima describe the values before the Hadamard");
     constexpr int BITS = Fmt<FMT>::bits;
     const int64_t R = p.rows, C = p.cols;
@@ -459,8 +466,31 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
                 dst[q] = w & (static_cast<uint64_t>(keep) << 32 | keep);
             }
         }
-        store_scale(p, oc, gr0 >> 5, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
+        const uint32_t sbyte = nan_block ? 0xffu : static_cast<uint32_t>(e + 127);
+        if (satom)
+            satom[((oc & 31) << 4) + (((oc >> 5) & 3) << 2) + ((gr0 >> 5) & 3)] = static_cast<uint8_t>(sbyte);
+        else
+            store_scale(p, oc, gr0 >> 5, sbyte);
     }
+}
+
+// A column tile's scales: 128 columns (outer rows of the output) x 4 blocks
+// down the tile, exactly one 512-byte atom of the MMA layout (the tile's first
+// column and row are multiples of 128).  For a full tile the encoders write
+// the atom's bytes into shared memory and, after the tile's barrier, warp j
+// writes copy j of it (one copy in the MMA layout, four in the x4 layout) with
+// one 16-byte store per lane: 16 or 64 whole 32-byte sectors per tile instead
+// of 512 or 2048 scattered single bytes.
+__device__ __forceinline__ bool tile_stages_scales(const CastParams &p, int64_t r0, int64_t c0) {
+    return p.stage_scales && r0 + COL_TILE_R <= p.rows && c0 + COL_TILE_C <= p.cols;
+}
+__device__ __forceinline__ void write_scale_atom(const CastParams &p, const uint8_t *satom, int64_t r0, int64_t c0,
+                                                 int warp, int lane) {
+    const int copies = p.mma_scales == SL_MMA_X4 ? 4 : 1;
+    if (warp >= copies) return;
+    const int64_t atom = (c0 >> 7) * p.k_groups + (r0 >> 7);
+    uint8_t *dst = p.scales + (atom << (copies == 4 ? 11 : 9)) + warp * 512;
+    reinterpret_cast<uint4 *>(dst)[lane] = reinterpret_cast<const uint4 *>(satom)[lane];
 }
 
 // After a staging wait gave up at tile use `use` (buffer `buf`): wait, again
@@ -531,6 +561,8 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p,
 
         const int64_t r0 = (t / tiles_c) * COL_TILE_R, c0 = (t % tiles_c) * COL_TILE_C;
         const int64_t gc = c0 + 2 * pair, gr0 = r0 + blk * 32;
+        const bool stage_sc = tile_stages_scales(p, r0, c0);
+        uint8_t *const satom = stage_sc ? st.atoms + buf * 512 : nullptr;
         if (ok && gc < C && gr0 < R) {
             const TIn *tile = reinterpret_cast<const TIn *>(tiles + buf * TILE_BYTES);
             // x[j] = (column gc, column gc + 1) at row gr0 + j, as packed f32x2
@@ -549,11 +581,12 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p,
                     if (HAD && DEFM && default_mask_negates(j)) x[j] ^= 0x8000000080000000ull;
                 }
             }
-            if (BF16_IN && !HAD) encode_col_pair<FMT, SR, false, true>(p, x, gc, gr0, bf16_pair_max<32>(words));
-            else encode_col_pair<FMT, SR, HAD, false, DEFM>(p, x, gc, gr0);
+            if (BF16_IN && !HAD) encode_col_pair<FMT, SR, false, true>(p, x, gc, gr0, bf16_pair_max<32>(words), satom);
+            else encode_col_pair<FMT, SR, HAD, false, DEFM>(p, x, gc, gr0, 0u, satom);
         }
-        // everyone is done with `buf` before it is refilled; with TMA staging
-        // a wait that gave up (in any thread) ends the CTA's loop
+        // everyone is done with `buf` (and has written its scale bytes) before
+        // it is refilled; with TMA staging a wait that gave up (in any thread)
+        // ends the CTA's loop
         if (TMA) {
             if (!__syncthreads_and(ok)) {
                 if (threadIdx.x == 0) drain_staged(st.bars, buf, use, tn < n_tiles);
@@ -562,6 +595,7 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_cols_kernel(CastParams p,
         } else {
             __syncthreads();
         }
+        if (stage_sc) write_scale_atom(p, satom, r0, c0, warp, lane);
     }
     if (!TMA) cp_async_wait_all();
 }
@@ -661,6 +695,8 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
 
         const uint8_t *tile = tiles + buf * TILE_BYTES;
         const int64_t r0 = (t / tiles_c) * COL_TILE_R, c0 = (t % tiles_c) * COL_TILE_C;
+        const bool stage_sc = tile_stages_scales(pc, r0, c0);
+        uint8_t *const satom = stage_sc ? st.atoms + buf * 512 : nullptr;
         // ---- column blocks ----
         const int64_t gc = c0 + 2 * pair, gr0 = r0 + blk * 32;
         if (ok && gc < C && gr0 < R) {
@@ -683,11 +719,11 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
             }
             if (BF16_IN && !HAD) {
                 const uint32_t m16 = bf16_pair_max<32>(words);
-                if (sr_cols) encode_col_pair<FMT, true, false, true>(pc, x, gc, gr0, m16);
-                else encode_col_pair<FMT, false, false, true>(pc, x, gc, gr0, m16);
+                if (sr_cols) encode_col_pair<FMT, true, false, true>(pc, x, gc, gr0, m16, satom);
+                else encode_col_pair<FMT, false, false, true>(pc, x, gc, gr0, m16, satom);
             } else {
-                if (sr_cols) encode_col_pair<FMT, true, HAD, false, DEFM>(pc, x, gc, gr0);
-                else encode_col_pair<FMT, false, HAD, false, DEFM>(pc, x, gc, gr0);
+                if (sr_cols) encode_col_pair<FMT, true, HAD, false, DEFM>(pc, x, gc, gr0, 0u, satom);
+                else encode_col_pair<FMT, false, HAD, false, DEFM>(pc, x, gc, gr0, 0u, satom);
             }
         }
         // ---- row blocks ----
@@ -726,8 +762,9 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
                 else encode_row_block<FMT, false, false>(pr, row, kb, b);
             }
         }
-        // everyone is done with `buf` before it is refilled; with TMA staging
-        // a wait that gave up (in any thread) ends the CTA's loop
+        // everyone is done with `buf` (and has written its scale bytes) before
+        // it is refilled; with TMA staging a wait that gave up (in any thread)
+        // ends the CTA's loop
         if (TMA) {
             if (!__syncthreads_and(ok)) {
                 if (threadIdx.x == 0) drain_staged(st.bars, buf, use, tn < n_tiles);
@@ -736,6 +773,7 @@ __global__ void __launch_bounds__(COL_THREADS, 2) cast_dual_kernel(CastParams pr
         } else {
             __syncthreads();
         }
+        if (stage_sc) write_scale_atom(pc, satom, r0, c0, warp, lane);
     }
     if (!TMA) cp_async_wait_all();
 }
@@ -918,7 +956,7 @@ static bool make_input_map(CUtensorMap *map, const CastParams &p, bool bf16, boo
 // Dynamic shared memory of the column and dual casts: two tile buffers, their
 // two staging barriers, and slack to align the buffers for TMA.
 static int staged_smem_bytes(int in_bytes, int align) {
-    return 2 * COL_TILE_R * COL_TILE_C * in_bytes + 16 + align;
+    return 2 * COL_TILE_R * COL_TILE_C * in_bytes + 16 + 2 * 512 + align;
 }
 
 // Column cast: two tile buffers of dynamic shared memory, a resident grid.
@@ -1052,6 +1090,7 @@ cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st) {
     p.sr_base = a.sr_base;
     p.sr_stride = a.sr_stride;
     p.skip_first = 0;
+    p.stage_scales = (a.sl == SL_MMA || a.sl == SL_MMA_X4) && (reinterpret_cast<uintptr_t>(a.scales) & 15u) == 0;
     if (a.block_axis == 0) {         // the one-shot hook applies to staged (column) casts
         p.skip_first = t_skip_first ? 1 : 0;
         t_skip_first = false;
@@ -1127,6 +1166,8 @@ cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st
     pc.sr_stride = a.sr_stride_cols;
     pr.skip_first = 0;
     pc.skip_first = t_skip_first ? 1 : 0;
+    pr.stage_scales = 0;
+    pc.stage_scales = (a.sl == SL_MMA || a.sl == SL_MMA_X4) && (reinterpret_cast<uintptr_t>(a.scales_cols) & 15u) == 0;
     t_skip_first = false;
     const int sr_r = a.rnd_rows == MX_SR, sr_c = a.rnd_cols == MX_SR;
     switch (a.fmt) {

@@ -125,3 +125,27 @@ def test_staging_wait_reports_timeout(oracle, kind):
         same(col_cast(sx, "e2m1", "sr", 3, True), want, kind)
     else:
         same(dual_cast(sx, "e2m1", "rne", "sr", True), oracle_dual(oracle, small, "e2m1", "rne", "sr", True), kind)
+
+
+# The scales of a full 128 x 128 column tile leave through shared memory as one
+# atom (and its copies); ragged tiles, the plain layout and a scale buffer
+# that is not 16-byte aligned keep the per-byte stores.  Every path gives the
+# oracle's bytes, and the bytes around an offset scale buffer stay untouched.
+@pytest.mark.parametrize("sl", ["mma", "mma_x4", "plain"])
+@pytest.mark.parametrize("offset", [0, 1])
+def test_column_scales_staged_and_scattered(oracle, sl, offset):
+    x = ragged_input(384, 416, 920 + offset, True)
+    R, C = x.shape
+    layout = {"plain": 0, "mma": 1, "mma_x4": 2}[sl]
+    n = mx.scales_bytes(sl, C, R)
+    codes = torch.full((C, mx.codes_row_bytes("e2m1", R)), FILL, dtype=torch.uint8, device=dev())
+    buf = torch.full((n + 32,), FILL, dtype=torch.uint8, device=dev())
+    scales = buf[offset:offset + n]
+    mx.quantize(to_device(x), 0, "e2m1", rnd="sr", seed=4, hadamard=True, sign_mask=MASK, scale_layout=sl,
+                codes=codes, scales=scales)
+    torch.cuda.synchronize()
+    wc, ws = oracle.quantize(x, 0, oracle.FORMATS["e2m1"], rnd=1, seed=4, hadamard=True, sign_mask=MASK,
+                             scale_layout=layout, fill=FILL)
+    got = host(buf)
+    same([host(codes), got[offset:offset + n]], [wc, ws.reshape(-1)[:n]], (sl, offset))
+    assert (got[:offset] == FILL).all() and (got[offset + n:] == FILL).all()
