@@ -150,7 +150,9 @@ typedef enum {
  * Elements are rounded to the grid with overflow clamped to +-max; FP formats
  * keep the sign of zero.
  * Errors: MX_ERR_ARG, MX_ERR_ALIGN, MX_ERR_SHAPE (inner % 32 != 0),
- * MX_ERR_UNSUPPORTED, MX_ERR_SR_RANGE, MX_ERR_CUDA.
+ * MX_ERR_UNSUPPORTED, MX_ERR_SR_RANGE, MX_ERR_CUDA; MX_ERR_TIMEOUT later through
+ * mx_last_device_status if a column cast (block_axis 0) gave up its bounded
+ * wait for a tile's copy into shared memory (its outputs are then incomplete).
  */
 MX_API int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
                 int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
@@ -422,8 +424,9 @@ MX_API size_t mx_scales_bytes(mx_scale_layout sl, int64_t outer, int64_t inner);
 MX_API size_t mx_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Synchronises `stream`, then returns and clears the current device's status
- * word: MX_OK, or MX_ERR_TIMEOUT if a kernel gave up a bounded wait since the
- * last call.  MX_ERR_CUDA if the synchronisation itself failed. */
+ * words (one for the GEMM kernels, one for the casts): MX_OK, or
+ * MX_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call.
+ * MX_ERR_CUDA if the synchronisation itself failed. */
 MX_API int mx_last_device_status(void *stream);
 
 /* Static description of a status code. */
