@@ -117,7 +117,9 @@ typedef enum {
     MX_ERR_UNSUPPORTED = -4,  /* valid request that this build does not implement       */
     MX_ERR_SR_RANGE = -5,     /* stochastic rounding index space exceeds 2^34 elements  */
     MX_ERR_CUDA = -6,         /* a CUDA runtime/driver call or launch failed            */
-    MX_ERR_TIMEOUT = -7       /* a bounded device-side wait expired (see below)         */
+    MX_ERR_TIMEOUT = -7,      /* a bounded device-side wait expired (see below)         */
+    MX_ERR_BOUNDS = -8        /* debug build only: a device store or load fell outside
+                                 its buffer and was skipped (see mx_last_device_status) */
 } mx_status;
 
 /*
@@ -426,7 +428,12 @@ MX_API size_t mx_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 /* Synchronises `stream`, then returns and clears the current device's status
  * words (one for the GEMM kernels, one for the casts): MX_OK, or
  * MX_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call.
- * MX_ERR_CUDA if the synchronisation itself failed. */
+ * MX_ERR_CUDA if the synchronisation itself failed.  In the debug build
+ * (libmx_debug.so, compiled with MX_DEBUG) every code and scale store of the
+ * casts and the quantizing epilogue, and every code and scale load of the
+ * decode, checks its byte range against its buffer's size first; a range
+ * outside the buffer is skipped and reported here as MX_ERR_BOUNDS (after a
+ * timeout, which takes precedence).  The release build has no such checks. */
 MX_API int mx_last_device_status(void *stream);
 
 /* Static description of a status code. */

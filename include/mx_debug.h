@@ -61,6 +61,18 @@ MX_API int mx_debug_cast_force_cpasync(int on);
  */
 MX_API int mx_debug_cast_skip_tile(int on);
 
+/*
+ * mx_debug_cast_cut_codes_cap -- one shot, for the next mx_quantize (or
+ * shard) call of the calling host thread: the size of the codes buffer the
+ * kernels are told is `bytes` smaller than the true one.  Only the debug
+ * build (libmx_debug.so, MX_DEBUG) checks stores against that size: there the
+ * blocks whose codes would reach past it are not written and
+ * mx_last_device_status reports MX_ERR_BOUNDS, which tests the bounds checks
+ * without any access outside a real buffer.  The release build ignores it.
+ * Returns MX_OK, or MX_ERR_ARG for a negative size.
+ */
+MX_API int mx_debug_cast_cut_codes_cap(int64_t bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -3,13 +3,36 @@
 // point allocates device memory or synchronises, except
 // mx_last_device_status, which synchronises the given stream by contract.
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "mx.h"
 #include "mx_internal.h"
 
 namespace {
+
+// Optional NVTX ranges (environment MX_NVTX=1, read once per process): every
+// entry point that launches work marks a range named after itself, so a
+// profiler's timeline shows the library's calls.  Off by default; NVTX's
+// header-only API costs nothing when no tool is attached.
+bool nvtx_on() {
+    static const bool on = [] {
+        const char *e = std::getenv("MX_NVTX");
+        return e != nullptr && e[0] == '1';
+    }();
+    return on;
+}
+struct NvtxRange {
+    bool on;
+    explicit NvtxRange(const char *name) : on(nvtx_on()) {
+        if (on) nvtxRangePushA(name);
+    }
+    ~NvtxRange() {
+        if (on) nvtxRangePop();
+    }
+};
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices];   // 0 = not queried yet
@@ -61,6 +84,7 @@ const char *mx_status_str(int status) {
         case MX_ERR_SR_RANGE: return "MX_ERR_SR_RANGE: stochastic-rounding index space exceeds 2^34";
         case MX_ERR_CUDA: return "MX_ERR_CUDA: CUDA call or kernel launch failed";
         case MX_ERR_TIMEOUT: return "MX_ERR_TIMEOUT: a bounded device wait expired";
+        case MX_ERR_BOUNDS: return "MX_ERR_BOUNDS: a debug-build bounds check skipped an access";
         default: return "unknown mx status";
     }
 }
@@ -200,6 +224,7 @@ int mx_quantize(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t
                 int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
                 const mx_precond *pre, void *codes, void *scales, mx_scale_layout sl,
                 void *stream) {
+    const NvtxRange nvtx_range("mx_quantize");
     return quantize_impl(x, xdt, rows, cols, ldx, block_axis, fmt, rnd, seed, pre, nullptr, codes, scales, sl,
                          stream);
 }
@@ -208,6 +233,7 @@ int mx_quantize_shard(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, i
                       int block_axis, mx_fmt fmt, mx_round rnd, uint64_t seed,
                       const mx_precond *pre, const mx_shard *shard, void *codes, void *scales,
                       mx_scale_layout sl, void *stream) {
+    const NvtxRange nvtx_range("mx_quantize_shard");
     if (!shard) return MX_ERR_ARG;
     return quantize_impl(x, xdt, rows, cols, ldx, block_axis, fmt, rnd, seed, pre, shard, codes, scales, sl,
                          stream);
@@ -217,6 +243,7 @@ int mx_quantize_dual(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, in
                      mx_round rnd_rows, uint64_t seed_rows, mx_round rnd_cols, uint64_t seed_cols,
                      const mx_precond *pre_cols, void *codes_rows, void *scales_rows, void *codes_cols,
                      void *scales_cols, mx_scale_layout sl, void *stream) {
+    const NvtxRange nvtx_range("mx_quantize_dual");
     return quantize_dual_impl(x, xdt, rows, cols, ldx, fmt, rnd_rows, seed_rows, rnd_cols, seed_cols, pre_cols,
                               nullptr, codes_rows, scales_rows, codes_cols, scales_cols, sl, stream);
 }
@@ -226,6 +253,7 @@ int mx_quantize_dual_shard(const void *x, mx_dtype xdt, int64_t rows, int64_t co
                            const mx_precond *pre_cols, const mx_shard *shard, void *codes_rows,
                            void *scales_rows, void *codes_cols, void *scales_cols, mx_scale_layout sl,
                            void *stream) {
+    const NvtxRange nvtx_range("mx_quantize_dual_shard");
     if (!shard) return MX_ERR_ARG;
     return quantize_dual_impl(x, xdt, rows, cols, ldx, fmt, rnd_rows, seed_rows, rnd_cols, seed_cols, pre_cols,
                               shard, codes_rows, scales_rows, codes_cols, scales_cols, sl, stream);
@@ -244,6 +272,7 @@ int64_t mx_nvfp4_domains(int64_t rows, int64_t domain_rows) {
 
 int mx_quantize_nvfp4(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, int64_t domain_rows,
                       void *codes, void *scales, mx_scale_layout sl, float *enc_scales, void *stream) {
+    const NvtxRange nvtx_range("mx_quantize_nvfp4");
     if (xdt != MX_F32 && xdt != MX_BF16) return MX_ERR_ARG;
     if (!valid_layout(sl)) return MX_ERR_ARG;
     if (rows < 0 || cols < 0 || domain_rows < 0) return MX_ERR_ARG;
@@ -264,6 +293,7 @@ int mx_quantize_nvfp4(const void *x, mx_dtype xdt, int64_t rows, int64_t cols, i
 
 int mx_dequantize(const void *codes, const void *scales, mx_fmt fmt, mx_scale_layout sl,
                   int64_t outer, int64_t inner, void *y, mx_dtype ydt, int64_t ldy, void *stream) {
+    const NvtxRange nvtx_range("mx_dequantize");
     if (elem_bits(fmt) == 0 || (ydt != MX_F32 && ydt != MX_BF16)) return MX_ERR_ARG;
     if (!valid_layout(sl)) return MX_ERR_ARG;
     if (outer < 0 || inner < 0) return MX_ERR_ARG;
@@ -383,6 +413,7 @@ int mx_gemm(const void *a_codes, const void *a_scales, mx_fmt fa,
             const void *b_codes, const void *b_scales, mx_fmt fb,
             int64_t M, int64_t N, int64_t K, float alpha,
             void *c, mx_dtype cdt, int64_t ldc, void *workspace, size_t ws_bytes, void *stream) {
+    const NvtxRange nvtx_range("mx_gemm");
     (void)workspace;
     (void)ws_bytes;
     return gemm_impl(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha, c, cdt, ldc, false, stream);
@@ -392,6 +423,7 @@ int mx_gemm_x4(const void *a_codes, const void *a_scales, mx_fmt fa,
                const void *b_codes, const void *b_scales, mx_fmt fb,
                int64_t M, int64_t N, int64_t K, float alpha,
                void *c, mx_dtype cdt, int64_t ldc, void *stream) {
+    const NvtxRange nvtx_range("mx_gemm_x4");
     return gemm_impl(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha, c, cdt, ldc, true, stream);
 }
 
@@ -400,6 +432,7 @@ int mx_gemm_quantize(const void *a_codes, const void *a_scales, mx_fmt fa,
                      int64_t M, int64_t N, int64_t K, float alpha,
                      mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
                      void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream) {
+    const NvtxRange nvtx_range("mx_gemm_quantize");
     return gemm_quantize_impl(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha, out_fmt, out_rnd,
                               out_seed, out_codes, out_scales, out_sl, false, stream);
 }
@@ -409,6 +442,7 @@ int mx_gemm_quantize_x4(const void *a_codes, const void *a_scales, mx_fmt fa,
                         int64_t M, int64_t N, int64_t K, float alpha,
                         mx_fmt out_fmt, mx_round out_rnd, uint64_t out_seed,
                         void *out_codes, void *out_scales, mx_scale_layout out_sl, void *stream) {
+    const NvtxRange nvtx_range("mx_gemm_quantize_x4");
     return gemm_quantize_impl(a_codes, a_scales, fa, b_codes, b_scales, fb, M, N, K, alpha, out_fmt, out_rnd,
                               out_seed, out_codes, out_scales, out_sl, true, stream);
 }
@@ -456,6 +490,7 @@ int mx_gemm_nvfp4(const void *a_codes, const void *a_scales, const float *a_enc,
                   const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
                   int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
                   void *stream) {
+    const NvtxRange nvtx_range("mx_gemm_nvfp4");
     return gemm_nvfp4_impl(a_codes, a_scales, a_enc, a_domain_rows, b_codes, b_scales, b_enc, b_domain_rows, M, N,
                            K, alpha, c, cdt, ldc, false, stream);
 }
@@ -464,15 +499,19 @@ int mx_gemm_nvfp4_x4(const void *a_codes, const void *a_scales, const float *a_e
                      const void *b_codes, const void *b_scales, const float *b_enc, int64_t b_domain_rows,
                      int64_t M, int64_t N, int64_t K, float alpha, void *c, mx_dtype cdt, int64_t ldc,
                      void *stream) {
+    const NvtxRange nvtx_range("mx_gemm_nvfp4_x4");
     return gemm_nvfp4_impl(a_codes, a_scales, a_enc, a_domain_rows, b_codes, b_scales, b_enc, b_domain_rows, M, N,
                            K, alpha, c, cdt, ldc, true, stream);
 }
 
 int mx_last_device_status(void *stream) {
-    // the GEMMs' and the casts' status words, both read and cleared
+    // the GEMMs', the casts' and the NVFP4 unit's status words, all read and
+    // cleared; a timeout takes precedence over a debug-build bounds report
     const int g = mx_read_device_status(static_cast<cudaStream_t>(stream));
     const int c = mx_read_cast_status();
-    return g != MX_OK ? g : c;
+    const int n = mx_read_nvfp4_bounds_status();
+    if (g == MX_ERR_TIMEOUT || c == MX_ERR_TIMEOUT) return MX_ERR_TIMEOUT;
+    return g != MX_OK ? g : (c != MX_OK ? c : n);
 }
 
 }  // extern "C"

@@ -43,12 +43,13 @@ struct CastParams {
     uint64_t sr_base, sr_stride;
     int skip_first;      // testing hook: CTA 0 withholds the copy of its first staged tile
     int stage_scales;    // column casts: a full tile's scale atom goes out through shared memory
+    uint64_t codes_cap, scales_cap;   // buffer sizes in bytes (checked by the debug build)
 };
 
 __device__ __forceinline__ void store_scale(const CastParams &p, int64_t o, int64_t kb, uint32_t s) {
     // scale buffers are far below 4 GiB: offsets in 32-bit arithmetic
     put_scale(p.scales, p.mma_scales, static_cast<uint32_t>(o), static_cast<uint32_t>(kb),
-              static_cast<uint32_t>(p.k_blocks), static_cast<uint32_t>(p.k_groups), s);
+              static_cast<uint32_t>(p.k_blocks), static_cast<uint32_t>(p.k_groups), s, p.scales_cap);
 }
 
 // ---------------------------------------------------------------------------
@@ -111,6 +112,8 @@ __device__ __forceinline__ BlockSink row_sink(const CastParams &p) {
     o.key = p.key;
     o.sr_base = p.sr_base;
     o.sr_stride = p.sr_stride;
+    o.codes_cap = p.codes_cap;
+    o.scales_cap = p.scales_cap;
     return o;
 }
 
@@ -442,7 +445,9 @@ __device__ __forceinline__ void encode_col_pair(const CastParams &p, uint64_t (&
                 pw[w] = cvt_pair<FMT>(v[4 * w], v[4 * w + 1]) | (cvt_pair<FMT>(v[4 * w + 2], v[4 * w + 3]) << (2 * SLOT));
         }
         const uint32_t keep = nan_block ? 0u : 0xffffffffu;     // a NaN/Inf block stores zero codes
-        if (BITS == 8) {
+        if (!in_bounds(static_cast<uint64_t>(oc * (R * BITS / 8) + gr0 * BITS / 8), 32 * BITS / 8, p.codes_cap)) {
+            // (debug build) the block's codes fall outside the buffer: skip them
+        } else if (BITS == 8) {
             uint4 *dst = reinterpret_cast<uint4 *>(p.codes + oc * R + gr0);
             dst[0] = make_uint4(pw[0] & keep, pw[1] & keep, pw[2] & keep, pw[3] & keep);
             dst[1] = make_uint4(pw[4] & keep, pw[5] & keep, pw[6] & keep, pw[7] & keep);
@@ -489,8 +494,9 @@ __device__ __forceinline__ void write_scale_atom(const CastParams &p, const uint
     const int copies = p.mma_scales == SL_MMA_X4 ? 4 : 1;
     if (warp >= copies) return;
     const int64_t atom = (c0 >> 7) * p.k_groups + (r0 >> 7);
-    uint8_t *dst = p.scales + (atom << (copies == 4 ? 11 : 9)) + warp * 512;
-    reinterpret_cast<uint4 *>(dst)[lane] = reinterpret_cast<const uint4 *>(satom)[lane];
+    const int64_t off = (atom << (copies == 4 ? 11 : 9)) + warp * 512;
+    if (!in_bounds(static_cast<uint64_t>(off), 512, p.scales_cap)) return;
+    reinterpret_cast<uint4 *>(p.scales + off)[lane] = reinterpret_cast<const uint4 *>(satom)[lane];
 }
 
 // After a staging wait gave up at tile use `use` (buffer `buf`): wait, again
@@ -833,6 +839,7 @@ struct DequantParams {
     int64_t outer, inner, k_blocks, k_groups;
     void *y;
     int64_t ldy;
+    uint64_t codes_cap, scales_cap;   // buffer sizes in bytes (checked by the debug build)
 };
 
 template <int FMT, bool BF16_OUT>
@@ -850,6 +857,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
         const int64_t so = p.mma_scales == SL_MMA_X4 ? static_cast<int64_t>(x4_scale_offset32(
                                static_cast<uint32_t>(o), static_cast<uint32_t>(kb), static_cast<uint32_t>(p.k_groups)))
                            : p.mma_scales == SL_MMA ? mma_scale_offset(o, kb, p.k_groups) : o * p.k_blocks + kb;
+        if (!in_bounds(static_cast<uint64_t>(so), 1, p.scales_cap) ||
+            !in_bounds(static_cast<uint64_t>(o * (p.inner * BITS / 8) + oc * BITS), BITS, p.codes_cap))
+            continue;                                   // (debug build) outside a buffer: skipped
         const uint32_t s = p.scales[so];
         uint32_t pairs[4];
         if (BITS == 8) {
@@ -935,6 +945,7 @@ static cudaError_t launch_overlapped(int grid, int block, int smem, cudaStream_t
 // Testing hooks (include/mx_debug.h), per host thread.
 thread_local bool t_force_cpasync = false;
 thread_local bool t_skip_first = false;
+thread_local uint64_t t_codes_cap_cut = 0;
 
 // Tensor map of a cast's input for TMA staging: the rows x cols tensor in
 // boxes of 128 rows x 128 columns, unswizzled (column cast), or x 128 bytes
@@ -1091,6 +1102,10 @@ cudaError_t mx_launch_quantize(const MxQuantizeArgs &a, cudaStream_t st) {
     p.sr_stride = a.sr_stride;
     p.skip_first = 0;
     p.stage_scales = (a.sl == SL_MMA || a.sl == SL_MMA_X4) && (reinterpret_cast<uintptr_t>(a.scales) & 15u) == 0;
+    p.codes_cap = mx_codes_bytes(static_cast<mx_fmt>(a.fmt), a.block_axis == 1 ? a.rows : a.cols, inner);
+    p.scales_cap = mx_scales_bytes(static_cast<mx_scale_layout>(a.sl), a.block_axis == 1 ? a.rows : a.cols, inner);
+    p.codes_cap -= t_codes_cap_cut < p.codes_cap ? t_codes_cap_cut : p.codes_cap;   // testing hook, one shot
+    t_codes_cap_cut = 0;
     if (a.block_axis == 0) {         // the one-shot hook applies to staged (column) casts
         p.skip_first = t_skip_first ? 1 : 0;
         t_skip_first = false;
@@ -1119,6 +1134,8 @@ cudaError_t mx_launch_dequantize(const MxDequantArgs &a, cudaStream_t st) {
     p.k_groups = (p.k_blocks + 3) / 4;
     p.y = a.y;
     p.ldy = a.ldy;
+    p.codes_cap = mx_codes_bytes(static_cast<mx_fmt>(a.fmt), a.outer, a.inner);
+    p.scales_cap = mx_scales_bytes(static_cast<mx_scale_layout>(a.sl), a.outer, a.inner);
     const int grid = grid_for(a.outer * (a.inner / 8), 256, a.num_sms * 8);
     const bool bf = a.ydt == MX_BF16;
 #define MX_DQ(F)                                                                                      \
@@ -1168,6 +1185,10 @@ cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st
     pc.skip_first = t_skip_first ? 1 : 0;
     pr.stage_scales = 0;
     pc.stage_scales = (a.sl == SL_MMA || a.sl == SL_MMA_X4) && (reinterpret_cast<uintptr_t>(a.scales_cols) & 15u) == 0;
+    pr.codes_cap = mx_codes_bytes(static_cast<mx_fmt>(a.fmt), a.rows, a.cols);
+    pr.scales_cap = mx_scales_bytes(static_cast<mx_scale_layout>(a.sl), a.rows, a.cols);
+    pc.codes_cap = mx_codes_bytes(static_cast<mx_fmt>(a.fmt), a.cols, a.rows);
+    pc.scales_cap = mx_scales_bytes(static_cast<mx_scale_layout>(a.sl), a.cols, a.rows);
     t_skip_first = false;
     const int sr_r = a.rnd_rows == MX_SR, sr_c = a.rnd_cols == MX_SR;
     switch (a.fmt) {
@@ -1181,13 +1202,16 @@ cudaError_t mx_launch_quantize_dual(const MxQuantizeDualArgs &a, cudaStream_t st
     return cudaErrorInvalidValue;
 }
 
-// Reads and clears the casts' status word (after the caller synchronised).
+// Reads and clears the casts' status word and, in this unit, the debug
+// build's bounds word (after the caller synchronised); a timeout comes first.
 int mx_read_cast_status() {
-    int v = 0;
+    int v = 0, b = 0;
     if (cudaMemcpyFromSymbol(&v, mxk::g_cast_status, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&b, mxk::g_bounds_status, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
     const int zero = 0;
     if (cudaMemcpyToSymbol(mxk::g_cast_status, &zero, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
-    return v;
+    if (cudaMemcpyToSymbol(mxk::g_bounds_status, &zero, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
+    return v != MX_OK ? v : b;
 }
 
 extern "C" int mx_debug_cast_force_cpasync(int on) {
@@ -1197,5 +1221,11 @@ extern "C" int mx_debug_cast_force_cpasync(int on) {
 
 extern "C" int mx_debug_cast_skip_tile(int on) {
     mxk::t_skip_first = on != 0;
+    return MX_OK;
+}
+
+extern "C" int mx_debug_cast_cut_codes_cap(int64_t bytes) {
+    if (bytes < 0) return MX_ERR_ARG;
+    mxk::t_codes_cap_cut = static_cast<uint64_t>(bytes);
     return MX_OK;
 }

@@ -254,16 +254,38 @@ __device__ __forceinline__ uint32_t x4_scale_offset32(uint32_t o, uint32_t kb, u
     return (atom << 11) + ((o & 31u) << 4) + (((o >> 5) & 3u) << 2) + (kb & 3u);
 }
 
+// Debug build (MX_DEBUG, libmx_debug.so): a store or load of `bytes` bytes at
+// offset `off` of a buffer of `cap` bytes goes ahead only inside the buffer;
+// otherwise this translation unit's bounds word records MX_ERR_BOUNDS (read by
+// mx_last_device_status) and the caller skips the access.  The release build
+// compiles the check away.
+namespace {
+__device__ int g_bounds_status;
+}
+__device__ __forceinline__ bool in_bounds(uint64_t off, uint64_t bytes, uint64_t cap) {
+#ifdef MX_DEBUG
+    if (off + bytes <= cap) return true;
+    atomicExch(&g_bounds_status, MX_ERR_BOUNDS);
+    return false;
+#else
+    (void)off; (void)bytes; (void)cap;
+    return true;
+#endif
+}
+
 // Writes scale byte s of (o, kb) in layout sl (plain rows of k_blocks bytes,
-// MMA atoms, or the four copies of the x4 layout).
+// MMA atoms, or the four copies of the x4 layout) into a buffer of cap bytes.
 __device__ __forceinline__ void put_scale(uint8_t *scales, int sl, uint32_t o, uint32_t kb, uint32_t k_blocks,
-                                          uint32_t k_groups, uint32_t s) {
+                                          uint32_t k_groups, uint32_t s, uint64_t cap) {
     if (sl == SL_MMA_X4) {
         const uint32_t off = x4_scale_offset32(o, kb, k_groups);
+        if (!in_bounds(off, 3u * 512u + 1u, cap)) return;
 #pragma unroll
         for (uint32_t j = 0; j < 4; ++j) scales[off + 512u * j] = static_cast<uint8_t>(s);
     } else {
-        scales[sl == SL_MMA ? mma_scale_offset32(o, kb, k_groups) : o * k_blocks + kb] = static_cast<uint8_t>(s);
+        const uint32_t off = sl == SL_MMA ? mma_scale_offset32(o, kb, k_groups) : o * k_blocks + kb;
+        if (!in_bounds(off, 1, cap)) return;
+        scales[off] = static_cast<uint8_t>(s);
     }
 }
 

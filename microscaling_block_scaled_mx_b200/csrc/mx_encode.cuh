@@ -22,12 +22,13 @@ struct BlockSink {
     // stochastic-rounding position of element (row, i): sr_base + row * sr_stride + i
     // (a whole tensor: 0 and inner; a shard: its place in the whole tensor's output)
     uint64_t sr_base, sr_stride;
+    uint64_t codes_cap, scales_cap;   // buffer sizes in bytes (checked by the debug build)
 };
 
 __device__ __forceinline__ void sink_scale(const BlockSink &o, int64_t row, int64_t kb, uint32_t s) {
     // scale buffers are far below 4 GiB: offsets in 32-bit arithmetic
     put_scale(o.scales, o.mma_scales, static_cast<uint32_t>(row), static_cast<uint32_t>(kb), o.k_blocks,
-              o.k_groups, s);
+              o.k_groups, s, o.scales_cap);
 }
 
 __device__ __forceinline__ uint64_t f2_mul_ftz(uint64_t a, uint64_t b) {
@@ -88,8 +89,9 @@ __device__ __forceinline__ void encode_block32_amax(const BlockSink &o, int64_t 
 #pragma unroll
             for (int i = 0; i < 8; ++i) c[i] = 0u;
         }
-        store_code32<V32>(o.codes + row * o.inner + kb * 32, make_uint4(c[0], c[1], c[2], c[3]),
-                          make_uint4(c[4], c[5], c[6], c[7]));
+        if (in_bounds(static_cast<uint64_t>(row * o.inner + kb * 32), 32, o.codes_cap))
+            store_code32<V32>(o.codes + row * o.inner + kb * 32, make_uint4(c[0], c[1], c[2], c[3]),
+                              make_uint4(c[4], c[5], c[6], c[7]));
         sink_scale(o, row, kb, nan_block ? 0xffu : static_cast<uint32_t>(e + 127));
         return;
     }
@@ -121,8 +123,11 @@ __device__ __forceinline__ void encode_block32_amax(const BlockSink &o, int64_t 
             pw[w] = cvt_pair<FMT>(u[4 * w], u[4 * w + 1]) | (cvt_pair<FMT>(u[4 * w + 2], u[4 * w + 3]) << (2 * SLOT));
     }
     const uint32_t keep = nan_block ? 0u : 0xffffffffu;     // a NaN/Inf block stores zero codes
-    uint8_t *dst = o.codes + row * (o.inner * BITS / 8) + kb * (32 * BITS / 8);
-    if (BITS == 8) {
+    const int64_t code_off = row * (o.inner * BITS / 8) + kb * (32 * BITS / 8);
+    uint8_t *dst = o.codes + code_off;
+    if (!in_bounds(static_cast<uint64_t>(code_off), 32 * BITS / 8, o.codes_cap)) {
+        // (debug build) the block's codes fall outside the buffer: skip them
+    } else if (BITS == 8) {
         store_code32<V32>(dst, make_uint4(pw[0] & keep, pw[1] & keep, pw[2] & keep, pw[3] & keep),
                           make_uint4(pw[4] & keep, pw[5] & keep, pw[6] & keep, pw[7] & keep));
     } else if (BITS == 4) {

@@ -108,6 +108,7 @@ struct MxOut {
     int sr;              // stochastic rounding (else RNE)
     int mma;             // scale layout: 0 plain, 1 MMA, 2 MMA x4
     uint32_t key;        // stochastic-rounding seed key
+    uint64_t codes_cap, scales_cap;   // buffer sizes in bytes (checked by the debug build)
 };
 
 struct Params {
@@ -318,6 +319,8 @@ __device__ __forceinline__ void quantize_chunk(const Params &p, int m, int n0, c
     o.key = p.q.key;
     o.sr_base = 0;
     o.sr_stride = static_cast<uint64_t>(p.N);
+    o.codes_cap = p.q.codes_cap;
+    o.scales_cap = p.q.scales_cap;
     const int kb = n0 >> 5;
     const bool sr = p.q.sr != 0;
     switch (p.q.fmt) {
@@ -1544,6 +1547,8 @@ MxOut mx_out(const MxGemmArgs &a) {
     q.sr = a.q_rnd == MX_SR;
     q.mma = a.q_sl;
     q.key = fmix32_host(static_cast<uint32_t>(a.q_seed)) ^ static_cast<uint32_t>(a.q_seed >> 32);
+    q.codes_cap = a.q_codes ? mx_codes_bytes(static_cast<mx_fmt>(a.q_fmt), a.M, a.N) : 0;
+    q.scales_cap = a.q_codes ? mx_scales_bytes(static_cast<mx_scale_layout>(a.q_sl), a.M, a.N) : 0;
     return q;
 }
 
@@ -1729,9 +1734,11 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st) {
 
 int mx_read_device_status(cudaStream_t st) {
     if (cudaStreamSynchronize(st) != cudaSuccess) return MX_ERR_CUDA;
-    int v = 0;
+    int v = 0, b = 0;
     if (cudaMemcpyFromSymbol(&v, g_mx_status, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&b, mxk::g_bounds_status, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_mx_status, &zero, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
-    return v;
+    if (cudaMemcpyToSymbol(mxk::g_bounds_status, &zero, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
+    return v != MX_OK ? v : b;        // the debug build's bounds word after a timeout
 }

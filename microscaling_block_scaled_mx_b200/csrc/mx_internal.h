@@ -109,6 +109,8 @@ int mx_launch_gemm(const MxGemmArgs &a, cudaStream_t st);
 int mx_read_device_status(cudaStream_t st);
 // reads and clears the cast kernels' status word (the caller has synchronised)
 int mx_read_cast_status();
+// reads and clears the NVFP4 unit's debug-build bounds word (the caller has synchronised)
+int mx_read_nvfp4_bounds_status();
 
 namespace mxg {
 // Encodes (or takes from a per-process cache) a 2-D tiled tensor map: d0 x d1

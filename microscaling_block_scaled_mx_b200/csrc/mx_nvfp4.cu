@@ -49,6 +49,7 @@ struct NvParams {
     int64_t n_dom;         // domains
     int parts;             // CTAs per domain
     uint32_t row_step, kb_step;   // THREADS blocks = row_step rows + kb_step blocks
+    uint64_t codes_cap, scales_cap;   // buffer sizes in bytes (checked by the debug build)
 };
 
 __device__ __forceinline__ float encode_scale(float amax) {
@@ -125,9 +126,10 @@ __device__ __forceinline__ void quant_block(const NvParams &p, int64_t row, int6
         }
         c = make_uint2(w[0], w[1]);
     }
-    *reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + kb * 8) = c;
+    if (mxk::in_bounds(static_cast<uint64_t>(row * (p.cols / 2) + kb * 8), 8, p.codes_cap))
+        *reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + kb * 8) = c;
     mxk::put_scale(p.scales, p.mma, static_cast<uint32_t>(row), static_cast<uint32_t>(kb), p.k_blocks, p.k_groups,
-                   s);
+                   s, p.scales_cap);
 }
 
 // bf16 input, a block as the 8 words of its 16 values (element 2i in the low
@@ -193,8 +195,9 @@ __device__ __forceinline__ void quant_block_bf16(const NvParams &p, int64_t row,
         }
         c = make_uint2(q[0], q[1]);
     }
-    *reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + kb * 8) = c;
-    mxk::put_scale(p.scales, p.mma, static_cast<uint32_t>(row), kb, p.k_blocks, p.k_groups, s);
+    if (mxk::in_bounds(static_cast<uint64_t>(row * (p.cols / 2) + kb * 8), 8, p.codes_cap))
+        *reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + kb * 8) = c;
+    mxk::put_scale(p.scales, p.mma, static_cast<uint32_t>(row), kb, p.k_blocks, p.k_groups, s, p.scales_cap);
 }
 
 // largest value over the CTA (every thread gets it)
@@ -362,6 +365,8 @@ cudaError_t mx_launch_quantize_nvfp4(const MxNvfp4Args &a, cudaStream_t st) {
     p.mma = a.sl;
     p.k_blocks = static_cast<uint32_t>(a.cols / NV_BLOCK);
     p.k_groups = (p.k_blocks + 3) / 4;
+    p.codes_cap = static_cast<uint64_t>(a.rows) * static_cast<uint64_t>(a.cols / 2);
+    p.scales_cap = mx_nvfp4_scales_bytes(static_cast<mx_scale_layout>(a.sl), a.rows, a.cols);
     p.enc = a.enc_scales;
     p.lines = (a.domain_rows == 0 || a.domain_rows > a.rows) ? a.rows : a.domain_rows;
     p.n_dom = (a.rows + p.lines - 1) / p.lines;
@@ -375,4 +380,14 @@ cudaError_t mx_launch_quantize_nvfp4(const MxNvfp4Args &a, cudaStream_t st) {
     p.row_step = static_cast<uint32_t>(THREADS / p.k_blocks);
     p.kb_step = static_cast<uint32_t>(THREADS % p.k_blocks);
     return a.xdt == MX_BF16 ? run<true>(p, st) : run<false>(p, st);
+}
+
+// Reads and clears this unit's debug-build bounds word (after the caller
+// synchronised).
+int mx_read_nvfp4_bounds_status() {
+    int b = 0;
+    if (cudaMemcpyFromSymbol(&b, mxk::g_bounds_status, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(mxk::g_bounds_status, &zero, sizeof(int)) != cudaSuccess) return MX_ERR_CUDA;
+    return b;
 }

@@ -29,7 +29,7 @@ DEFAULT_SIGN_MASK = 0x6A09E667
 MX_OK = 0
 STATUS_NAMES = {0: "MX_OK", -1: "MX_ERR_ARG", -2: "MX_ERR_ALIGN", -3: "MX_ERR_SHAPE",
                 -4: "MX_ERR_UNSUPPORTED", -5: "MX_ERR_SR_RANGE", -6: "MX_ERR_CUDA",
-                -7: "MX_ERR_TIMEOUT"}
+                -7: "MX_ERR_TIMEOUT", -8: "MX_ERR_BOUNDS"}
 
 
 class MxError(RuntimeError):
@@ -121,6 +121,8 @@ def lib() -> ctypes.CDLL:
             L.mx_debug_cast_force_cpasync.argtypes = [i32]
             L.mx_debug_cast_skip_tile.restype = i32
             L.mx_debug_cast_skip_tile.argtypes = [i32]
+            L.mx_debug_cast_cut_codes_cap.restype = i32
+            L.mx_debug_cast_cut_codes_cap.argtypes = [i64]
             _lib = L
     return _lib
 

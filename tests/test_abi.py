@@ -42,6 +42,19 @@ def test_library_exports_every_declared_symbol(mx):
     assert L.mx_abi_version() == 1
 
 
+def test_debug_library_exports_every_declared_symbol():
+    # libmx_debug.so (MX_DEBUG bounds checks) is built beside libmx.so by the
+    # package build; it must offer the same boundary
+    import ctypes
+    from microscaling_block_scaled_mx_b200 import build as B
+    if not os.path.exists(B.DEBUG_LIB):
+        pytest.skip("libmx_debug.so not built")
+    L = ctypes.CDLL(B.DEBUG_LIB)
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert L.mx_abi_version() == 1
+
+
 def test_status_strings(mx):
     for code, name in mx.STATUS_NAMES.items():
         assert mx.status_str(code).startswith(name)
