@@ -28,16 +28,28 @@ CALLS = textwrap.dedent("""
     import numpy as np, torch
     from microscaling_block_scaled_mx_b200 import inputs as I
     def run(mx, dev):
+        # every output starts as 0xAB, so the padding bytes of the scale
+        # layouts compare equal too
+        u8 = lambda n: torch.full((max(n, 1),), 0xAB, dtype=torch.uint8, device=dev)
         rng = np.random.default_rng(77)
         x = torch.from_numpy(I.to_bf16_bits(rng.standard_normal((384, 416)).astype(np.float32)).view(np.int16)
                              ).view(torch.bfloat16).to(dev)
+        R, C = x.shape
+        L = mx.lib()
         out = {}
-        out["rows"] = mx.quantize(x, 1, "e4m3")
-        out["cols_x4"] = mx.quantize(x, 0, "e2m1", rnd="sr", seed=5, hadamard=True, scale_layout="mma_x4")
-        out["dual"] = mx.quantize_dual(x, "e2m1", rnd_cols="sr", seed_cols=6, hadamard=True)
-        out["nvfp4"] = mx.quantize_nvfp4(x, 128)
+        out["rows"] = (u8(R * C), u8(mx.scales_bytes("mma", R, C)))
+        mx.quantize(x, 1, "e4m3", codes=out["rows"][0].view(R, C), scales=out["rows"][1])
+        out["cols_x4"] = (u8(C * R // 2), u8(mx.scales_bytes("mma_x4", C, R)))
+        mx.quantize(x, 0, "e2m1", rnd="sr", seed=5, hadamard=True, scale_layout="mma_x4",
+                    codes=out["cols_x4"][0].view(C, R // 2), scales=out["cols_x4"][1])
+        out["dual"] = (u8(R * C // 2).view(R, C // 2), u8(mx.scales_bytes("mma", R, C)),
+                       u8(C * R // 2).view(C, R // 2), u8(mx.scales_bytes("mma", C, R)))
+        mx.quantize_dual(x, "e2m1", rnd_cols="sr", seed_cols=6, hadamard=True, out=out["dual"])
+        out["nvfp4"] = (u8(R * C // 2).view(R, C // 2), u8(L.mx_nvfp4_scales_bytes(1, R, C)),
+                        torch.zeros(L.mx_nvfp4_domains(R, 128), dtype=torch.float32, device=dev))
+        mx.quantize_nvfp4(x, 128, out=out["nvfp4"])
         c, s = out["rows"]
-        out["decode"] = (mx.dequantize(c, s, "e4m3", 384, 416),)
+        out["decode"] = (mx.dequantize(c.view(R, C), s, "e4m3", R, C),)
         a = mx.quantize(x[:256, :384].contiguous(), 1, "e4m3")
         b = mx.quantize(x[128:384, :384].contiguous(), 1, "e4m3")
         out["gemm_q"] = mx.gemm_quantize(a[0], a[1], b[0], b[1], 256, 256, 384, fa="e4m3", out_fmt="e2m1")
