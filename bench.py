@@ -54,18 +54,18 @@ MEASURED_TRAFFIC = {
     # --cache-control none, so each launch also carries the write-back of its
     # predecessor's output still in L2 (steady state: reads + writes of one cast)
     "cast_rows": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                  "470cee7944bfdf674cfe577bd4793cd0b287c6d30ed2e89c57f505d217258a36",
-                  {"e4m3_bf16_8192x8192": 134243584 + 69091072, "e5m2_bf16_8192x8192": 134252288 + 67738880,
-                   "e2m3_bf16_8192x8192": 134226944 + 52333312, "e3m2_bf16_8192x8192": 134219776 + 52260864,
-                   "e2m1_bf16_8192x8192": 134220032 + 35634176, "int8_bf16_8192x8192": 134220544 + 68231680}),
+                  "8b734928cc1e08710e6c1619c3ea512a525f233816c157ec451316e7aef9c23a",
+                  {"e4m3_bf16_8192x8192": 134282752 + 70009600, "e5m2_bf16_8192x8192": 134250496 + 66572800,
+                   "e2m3_bf16_8192x8192": 134224640 + 53562112, "e3m2_bf16_8192x8192": 134220544 + 52639744,
+                   "e2m1_bf16_8192x8192": 134220288 + 36188160, "int8_bf16_8192x8192": 134219776 + 68327680}),
     # the GEMMs: default cache control (L2 flushed before the launch), so reads
     # show re-reads and writes count only what left L2 during the launch; "x4":
     # operands with x4 scales
     "gemm": (("mx_gemm.cu", "mx_encode.cuh"),
-             "bad3a233a9d970735d12687459dc70e60e65b4769370a43f0e29800d55358190",
-             {"e2m1_x4_8192x6144x4096": 37595136 + 56642816, "e2m1_x4_8192x14336x4096": 59562496 + 189831936,
-              "e2m1_x4_8192x4096x14336": 142597376 + 51500288, "e4m3_8192x3072x768": 8974592 + 778496,
-              "e4m3_8192x768x3072": 28427008 + 0, "e2m1_x4_4096x14336x16384": 416875520 + 210363136}),
+             "6857d04b731b1d6b91f472390b0595c1f8be37ebd11ed4d86eb7c5ae9c88039c",
+             {"e2m1_x4_8192x6144x4096": 37304320 + 56930816, "e2m1_x4_8192x14336x4096": 59648768 + 188995584,
+              "e2m1_x4_8192x4096x14336": 140673536 + 52436736, "e4m3_8192x3072x768": 8976384 + 1790208,
+              "e4m3_8192x768x3072": 28427264 + 0, "e2m1_x4_4096x14336x16384": 456610048 + 210655232}),
 }
 
 
@@ -75,13 +75,13 @@ MEASURED_TRAFFIC = {
 # issue roofline of those casts: at most 4 warp instructions per clock per SM.
 MEASURED_INSTR = {
     "cast_cols_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                         "470cee7944bfdf674cfe577bd4793cd0b287c6d30ed2e89c57f505d217258a36",
+                         "8b734928cc1e08710e6c1619c3ea512a525f233816c157ec451316e7aef9c23a",
                          {"e2m1_bf16_x4_16384x4096": 27130504 / (16384 * 4096),
                           "e2m1_bf16_x4_16384x14336": 94438024 / (16384 * 14336)}),
     "cast_dual_had_sr": (("mx_cast.cu", "mx_device.cuh", "mx_encode.cuh"),
-                         "470cee7944bfdf674cfe577bd4793cd0b287c6d30ed2e89c57f505d217258a36",
-                         {"e2m1_bf16_16384x4096": 41284616 / (16384 * 4096),
-                          "e2m1_bf16_16384x14336": 144083976 / (16384 * 14336)}),
+                         "8b734928cc1e08710e6c1619c3ea512a525f233816c157ec451316e7aef9c23a",
+                         {"e2m1_bf16_16384x4096": 40931272 / (16384 * 4096),
+                          "e2m1_bf16_16384x14336": 142829512 / (16384 * 14336)}),
 }
 
 
