@@ -430,8 +430,8 @@ MX_API size_t mx_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * MX_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call.
  * MX_ERR_CUDA if the synchronisation itself failed.  In the debug build
  * (libmx_debug.so, compiled with MX_DEBUG) every code and scale store of the
- * casts and the quantizing epilogue, and every code and scale load of the
- * decode, checks its byte range against its buffer's size first; a range
+ * casts and the NVFP4 cast, and every code and scale load of the decode,
+ * checks its byte range against its buffer's size first; a range
  * outside the buffer is skipped and reported here as MX_ERR_BOUNDS (after a
  * timeout, which takes precedence).  The release build has no such checks. */
 MX_API int mx_last_device_status(void *stream);
