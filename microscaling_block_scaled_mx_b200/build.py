@@ -1,8 +1,8 @@
 """Build libmx.so (the C-ABI library) in-tree with nvcc for sm_100a, and on
-request libmx_debug.so: the same sources compiled with MX_DEBUG, whose
-kernels check every code and scale store (and the decode's loads) against
-the buffer sizes and report a range outside a buffer as MX_ERR_BOUNDS
-instead of touching it.
+request libmx_debug.so: the same sources compiled with MX_DEBUG, whose cast
+kernels (MX, dual and NVFP4) check every code and scale store, and the
+decode its loads, against the buffer sizes, and report a range outside a
+buffer as MX_ERR_BOUNDS instead of touching it.
 
 Usage: python -m microscaling_block_scaled_mx_b200.build [--force] [--debug]
 """
